@@ -1,0 +1,305 @@
+"""Pins of the oracle: checks against what the paper and mathematics fix.
+
+Every pin takes an ``Oracle`` and raises AssertionError on a mismatch.  None of
+them re-types the oracle's formulas: they compare against numpy/torch library
+routines (einsum, lexsort, scaled_dot_product_attention), brute force over
+tiny inputs, closed forms and hand-derived cases under tests/golden/.  The
+planted-mistake test runs all of them against deliberately wrong builds of the
+oracle and requires each build to fail at least one pin.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from helpers import (bf16_bits_to_f64, brute_expand, f32_to_bf16_bits, golden, lexsort_topk,
+                     numpy_scores, rand_bf16, sdpa_group, subset_topk)
+from long_context_decoding_anchor_b200 import synth
+from oracle import (CHAIN_ANCHOR, CHAIN_PREV, MODE_DENSE_ANCHOR, MODE_REFINE,
+                    MODE_STATIC_REUSE, bf16_bits)
+
+
+# -- Eq. (1): relevance score ---------------------------------------------------
+def pin_score_bruteforce(o):
+    """Scores equal numpy.einsum over group and head dim, 64-256 tokens."""
+    rng = np.random.default_rng(11)
+    for G, d, L in [(4, 64, 64), (2, 128, 256), (1, 16, 100), (8, 64, 128), (3, 32, 77)]:
+        q = rand_bf16(rng, (G, d))
+        k = rand_bf16(rng, (L, d))
+        scale = 1.0 / math.sqrt(d)
+        ref = numpy_scores(q, k, scale)
+        got = o.score(q, k, scale=scale)
+        assert np.allclose(got, ref, rtol=1e-12, atol=1e-12), "score vs einsum"
+        pos = np.sort(rng.choice(L, size=L // 3, replace=False)).astype(np.int32)
+        got = o.score(q, k, pos=pos, scale=scale)
+        assert np.allclose(got, ref[pos], rtol=1e-12, atol=1e-12), "score on a position list"
+
+
+def pin_score_hand(o):
+    """Hand case: q=(1,0), k_i=(i,0): scores increase, top-kappa = last kappa."""
+    g = golden("score_hand_case")
+    L, kappa = g["L"], g["kappa"]
+    q = f32_to_bf16_bits(np.array([[1.0, 0.0]], dtype=np.float32))
+    k = f32_to_bf16_bits(np.stack([np.arange(L), np.zeros(L)], 1).astype(np.float32))
+    s = o.score(q, k, scale=1.0)
+    assert np.array_equal(s, np.arange(L, dtype=np.float64)), "hand scores"
+    idx, keff = o.topk(s, kappa)
+    assert keff == kappa and list(idx) == g["expected_topk"], "hand top-kappa"
+
+
+# -- Eq. (2)/(6): exact top-kappa ------------------------------------------------
+def pin_topk_golden(o):
+    for c in golden("topk_cases")["cases"]:
+        pos = c.get("positions")
+        idx, keff = o.topk(np.array(c["scores"], dtype=np.float64), c["kappa"],
+                           pos=None if pos is None else np.array(pos))
+        assert list(idx) == c["expected"], f"topk golden {c}"
+        assert keff == sum(1 for x in c["expected"] if x >= 0)
+
+
+def pin_topk_lexsort(o):
+    """Top-kappa equals numpy.lexsort on (-score, position), ties included."""
+    rng = np.random.default_rng(12)
+    for n, kappa, ties in [(1000, 37, False), (1000, 37, True), (300, 300, True), (50, 80, True),
+                           (4096, 256, True), (1, 1, False), (257, 256, True)]:
+        s = rng.integers(-5, 6, n).astype(np.float64) if ties else rng.standard_normal(n)
+        if ties:
+            s[rng.random(n) < 0.1] = -0.0
+        pos = np.sort(rng.choice(4 * n, size=n, replace=False)).astype(np.int32)
+        for p in (None, pos):
+            idx, keff = o.topk(s, kappa, pos=p)
+            assert np.array_equal(idx, lexsort_topk(s, kappa, p)), "topk vs lexsort"
+            assert keff == min(kappa, n)
+
+
+def pin_topk_all_equal(o):
+    for n, kappa in [(10, 3), (4096, 256), (5, 5)]:
+        idx, _ = o.topk(np.full(n, 0.25), kappa)
+        assert list(idx) == list(range(kappa)), "all-equal scores select {0..kappa-1}"
+
+
+def pin_topk_subsets(o):
+    """Brute force over all kappa-subsets of at most 10 tokens."""
+    rng = np.random.default_rng(13)
+    for trial in range(40):
+        n = int(rng.integers(1, 11))
+        kappa = int(rng.integers(1, n + 2))
+        s = rng.integers(-2, 3, n).astype(np.float64)
+        ref, count = subset_topk(s, kappa)
+        assert count == 1, "the tie rule makes the top-kappa subset unique"
+        idx, _ = o.topk(s, kappa)
+        assert np.array_equal(idx, ref), "topk vs subset brute force"
+
+
+# -- positional proposal ---------------------------------------------------------
+def pin_expand_golden(o):
+    for c in golden("expand_cases")["cases"]:
+        got = o.expand(c["L"], np.array(c["idx_prev"], dtype=np.int32), c["r"])
+        assert list(got) == c["expected"], f"expand golden {c}"
+
+
+def pin_expand_bruteforce(o):
+    rng = np.random.default_rng(14)
+    for trial in range(60):
+        L = int(rng.integers(1, 300))
+        r = int(rng.integers(0, 12))
+        n = int(rng.integers(1, 40))
+        idx = rng.integers(-3, L + 3, n).astype(np.int32)
+        got = o.expand(L, idx, r)
+        assert np.array_equal(got, brute_expand(L, idx, r)), "expand vs set brute force"
+
+
+# -- SparseAttn -------------------------------------------------------------------
+def pin_attention_sdpa(o):
+    """Attention over an index set equals torch SDPA (fp64) with a mask; with
+    kappa = L it is dense attention."""
+    rng = np.random.default_rng(15)
+    for G, d, L, nsel in [(4, 64, 96, 96), (2, 128, 200, 31), (1, 32, 64, 64), (8, 64, 150, 40)]:
+        q, k, v = rand_bf16(rng, (G, d), 2.0), rand_bf16(rng, (L, d)), rand_bf16(rng, (L, d))
+        idx = np.sort(rng.choice(L, size=nsel, replace=False)).astype(np.int32)
+        idx = np.concatenate([idx, -np.ones(3, dtype=np.int32)])
+        scale = 1.0 / math.sqrt(d)
+        got, wsum = o.attention(q, k, v, idx, scale)
+        ref = sdpa_group(q, k, v, idx, scale)
+        assert np.allclose(got, ref, rtol=1e-10, atol=1e-12), "attention vs SDPA"
+        assert np.allclose(wsum, 1.0, rtol=0, atol=1e-12), "softmax weights sum to 1"
+
+
+def pin_attention_closed_forms(o):
+    # Two keys, d = 2, scale 1: logits 0 and 1, weights 1/(1+e) and e/(1+e).
+    q = f32_to_bf16_bits(np.array([[1.0, 0.0]], np.float32))
+    k = f32_to_bf16_bits(np.array([[0.0, 0.0], [1.0, 0.0]], np.float32))
+    v = f32_to_bf16_bits(np.array([[1.0, 0.0], [0.0, 1.0]], np.float32))
+    got, wsum = o.attention(q, k, v, np.array([0, 1], np.int32), scale=1.0)
+    e = math.e
+    assert np.allclose(got[0], [1 / (1 + e), e / (1 + e)], rtol=1e-14, atol=1e-15), "two-key closed form"
+    # Same keys with the default 1/sqrt(d) scale: logits 0 and 1/sqrt(2).
+    got, _ = o.attention(q, k, v, np.array([0, 1], np.int32))
+    w1 = 1.0 / (1.0 + math.exp(-1.0 / math.sqrt(2.0)))
+    assert np.allclose(got[0], [1 - w1, w1], rtol=1e-14, atol=1e-15), "default scale"
+    # All logits equal (identical key rows): the output is the mean of the V rows.
+    rng = np.random.default_rng(16)
+    G, d, L = 4, 64, 50
+    qg = rand_bf16(rng, (G, d))
+    krow = rand_bf16(rng, (1, d))
+    kk = np.repeat(krow, L, 0)
+    vv = rand_bf16(rng, (L, d))
+    idx = np.arange(0, L, 2, dtype=np.int32)
+    got, wsum = o.attention(qg, kk, vv, idx)
+    mean = bf16_bits_to_f64(vv)[idx].mean(0)
+    assert np.allclose(got, np.broadcast_to(mean, (G, d)), rtol=1e-13, atol=1e-14), "equal logits -> mean of V"
+    # Empty selection: zero output, zero weight.
+    got, wsum = o.attention(qg, kk, vv, -np.ones(4, np.int32))
+    assert np.all(got == 0.0) and np.all(wsum == 0.0), "empty selection"
+
+
+# -- Algorithm 1: decode step ----------------------------------------------------
+def _hand_inputs():
+    g = golden("decode_hand_case")
+    L, N = g["L"], len(g["x"])
+    q = np.zeros((N, 1, 1, 2), np.float32)
+    q[..., 0] = 1.0
+    ks, vs = [], []
+    for l in range(N):
+        k = np.zeros((1, 1, L, 2), np.float32)
+        for p, x in g["x"][l].items():
+            k[0, 0, int(p), 0] = x
+        v = np.stack([np.arange(L), np.ones(L)], 1).astype(np.float32).reshape(1, 1, L, 2)
+        ks.append(f32_to_bf16_bits(k))
+        vs.append(f32_to_bf16_bits(v))
+    return g, f32_to_bf16_bits(q), ks, vs, np.array([L], np.int32)
+
+
+def pin_decode_hand(o):
+    g, q, ks, vs, lens = _hand_inputs()
+    cases = {"refine_prev": (MODE_REFINE, CHAIN_PREV), "refine_anchor": (MODE_REFINE, CHAIN_ANCHOR),
+             "static_reuse": (MODE_STATIC_REUSE, CHAIN_PREV), "dense_anchor": (MODE_DENSE_ANCHOR, CHAIN_PREV)}
+    for name, (mode, chain) in cases.items():
+        _, idx = o.decode_step(q, ks, vs, lens, g["kappa"], g["r"], g["anchor_mask"],
+                               mode=mode, chain=chain, scale=g["scale"])
+        assert idx[:, 0, 0, :].tolist() == g["expected"][name], f"hand decode {name}"
+
+
+def small_workloads():
+    """Small synthetic workloads (64-256 tokens) with the generator's structure."""
+    w1 = synth.WORKLOADS[1].replace(max_len=256, n_layers=4, kappa=16, radius=2, n_clusters=4,
+                                    drift=4)
+    w2 = synth.WORKLOADS[2].replace(batch=2, max_len=192, n_layers=5, n_q_heads=8, n_kv_heads=2,
+                                    head_dim=64, kappa=24, radius=3, anchor_every=3, n_clusters=4,
+                                    drift=5, ragged=(100, 192))
+    w3 = synth.WORKLOADS[5].replace(max_len=64, n_layers=3, n_q_heads=8, n_kv_heads=1,
+                                    head_dim=32, kappa=8, radius=1, anchor_every=8,
+                                    n_clusters=2, drift=2)
+    return [w1, w2, w3]
+
+
+def _bits(inp):
+    q = bf16_bits(inp["q"])
+    ks = [bf16_bits(t) for t in inp["k"]]
+    vs = [bf16_bits(t) for t in inp["v"]]
+    return q, ks, vs, inp["lens"].cpu().numpy().astype(np.int32)
+
+
+def _numpy_chain(w, q, ks, lens, mode, chain, r):
+    """The decode step's selections recomputed with numpy: einsum scores,
+    lexsort top-kappa, set-based proposal."""
+    N, B, Hq, d = q.shape
+    H, G = w.n_kv_heads, w.group
+    scale = 1.0 / math.sqrt(d)
+    mask = w.anchor_mask()
+    idx = np.zeros((N, B, H, w.kappa), dtype=np.int64)
+    last_anchor = 0
+    for l in range(N):
+        anchor = mode == MODE_DENSE_ANCHOR or mask[l]
+        src = last_anchor if chain == CHAIN_ANCHOR else l - 1
+        for b in range(B):
+            L = int(lens[b])
+            for h in range(H):
+                qg = q[l, b, h * G:(h + 1) * G]
+                kr = ks[l][b, h, :L]
+                if anchor:
+                    idx[l, b, h] = lexsort_topk(numpy_scores(qg, kr, scale), w.kappa)
+                elif mode == MODE_STATIC_REUSE:
+                    idx[l, b, h] = idx[src, b, h]
+                else:
+                    P = brute_expand(L, idx[src, b, h], r)
+                    idx[l, b, h] = lexsort_topk(numpy_scores(qg, kr, scale, P), w.kappa, P)
+        if anchor:
+            last_anchor = l
+    return idx
+
+
+def pin_decode_numpy_chain(o):
+    """Every mode/chain of the decode step equals the numpy recomputation."""
+    for w in small_workloads():
+        q, ks, vs, lens = _bits(synth.make_inputs(w))
+        for mode, chain in [(MODE_REFINE, CHAIN_PREV), (MODE_REFINE, CHAIN_ANCHOR),
+                            (MODE_STATIC_REUSE, CHAIN_PREV), (MODE_DENSE_ANCHOR, CHAIN_PREV)]:
+            _, idx = o.decode_step(q, ks, vs, lens, w.kappa, w.radius, w.anchor_mask(),
+                                   mode=mode, chain=chain)
+            ref = _numpy_chain(w, q, ks, lens, mode, chain, w.radius)
+            assert np.array_equal(idx, ref), f"decode chain vs numpy ({w.name}, {mode}, {chain})"
+
+
+def pin_decode_outputs_sdpa(o):
+    """Each layer's output equals masked SDPA over that layer's selection."""
+    for w in small_workloads()[:2]:
+        q, ks, vs, lens = _bits(synth.make_inputs(w))
+        out, idx = o.decode_step(q, ks, vs, lens, w.kappa, w.radius, w.anchor_mask())
+        N, B, Hq, d = q.shape
+        G = w.group
+        for l in range(N):
+            for b in range(B):
+                L = int(lens[b])
+                for h in range(w.n_kv_heads):
+                    ref = sdpa_group(q[l, b, h * G:(h + 1) * G], ks[l][b, h, :L], vs[l][b, h, :L],
+                                     idx[l, b, h], 1.0 / math.sqrt(d))
+                    assert np.allclose(out[l, b, h * G:(h + 1) * G], ref, rtol=1e-10, atol=1e-12), \
+                        "decode output vs SDPA"
+
+
+def pin_decode_invariants(o):
+    """Invariants the method fixes:
+    r >= L: the refined selection is the exact per-layer top-kappa;
+    r = 0 refinement selects the same sets as static reuse;
+    static reuse repeats the anchor's selection on every layer;
+    kappa = L: every layer's output is dense attention."""
+    w = small_workloads()[1]
+    q, ks, vs, lens = _bits(synth.make_inputs(w))
+    mask = w.anchor_mask()
+    _, dense = o.decode_step(q, ks, vs, lens, w.kappa, w.radius, mask, mode=MODE_DENSE_ANCHOR)
+    _, wide = o.decode_step(q, ks, vs, lens, w.kappa, w.max_len, mask, mode=MODE_REFINE)
+    assert np.array_equal(wide, dense), "r >= L equals per-layer exact selection"
+    _, r0 = o.decode_step(q, ks, vs, lens, w.kappa, 0, mask, mode=MODE_REFINE)
+    _, st = o.decode_step(q, ks, vs, lens, w.kappa, w.radius, mask, mode=MODE_STATIC_REUSE)
+    assert np.array_equal(r0, st), "r = 0 refinement equals static reuse"
+    last = 0
+    for l in range(len(mask)):
+        if mask[l]:
+            last = l
+            assert np.array_equal(st[l], dense[l]), "anchor layers select exactly"
+        assert np.array_equal(st[l], st[last]), "static reuse repeats the anchor"
+    # kappa = Lmax: sparse attention over everything = dense attention.
+    out, idx = o.decode_step(q, ks, vs, lens, w.max_len, w.radius, mask, mode=MODE_REFINE)
+    N, B, Hq, d = q.shape
+    G = w.group
+    for l in range(N):
+        for b in range(B):
+            L = int(lens[b])
+            for h in range(w.n_kv_heads):
+                assert np.array_equal(idx[l, b, h, :L], np.arange(L)), "kappa=L selects all"
+                ref = sdpa_group(q[l, b, h * G:(h + 1) * G], ks[l][b, h, :L], vs[l][b, h, :L],
+                                 np.arange(L), 1.0 / math.sqrt(d))
+                assert np.allclose(out[l, b, h * G:(h + 1) * G], ref, rtol=1e-10, atol=1e-12), \
+                    "kappa = L equals dense attention"
+
+
+ALL_PINS = [pin_score_bruteforce, pin_score_hand, pin_topk_golden, pin_topk_lexsort,
+            pin_topk_all_equal, pin_topk_subsets, pin_expand_golden, pin_expand_bruteforce,
+            pin_attention_sdpa, pin_attention_closed_forms, pin_decode_hand,
+            pin_decode_numpy_chain, pin_decode_outputs_sdpa, pin_decode_invariants]
+
+__all__ = ["ALL_PINS", "small_workloads"] + [p.__name__ for p in ALL_PINS]
+_ = torch  # torch is used through helpers.sdpa_group and synth
