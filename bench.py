@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark: Prism Attention decode step at 128K context on B200.
+
+Workload (the 128K long-context decode): batch 1, context 131072, 32 layers
+(anchor every 4), 32 query / 8 KV heads, head_dim 128, kappa 2048, r 8, bf16
+KV cache (~17 GB) from the seeded synthetic generator.  A step is one
+prism_decode_step over all 32 layers (anchor scoring + exact top-kappa on
+anchor layers, +-r proposal / rescoring / top-kappa on refined layers, sparse
+GQA attention on every layer), replayed from a CUDA graph with every input
+already in HBM.  Every step touches ~4 GB of distinct K/V bytes, far more than
+the 126 MB L2, so no flush is needed between steps.
+
+One JSON line on rank 0.  ``--impl reference`` times the oracle (plain C,
+fp64) on the host cores instead, on a bounded sample of the same workload.
+Multi-GPU (torchrun): every rank runs its own replica (no collective on the
+data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("decode-step µs/layer at 128K ctx; index+attn HBM GB/s as fraction of "
+          "B200 peak")
+UNIT = "us/layer"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["prism", "reference"], default="prism")
+    ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches")
+    ap.add_argument("--cpu-layers", type=int, default=8,
+                    help="layers of the workload in the CPU-baseline sample")
+    ap.add_argument("--ref-layers", type=int, default=4,
+                    help="layers per step of the reference (oracle) arm")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.path = tempfile.mktemp(prefix="prism_clocks_", suffix=".csv")
+        self.proc = None
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", gpu_id], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id_for(dev) -> str:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index or 0)
+
+
+# --------------------------------------------------------------------------- helpers
+def anchor_bytes(w, lens):
+    return int(sum(int(L) for L in lens)) * w.n_kv_heads * w.head_dim * 2
+
+
+def kernel_traffic(src_paths, profile_md):
+    """DRAM bytes per launch of the anchor scoring kernel from a committed ncu
+    summary, valid only while the kernel's sources are unchanged."""
+    try:
+        text = open(profile_md).read()
+    except OSError:
+        return None
+    h = hashlib.sha256()
+    for p in src_paths:
+        h.update(open(p, "rb").read())
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_sha or not m_tr or m_sha.group(1) != h.hexdigest():
+        return None
+    return int(m_tr.group(1))
+
+
+def oracle_sample(w, inp, layers, heads):
+    """Host copies (uint16 bits) of layers x KV heads of the workload."""
+    from oracle import bf16_bits
+    G = w.group
+    h0, h1 = heads
+    q = bf16_bits(inp["q"][layers[0]:layers[-1] + 1, :, h0 * G:h1 * G])
+    ks = [bf16_bits(inp["k"][l][:, h0:h1]) for l in layers]
+    vs = [bf16_bits(inp["v"][l][:, h0:h1]) for l in layers]
+    lens = inp["lens"].cpu().numpy()
+    mask = [inp["anchor_mask"][l] for l in layers]
+    return q, ks, vs, lens, mask
+
+
+def time_oracle(w, sample, reps=1):
+    import oracle
+    o = oracle.load()
+    q, ks, vs, lens, mask = sample
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        o.decode_step(q, ks, vs, lens, w.kappa, w.radius, mask)
+    return (time.perf_counter() - t0) / reps, o.num_threads()
+
+
+# --------------------------------------------------------------------------- arms
+def run_reference(args, rank, world):
+    """The oracle on the host cores, on a bounded sample of the workload."""
+    import torch
+    from long_context_decoding_anchor_b200 import synth
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    layers = list(range(args.ref_layers))
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = synth.make_inputs(w, device=dev, layers=layers)
+    sample = oracle_sample(w, inp, layers, (0, w.n_kv_heads))
+    del inp
+    for _ in range(args.warmup):
+        time_oracle(w, sample)
+    times = []
+    threads = 1
+    for _ in range(args.steps):
+        t, threads = time_oracle(w, sample)
+        times.append(t)
+    ms = statistics.mean(times) * 1e3
+    value = ms * 1e3 / len(layers)
+    cores = min(threads, w.rows)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{w.name}: {w.describe()}", "sample_layers": layers,
+                   "kv_heads": w.n_kv_heads},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"layers {layers[0]}-{layers[-1]} (1 anchor + "
+                                   f"{len(layers) - 1} refined) x all {w.n_kv_heads} KV heads "
+                                   f"of the 128K workload, per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_prism(args, rank, world, dev):
+    import torch
+    import long_context_decoding_anchor_b200 as prism
+    from long_context_decoding_anchor_b200 import build as prism_build, synth
+    from long_context_decoding_anchor_b200.runner import DecodeStepGraph
+
+    if not os.path.exists(prism.LIB_PATH):
+        prism_build.build()
+    prism.lib()
+    w = synth.WORKLOADS[args.workload]
+    inp = synth.make_inputs(w, device=dev)
+    cfg = prism.Config.from_workload(w)
+    ws = prism.workspace(cfg, dev)
+    N = w.n_layers
+    lens_h = inp["lens"].cpu().tolist()
+    torch.cuda.synchronize(dev)
+
+    # -- eager reference run: selections (for |P| accounting) and status check
+    out_e, idx_e = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                           want_idx=True, ws=ws)
+    st, detail = prism.prism_check_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} {detail}")
+    mask = w.anchor_mask()
+    prop_sizes = []
+    last_anchor = 0
+    for l in range(N):
+        if mask[l]:
+            last_anchor = l
+            continue
+        _, _, _, cc = prism.prism_index_refine(cfg, inp["q"][l], inp["k"][l], inp["lens"],
+                                               idx_e[l - 1].contiguous(), cand_cap=1, ws=ws)
+        prop_sizes.append(int(cc.sum()))
+    n_anchor = sum(mask)
+    kappa_eff = sum(min(w.kappa, int(L)) for L in lens_h) * w.n_kv_heads
+    gather = kappa_eff * w.head_dim * 2 * 2
+    a_bytes = anchor_bytes(w, lens_h)
+    step_bytes = n_anchor * a_bytes + sum(prop_sizes) * w.head_dim * 2 + N * gather
+
+    # -- the timed step: CUDA-graph replay of the whole decode step
+    if args.no_graph:
+        runner = None
+        launches_per_step = None
+
+        def step():
+            prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], out=out_e,
+                                    ws=ws)
+        n0 = prism.lib().prism_launch_count()
+        step()
+        launches_per_step = int(prism.lib().prism_launch_count() - n0)
+    else:
+        runner = DecodeStepGraph(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], ws=ws)
+        launches_per_step = runner.launches
+        step = runner.replay
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(gpu_id_for(dev))
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    st, detail = prism.prism_check_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status after timing {st} {detail}")
+    value = ms * 1e3 / (N * world)
+    peak, peak_kind = peaks()
+    step_gbs = step_bytes / (ms * 1e-3) / 1e9
+
+    # -- dominant kernel: anchor scoring alone, CUDA events around each launch
+    anchors = [l for l in range(N) if mask[l]]
+    S = torch.empty((w.batch, w.n_kv_heads, w.max_len), dtype=torch.float32, device=dev)
+    L = prism.lib()
+    import ctypes
+    cfgp = ctypes.byref(cfg)
+
+    def score_launch(l):
+        rc = L.prism_score_anchor(cfgp, ctypes.c_void_p(inp["q"][l].data_ptr()),
+                                  ctypes.c_void_p(inp["k"][l].data_ptr()),
+                                  ctypes.c_void_p(inp["lens"].data_ptr()),
+                                  ctypes.c_void_p(S.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                  ws.numel(), ctypes.c_void_p(stream.cuda_stream))
+        if rc != 0:
+            raise RuntimeError(f"prism_score_anchor: {rc}")
+    for i in range(3):
+        score_launch(anchors[i % len(anchors)])
+    n_k = max(args.steps, 16)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_k)]
+    for i in range(n_k):
+        evs[i][0].record(stream)
+        score_launch(anchors[i % len(anchors)])
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    t_score = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e-3
+    ach = a_bytes / t_score / 1e9
+    score_src = [os.path.join(ROOT, "long_context_decoding_anchor_b200", "csrc", f)
+                 for f in ("score.cu", "prism_internal.cuh")]
+    traffic = kernel_traffic(score_src, os.path.join(ROOT, "profiles", "anchor_score_128k.md"))
+
+    # -- per-stage breakdown (events around each public stage call)
+    def timed(fn, reps=8):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        fn(0)
+        for i in range(reps):
+            ev[i][0].record(stream)
+            fn(i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+    refines = [l for l in range(N) if not mask[l]]
+    idx_tmp = torch.empty((w.batch, w.n_kv_heads, w.kappa), dtype=torch.int32, device=dev)
+    out_tmp = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+    br = {
+        "anchor_index": timed(lambda i: prism.prism_index_anchor(
+            cfg, inp["q"][anchors[i % len(anchors)]], inp["k"][anchors[i % len(anchors)]],
+            inp["lens"], idx_out=idx_tmp, ws=ws, stream=stream)),
+        "refine_index": timed(lambda i: prism.prism_index_refine(
+            cfg, inp["q"][refines[i % len(refines)]], inp["k"][refines[i % len(refines)]],
+            inp["lens"], idx_e[refines[i % len(refines)] - 1].contiguous(), idx_out=idx_tmp,
+            ws=ws, stream=stream)),
+        "sparse_attn": timed(lambda i: prism.prism_sparse_decode(
+            cfg, inp["q"][i % N], inp["k"][i % N], inp["v"][i % N], inp["lens"],
+            idx_e[i % N].contiguous(), out=out_tmp, ws=ws, stream=stream)),
+        "anchor_score_kernel": t_score * 1e6,
+    }
+    br["anchor_layer"] = br["anchor_index"] + br["sparse_attn"]
+    br["refine_layer"] = br["refine_index"] + br["sparse_attn"]
+
+    # -- end to end through the public call, host buffers, copies in the timed region
+    e2e = None
+    if not args.skip_e2e:
+        q_h = inp["q"].cpu().pin_memory()
+        lens_hp = inp["lens"].cpu().pin_memory()
+        out_h = torch.empty(out_e.shape, dtype=out_e.dtype).pin_memory()
+        q_d = torch.empty_like(inp["q"])
+        out_d = torch.empty_like(out_e)
+
+        def e2e_step():
+            q_d.copy_(q_h, non_blocking=True)
+            inp["lens"].copy_(lens_hp, non_blocking=True)
+            prism.prism_decode_step(cfg, q_d, inp["k"], inp["v"], inp["lens"], out=out_d, ws=ws,
+                                    stream=stream)
+            out_h.copy_(out_d, non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e2e = a.elapsed_time(b) / args.steps
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": ms_e2e * 1e3 / (N * world), "unit": UNIT,
+               "h2d_bytes_per_step": q_h.numel() * 2 + lens_hp.numel() * 4,
+               "d2h_bytes_per_step": out_h.numel() * 2,
+               "path": "prism_decode_step (eager, public C ABI) with pinned host q/len in "
+                       "and out back, KV cache resident"}
+
+    # -- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if not args.skip_cpu and rank == 0 and world == 1:
+        layers = list(range(min(args.cpu_layers, N)))
+        sample = oracle_sample(w, inp, layers, (0, w.n_kv_heads))
+        t_cpu, threads = time_oracle(w, sample)
+        cpu = {"value": t_cpu * 1e6 / len(layers), "unit": UNIT,
+               "cores": min(threads, w.rows), "kind": "oracle",
+               "sample": f"layers 0-{layers[-1]} ({sum(mask[:len(layers)])} anchor + "
+                         f"{len(layers) - sum(mask[:len(layers)])} refined) x all "
+                         f"{w.n_kv_heads} KV heads, one pass ({t_cpu:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: {w.describe()}", "global_batch": w.batch * world,
+                       "seq_len": w.max_len, "parallelism": f"replicas x{world}",
+                       "graph": not args.no_graph,
+                       "l2": "no flush: each step reads ~%.1f GB of distinct K/V, > 126 MB L2"
+                             % (step_bytes / 1e9)},
+            "layers_per_s": 1e6 / value,
+            "step_hbm": {"algorithmic_bytes": step_bytes, "gbs": step_gbs,
+                         "frac": step_gbs / peak, "peak": peak, "peak_kind": peak_kind,
+                         "proposal_sizes": {"mean_per_row": statistics.mean(prop_sizes)
+                                            / w.rows if prop_sizes else 0}},
+            "roofline": {"kernel": "k_anchor_score", "bound": "hbm", "achieved": ach,
+                         "peak": peak, "unit": "GB/s", "frac": ach / peak, "traffic": traffic,
+                         "bytes_per_launch": a_bytes, "us_per_launch": t_score * 1e6,
+                         "peak_kind": peak_kind},
+            "breakdown_us": br,
+            "gpu_launches": launches_per_step * args.steps,
+            "launches_per_step": launches_per_step,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if runner is not None:
+        del runner
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=dev)
+    try:
+        run_prism(args, rank, world, dev)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

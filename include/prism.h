@@ -1,0 +1,221 @@
+/*
+ * prism.h -- C ABI of the Prism Attention decode hot path on B200 (sm_100a).
+ *
+ * Source of every operation: "Prism Attention: Proposal-Refined Index Sharing
+ * Mechanism for Efficient LLMs Inference" (arXiv 2610.22985), section 4.1
+ * (equations (1)-(6)) and Algorithm 1 (PrismAttention decoding at step t).
+ *
+ * The decode step walks a group of layers.  An anchor (proposal) layer scores
+ * every cached token and keeps the exact top-kappa tokens; a refined layer
+ * expands the source selection by +-r positions into a deduplicated proposal
+ * set, rescores only that set with its own query and keys, and keeps its own
+ * top-kappa; every layer then runs sparse GQA decode attention over its
+ * kappa selected K/V rows.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named q, k, v, out, idx*, cand*, len, ws are DEVICE pointers on
+ *    the current CUDA device; the caller owns every buffer.  The library
+ *    allocates nothing and keeps no state between calls other than a few
+ *    per-device attribute caches.
+ *  - Layouts (row-major, no padding between rows):
+ *      q    bf16 [B][Hq][d]            one decode query per sequence
+ *      k, v bf16 [B][Hkv][Lmax][d]     KV cache of one layer; position i of
+ *                                       sequence b is row i of every head
+ *      len  int32 [B]                  context length of each sequence,
+ *                                       0 <= len[b] <= Lmax
+ *      idx  int32 [B][Hkv][kappa]      a selection: token positions in
+ *                                       ascending order, then -1 padding
+ *    Query head j reads KV head j / (Hq / Hkv).
+ *  - Alignment: q, k, v, out 16 bytes; int32 arrays 4 bytes; ws 256 bytes.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream), makes no host synchronisation, allocates no memory and
+ *    can be captured into a CUDA graph.
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid argument returns PRISM_ERR_INVALID_ARG (or PRISM_ERR_UNSUPPORTED
+ *    for a shape the kernels do not cover, PRISM_ERR_WORKSPACE for a short
+ *    workspace) and launches nothing.  A launch failure returns
+ *    PRISM_ERR_CUDA.
+ *  - Device-side contract violations (len[b] outside [0, Lmax], a selected
+ *    index outside [0, len[b])) are clamped or skipped by the kernels, which
+ *    also record the first such event in the workspace status word; a wait
+ *    that runs past its time limit records PRISM_ERR_TIMEOUT there.  Read it
+ *    with prism_check_device_status().
+ *  - Scores are fp32 (bf16 inputs, fp32 accumulation).  Ties in a top-kappa
+ *    selection go to the lower position; -0.0 ties with +0.0.
+ */
+#ifndef PRISM_H
+#define PRISM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PRISM_API __attribute__((visibility("default")))
+#else
+#define PRISM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PRISM_OK = 0,
+    PRISM_ERR_INVALID_ARG = 1,
+    PRISM_ERR_UNSUPPORTED = 2,
+    PRISM_ERR_WORKSPACE = 3,
+    PRISM_ERR_CUDA = 4,
+    PRISM_ERR_TIMEOUT = 5,
+    PRISM_ERR_DEVICE = 6
+} prism_status_t;
+
+/* Decode-step variants (Algorithm 1 and its special cases).
+ * REFINE:        anchor layers select exactly (Eq. (1)-(2)); other layers
+ *                expand +-radius, rescore (Eq. (5)) and reselect (Eq. (6)).
+ * STATIC_REUSE:  other layers reuse the source selection unchanged (Eq. (3)).
+ * DENSE_ANCHOR:  every layer is an anchor layer (per-layer exact top-kappa). */
+typedef enum {
+    PRISM_MODE_REFINE = 0,
+    PRISM_MODE_STATIC_REUSE = 1,
+    PRISM_MODE_DENSE_ANCHOR = 2
+} prism_mode_t;
+
+/* Source selection of a refined layer.
+ * PREV:   the previous layer's final selection (default).
+ * ANCHOR: the most recent anchor layer's selection (the association f(S) of
+ *         Algorithm 1). */
+typedef enum {
+    PRISM_CHAIN_PREV = 0,
+    PRISM_CHAIN_ANCHOR = 1
+} prism_chain_t;
+
+/* Shape and policy of one decode step.  All fields are plain int32/float so
+ * that the struct has the same layout from C, C++ and Python (ctypes). */
+typedef struct {
+    int32_t batch;          /* B >= 1                                         */
+    int32_t n_q_heads;      /* Hq >= 1                                        */
+    int32_t n_kv_heads;     /* Hkv >= 1, Hq % Hkv == 0, G = Hq/Hkv in {1,2,4,8,16} */
+    int32_t head_dim;       /* d in {64, 128}                                 */
+    int32_t max_len;        /* Lmax, 1 <= Lmax <= PRISM_MAX_LEN               */
+    int32_t kappa;          /* sparse budget, 1 <= kappa <= PRISM_MAX_LEN     */
+    int32_t radius;         /* proposal radius r >= 0                         */
+    int32_t n_layers;       /* N >= 1 (prism_decode_step only)                */
+    const uint8_t *anchor_mask; /* HOST array [N]; nonzero = anchor layer;
+                                   mask[0] must be nonzero unless DENSE_ANCHOR
+                                   (prism_decode_step only; may be NULL for the
+                                   single-stage calls)                        */
+    int32_t mode;           /* prism_mode_t                                   */
+    int32_t chain;          /* prism_chain_t                                  */
+    float scale;            /* score/logit scale; 0 means 1/sqrt(d)           */
+} prism_config_t;
+
+#define PRISM_MAX_LEN (1 << 20)
+#define PRISM_MAX_BATCH_ROWS 65535   /* B * Hkv */
+
+/* Bytes of workspace every call below needs for `cfg` (the same figure serves
+ * all of them).  The workspace holds scores, candidate lists, histograms,
+ * selections and attention partials; its first 256 bytes are the device
+ * status word.  Pass it 256-byte aligned.  Its contents need no
+ * initialisation and are scratch between calls, except the status word,
+ * which persists until prism_check_device_status() reads it.
+ * Errors: PRISM_ERR_INVALID_ARG / PRISM_ERR_UNSUPPORTED for a bad config. */
+PRISM_API prism_status_t prism_workspace_size(const prism_config_t *cfg, size_t *bytes);
+
+/* Anchor layer index construction: Eq. (1) over every cached token, then the
+ * exact top-kappa of Eq. (2).
+ *   s[b][h][i] = scale * sum_{j in G(h)} <q[b][j], k[b][h][i]>, i < len[b]
+ *   idx_out[b][h] = the min(kappa, len[b]) positions with the largest s,
+ *                   ties to the lower position, ascending, -1 padded.
+ * q          bf16 [B][Hq][d]           k bf16 [B][Hkv][Lmax][d]
+ * len        int32 [B]                 idx_out int32 [B][Hkv][kappa] (written)
+ * scores_out fp32 [B][Hkv][Lmax] or NULL; when given, receives s (entries at
+ *            i >= len[b] are left untouched).                                */
+PRISM_API prism_status_t prism_index_anchor(const prism_config_t *cfg, const void *q,
+                                  const void *k, const int32_t *len,
+                                  int32_t *idx_out, float *scores_out,
+                                  void *ws, size_t ws_bytes, void *stream);
+
+/* Anchor scoring only: Eq. (1) over every cached token, exactly one kernel
+ * launch (the streaming kernel that prism_index_anchor starts with).  Meant
+ * for timing that kernel on its own and for diagnostics.
+ * scores_out fp32 [B][Hkv][Lmax] (written for i < len[b]).  The first-digit
+ * histogram region of the workspace is accumulated, not reset, by this call;
+ * the other calls reset it before use. */
+PRISM_API prism_status_t prism_score_anchor(const prism_config_t *cfg, const void *q,
+                                  const void *k, const int32_t *len,
+                                  float *scores_out, void *ws, size_t ws_bytes,
+                                  void *stream);
+
+/* Refined layer index refinement: proposal P = { p : |p - i| <= radius for
+ * some i in idx_prev[b][h], 0 <= p < len[b] } (a set, so duplicates vanish);
+ * the scores of Eq. (5) on P only, with this layer's q and k; then the
+ * top-kappa of Eq. (6) over P, same tie and order rules as the anchor.
+ * idx_prev   int32 [B][Hkv][kappa]: entries < 0 are padding and skipped; any
+ *            order is accepted.
+ * idx_out    int32 [B][Hkv][kappa] (written; may not alias idx_prev).
+ * cand_pos, cand_score, cand_count: optional diagnostic copies of P (all
+ *            three NULL, or all three given): cand_pos int32 [B][Hkv][cand_cap]
+ *            ascending positions, cand_score fp32 [B][Hkv][cand_cap] their
+ *            scores, cand_count int32 [B][Hkv] = |P| (entries beyond
+ *            cand_cap are not stored).                                       */
+PRISM_API prism_status_t prism_index_refine(const prism_config_t *cfg, const void *q,
+                                  const void *k, const int32_t *len,
+                                  const int32_t *idx_prev, int32_t *idx_out,
+                                  int32_t *cand_pos, float *cand_score,
+                                  int32_t *cand_count, int32_t cand_cap,
+                                  void *ws, size_t ws_bytes, void *stream);
+
+/* Sparse GQA decode attention (the SparseAttn step of Algorithm 1): for every
+ * query head j of KV head h,
+ *   z_i = scale * <q[b][j], k[b][h][i]>,  i in idx[b][h] (entries < 0 skipped)
+ *   out[b][j] = sum_i softmax(z)_i * v[b][h][i]   (0 if nothing is selected)
+ * computed split-K with an online softmax and a final combine.
+ * idx   int32 [B][Hkv][n_idx], 1 <= n_idx <= kappa   out bf16 [B][Hq][d]     */
+PRISM_API prism_status_t prism_sparse_decode(const prism_config_t *cfg, const void *q,
+                                   const void *k, const void *v,
+                                   const int32_t *len, const int32_t *idx,
+                                   int32_t n_idx, void *out, void *ws,
+                                   size_t ws_bytes, void *stream);
+
+/* One decode step over cfg->n_layers layers (Algorithm 1), per cfg->mode and
+ * cfg->chain, every layer ending in sparse attention over its own selection.
+ * q        bf16 [N][B][Hq][d] (device)
+ * k, v     HOST arrays of N device pointers, each bf16 [B][Hkv][Lmax][d]
+ * len      int32 [B] (device)
+ * out      bf16 [N][B][Hq][d] (written)
+ * idx_out  int32 [N][B][Hkv][kappa] or NULL: every layer's selection.        */
+PRISM_API prism_status_t prism_decode_step(const prism_config_t *cfg, const void *q,
+                                 const void *const *k, const void *const *v,
+                                 const int32_t *len, void *out,
+                                 int32_t *idx_out, void *ws, size_t ws_bytes,
+                                 void *stream);
+
+/* Synchronises `stream`, reads the workspace status word and clears it.
+ * Returns PRISM_OK, PRISM_ERR_TIMEOUT (a bounded wait ran out) or
+ * PRISM_ERR_DEVICE (a device-side contract violation); `detail` (nullable)
+ * receives {code, where, value, 0}. */
+PRISM_API prism_status_t prism_check_device_status(void *ws, size_t ws_bytes,
+                                         void *stream, uint32_t detail[4]);
+
+/* Test hook for the bounded waits: launches one CTA that waits on a barrier
+ * nothing will complete, for at most `limit_ns` nanoseconds, then records
+ * PRISM_ERR_TIMEOUT in the status word and returns.  It never hangs. */
+PRISM_API prism_status_t prism_debug_wait_timeout(void *ws, size_t ws_bytes,
+                                        uint64_t limit_ns, void *stream);
+
+/* Static, human-readable name of a status code. */
+PRISM_API const char *prism_status_string(prism_status_t status);
+
+/* Number of kernels the calling host thread has launched through this
+ * library since it was loaded (memsets and copies excluded). */
+PRISM_API uint64_t prism_launch_count(void);
+
+/* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
+PRISM_API int32_t prism_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PRISM_H */

@@ -1,1 +1,286 @@
-"""Prism Attention decode hot path for B200 (sm_100a)."""
+"""Prism Attention decode hot path for B200 (sm_100a): Python binding.
+
+A thin ctypes layer over the C ABI of ``libprism.so`` (declared in
+``include/prism.h``).  It only marshals arguments: torch tensors provide
+device memory and streams, every step of the computation runs in the CUDA
+kernels of the library.  There is no fallback: if the library is missing or
+cannot be loaded, every call raises.
+
+Functions carry the C names:
+  prism_workspace_size, prism_index_anchor, prism_index_refine,
+  prism_sparse_decode, prism_decode_step, prism_check_device_status,
+  prism_debug_wait_timeout
+plus ``Config`` (the prism_config_t struct) and ``workspace()``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libprism.so")
+
+MODE_REFINE, MODE_STATIC_REUSE, MODE_DENSE_ANCHOR = 0, 1, 2
+CHAIN_PREV, CHAIN_ANCHOR = 0, 1
+STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED",
+          3: "PRISM_ERR_WORKSPACE", 4: "PRISM_ERR_CUDA", 5: "PRISM_ERR_TIMEOUT",
+          6: "PRISM_ERR_DEVICE"}
+EXPORTS = ("prism_workspace_size", "prism_index_anchor", "prism_index_refine",
+           "prism_sparse_decode", "prism_decode_step", "prism_check_device_status",
+           "prism_debug_wait_timeout", "prism_score_anchor", "prism_status_string",
+           "prism_version", "prism_launch_count")
+
+
+class PrismError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({_status_text(status)})")
+
+
+class Config(ctypes.Structure):
+    """prism_config_t."""
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("max_len", ctypes.c_int32), ("kappa", ctypes.c_int32),
+                ("radius", ctypes.c_int32), ("n_layers", ctypes.c_int32),
+                ("anchor_mask", ctypes.POINTER(ctypes.c_uint8)),
+                ("mode", ctypes.c_int32), ("chain", ctypes.c_int32),
+                ("scale", ctypes.c_float)]
+
+    @classmethod
+    def make(cls, batch, n_q_heads, n_kv_heads, head_dim, max_len, kappa, radius=0,
+             n_layers=1, anchor_mask: Optional[Sequence[int]] = None, mode=MODE_REFINE,
+             chain=CHAIN_PREV, scale=0.0) -> "Config":
+        c = cls(batch, n_q_heads, n_kv_heads, head_dim, max_len, kappa, radius, n_layers,
+                None, mode, chain, scale)
+        if anchor_mask is not None:
+            arr = (ctypes.c_uint8 * len(anchor_mask))(*[1 if x else 0 for x in anchor_mask])
+            c._mask_keepalive = arr
+            c.anchor_mask = ctypes.cast(arr, ctypes.POINTER(ctypes.c_uint8))
+        return c
+
+    @classmethod
+    def from_workload(cls, w, **kw) -> "Config":
+        args = dict(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                    head_dim=w.head_dim, max_len=w.max_len, kappa=w.kappa, radius=w.radius,
+                    n_layers=w.n_layers, anchor_mask=w.anchor_mask())
+        args.update(kw)
+        return cls.make(**args)
+
+    @property
+    def rows(self) -> int:
+        return self.batch * self.n_kv_heads
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libprism.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m long_context_decoding_anchor_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32, u64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_uint64
+        cfgp = ctypes.POINTER(Config)
+        L.prism_workspace_size.argtypes = [cfgp, ctypes.POINTER(sz)]
+        L.prism_index_anchor.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_score_anchor.argtypes = [cfgp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_score_anchor.restype = ctypes.c_int
+        L.prism_launch_count.restype = ctypes.c_uint64
+        L.prism_launch_count.argtypes = []
+        L.prism_index_refine.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
+        L.prism_sparse_decode.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
+        L.prism_decode_step.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_check_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)]
+        L.prism_debug_wait_timeout.argtypes = [vp, sz, u64, vp]
+        L.prism_status_string.argtypes = [ctypes.c_int]
+        L.prism_status_string.restype = ctypes.c_char_p
+        L.prism_version.restype = i32
+        for name in EXPORTS[:8]:
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _status_text(st: int) -> str:
+    try:
+        return lib().prism_status_string(st).decode()
+    except Exception:
+        return "?"
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise PrismError(st, where)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def prism_workspace_size(cfg: Config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().prism_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "prism_workspace_size")
+    return n.value
+
+
+def workspace(cfg: Config, device=None) -> torch.Tensor:
+    """A workspace buffer for ``cfg`` (uint8; torch allocations are 512-byte aligned)."""
+    return torch.empty(prism_workspace_size(cfg), dtype=torch.uint8,
+                       device=device or torch.device("cuda"))
+
+
+def prism_index_anchor(cfg: Config, q, k, lens, idx_out=None, scores_out=None, ws=None,
+                       stream=None):
+    B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
+    _need(q, "q", torch.bfloat16, (B, Hq, d))
+    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need(lens, "lens", torch.int32, (B,))
+    if idx_out is None:
+        idx_out = torch.empty((B, Hkv, cfg.kappa), dtype=torch.int32, device=q.device)
+    _need(idx_out, "idx_out", torch.int32, (B, Hkv, cfg.kappa))
+    if scores_out is not None:
+        _need(scores_out, "scores_out", torch.float32, (B, Hkv, L))
+    ws = workspace(cfg, q.device) if ws is None else ws
+    _check(lib().prism_index_anchor(ctypes.byref(cfg), _p(q), _p(k), _p(lens), _p(idx_out),
+                                    _p(scores_out), _p(ws), ws.numel(), _stream(stream)),
+           "prism_index_anchor")
+    return idx_out
+
+
+def prism_score_anchor(cfg: Config, q, k, lens, scores_out=None, ws=None, stream=None):
+    """Eq. (1) only: one launch of the anchor scoring kernel."""
+    B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
+    _need(q, "q", torch.bfloat16, (B, Hq, d))
+    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need(lens, "lens", torch.int32, (B,))
+    if scores_out is None:
+        scores_out = torch.empty((B, Hkv, L), dtype=torch.float32, device=q.device)
+    _need(scores_out, "scores_out", torch.float32, (B, Hkv, L))
+    ws = workspace(cfg, q.device) if ws is None else ws
+    _check(lib().prism_score_anchor(ctypes.byref(cfg), _p(q), _p(k), _p(lens), _p(scores_out),
+                                    _p(ws), ws.numel(), _stream(stream)),
+           "prism_score_anchor")
+    return scores_out
+
+
+def prism_index_refine(cfg: Config, q, k, lens, idx_prev, idx_out=None, cand_cap=0, ws=None,
+                       stream=None):
+    """Returns idx_out, or (idx_out, cand_pos, cand_score, cand_count) when cand_cap > 0."""
+    B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
+    _need(q, "q", torch.bfloat16, (B, Hq, d))
+    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need(lens, "lens", torch.int32, (B,))
+    _need(idx_prev, "idx_prev", torch.int32, (B, Hkv, cfg.kappa))
+    if idx_out is None:
+        idx_out = torch.empty((B, Hkv, cfg.kappa), dtype=torch.int32, device=q.device)
+    _need(idx_out, "idx_out", torch.int32, (B, Hkv, cfg.kappa))
+    cp = cs = cc = None
+    if cand_cap > 0:
+        cp = torch.empty((B, Hkv, cand_cap), dtype=torch.int32, device=q.device)
+        cs = torch.empty((B, Hkv, cand_cap), dtype=torch.float32, device=q.device)
+        cc = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    ws = workspace(cfg, q.device) if ws is None else ws
+    _check(lib().prism_index_refine(ctypes.byref(cfg), _p(q), _p(k), _p(lens), _p(idx_prev),
+                                    _p(idx_out), _p(cp), _p(cs), _p(cc), int(cand_cap), _p(ws),
+                                    ws.numel(), _stream(stream)),
+           "prism_index_refine")
+    return (idx_out, cp, cs, cc) if cand_cap > 0 else idx_out
+
+
+def prism_sparse_decode(cfg: Config, q, k, v, lens, idx, out=None, ws=None, stream=None):
+    B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
+    _need(q, "q", torch.bfloat16, (B, Hq, d))
+    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need(v, "v", torch.bfloat16, (B, Hkv, L, d))
+    _need(lens, "lens", torch.int32, (B,))
+    if idx.dim() != 3 or tuple(idx.shape[:2]) != (B, Hkv):
+        raise ValueError("idx must be [B][Hkv][n_idx]")
+    _need(idx, "idx", torch.int32)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, d))
+    ws = workspace(cfg, q.device) if ws is None else ws
+    _check(lib().prism_sparse_decode(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(lens), _p(idx),
+                                     int(idx.shape[2]), _p(out), _p(ws), ws.numel(),
+                                     _stream(stream)),
+           "prism_sparse_decode")
+    return out
+
+
+def prism_decode_step(cfg: Config, q, k_layers, v_layers, lens, out=None, idx_out=None,
+                      ws=None, stream=None, want_idx=False):
+    N, B, Hq, Hkv, d, L = (cfg.n_layers, cfg.batch, cfg.n_q_heads, cfg.n_kv_heads,
+                           cfg.head_dim, cfg.max_len)
+    _need(q, "q", torch.bfloat16, (N, B, Hq, d))
+    if len(k_layers) != N or len(v_layers) != N:
+        raise ValueError("need one K and one V tensor per layer")
+    for i, (kk, vv) in enumerate(zip(k_layers, v_layers)):
+        _need(kk, f"k[{i}]", torch.bfloat16, (B, Hkv, L, d))
+        _need(vv, f"v[{i}]", torch.bfloat16, (B, Hkv, L, d))
+    _need(lens, "lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((N, B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (N, B, Hq, d))
+    if idx_out is None and want_idx:
+        idx_out = torch.empty((N, B, Hkv, cfg.kappa), dtype=torch.int32, device=q.device)
+    if idx_out is not None:
+        _need(idx_out, "idx_out", torch.int32, (N, B, Hkv, cfg.kappa))
+    kp = (ctypes.c_void_p * N)(*[kk.data_ptr() for kk in k_layers])
+    vp = (ctypes.c_void_p * N)(*[vv.data_ptr() for vv in v_layers])
+    ws = workspace(cfg, q.device) if ws is None else ws
+    _check(lib().prism_decode_step(ctypes.byref(cfg), _p(q), ctypes.cast(kp, ctypes.c_void_p),
+                                   ctypes.cast(vp, ctypes.c_void_p), _p(lens), _p(out),
+                                   _p(idx_out), _p(ws), ws.numel(), _stream(stream)),
+           "prism_decode_step")
+    return (out, idx_out) if idx_out is not None else out
+
+
+def prism_check_device_status(ws: torch.Tensor, stream=None):
+    """Synchronises; returns (status, [code, where, value, 0]) and clears the word."""
+    detail = (ctypes.c_uint32 * 4)()
+    st = lib().prism_check_device_status(_p(ws), ws.numel(), _stream(stream), detail)
+    return st, list(detail)
+
+
+def prism_debug_wait_timeout(ws: torch.Tensor, limit_ns: int, stream=None):
+    _check(lib().prism_debug_wait_timeout(_p(ws), ws.numel(), int(limit_ns), _stream(stream)),
+           "prism_debug_wait_timeout")
+
+
+def raw_status(fn_name: str, *args) -> int:
+    """Call a C entry point with raw ctypes arguments; returns the status code
+    (used by the argument-validation tests)."""
+    return getattr(lib(), fn_name)(*args)
+
+
+__all__ = ["Config", "PrismError", "lib", "workspace", "prism_workspace_size",
+           "prism_index_anchor", "prism_index_refine", "prism_sparse_decode",
+           "prism_decode_step", "prism_check_device_status", "prism_debug_wait_timeout",
+           "prism_score_anchor", "raw_status", "MODE_REFINE", "MODE_STATIC_REUSE", "MODE_DENSE_ANCHOR",
+           "CHAIN_PREV", "CHAIN_ANCHOR", "EXPORTS", "LIB_PATH"]

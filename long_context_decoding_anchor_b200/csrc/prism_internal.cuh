@@ -1,0 +1,350 @@
+// prism_internal.cuh -- device helpers and launch interfaces shared by the
+// kernels of the Prism Attention decode hot path (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace prism {
+
+// First-level radix digit of a score key (the top 11 bits).
+constexpr int kHistBits = 11;
+constexpr int kHistBins = 1 << kHistBits;
+constexpr int kMaxLen = 1 << 20;
+
+// Device status word (first bytes of the workspace).
+struct DevStatus {
+    uint32_t code;    // 0 = ok, else one of the kDevErr* values
+    uint32_t where;   // which kernel reported
+    uint32_t value;   // offending value (a length, an index, a stage)
+    uint32_t pad;
+};
+enum : uint32_t {
+    kDevErrNone = 0,
+    kDevErrTimeout = 1,
+    kDevErrBadLen = 2,
+    kDevErrBadIndex = 3,
+    kDevErrInternal = 4,
+};
+enum : uint32_t {
+    kWhereScore = 1,
+    kWhereRescore = 2,
+    kWhereExpand = 3,
+    kWhereCollect = 4,
+    kWhereFinalize = 5,
+    kWhereAttn = 6,
+    kWhereDebugWait = 7,
+};
+
+// Per (batch, KV head) row counters; zeroed at the start of every public call
+// and left zeroed by the kernels that consume them.
+struct RowCtl {
+    int32_t n_sel;     // items strictly above the threshold digit (collect)
+    int32_t n_tie;     // items on the threshold digit (collect)
+    int32_t n_prop;    // |P| of the refine proposal (expand)
+    int32_t pad;
+};
+
+__device__ __forceinline__ void report(DevStatus *st, uint32_t code, uint32_t where,
+                                       uint32_t value) {
+    if (atomicCAS(&st->code, 0u, code) == 0u) {
+        st->where = where;
+        st->value = value;
+    }
+}
+
+// Clamped context length of batch entry b (reports values outside [0, Lmax]).
+__device__ __forceinline__ int load_len(const int32_t *len, int b, int Lmax, DevStatus *st,
+                                        uint32_t where) {
+    int L = __ldg(len + b);
+    if (L < 0 || L > Lmax) {
+        report(st, kDevErrBadLen, where, (uint32_t)L);
+        L = L < 0 ? 0 : Lmax;
+    }
+    return L;
+}
+
+// Order-preserving unsigned key of an fp32 score: a > b  <=>  key(a) > key(b).
+// -0.0 is folded onto +0.0 so the two tie.
+__device__ __forceinline__ uint32_t score_key(float s) {
+    uint32_t u = __float_as_uint(s);
+    u = (u == 0x80000000u) ? 0u : u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// bf16 halves of a 32-bit word, widened exactly to fp32.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float dot8(const uint4 &kv, const float *q) {
+    float a = bf16_lo(kv.x) * q[0];
+    a = fmaf(bf16_hi(kv.x), q[1], a);
+    a = fmaf(bf16_lo(kv.y), q[2], a);
+    a = fmaf(bf16_hi(kv.y), q[3], a);
+    a = fmaf(bf16_lo(kv.z), q[4], a);
+    a = fmaf(bf16_hi(kv.z), q[5], a);
+    a = fmaf(bf16_lo(kv.w), q[6], a);
+    a = fmaf(bf16_hi(kv.w), q[7], a);
+    return a;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Transposing butterfly reduction.  Each lane of an NL-lane group holds NV
+// partial sums (one per item); after the call the lane holds in v[0] the full
+// group sum of item `transpose_item<NV, NL>(lane)` (for NV <= NL).  Costs
+// NV-1 + log2(NL/NV) shuffles instead of NV*log2(NL).
+template <int NV, int NL>
+__device__ __forceinline__ void transpose_reduce(float (&v)[NV], int lane) {
+    static_assert((NV & (NV - 1)) == 0 && (NL & (NL - 1)) == 0, "powers of two");
+    static_assert(NV <= NL, "at most one item per lane after the reduction");
+    int cnt = NV;
+#pragma unroll
+    for (int m = NL / 2; m >= 1; m >>= 1) {
+        if (cnt > 1) {
+            const bool upper = (lane & m) != 0;
+#pragma unroll
+            for (int i = 0; i < NV / 2; ++i) {
+                if (i < cnt / 2) {
+                    float keep = upper ? v[i + cnt / 2] : v[i];
+                    float send = upper ? v[i] : v[i + cnt / 2];
+                    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                }
+            }
+            cnt >>= 1;
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], m);
+        }
+    }
+}
+
+// Which item a lane holds after transpose_reduce<NV, NL>.
+template <int NV, int NL>
+__device__ __forceinline__ int transpose_item(int lane) {
+    int item = 0;
+    int bit = NV / 2;
+#pragma unroll
+    for (int m = NL / 2; m >= 1 && bit >= 1; m >>= 1, bit >>= 1)
+        if (lane & m) item |= bit;
+    return item;
+}
+
+// Whether this lane is the one (of NL/NV equal copies) that stores the item.
+template <int NV, int NL>
+__device__ __forceinline__ bool transpose_writer(int lane) {
+    return (lane & (NL / NV - 1)) == 0;
+}
+
+// ---- mbarrier / bulk-copy (TMA) primitives -------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase of `parity` to complete; false after limit_ns
+// (or after an iteration cap, should the timer misbehave).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0; it < (1u << 28); ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31u) == 31u && global_timer_ns() - t0 > limit_ns) return false;
+    }
+    return false;
+}
+// Evict-first L2 policy for data read exactly once (the streamed key cache).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+// 1-D bulk copy global -> shared, completing on `bar` (bytes % 16 == 0, both
+// addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// ---- cp.async (16-byte) gather primitives ---------------------------------
+// src_bytes = 0 zero-fills the destination without reading global memory.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// ---- block-wide exclusive scan (int), blockDim.x a multiple of 32 ---------
+// `scratch` holds at least 33 ints.  Returns the exclusive prefix of `x`;
+// *total receives the block sum.  Contains __syncthreads().
+__device__ __forceinline__ int block_exclusive_scan(int x, int *scratch, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = blockDim.x >> 5;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nwarps ? scratch[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < nwarps) scratch[lane] = wi - w;
+        if (lane == 31) scratch[32] = wi;
+    }
+    __syncthreads();
+    int res = scratch[warp] + incl - x;
+    *total = scratch[32];
+    __syncthreads();
+    return res;
+}
+
+// Threshold digit of a histogram: the bin `bsel` such that the number of items
+// in bins above it is < need <= that number + hist[bsel].  `hist` is in shared
+// memory with `nbins` entries (a multiple of blockDim.x).  Writes bsel and the
+// count above it to out[0], out[1].  Contains __syncthreads().
+__device__ __forceinline__ void find_threshold_bin(const uint32_t *hist, int nbins, int need,
+                                                   int *scratch, int *out) {
+    const int per = nbins / blockDim.x;
+    // Thread t owns bins [nbins - (t+1)*per, nbins - t*per): thread 0 the top.
+    const int hi = nbins - threadIdx.x * per;
+    int local = 0;
+    for (int i = 1; i <= per; ++i) local += (int)hist[hi - i];
+    int total;
+    int above = block_exclusive_scan(local, scratch, &total);
+    if (above < need && above + local >= need) {
+        int acc = above;
+        for (int i = 1; i <= per; ++i) {
+            int h = (int)hist[hi - i];
+            if (acc + h >= need) {
+                out[0] = hi - i;
+                out[1] = acc;
+                break;
+            }
+            acc += h;
+        }
+    }
+    __syncthreads();
+}
+
+// ---- launch interfaces (host side, defined in the .cu files) -------------
+// Kernels launched by the calling host thread (see prism_launch_count()).
+void count_launches(int n);
+
+struct ScoreArgs {
+    const void *q;          // bf16 [B][Hq][d]
+    const void *k;          // bf16 [B][Hkv][Lmax][d]
+    const int32_t *len;     // [B]
+    int B, Hkv, G, d, Lmax;
+    float scale;
+    float *S;               // fp32 [rows][Lmax]: anchor scores / refine candidate scores
+    uint32_t *hist;         // [rows][kHistBins]
+    const int32_t *cpos;    // refine: [rows][Lmax] proposal positions (ascending)
+    RowCtl *ctl;            // [rows]
+    DevStatus *st;
+    uint64_t wait_ns;
+};
+
+cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s);
+cudaError_t launch_refine_rescore(const ScoreArgs &a, long long max_prop, cudaStream_t s);
+
+struct ExpandArgs {
+    const int32_t *idx_prev;   // [rows][kappa]
+    const int32_t *len;
+    int B, Hkv, Lmax, kappa, radius;
+    int32_t *cpos;             // [rows][Lmax]
+    RowCtl *ctl;
+    DevStatus *st;
+};
+cudaError_t launch_expand(const ExpandArgs &a, cudaStream_t s);
+
+struct SelectArgs {
+    const float *S;            // [rows][Lmax] scores (anchor: by position; refine: by proposal slot)
+    const int32_t *cpos;       // refine: [rows][Lmax] positions; nullptr for the anchor
+    const int32_t *len;
+    int B, Hkv, Lmax, kappa;
+    uint32_t *hist;            // [rows][kHistBins]
+    RowCtl *ctl;
+    int32_t *sel;              // [rows][kappa] positions above the threshold digit
+    uint64_t *tie;             // [rows][Lmax] (key << 32 | position) on the threshold digit
+    int32_t *idx_out;          // [rows][kappa]
+    DevStatus *st;
+};
+cudaError_t launch_select(const SelectArgs &a, long long max_items, cudaStream_t s);
+
+struct AttnArgs {
+    const void *q;             // bf16 [B][Hq][d]
+    const void *k, *v;         // bf16 [B][Hkv][Lmax][d]
+    const int32_t *len;
+    const int32_t *idx;        // [rows][idx_stride]
+    int idx_stride, n_idx;
+    int B, Hkv, G, d, Lmax;
+    float scale;
+    float *part_acc;           // [rows][nsplit][G][d]
+    float *part_ml;            // [rows][nsplit][G][2]
+    void *out;                 // bf16 [B][Hq][d]
+    DevStatus *st;
+};
+constexpr int kAttnChunk = 64;
+cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s);
+
+cudaError_t launch_export_candidates(const float *S, const int32_t *cpos, const RowCtl *ctl,
+                                     int rows, int Lmax, int32_t *cand_pos, float *cand_score,
+                                     int32_t *cand_count, int cand_cap, cudaStream_t s);
+
+cudaError_t launch_debug_wait(DevStatus *st, uint64_t limit_ns, cudaStream_t s);
+
+}  // namespace prism

@@ -1,0 +1,155 @@
+"""C-ABI boundary on the CPU: the library loads, exports every entry point
+that include/prism.h declares, and rejects invalid arguments on the host
+before anything is launched (no GPU needed, no device memory touched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_decoding_anchor_b200 as prism
+from long_context_decoding_anchor_b200 import build as prism_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "prism.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    prism_build.build()
+    return prism.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"PRISM_API\s+[\w\s\*]+?\b(prism_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for required in ("prism_index_anchor", "prism_index_refine", "prism_sparse_decode",
+                     "prism_decode_step", "prism_workspace_size"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), f"{name} declared in prism.h but not exported"
+    assert set(prism.EXPORTS) <= set(declared_symbols())
+
+
+def test_status_strings(L):
+    for code in range(7):
+        assert len(L.prism_status_string(code)) > 0
+    assert L.prism_version() >= 100
+
+
+def _cfg(**kw):
+    base = dict(batch=1, n_q_heads=8, n_kv_heads=2, head_dim=64, max_len=4096, kappa=256,
+                radius=4, n_layers=4, anchor_mask=[1, 0, 0, 0])
+    base.update(kw)
+    return prism.Config.make(**base)
+
+
+def test_workspace_size_monotone(L):
+    small = prism.prism_workspace_size(_cfg())
+    big = prism.prism_workspace_size(_cfg(max_len=8192))
+    assert 0 < small < big
+    assert prism.prism_workspace_size(_cfg(batch=2)) > small
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(head_dim=96), 2), (dict(head_dim=32), 2), (dict(n_q_heads=12, n_kv_heads=8), 1),
+    (dict(n_q_heads=24, n_kv_heads=8), 2), (dict(n_q_heads=32, n_kv_heads=2, head_dim=64), 2),
+    (dict(kappa=0), 1), (dict(radius=-1), 1), (dict(max_len=0), 1),
+    (dict(max_len=(1 << 20) + 1), 2), (dict(batch=0), 1), (dict(mode=3), 1), (dict(chain=2), 1),
+    (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1), (dict(batch=70000, n_kv_heads=1,
+                                                                  n_q_heads=1), 2),
+])
+def test_invalid_config_rejected(L, bad, status):
+    c = _cfg(**bad)
+    n = ctypes.c_size_t(0)
+    assert L.prism_workspace_size(ctypes.byref(c), ctypes.byref(n)) == status
+
+
+# Fake device addresses: validation must reject the call before any use.
+A16 = ctypes.c_void_p(0x10000)
+A4 = ctypes.c_void_p(0x10004)
+MIS = ctypes.c_void_p(0x10002)
+
+
+def test_anchor_argument_validation(L):
+    c = _cfg()
+    ws_n = prism.prism_workspace_size(c)
+    ws = ctypes.c_void_p(0x100000)
+    f = L.prism_index_anchor
+    cp = ctypes.byref(c)
+    assert f(cp, None, A16, A4, A4, None, ws, ws_n, None) == 1          # null q
+    assert f(cp, A16, None, A4, A4, None, ws, ws_n, None) == 1          # null k
+    assert f(cp, A16, A16, None, A4, None, ws, ws_n, None) == 1         # null len
+    assert f(cp, A16, A16, A4, None, None, ws, ws_n, None) == 1         # null idx_out
+    assert f(cp, MIS, A16, A4, A4, None, ws, ws_n, None) == 1           # q misaligned
+    assert f(cp, A16, MIS, A4, A4, None, ws, ws_n, None) == 1           # k misaligned
+    assert f(cp, A16, A16, A4, A4, None, ctypes.c_void_p(0x100010), ws_n, None) == 1  # ws align
+    assert f(cp, A16, A16, A4, A4, None, ws, ws_n - 1, None) == 3       # short workspace
+    assert f(cp, A16, A16, A4, A4, None, None, ws_n, None) == 1         # null workspace
+
+
+def test_refine_argument_validation(L):
+    c = _cfg()
+    ws_n = prism.prism_workspace_size(c)
+    ws = ctypes.c_void_p(0x100000)
+    f = L.prism_index_refine
+    cp = ctypes.byref(c)
+    same = ctypes.c_void_p(0x20000)
+    assert f(cp, A16, A16, A4, same, same, None, None, None, 0, ws, ws_n, None) == 1   # alias
+    assert f(cp, A16, A16, A4, A4, ctypes.c_void_p(0x30000), A4, None, None, 16, ws, ws_n,
+             None) == 1                                                   # partial cand outputs
+    assert f(cp, A16, A16, A4, A4, ctypes.c_void_p(0x30000), A4, A4, A4, 0, ws, ws_n,
+             None) == 1                                                   # cand_cap 0
+    assert f(cp, A16, A16, A4, None, A4, None, None, None, 0, ws, ws_n, None) == 1
+
+
+def test_sparse_decode_argument_validation(L):
+    c = _cfg()
+    ws_n = prism.prism_workspace_size(c)
+    ws = ctypes.c_void_p(0x100000)
+    f = L.prism_sparse_decode
+    cp = ctypes.byref(c)
+    assert f(cp, A16, A16, A16, A4, A4, 0, A16, ws, ws_n, None) == 1         # n_idx 0
+    assert f(cp, A16, A16, A16, A4, A4, 257, A16, ws, ws_n, None) == 1       # n_idx > kappa
+    assert f(cp, A16, A16, MIS, A4, A4, 16, A16, ws, ws_n, None) == 1        # v misaligned
+    assert f(cp, A16, A16, A16, A4, A4, 16, MIS, ws, ws_n, None) == 1        # out misaligned
+
+
+def test_decode_step_argument_validation(L):
+    ws = ctypes.c_void_p(0x100000)
+    c = _cfg(anchor_mask=[0, 1, 0, 0])
+    ws_n = prism.prism_workspace_size(c)
+    kp = (ctypes.c_void_p * 4)(*[0x40000 + 0x100 * i for i in range(4)])
+    f = L.prism_decode_step
+    assert f(ctypes.byref(c), A16, kp, kp, A4, A16, None, ws, ws_n, None) == 1  # layer 0 not anchor
+    c = _cfg()
+    bad = (ctypes.c_void_p * 4)(0x40000, 0x40008, 0x40100, 0x40200)             # k[1] misaligned
+    assert f(ctypes.byref(c), A16, bad, kp, A4, A16, None, ws, ws_n, None) == 1
+    nul = (ctypes.c_void_p * 4)(0x40000, None, 0x40100, 0x40200)
+    assert f(ctypes.byref(c), A16, kp, nul, A4, A16, None, ws, ws_n, None) == 1
+    c = _cfg(n_layers=0)
+    assert f(ctypes.byref(c), A16, kp, kp, A4, A16, None, ws, ws_n, None) == 1
+    c = _cfg(anchor_mask=None)
+    assert f(ctypes.byref(c), A16, kp, kp, A4, A16, None, ws, ws_n, None) == 1  # mask required
+
+
+def test_debug_wait_validation(L):
+    assert L.prism_debug_wait_timeout(None, 256, 1000, None) == 1
+    assert L.prism_debug_wait_timeout(ctypes.c_void_p(0x100000), 256, 0, None) == 1
+    assert L.prism_check_device_status(ctypes.c_void_p(0x100010), 256, None, None) == 1
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    c = _cfg()
+    with pytest.raises(ValueError):
+        prism.prism_index_anchor(c, torch.zeros(1, 8, 64, dtype=torch.bfloat16),
+                                 torch.zeros(1, 2, 4096, 64, dtype=torch.bfloat16),
+                                 torch.zeros(1, dtype=torch.int32))

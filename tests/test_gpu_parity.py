@@ -1,0 +1,161 @@
+"""CUDA path against the oracle on seeded synthetic inputs (GPU only).
+
+Sizes span several tiles and ragged tails; the tiny and 32K workloads run at
+their full sizes, the batched ragged one at reduced batch; the 128K and 512K
+workloads are covered by tests/test_gpu_fullsize.py on sampled rows."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_decoding_anchor_b200 as prism
+from long_context_decoding_anchor_b200 import synth
+from gpu_checks import (check_anchor, check_attention, check_refine, layerwise_step_check,
+                        recall)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    prism.lib()   # the library must load: no fallback
+
+
+def _inputs(w, layers=None):
+    return synth.make_inputs(w, device="cuda", layers=layers)
+
+
+SHAPES = {
+    # name: workload overrides (kept small: several tiles, ragged tails)
+    "tiny-full": synth.WORKLOADS[1],
+    "d128-g4": synth.WORKLOADS[2].replace(max_len=5000, n_layers=3, kappa=200, radius=3,
+                                          n_clusters=8),
+    "d128-g8-ragged": synth.WORKLOADS[4].replace(batch=3, max_len=3001, n_layers=3,
+                                                 n_q_heads=64, kappa=128, radius=2,
+                                                 ragged=(700, 3001), n_clusters=6),
+    "d128-g16": synth.WORKLOADS[5].replace(max_len=2304, n_layers=2, n_q_heads=32,
+                                           n_kv_heads=2, kappa=96, radius=5, n_clusters=4),
+    "d64-g1": synth.WORKLOADS[1].replace(max_len=1000, n_layers=3, n_q_heads=2,
+                                         n_kv_heads=2, kappa=100, radius=1),
+    "d64-g2-batch": synth.WORKLOADS[1].replace(batch=4, max_len=777, n_layers=2,
+                                               n_q_heads=4, n_kv_heads=2, kappa=64,
+                                               radius=2, ragged=(1, 777), n_clusters=3),
+    "d64-g8": synth.WORKLOADS[1].replace(max_len=1500, n_layers=2, n_q_heads=16,
+                                         n_kv_heads=2, kappa=300, radius=4),
+}
+
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_anchor_refine_attention_stages(oracle, name):
+    w = SHAPES[name]
+    inp = _inputs(w, layers=[0, 1])
+    cfg = prism.Config.from_workload(w)
+    q0, k0, v0, lens = inp["q"][0], inp["k"][0], inp["v"][0], inp["lens"]
+    S = torch.empty((w.batch, w.n_kv_heads, w.max_len), dtype=torch.float32, device="cuda")
+    ws = prism.workspace(cfg)
+    idx0 = prism.prism_index_anchor(cfg, q0, k0, lens, scores_out=S, ws=ws)
+    check_anchor(oracle, cfg, q0, k0, lens, idx0, S)
+    out0 = prism.prism_sparse_decode(cfg, q0, k0, v0, lens, idx0, ws=ws)
+    check_attention(oracle, cfg, q0, k0, v0, lens, idx0, out0)
+    q1, k1, v1 = inp["q"][1], inp["k"][1], inp["v"][1]
+    idx1, cp, cs, cc = prism.prism_index_refine(cfg, q1, k1, lens, idx0, cand_cap=w.max_len, ws=ws)
+    check_refine(oracle, cfg, q1, k1, lens, idx0, idx1, cp, cs, cc)
+    out1 = prism.prism_sparse_decode(cfg, q1, k1, v1, lens, idx1, ws=ws)
+    check_attention(oracle, cfg, q1, k1, v1, lens, idx1, out1)
+    st, detail = prism.prism_check_device_status(ws)
+    assert st == 0, detail
+
+
+@pytest.mark.parametrize("wkey", [1, 2])
+def test_decode_step_full_workload(oracle, wkey):
+    """The tiny (4K) and 32K workloads at full size, every layer."""
+    w = synth.WORKLOADS[wkey]
+    inp = _inputs(w)
+    cfg = prism.Config.from_workload(w)
+    out, idx = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                       want_idx=True)
+    stats = {}
+    layerwise_step_check(oracle, cfg, inp, out, idx, stats=stats)
+    # End to end: recall of the GPU chain against the oracle's fp64 chain.
+    from oracle import bf16_bits
+    ref_out, ref_idx = oracle.decode_step(bf16_bits(inp["q"]), [bf16_bits(t) for t in inp["k"]],
+                                          [bf16_bits(t) for t in inp["v"]],
+                                          inp["lens"].cpu().numpy(), w.kappa, w.radius,
+                                          w.anchor_mask())
+    gi = idx.cpu().numpy()
+    for l in range(w.n_layers):
+        for b in range(w.batch):
+            for h in range(w.n_kv_heads):
+                assert recall(gi[l, b, h], ref_idx[l, b, h]) >= 0.999, (l, b, h)
+    assert np.max(np.abs(out.float().cpu().numpy() - ref_out)) < 5e-2
+
+
+def test_decode_step_batched_ragged(oracle):
+    """The batched ragged workload's structure at reduced batch and length."""
+    w = synth.WORKLOADS[4].replace(batch=4, max_len=6000, ragged=(1500, 6000), n_layers=6,
+                                   kappa=256, n_clusters=16)
+    inp = _inputs(w)
+    cfg = prism.Config.from_workload(w)
+    out, idx = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                       want_idx=True)
+    layerwise_step_check(oracle, cfg, inp, out, idx)
+
+
+@pytest.mark.parametrize("mode,chain", [(prism.MODE_STATIC_REUSE, prism.CHAIN_PREV),
+                                        (prism.MODE_DENSE_ANCHOR, prism.CHAIN_PREV),
+                                        (prism.MODE_REFINE, prism.CHAIN_ANCHOR)])
+def test_decode_step_modes(oracle, mode, chain):
+    w = synth.WORKLOADS[1].replace(max_len=3000, n_layers=5, anchor_every=3)
+    inp = _inputs(w)
+    cfg = prism.Config.from_workload(w, mode=mode, chain=chain)
+    out, idx = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                       want_idx=True)
+    layerwise_step_check(oracle, cfg, inp, out, idx)
+    if mode == prism.MODE_STATIC_REUSE:
+        assert torch.equal(idx[1], idx[0]) and torch.equal(idx[2], idx[0])
+
+
+def test_decode_step_without_idx_out_matches(oracle):
+    """idx_out is optional; the outputs are identical either way."""
+    w = synth.WORKLOADS[1].replace(max_len=2500, n_layers=6, anchor_every=4)
+    inp = _inputs(w)
+    for chain in (prism.CHAIN_PREV, prism.CHAIN_ANCHOR):
+        cfg = prism.Config.from_workload(w, chain=chain)
+        out_a, _ = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                           want_idx=True)
+        out_b = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"])
+        assert torch.equal(out_a, out_b)
+
+
+def test_invariants_on_gpu(oracle):
+    """r = 0 equals static reuse; r >= L equals per-layer exact selection;
+    kappa >= L is dense attention."""
+    w = synth.WORKLOADS[1].replace(max_len=1200, n_layers=4, kappa=64)
+    inp = _inputs(w)
+    base = dict(n_layers=w.n_layers)
+    run = lambda **kw: prism.prism_decode_step(prism.Config.from_workload(w, **{**base, **kw}),
+                                               inp["q"], inp["k"], inp["v"], inp["lens"],
+                                               want_idx=True)
+    _, r0 = run(radius=0)
+    _, st = run(mode=prism.MODE_STATIC_REUSE)
+    assert torch.equal(r0, st)
+    _, wide = run(radius=w.max_len)
+    _, dense = run(mode=prism.MODE_DENSE_ANCHOR)
+    assert torch.equal(wide, dense)
+    out, idx = run(kappa=w.max_len)
+    assert torch.equal(idx[:, 0, :, :w.max_len].cpu(),
+                       torch.arange(w.max_len, dtype=torch.int32).expand(w.n_layers, 2, -1))
+    from oracle import bf16_bits
+    from helpers import sdpa_group
+    qh = bf16_bits(inp["q"])
+    G = w.group
+    for l in range(w.n_layers):
+        kh, vh = bf16_bits(inp["k"][l]), bf16_bits(inp["v"][l])
+        for h in range(w.n_kv_heads):
+            ref = sdpa_group(qh[l, 0, h * G:(h + 1) * G], kh[0, h], vh[0, h],
+                             np.arange(w.max_len), 1.0 / math.sqrt(w.head_dim))
+            got = out[l, 0, h * G:(h + 1) * G].float().cpu().numpy()
+            assert np.all(np.abs(got - ref) <= 2e-2 + 1e-2 * np.abs(ref))
