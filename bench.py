@@ -46,9 +46,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["prism", "reference"], default="prism")
     ap.add_argument("--workload", type=int, default=3)
     ap.add_argument("--no-graph", action="store_true", help="time eager launches")
-    ap.add_argument("--cpu-layers", type=int, default=8,
+    ap.add_argument("--cpu-layers", type=int, default=16,
                     help="layers of the workload in the CPU-baseline sample")
-    ap.add_argument("--ref-layers", type=int, default=4,
+    ap.add_argument("--ref-layers", type=int, default=8,
                     help="layers per step of the reference (oracle) arm")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")

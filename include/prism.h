@@ -116,9 +116,11 @@ typedef struct {
 /* Bytes of workspace every call below needs for `cfg` (the same figure serves
  * all of them).  The workspace holds scores, candidate lists, histograms,
  * selections and attention partials; its first 256 bytes are the device
- * status word.  Pass it 256-byte aligned.  Its contents need no
- * initialisation and are scratch between calls, except the status word,
- * which persists until prism_check_device_status() reads it.
+ * status word.  Pass it 256-byte aligned.  Zero the status word (the first
+ * 256 bytes) once after allocating the workspace, e.g. by allocating it
+ * zero-filled; the rest needs no initialisation and is scratch between
+ * calls.  The status word persists across calls until
+ * prism_check_device_status() reads and clears it.
  * Errors: PRISM_ERR_INVALID_ARG / PRISM_ERR_UNSUPPORTED for a bad config. */
 PRISM_API prism_status_t prism_workspace_size(const prism_config_t *cfg, size_t *bytes);
 

@@ -150,8 +150,9 @@ def prism_workspace_size(cfg: Config) -> int:
 
 
 def workspace(cfg: Config, device=None) -> torch.Tensor:
-    """A workspace buffer for ``cfg`` (uint8; torch allocations are 512-byte aligned)."""
-    return torch.empty(prism_workspace_size(cfg), dtype=torch.uint8,
+    """A zero-filled workspace buffer for ``cfg`` (uint8; torch allocations are
+    512-byte aligned).  Zero-filled so that the status word starts clear."""
+    return torch.zeros(prism_workspace_size(cfg), dtype=torch.uint8,
                        device=device or torch.device("cuda"))
 
 
