@@ -52,6 +52,10 @@ def parse_args():
                     help="layers per step of the reference (oracle) arm")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="only run --steps eager decode steps (for ncu captures)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the workload's layer count (profiling a smaller case)")
     return ap.parse_args()
 
 
@@ -216,7 +220,20 @@ def run_prism(args, rank, world, dev):
         prism_build.build()
     prism.lib()
     w = synth.WORKLOADS[args.workload]
+    if args.layers:
+        w = w.replace(n_layers=args.layers)
     inp = synth.make_inputs(w, device=dev)
+    if args.profile:
+        cfg = prism.Config.from_workload(w)
+        ws = prism.workspace(cfg, dev)
+        for _ in range(args.steps):
+            prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], ws=ws)
+        torch.cuda.synchronize(dev)
+        st, detail = prism.prism_check_device_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status {st} {detail}")
+        print(f"profile run: {args.steps} eager steps of {w.name} ({w.n_layers} layers)")
+        return
     cfg = prism.Config.from_workload(w)
     ws = prism.workspace(cfg, dev)
     N = w.n_layers

@@ -16,8 +16,9 @@
  * --------------------------------
  *  - Pointers named q, k, v, out, idx*, cand*, len, ws are DEVICE pointers on
  *    the current CUDA device; the caller owns every buffer.  The library
- *    allocates nothing and keeps no state between calls other than a few
- *    per-device attribute caches.
+ *    allocates no device memory.  Between calls it keeps only per-device
+ *    caches: the SM count, and (for prism_decode_step) three helper streams
+ *    and a pool of events, created on first use and kept until exit.
  *  - Layouts (row-major, no padding between rows):
  *      q    bf16 [B][Hq][d]            one decode query per sequence
  *      k, v bf16 [B][Hkv][Lmax][d]     KV cache of one layer; position i of
@@ -29,8 +30,10 @@
  *    Query head j reads KV head j / (Hq / Hkv).
  *  - Alignment: q, k, v, out 16 bytes; int32 arrays 4 bytes; ws 256 bytes.
  *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
- *    default stream), makes no host synchronisation, allocates no memory and
- *    can be captured into a CUDA graph.
+ *    default stream), makes no host synchronisation and can be captured into
+ *    a CUDA graph.  prism_decode_step forks work from `stream` onto its
+ *    helper streams and joins it back before returning control of `stream`:
+ *    work enqueued on `stream` afterwards sees every result.
  *  - Arguments are validated on the host before anything is launched; an
  *    invalid argument returns PRISM_ERR_INVALID_ARG (or PRISM_ERR_UNSUPPORTED
  *    for a shape the kernels do not cover, PRISM_ERR_WORKSPACE for a short
@@ -100,7 +103,7 @@ typedef struct {
     int32_t max_len;        /* Lmax, 1 <= Lmax <= PRISM_MAX_LEN               */
     int32_t kappa;          /* sparse budget, 1 <= kappa <= PRISM_MAX_LEN     */
     int32_t radius;         /* proposal radius r >= 0                         */
-    int32_t n_layers;       /* N >= 1 (prism_decode_step only)                */
+    int32_t n_layers;       /* N >= 1 for prism_decode_step, <= PRISM_MAX_LAYERS */
     const uint8_t *anchor_mask; /* HOST array [N]; nonzero = anchor layer;
                                    mask[0] must be nonzero unless DENSE_ANCHOR
                                    (prism_decode_step only; may be NULL for the
@@ -108,13 +111,21 @@ typedef struct {
     int32_t mode;           /* prism_mode_t                                   */
     int32_t chain;          /* prism_chain_t                                  */
     float scale;            /* score/logit scale; 0 means 1/sqrt(d)           */
+    int32_t flags;          /* PRISM_FLAG_* bits, 0 by default                */
 } prism_config_t;
+
+/* prism_decode_step schedules anchor scoring, selections and attention as a
+ * DAG over helper streams; this flag enqueues everything, in layer order, on
+ * the caller's stream instead (same results, bit for bit). */
+#define PRISM_FLAG_SERIAL 1
 
 #define PRISM_MAX_LEN (1 << 20)
 #define PRISM_MAX_BATCH_ROWS 65535   /* B * Hkv */
+#define PRISM_MAX_LAYERS 4096
 
 /* Bytes of workspace every call below needs for `cfg` (the same figure serves
- * all of them).  The workspace holds scores, candidate lists, histograms,
+ * all of them; it grows with n_layers, which the single-stage calls may leave
+ * at 0 or 1).  The workspace holds scores, candidate lists, histograms,
  * selections and attention partials; its first 256 bytes are the device
  * status word.  Pass it 256-byte aligned.  Zero the status word (the first
  * 256 bytes) once after allocating the workspace, e.g. by allocating it

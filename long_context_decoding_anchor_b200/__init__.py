@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_PKG, "libprism.so")
 
 MODE_REFINE, MODE_STATIC_REUSE, MODE_DENSE_ANCHOR = 0, 1, 2
 CHAIN_PREV, CHAIN_ANCHOR = 0, 1
+FLAG_SERIAL = 1
 STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED",
           3: "PRISM_ERR_WORKSPACE", 4: "PRISM_ERR_CUDA", 5: "PRISM_ERR_TIMEOUT",
           6: "PRISM_ERR_DEVICE"}
@@ -48,14 +49,14 @@ class Config(ctypes.Structure):
                 ("radius", ctypes.c_int32), ("n_layers", ctypes.c_int32),
                 ("anchor_mask", ctypes.POINTER(ctypes.c_uint8)),
                 ("mode", ctypes.c_int32), ("chain", ctypes.c_int32),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("flags", ctypes.c_int32)]
 
     @classmethod
     def make(cls, batch, n_q_heads, n_kv_heads, head_dim, max_len, kappa, radius=0,
              n_layers=1, anchor_mask: Optional[Sequence[int]] = None, mode=MODE_REFINE,
-             chain=CHAIN_PREV, scale=0.0) -> "Config":
+             chain=CHAIN_PREV, scale=0.0, flags=0) -> "Config":
         c = cls(batch, n_q_heads, n_kv_heads, head_dim, max_len, kappa, radius, n_layers,
-                None, mode, chain, scale)
+                None, mode, chain, scale, flags)
         if anchor_mask is not None:
             arr = (ctypes.c_uint8 * len(anchor_mask))(*[1 if x else 0 for x in anchor_mask])
             c._mask_keepalive = arr
@@ -284,4 +285,4 @@ __all__ = ["Config", "PrismError", "lib", "workspace", "prism_workspace_size",
            "prism_index_anchor", "prism_index_refine", "prism_sparse_decode",
            "prism_decode_step", "prism_check_device_status", "prism_debug_wait_timeout",
            "prism_score_anchor", "raw_status", "MODE_REFINE", "MODE_STATIC_REUSE", "MODE_DENSE_ANCHOR",
-           "CHAIN_PREV", "CHAIN_ANCHOR", "EXPORTS", "LIB_PATH"]
+           "CHAIN_PREV", "CHAIN_ANCHOR", "FLAG_SERIAL", "EXPORTS", "LIB_PATH"]

@@ -7,8 +7,8 @@
 // and V rows once for all G query heads with 16-byte cp.async copies into
 // shared memory (rows of padding slots are zero-filled, not read), forms the
 // G x 64 logits, and writes an unnormalised partial (running max m, sum l,
-// accumulator acc[d]) per query head.  k_attn_combine merges the partials of
-// a row with the usual rescaling by exp(m_s - M).
+// accumulator acc[d]) per query head.  The last CTA of a row to finish merges
+// the row's partials with the usual rescaling by exp(m_s - M).
 #include <cuda_bf16.h>
 
 #include "prism_internal.cuh"
@@ -30,6 +30,81 @@ struct AttnCfg {
     static constexpr int kChunksPerRow = D / 8;
     static_assert(G <= kNL, "group larger than lanes per row");
 };
+
+// Merge the split-K partials of one (batch, KV head) row:
+//   O_j = sum_s exp(m_s - M) acc_s / sum_s exp(m_s - M) l_s,  M = max_s m_s.
+// `wbuf` holds at least G * kAttnChunk floats (the split weights are cached
+// there when the row has at most kAttnChunk splits).
+template <int D, int G>
+__device__ void combine_row(const AttnArgs &a, int row, int b, int h, int nsplit, float *wbuf) {
+    __shared__ float Mh[G], inv_den[G];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float *pm = a.part_ml + (size_t)row * nsplit * G * 2;
+    const bool cache = nsplit <= kAttnChunk;
+    for (int g = warp; g < G; g += 4) {
+        float M = -INFINITY;
+        for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, __ldcg(pm + ((size_t)s * G + g) * 2));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float den = 0.f;
+        for (int s = lane; s < nsplit; s += 32) {
+            const float m = __ldcg(pm + ((size_t)s * G + g) * 2);
+            const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : __expf(m - M);
+            if (cache) wbuf[g * kAttnChunk + s] = w;
+            den = fmaf(w, __ldcg(pm + ((size_t)s * G + g) * 2 + 1), den);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        if (lane == 0) {
+            Mh[g] = M;
+            inv_den[g] = den > 0.f ? 1.f / den : 0.f;
+        }
+    }
+    __syncthreads();
+    // Each thread owns float4 columns of the [G][D] accumulator; the partials
+    // of 16 splits are loaded at a time so their L2 round trips overlap.
+    constexpr int kC4 = G * D / 4;
+    constexpr int kBatch = 16;
+    const float4 *pa4 = reinterpret_cast<const float4 *>(a.part_acc + (size_t)row * nsplit * G * D);
+    uint16_t *out = static_cast<uint16_t *>(a.out) + ((size_t)b * a.Hkv * G + (size_t)h * G) * D;
+    for (int c4 = threadIdx.x; c4 < kC4; c4 += blockDim.x) {
+        const int g = (c4 * 4) / D;
+        const float Mg = Mh[g];
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (Mg != -INFINITY) {
+            for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
+                float4 v[kBatch];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u)
+                    v[u] = s0 + u < nsplit ? __ldcg(pa4 + (size_t)(s0 + u) * kC4 + c4)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int sp = s0 + u;
+                    if (sp >= nsplit) break;
+                    float w;
+                    if (cache) {
+                        w = wbuf[g * kAttnChunk + sp];
+                    } else {
+                        const float m = __ldcg(pm + ((size_t)sp * G + g) * 2);
+                        w = m == -INFINITY ? 0.f : __expf(m - Mg);
+                    }
+                    acc.x = fmaf(w, v[u].x, acc.x);
+                    acc.y = fmaf(w, v[u].y, acc.y);
+                    acc.z = fmaf(w, v[u].z, acc.z);
+                    acc.w = fmaf(w, v[u].w, acc.w);
+                }
+            }
+        }
+        const float sc = inv_den[g];
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * sc, acc.y * sc);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * sc, acc.w * sc);
+        uint2 packed;
+        packed.x = *reinterpret_cast<const uint32_t *>(&lo);
+        packed.y = *reinterpret_cast<const uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(out + (size_t)c4 * 4) = packed;
+    }
+}
 
 template <int D, int G>
 __global__ void __launch_bounds__(128)
@@ -180,32 +255,18 @@ k_sparse_attn(AttnArgs a) {
         a.part_ml[(pbase + tid) * 2 + 0] = ml[tid][0];
         a.part_ml[(pbase + tid) * 2 + 1] = ml[tid][1];
     }
-}
 
-// Merge the split-K partials of one (batch, KV head) row: thread = element c
-// of head g.
-template <int D, int G>
-__global__ void __launch_bounds__(D)
-k_attn_combine(AttnArgs a, int nsplit) {
-    const int g = blockIdx.x, row = blockIdx.y, c = threadIdx.x;
-    const int b = row / a.Hkv, h = row % a.Hkv;
-    const float *pm = a.part_ml + (size_t)row * nsplit * G * 2;
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pm[((size_t)s * G + g) * 2]);
-    float o = 0.f;
-    if (M != -INFINITY) {
-        float num = 0.f, den = 0.f;
-        for (int s = 0; s < nsplit; ++s) {
-            const float m = pm[((size_t)s * G + g) * 2];
-            if (m == -INFINITY) continue;
-            const float w = __expf(m - M);
-            den = fmaf(w, pm[((size_t)s * G + g) * 2 + 1], den);
-            num = fmaf(w, a.part_acc[(((size_t)row * nsplit + s) * G + g) * D + c], num);
-        }
-        o = num / den;
-    }
-    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out);
-    out[((size_t)b * a.Hkv * G + (size_t)h * G + g) * D + c] = __float2bfloat16_rn(o);
+    // The last CTA of the row to finish merges the partials (no waiting: an
+    // atomic counter decides which CTA that is).
+    __shared__ int is_last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = atomicAdd(&a.ctl[row].done_attn, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    combine_row<D, G>(a, row, b, h, gridDim.x, &z[0][0]);
+    if (tid == 0) a.ctl[row].done_attn = 0;
 }
 
 template <int D, int G>
@@ -213,10 +274,6 @@ static cudaError_t launch_attn_dg(const AttnArgs &a, cudaStream_t s) {
     const int rows = a.B * a.Hkv;
     const int nsplit = (a.n_idx + kAttnChunk - 1) / kAttnChunk;
     k_sparse_attn<D, G><<<dim3(nsplit, rows), 128, 0, s>>>(a);
-    count_launches(1);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    k_attn_combine<D, G><<<dim3(G, rows), D, 0, s>>>(a, nsplit);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -1,11 +1,26 @@
 // prism_api.cu -- the C ABI (include/prism.h): host-side validation, the
-// workspace layout, and the stream-ordered orchestration of the decode step
-// (Algorithm 1 of "Prism Attention").
+// workspace layout, and the orchestration of the decode step (Algorithm 1 of
+// "Prism Attention").
+//
+// The decode step is a DAG, not a chain.  An anchor layer's scoring reads only
+// its own inputs, so it can run ahead of the refined layers; a layer's
+// attention reads only its own selection, so it can trail behind.  The step
+// therefore runs on three streams forked from the caller's stream and joined
+// back into it (events, so a CUDA-graph capture records the same DAG):
+//   A (low priority):  anchor scoring, at most two anchor layers ahead
+//                      (two workspace slots);
+//   M (high priority): selections in layer order -- each anchor layer's
+//                      top-kappa, each refined layer's rescoring + top-kappa;
+//   C (high priority): each layer's sparse attention once its selection is
+//                      done.
+// PRISM_FLAG_SERIAL runs everything on the caller's stream instead.
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "prism.h"
 #include "prism_internal.cuh"
@@ -22,31 +37,48 @@ namespace {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-struct Layout {
-    size_t status, hist, ctl, ctl_end;   // [hist, ctl_end) is zeroed per call
-    size_t S, cpos, tie, sel, idx[3], pacc, pml, total;
+constexpr int kSlots = 3;           // selection slots: 0, 1 anchors (ring), 2 refined layers
+constexpr int kRefineSlot = 2;
+
+// Buffers of one selection slot.
+struct SlotLayout {
+    size_t hist, ctl, S, tie, sel;
 };
+
+struct Layout {
+    size_t status;
+    size_t ctl_begin, ctl_end;      // [ctl_begin, ctl_end): histograms and counters, zeroed per call
+    SlotLayout slot[kSlots];
+    size_t attn_ctl;
+    size_t canon, idx_all, pacc, pml, total;
+};
+
+int n_layers_of(const prism_config_t &c) { return c.n_layers > 0 ? c.n_layers : 1; }
 
 Layout make_layout(const prism_config_t &c) {
     const size_t rows = (size_t)c.batch * c.n_kv_heads;
     const size_t G = (size_t)(c.n_q_heads / c.n_kv_heads);
     const size_t nsplit = ((size_t)c.kappa + kAttnChunk - 1) / kAttnChunk;
+    const size_t sel_elems = rows * (size_t)c.kappa;
     Layout l{};
     size_t off = 0;
     l.status = off; off = align256(off + sizeof(DevStatus));
-    l.hist = off;   off = align256(off + rows * kHistBins * sizeof(uint32_t));
-    l.ctl = off;    off = align256(off + rows * sizeof(RowCtl));
-    l.ctl_end = off;
-    l.S = off;      off = align256(off + rows * (size_t)c.max_len * sizeof(float));
-    l.cpos = off;   off = align256(off + rows * (size_t)c.max_len * sizeof(int32_t));
-    l.tie = off;    off = align256(off + rows * (size_t)c.max_len * sizeof(uint64_t));
-    l.sel = off;    off = align256(off + rows * (size_t)c.kappa * sizeof(int32_t));
-    for (int i = 0; i < 3; ++i) {
-        l.idx[i] = off;
-        off = align256(off + rows * (size_t)c.kappa * sizeof(int32_t));
+    l.ctl_begin = off;
+    for (int s = 0; s < kSlots; ++s) {
+        l.slot[s].hist = off; off = align256(off + rows * kHistBins * sizeof(uint32_t));
+        l.slot[s].ctl = off;  off = align256(off + rows * sizeof(RowCtl));
     }
-    l.pacc = off;   off = align256(off + rows * nsplit * G * (size_t)c.head_dim * sizeof(float));
-    l.pml = off;    off = align256(off + rows * nsplit * G * 2 * sizeof(float));
+    l.attn_ctl = off; off = align256(off + rows * sizeof(RowCtl));
+    l.ctl_end = off;
+    for (int s = 0; s < kSlots; ++s) {
+        l.slot[s].S = off;   off = align256(off + rows * (size_t)c.max_len * sizeof(float));
+        l.slot[s].tie = off; off = align256(off + rows * (size_t)c.max_len * sizeof(uint64_t));
+        l.slot[s].sel = off; off = align256(off + sel_elems * sizeof(int32_t));
+    }
+    l.canon = off;   off = align256(off + sel_elems * sizeof(int32_t));
+    l.idx_all = off; off = align256(off + (size_t)n_layers_of(c) * sel_elems * sizeof(int32_t));
+    l.pacc = off;    off = align256(off + rows * nsplit * G * (size_t)c.head_dim * sizeof(float));
+    l.pml = off;     off = align256(off + rows * nsplit * G * 2 * sizeof(float));
     l.total = off;
     return l;
 }
@@ -56,18 +88,20 @@ bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 prism_status_t check_config(const prism_config_t *c) {
     if (!c) return PRISM_ERR_INVALID_ARG;
     if (c->batch < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1 || c->max_len < 1 || c->kappa < 1 ||
-        c->radius < 0)
+        c->radius < 0 || c->n_layers < 0)
         return PRISM_ERR_INVALID_ARG;
     if (c->n_q_heads % c->n_kv_heads != 0) return PRISM_ERR_INVALID_ARG;
     if (!(c->scale >= 0.f) || std::isinf(c->scale)) return PRISM_ERR_INVALID_ARG;
     if (c->mode < PRISM_MODE_REFINE || c->mode > PRISM_MODE_DENSE_ANCHOR) return PRISM_ERR_INVALID_ARG;
     if (c->chain < PRISM_CHAIN_PREV || c->chain > PRISM_CHAIN_ANCHOR) return PRISM_ERR_INVALID_ARG;
+    if (c->flags & ~PRISM_FLAG_SERIAL) return PRISM_ERR_INVALID_ARG;
     if (c->head_dim != 64 && c->head_dim != 128) return PRISM_ERR_UNSUPPORTED;
     const int G = c->n_q_heads / c->n_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return PRISM_ERR_UNSUPPORTED;
     if (G > c->head_dim / 8) return PRISM_ERR_UNSUPPORTED;
     if (c->max_len > PRISM_MAX_LEN || c->kappa > PRISM_MAX_LEN) return PRISM_ERR_UNSUPPORTED;
     if ((long long)c->batch * c->n_kv_heads > PRISM_MAX_BATCH_ROWS) return PRISM_ERR_UNSUPPORTED;
+    if (c->n_layers > PRISM_MAX_LAYERS) return PRISM_ERR_UNSUPPORTED;
     return PRISM_OK;
 }
 
@@ -88,10 +122,12 @@ uint64_t wait_limit_ns() {
     return v;
 }
 
+constexpr int kMaxDevices = 64;
+
 int num_sms() {
-    static int cache[128] = {0};
+    static int cache[kMaxDevices] = {0};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
     if (cache[dev] == 0) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
@@ -101,15 +137,51 @@ int num_sms() {
     return cache[dev];
 }
 
-struct Ws {
-    DevStatus *st;
+// Helper streams and a pool of events, per device, created on first use and
+// kept until the process exits.
+struct DeviceHelpers {
+    cudaStream_t anchor = nullptr, chain = nullptr, attn = nullptr;
+    std::vector<cudaEvent_t> events;
+};
+std::mutex g_helpers_mu;
+DeviceHelpers g_helpers[kMaxDevices];
+
+prism_status_t helpers_for_current_device(size_t n_events, DeviceHelpers **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PRISM_ERR_CUDA;
+    DeviceHelpers &h = g_helpers[dev];
+    if (!h.anchor) {
+        int lo = 0, hi = 0;
+        if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return PRISM_ERR_CUDA;
+        // lo is the least urgent priority, hi the most urgent.
+        if (cudaStreamCreateWithPriority(&h.anchor, cudaStreamNonBlocking, lo) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&h.chain, cudaStreamNonBlocking, hi) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&h.attn, cudaStreamNonBlocking, hi) != cudaSuccess)
+            return PRISM_ERR_CUDA;
+    }
+    while (h.events.size() < n_events) {
+        cudaEvent_t e;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return PRISM_ERR_CUDA;
+        h.events.push_back(e);
+    }
+    *out = &h;
+    return PRISM_OK;
+}
+
+struct Slot {
     uint32_t *hist;
     RowCtl *ctl;
     float *S;
-    int32_t *cpos;
     uint64_t *tie;
     int32_t *sel;
-    int32_t *idx[3];
+};
+
+struct Ws {
+    DevStatus *st;
+    Slot slot[kSlots];
+    RowCtl *attn_ctl;
+    int32_t *canon;
+    int32_t *idx_all;
     float *pacc, *pml;
     uint8_t *base;
     Layout l;
@@ -122,13 +194,16 @@ prism_status_t carve(const prism_config_t &c, void *ws, size_t ws_bytes, Ws *w) 
     uint8_t *b = static_cast<uint8_t *>(ws);
     w->base = b;
     w->st = reinterpret_cast<DevStatus *>(b + w->l.status);
-    w->hist = reinterpret_cast<uint32_t *>(b + w->l.hist);
-    w->ctl = reinterpret_cast<RowCtl *>(b + w->l.ctl);
-    w->S = reinterpret_cast<float *>(b + w->l.S);
-    w->cpos = reinterpret_cast<int32_t *>(b + w->l.cpos);
-    w->tie = reinterpret_cast<uint64_t *>(b + w->l.tie);
-    w->sel = reinterpret_cast<int32_t *>(b + w->l.sel);
-    for (int i = 0; i < 3; ++i) w->idx[i] = reinterpret_cast<int32_t *>(b + w->l.idx[i]);
+    for (int s = 0; s < kSlots; ++s) {
+        w->slot[s].hist = reinterpret_cast<uint32_t *>(b + w->l.slot[s].hist);
+        w->slot[s].ctl = reinterpret_cast<RowCtl *>(b + w->l.slot[s].ctl);
+        w->slot[s].S = reinterpret_cast<float *>(b + w->l.slot[s].S);
+        w->slot[s].tie = reinterpret_cast<uint64_t *>(b + w->l.slot[s].tie);
+        w->slot[s].sel = reinterpret_cast<int32_t *>(b + w->l.slot[s].sel);
+    }
+    w->attn_ctl = reinterpret_cast<RowCtl *>(b + w->l.attn_ctl);
+    w->canon = reinterpret_cast<int32_t *>(b + w->l.canon);
+    w->idx_all = reinterpret_cast<int32_t *>(b + w->l.idx_all);
     w->pacc = reinterpret_cast<float *>(b + w->l.pacc);
     w->pml = reinterpret_cast<float *>(b + w->l.pml);
     return PRISM_OK;
@@ -144,58 +219,59 @@ prism_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? PRISM_OK :
 #define PRISM_CUDA(expr) PRISM_TRY(cuda_status(expr))
 
 prism_status_t zero_control(const Ws &w, cudaStream_t s) {
-    return cuda_status(cudaMemsetAsync(w.base + w.l.hist, 0, w.l.ctl_end - w.l.hist, s));
+    return cuda_status(cudaMemsetAsync(w.base + w.l.ctl_begin, 0, w.l.ctl_end - w.l.ctl_begin, s));
 }
 
-// Anchor: Eq. (1) over every token, then Eq. (2).
-prism_status_t run_anchor(const prism_config_t &c, const Ws &w, const void *q, const void *k,
-                          const int32_t *len, int32_t *idx_out, float *scores, cudaStream_t s) {
+ScoreArgs score_args(const prism_config_t &c, const Ws &w, const Slot &sl, const void *q,
+                     const void *k, const int32_t *len) {
     ScoreArgs sa{};
     sa.q = q; sa.k = k; sa.len = len;
     sa.B = c.batch; sa.Hkv = c.n_kv_heads; sa.G = c.n_q_heads / c.n_kv_heads;
     sa.d = c.head_dim; sa.Lmax = c.max_len; sa.scale = eff_scale(c);
-    sa.S = scores ? scores : w.S; sa.hist = w.hist; sa.cpos = nullptr; sa.ctl = w.ctl;
-    sa.st = w.st; sa.wait_ns = wait_limit_ns();
-    PRISM_CUDA(launch_anchor_score(sa, num_sms(), s));
+    sa.S = sl.S; sa.hist = sl.hist; sa.src = nullptr; sa.kappa = c.kappa; sa.radius = c.radius;
+    sa.ctl = sl.ctl; sa.st = w.st; sa.wait_ns = wait_limit_ns();
+    return sa;
+}
+
+SelectArgs select_args(const prism_config_t &c, const Ws &w, const Slot &sl, const float *S,
+                       const int32_t *src, const int32_t *len, int32_t *idx_out) {
     SelectArgs se{};
-    se.S = sa.S; se.cpos = nullptr; se.len = len;
+    se.S = S; se.src = src; se.len = len;
     se.B = c.batch; se.Hkv = c.n_kv_heads; se.Lmax = c.max_len; se.kappa = c.kappa;
-    se.hist = w.hist; se.ctl = w.ctl; se.sel = w.sel; se.tie = w.tie; se.idx_out = idx_out;
+    se.radius = c.radius;
+    se.hist = sl.hist; se.ctl = sl.ctl; se.sel = sl.sel; se.tie = sl.tie; se.idx_out = idx_out;
     se.st = w.st;
-    PRISM_CUDA(launch_select(se, c.max_len, s));
-    return PRISM_OK;
+    return se;
 }
 
-long long proposal_bound(const prism_config_t &c) {
-    const long long win = 2LL * c.radius + 1;
-    const long long b = (long long)c.kappa * win;
-    return b < c.max_len ? b : c.max_len;
+// Anchor scoring (Eq. (1)) into slot `slot`; scores go to `scores` if given.
+prism_status_t run_anchor_score(const prism_config_t &c, const Ws &w, int slot, const void *q,
+                                const void *k, const int32_t *len, float *scores,
+                                cudaStream_t s) {
+    ScoreArgs sa = score_args(c, w, w.slot[slot], q, k, len);
+    if (scores) sa.S = scores;
+    return cuda_status(launch_anchor_score(sa, num_sms(), s));
 }
 
-// Refined layer: +-r proposal, Eq. (5) on it, Eq. (6).
+// Anchor top-kappa (Eq. (2)) from slot `slot`.
+prism_status_t run_anchor_select(const prism_config_t &c, const Ws &w, int slot,
+                                 const int32_t *len, int32_t *idx_out, const float *scores,
+                                 cudaStream_t s) {
+    const Slot &sl = w.slot[slot];
+    return cuda_status(launch_select(select_args(c, w, sl, scores ? scores : sl.S, nullptr, len,
+                                                 idx_out), s));
+}
+
+// Refined layer: +-r proposal around the canonical source selection `src`,
+// Eq. (5) on it, Eq. (6).
 prism_status_t run_refine(const prism_config_t &c, const Ws &w, const void *q, const void *k,
-                          const int32_t *len, const int32_t *idx_prev, int32_t *idx_out,
+                          const int32_t *len, const int32_t *src, int32_t *idx_out,
                           cudaStream_t s) {
-    ExpandArgs ea{};
-    ea.idx_prev = idx_prev; ea.len = len; ea.B = c.batch; ea.Hkv = c.n_kv_heads;
-    ea.Lmax = c.max_len; ea.kappa = c.kappa; ea.radius = c.radius;
-    ea.cpos = w.cpos; ea.ctl = w.ctl; ea.st = w.st;
-    PRISM_CUDA(launch_expand(ea, s));
-    ScoreArgs sa{};
-    sa.q = q; sa.k = k; sa.len = len;
-    sa.B = c.batch; sa.Hkv = c.n_kv_heads; sa.G = c.n_q_heads / c.n_kv_heads;
-    sa.d = c.head_dim; sa.Lmax = c.max_len; sa.scale = eff_scale(c);
-    sa.S = w.S; sa.hist = w.hist; sa.cpos = w.cpos; sa.ctl = w.ctl;
-    sa.st = w.st; sa.wait_ns = wait_limit_ns();
-    const long long bound = proposal_bound(c);
-    PRISM_CUDA(launch_refine_rescore(sa, bound, s));
-    SelectArgs se{};
-    se.S = w.S; se.cpos = w.cpos; se.len = len;
-    se.B = c.batch; se.Hkv = c.n_kv_heads; se.Lmax = c.max_len; se.kappa = c.kappa;
-    se.hist = w.hist; se.ctl = w.ctl; se.sel = w.sel; se.tie = w.tie; se.idx_out = idx_out;
-    se.st = w.st;
-    PRISM_CUDA(launch_select(se, bound, s));
-    return PRISM_OK;
+    const Slot &sl = w.slot[kRefineSlot];
+    ScoreArgs sa = score_args(c, w, sl, q, k, len);
+    sa.src = src;
+    PRISM_CUDA(launch_refine_rescore(sa, s));
+    return cuda_status(launch_select(select_args(c, w, sl, sl.S, src, len, idx_out), s));
 }
 
 prism_status_t run_attn(const prism_config_t &c, const Ws &w, const void *q, const void *k,
@@ -206,8 +282,108 @@ prism_status_t run_attn(const prism_config_t &c, const Ws &w, const void *q, con
     aa.idx_stride = idx_stride; aa.n_idx = n_idx;
     aa.B = c.batch; aa.Hkv = c.n_kv_heads; aa.G = c.n_q_heads / c.n_kv_heads;
     aa.d = c.head_dim; aa.Lmax = c.max_len; aa.scale = eff_scale(c);
-    aa.part_acc = w.pacc; aa.part_ml = w.pml; aa.out = out; aa.st = w.st;
-    PRISM_CUDA(launch_sparse_attn(aa, s));
+    aa.part_acc = w.pacc; aa.part_ml = w.pml; aa.ctl = w.attn_ctl; aa.out = out; aa.st = w.st;
+    return cuda_status(launch_sparse_attn(aa, s));
+}
+
+// The decode step's launch sequence.  With hp == nullptr everything goes to
+// `s0`; otherwise the three streams of the DAG described at the top.  Every
+// event is recorded (on the host) before any wait on it is enqueued.
+prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
+                            const void *const *k, const void *const *v, const int32_t *len,
+                            void *out, int32_t *idx_out, cudaStream_t s0, DeviceHelpers *hp) {
+    const int N = c.n_layers;
+    const size_t rows = (size_t)c.batch * c.n_kv_heads;
+    const size_t sel_elems = rows * (size_t)c.kappa;
+    const size_t q_elems = (size_t)c.batch * c.n_q_heads * c.head_dim;
+    const uint16_t *qb = static_cast<const uint16_t *>(q);
+    uint16_t *ob = static_cast<uint16_t *>(out);
+    int32_t *idx_base = idx_out ? idx_out : w.idx_all;
+    auto is_anchor = [&](int l) { return c.mode == PRISM_MODE_DENSE_ANCHOR || c.anchor_mask[l] != 0; };
+    std::vector<int> anchors;
+    for (int l = 0; l < N; ++l)
+        if (is_anchor(l)) anchors.push_back(l);
+    const int NA = (int)anchors.size();
+
+    cudaStream_t sA = hp ? hp->anchor : s0, sM = hp ? hp->chain : s0, sC = hp ? hp->attn : s0;
+    // Events: fork, two joins, per anchor "scored" and "slot free", per layer "selected".
+    cudaEvent_t ev_fork = nullptr, ev_join_m = nullptr, ev_join_c = nullptr;
+    const cudaEvent_t *ev_scored = nullptr, *ev_free = nullptr, *ev_sel = nullptr;
+    if (hp) {
+        const cudaEvent_t *e = hp->events.data();
+        ev_fork = e[0];
+        ev_join_m = e[1];
+        ev_join_c = e[2];
+        ev_scored = e + 3;
+        ev_free = ev_scored + NA;
+        ev_sel = ev_free + NA;
+    }
+
+    PRISM_TRY(zero_control(w, s0));
+    if (hp) {
+        PRISM_CUDA(cudaEventRecord(ev_fork, s0));
+        PRISM_CUDA(cudaStreamWaitEvent(sA, ev_fork, 0));
+        PRISM_CUDA(cudaStreamWaitEvent(sM, ev_fork, 0));
+        PRISM_CUDA(cudaStreamWaitEvent(sC, ev_fork, 0));
+    }
+    auto score_anchor = [&](int g) -> prism_status_t {
+        const int l = anchors[g];
+        if (hp && g >= 2) PRISM_CUDA(cudaStreamWaitEvent(sA, ev_free[g - 2], 0));
+        PRISM_TRY(run_anchor_score(c, w, g % 2, qb + (size_t)l * q_elems, k[l], len, nullptr, sA));
+        if (hp) PRISM_CUDA(cudaEventRecord(ev_scored[g], sA));
+        return PRISM_OK;
+    };
+    // The anchor stream starts up to two anchors ahead.
+    if (hp) {
+        for (int g = 0; g < NA && g < 2; ++g) PRISM_TRY(score_anchor(g));
+    }
+
+    const int32_t *anchor_sel = nullptr;
+    const int32_t *prev_sel = nullptr;
+    int g = 0;
+    for (int l = 0; l < N; ++l) {
+        const void *ql = qb + (size_t)l * q_elems;
+        const int32_t *src = c.chain == PRISM_CHAIN_ANCHOR ? anchor_sel : prev_sel;
+        int32_t *dst = idx_base + (size_t)l * sel_elems;
+        const int32_t *cur = dst;
+        if (is_anchor(l)) {
+            if (hp) {
+                PRISM_CUDA(cudaStreamWaitEvent(sM, ev_scored[g], 0));
+            } else {
+                PRISM_TRY(score_anchor(g));
+            }
+            PRISM_TRY(run_anchor_select(c, w, g % 2, len, dst, nullptr, sM));
+            if (hp) {
+                PRISM_CUDA(cudaEventRecord(ev_free[g], sM));
+                if (g + 2 < NA) PRISM_TRY(score_anchor(g + 2));
+            }
+            anchor_sel = dst;
+            ++g;
+        } else if (c.mode == PRISM_MODE_STATIC_REUSE) {
+            if (idx_out) {
+                PRISM_CUDA(cudaMemcpyAsync(dst, src, sel_elems * sizeof(int32_t),
+                                           cudaMemcpyDeviceToDevice, sM));
+            } else {
+                cur = src;
+            }
+        } else {
+            PRISM_TRY(run_refine(c, w, ql, k[l], len, src, dst, sM));
+        }
+        if (hp) {
+            PRISM_CUDA(cudaEventRecord(ev_sel[l], sM));
+            PRISM_CUDA(cudaStreamWaitEvent(sC, ev_sel[l], 0));
+        }
+        PRISM_TRY(run_attn(c, w, ql, k[l], v[l], len, cur, c.kappa, c.kappa,
+                           ob + (size_t)l * q_elems, sC));
+        prev_sel = cur;
+    }
+    if (hp) {
+        // Every anchor score was waited on by M; join M and C into the caller's stream.
+        PRISM_CUDA(cudaEventRecord(ev_join_m, sM));
+        PRISM_CUDA(cudaEventRecord(ev_join_c, sC));
+        PRISM_CUDA(cudaStreamWaitEvent(s0, ev_join_m, 0));
+        PRISM_CUDA(cudaStreamWaitEvent(s0, ev_join_c, 0));
+    }
     return PRISM_OK;
 }
 
@@ -234,7 +410,8 @@ prism_status_t prism_index_anchor(const prism_config_t *cfg, const void *q, cons
     PRISM_TRY(carve(*cfg, ws, ws_bytes, &w));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     PRISM_TRY(zero_control(w, s));
-    return run_anchor(*cfg, w, q, k, len, idx_out, scores_out, s);
+    PRISM_TRY(run_anchor_score(*cfg, w, 0, q, k, len, scores_out, s));
+    return run_anchor_select(*cfg, w, 0, len, idx_out, scores_out, s);
 }
 
 prism_status_t prism_score_anchor(const prism_config_t *cfg, const void *q, const void *k,
@@ -246,14 +423,7 @@ prism_status_t prism_score_anchor(const prism_config_t *cfg, const void *q, cons
         return PRISM_ERR_INVALID_ARG;
     Ws w;
     PRISM_TRY(carve(*cfg, ws, ws_bytes, &w));
-    const prism_config_t &c = *cfg;
-    ScoreArgs sa{};
-    sa.q = q; sa.k = k; sa.len = len;
-    sa.B = c.batch; sa.Hkv = c.n_kv_heads; sa.G = c.n_q_heads / c.n_kv_heads;
-    sa.d = c.head_dim; sa.Lmax = c.max_len; sa.scale = eff_scale(c);
-    sa.S = scores_out; sa.hist = w.hist; sa.cpos = nullptr; sa.ctl = w.ctl;
-    sa.st = w.st; sa.wait_ns = wait_limit_ns();
-    return cuda_status(launch_anchor_score(sa, num_sms(), static_cast<cudaStream_t>(stream)));
+    return run_anchor_score(*cfg, w, 0, q, k, len, scores_out, static_cast<cudaStream_t>(stream));
 }
 
 prism_status_t prism_index_refine(const prism_config_t *cfg, const void *q, const void *k,
@@ -275,11 +445,16 @@ prism_status_t prism_index_refine(const prism_config_t *cfg, const void *q, cons
     PRISM_TRY(carve(*cfg, ws, ws_bytes, &w));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     PRISM_TRY(zero_control(w, s));
-    PRISM_TRY(run_refine(*cfg, w, q, k, len, idx_prev, idx_out, s));
+    CanonArgs ca{};
+    ca.idx = idx_prev; ca.len = len; ca.B = cfg->batch; ca.Hkv = cfg->n_kv_heads;
+    ca.Lmax = cfg->max_len; ca.kappa = cfg->kappa; ca.out = w.canon; ca.st = w.st;
+    PRISM_CUDA(launch_canonicalize(ca, s));
+    PRISM_TRY(run_refine(*cfg, w, q, k, len, w.canon, idx_out, s));
     if (all)
-        PRISM_CUDA(launch_export_candidates(w.S, w.cpos, w.ctl, cfg->batch * cfg->n_kv_heads,
-                                            cfg->max_len, cand_pos, cand_score, cand_count,
-                                            cand_cap, s));
+        PRISM_CUDA(launch_export_candidates(w.slot[kRefineSlot].S, w.canon, nullptr, len,
+                                            cfg->batch, cfg->n_kv_heads, cfg->max_len,
+                                            cfg->kappa, cfg->radius, cand_pos, cand_score,
+                                            cand_count, cand_cap, w.st, s));
     return PRISM_OK;
 }
 
@@ -295,8 +470,10 @@ prism_status_t prism_sparse_decode(const prism_config_t *cfg, const void *q, con
         return PRISM_ERR_INVALID_ARG;
     Ws w;
     PRISM_TRY(carve(*cfg, ws, ws_bytes, &w));
-    return run_attn(*cfg, w, q, k, v, len, idx, n_idx, n_idx, out,
-                    static_cast<cudaStream_t>(stream));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    PRISM_CUDA(cudaMemsetAsync(w.attn_ctl, 0,
+                               (size_t)cfg->batch * cfg->n_kv_heads * sizeof(RowCtl), s));
+    return run_attn(*cfg, w, q, k, v, len, idx, n_idx, n_idx, out, s);
 }
 
 prism_status_t prism_decode_step(const prism_config_t *cfg, const void *q, const void *const *k,
@@ -317,47 +494,11 @@ prism_status_t prism_decode_step(const prism_config_t *cfg, const void *q, const
     Ws w;
     PRISM_TRY(carve(c, ws, ws_bytes, &w));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    PRISM_TRY(zero_control(w, s));
-
-    const size_t rows = (size_t)c.batch * c.n_kv_heads;
-    const size_t sel_elems = rows * (size_t)c.kappa;
-    const size_t q_elems = (size_t)c.batch * c.n_q_heads * c.head_dim;
-    const uint16_t *qb = static_cast<const uint16_t *>(q);
-    uint16_t *ob = static_cast<uint16_t *>(out);
-
-    const int32_t *anchor_sel = nullptr;   // most recent anchor layer's selection
-    const int32_t *prev_sel = nullptr;     // previous layer's selection
-    int flip = 0;
-    for (int l = 0; l < c.n_layers; ++l) {
-        const bool anchor = c.mode == PRISM_MODE_DENSE_ANCHOR || c.anchor_mask[l];
-        const void *ql = qb + (size_t)l * q_elems;
-        const int32_t *src = c.chain == PRISM_CHAIN_ANCHOR ? anchor_sel : prev_sel;
-        const int32_t *cur = nullptr;
-        if (anchor) {
-            int32_t *dst = idx_out ? idx_out + (size_t)l * sel_elems : w.idx[2];
-            PRISM_TRY(run_anchor(c, w, ql, k[l], len, dst, nullptr, s));
-            cur = dst;
-            anchor_sel = dst;
-        } else if (c.mode == PRISM_MODE_STATIC_REUSE) {
-            if (idx_out) {
-                int32_t *dst = idx_out + (size_t)l * sel_elems;
-                PRISM_CUDA(cudaMemcpyAsync(dst, src, sel_elems * sizeof(int32_t),
-                                           cudaMemcpyDeviceToDevice, s));
-                cur = dst;
-            } else {
-                cur = src;
-            }
-        } else {
-            int32_t *dst = idx_out ? idx_out + (size_t)l * sel_elems : w.idx[flip];
-            flip ^= 1;
-            PRISM_TRY(run_refine(c, w, ql, k[l], len, src, dst, s));
-            cur = dst;
-        }
-        PRISM_TRY(run_attn(c, w, ql, k[l], v[l], len, cur, c.kappa, c.kappa,
-                           ob + (size_t)l * q_elems, s));
-        prev_sel = cur;
-    }
-    return PRISM_OK;
+    if (c.flags & PRISM_FLAG_SERIAL) return enqueue_step(c, w, q, k, v, len, out, idx_out, s, nullptr);
+    std::lock_guard<std::mutex> lock(g_helpers_mu);
+    DeviceHelpers *hp = nullptr;
+    PRISM_TRY(helpers_for_current_device(3 + 3 * (size_t)c.n_layers, &hp));
+    return enqueue_step(c, w, q, k, v, len, out, idx_out, s, hp);
 }
 
 prism_status_t prism_check_device_status(void *ws, size_t ws_bytes, void *stream,
@@ -405,6 +546,6 @@ const char *prism_status_string(prism_status_t st) {
 
 uint64_t prism_launch_count(void) { return g_launches; }
 
-int32_t prism_version(void) { return 100; }
+int32_t prism_version(void) { return 10100; }
 
 }  // extern "C"

@@ -29,7 +29,7 @@ enum : uint32_t {
 enum : uint32_t {
     kWhereScore = 1,
     kWhereRescore = 2,
-    kWhereExpand = 3,
+    kWhereCanon = 3,
     kWhereCollect = 4,
     kWhereFinalize = 5,
     kWhereAttn = 6,
@@ -37,12 +37,14 @@ enum : uint32_t {
 };
 
 // Per (batch, KV head) row counters; zeroed at the start of every public call
-// and left zeroed by the kernels that consume them.
+// that uses them and left zeroed by the kernels that consume them.
 struct RowCtl {
-    int32_t n_sel;     // items strictly above the threshold digit (collect)
-    int32_t n_tie;     // items on the threshold digit (collect)
-    int32_t n_prop;    // |P| of the refine proposal (expand)
-    int32_t pad;
+    int32_t n_sel;         // items strictly above the threshold digit (select)
+    int32_t n_tie;         // items on the threshold digit (select)
+    int32_t n_prop;        // |P| of the refine proposal (rescore)
+    uint32_t done_select;  // select CTAs of this row that have finished
+    uint32_t done_attn;    // attention CTAs of this row that have finished
+    int32_t pad[3];
 };
 
 __device__ __forceinline__ void report(DevStatus *st, uint32_t code, uint32_t where,
@@ -137,6 +139,34 @@ __device__ __forceinline__ int transpose_item(int lane) {
 template <int NV, int NL>
 __device__ __forceinline__ bool transpose_writer(int lane) {
     return (lane & (NL / NV - 1)) == 0;
+}
+
+// ---- positional proposal: owned ranges ------------------------------------
+// A canonical selection lists distinct positions in ascending order, then -1
+// padding.  With it, the proposal P = union of [i - r, i + r] clipped to
+// [0, L) splits into disjoint consecutive ranges: entry j owns the positions of
+// its window that no earlier entry's window covers,
+//   lo_j = max(i_j - r, i_{j-1} + r + 1, 0),  hi_j = min(i_j + r, L - 1),
+// so P is enumerated in ascending order, without duplicates, entry by entry.
+// A malformed entry (>= L, or not above its predecessor) is reported and owns
+// nothing; the ranges stay inside [0, L) either way.
+__device__ __forceinline__ int owned_range(const int32_t *src, int j, long long r, int L,
+                                           int *lo_out, DevStatus *st, uint32_t where) {
+    const int i = src[j];
+    if (i < 0) return 0;
+    const int prev = j > 0 ? src[j - 1] : -1;
+    if (i >= L || (prev >= 0 && i <= prev)) {
+        report(st, kDevErrBadIndex, where, (uint32_t)i);
+        return 0;
+    }
+    long long lo = (long long)i - r;
+    if (prev >= 0 && (long long)prev + r + 1 > lo) lo = (long long)prev + r + 1;
+    if (lo < 0) lo = 0;
+    long long hi = (long long)i + r;
+    if (hi > L - 1) hi = L - 1;
+    if (hi < lo) return 0;
+    *lo_out = (int)lo;
+    return (int)(hi - lo + 1);
 }
 
 // ---- mbarrier / bulk-copy (TMA) primitives -------------------------------
@@ -280,6 +310,39 @@ __device__ __forceinline__ void find_threshold_bin(const uint32_t *hist, int nbi
     __syncthreads();
 }
 
+// Enumeration of the proposal positions owned by entries [j0, j0 + kPropEntries)
+// of a canonical source selection: per-entry range starts in lo_s, exclusive
+// offsets in off_s[0..kPropEntries].  Returns the number of positions (all
+// threads).  Needs blockDim.x >= kPropEntries.  Contains __syncthreads().
+constexpr int kPropEntries = 64;
+__device__ __forceinline__ int proposal_slice(const int32_t *src_row, int j0, int kappa,
+                                              int radius, int L, int *lo_s, int *off_s,
+                                              int *scratch, DevStatus *st, uint32_t where) {
+    int cnt = 0, lo = 0;
+    const int t = threadIdx.x;
+    if (t < kPropEntries && j0 + t < kappa)
+        cnt = owned_range(src_row, j0 + t, radius, L, &lo, st, where);
+    int total;
+    const int ex = block_exclusive_scan(t < kPropEntries ? cnt : 0, scratch, &total);
+    if (t < kPropEntries) {
+        lo_s[t] = lo;
+        off_s[t] = ex;
+    }
+    if (t == 0) off_s[kPropEntries] = total;
+    __syncthreads();
+    return total;
+}
+
+// Position of enumeration index e of a proposal slice.
+__device__ __forceinline__ int slice_position(const int *lo_s, const int *off_s, int e) {
+    int a = 0, b = kPropEntries - 1;       // largest t with off_s[t] <= e
+    while (a < b) {
+        const int m = (a + b + 1) >> 1;
+        if (off_s[m] <= e) a = m; else b = m - 1;
+    }
+    return lo_s[a] + (e - off_s[a]);
+}
+
 // ---- launch interfaces (host side, defined in the .cu files) -------------
 // Kernels launched by the calling host thread (see prism_launch_count()).
 void count_launches(int n);
@@ -290,32 +353,32 @@ struct ScoreArgs {
     const int32_t *len;     // [B]
     int B, Hkv, G, d, Lmax;
     float scale;
-    float *S;               // fp32 [rows][Lmax]: anchor scores / refine candidate scores
+    float *S;               // fp32 [rows][Lmax], indexed by position
     uint32_t *hist;         // [rows][kHistBins]
-    const int32_t *cpos;    // refine: [rows][Lmax] proposal positions (ascending)
+    const int32_t *src;     // refine: canonical source selection [rows][kappa]
+    int kappa, radius;      // refine
     RowCtl *ctl;            // [rows]
     DevStatus *st;
     uint64_t wait_ns;
 };
 
 cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s);
-cudaError_t launch_refine_rescore(const ScoreArgs &a, long long max_prop, cudaStream_t s);
+cudaError_t launch_refine_rescore(const ScoreArgs &a, cudaStream_t s);
 
-struct ExpandArgs {
-    const int32_t *idx_prev;   // [rows][kappa]
-    const int32_t *len;
-    int B, Hkv, Lmax, kappa, radius;
-    int32_t *cpos;             // [rows][Lmax]
-    RowCtl *ctl;
-    DevStatus *st;
-};
-cudaError_t launch_expand(const ExpandArgs &a, cudaStream_t s);
-
-struct SelectArgs {
-    const float *S;            // [rows][Lmax] scores (anchor: by position; refine: by proposal slot)
-    const int32_t *cpos;       // refine: [rows][Lmax] positions; nullptr for the anchor
+struct CanonArgs {
+    const int32_t *idx;        // [rows][kappa], any order, duplicates, -1 padding
     const int32_t *len;
     int B, Hkv, Lmax, kappa;
+    int32_t *out;              // [rows][kappa] canonical: ascending, distinct, -1 padded
+    DevStatus *st;
+};
+cudaError_t launch_canonicalize(const CanonArgs &a, cudaStream_t s);
+
+struct SelectArgs {
+    const float *S;            // [rows][Lmax] scores indexed by position
+    const int32_t *src;        // refine: canonical source selection; nullptr for the anchor
+    const int32_t *len;
+    int B, Hkv, Lmax, kappa, radius;
     uint32_t *hist;            // [rows][kHistBins]
     RowCtl *ctl;
     int32_t *sel;              // [rows][kappa] positions above the threshold digit
@@ -323,7 +386,7 @@ struct SelectArgs {
     int32_t *idx_out;          // [rows][kappa]
     DevStatus *st;
 };
-cudaError_t launch_select(const SelectArgs &a, long long max_items, cudaStream_t s);
+cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
 
 struct AttnArgs {
     const void *q;             // bf16 [B][Hq][d]
@@ -335,15 +398,18 @@ struct AttnArgs {
     float scale;
     float *part_acc;           // [rows][nsplit][G][d]
     float *part_ml;            // [rows][nsplit][G][2]
+    RowCtl *ctl;
     void *out;                 // bf16 [B][Hq][d]
     DevStatus *st;
 };
 constexpr int kAttnChunk = 64;
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s);
 
-cudaError_t launch_export_candidates(const float *S, const int32_t *cpos, const RowCtl *ctl,
-                                     int rows, int Lmax, int32_t *cand_pos, float *cand_score,
-                                     int32_t *cand_count, int cand_cap, cudaStream_t s);
+cudaError_t launch_export_candidates(const float *S, const int32_t *src, const RowCtl *ctl,
+                                     const int32_t *len, int B, int Hkv, int Lmax, int kappa,
+                                     int radius, int32_t *cand_pos, float *cand_score,
+                                     int32_t *cand_count, int cand_cap, DevStatus *st,
+                                     cudaStream_t s);
 
 cudaError_t launch_debug_wait(DevStatus *st, uint64_t limit_ns, cudaStream_t s);
 

@@ -16,7 +16,8 @@
 // first radix digit of the top-kappa selection.
 //
 // k_refine_rescore scores only the proposal positions of a refined layer
-// (Eq. (5)): rows are gathered with 16-byte non-caching loads.
+// (Eq. (5)), enumerated from the owned ranges of the source selection; each
+// owned range is one bulk copy, and scores are stored by position.
 #include "prism_internal.cuh"
 
 namespace prism {
@@ -267,53 +268,79 @@ k_anchor_score(ScoreArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Refined layer: score only the proposal positions (Eq. (5)).
+// Refined layer: score only the proposal positions (Eq. (5)).  One CTA per 16
+// entries of the (canonical) source selection.  Each entry owns a contiguous
+// run of key rows, so the gather is one 1-D bulk copy (TMA) per run, issued by
+// 16 lanes of warp 0 into a shared-memory buffer that completes on an
+// mbarrier; nothing is held in registers while the copies fly.  The eight
+// warps then form 32 dot products per round each from shared memory, and the
+// transposing reduction leaves one score per lane, stored by position.
 template <int D>
 struct RescoreCfg {
-    static constexpr int kTile = 128;        // proposal slots per CTA
+    static constexpr int kEntries = 16;
     static constexpr int kWarps = 8;
     static constexpr int kThreads = 32 * kWarps;
     static constexpr int kNL = D / 8;
     static constexpr int kRPI = 32 / kNL;
-    static constexpr int kRowsPerWarp = kTile / kWarps;
-    static constexpr int kSteps = kRowsPerWarp / kRPI;
+    static constexpr int kRowsPerWarp = 32;
+    static constexpr int kSteps = kRowsPerWarp / kRPI;       // == kNL
+    static constexpr int kRowBytes = D * 2;
+    static constexpr int kCapRows = 48 * 1024 / kRowBytes;    // rows staged per round
+    static constexpr int kSmemBytes = kCapRows * kRowBytes;
+    static_assert(kSteps == kNL, "one score per lane after the reduction");
 };
 
 template <int D>
 __global__ void __launch_bounds__(RescoreCfg<D>::kThreads)
 k_refine_rescore(ScoreArgs a) {
     using C = RescoreCfg<D>;
+    extern __shared__ __align__(128) uint8_t rows_s[];
+    __shared__ uint64_t bar;
     __shared__ uint32_t hist_s[kHistBins];
+    __shared__ int lo_s[C::kEntries], cnt_s[C::kEntries], off_s[C::kEntries + 1];
+    __shared__ int pos_s[C::kCapRows];
+    __shared__ int fail_s;
     const int row = blockIdx.y;
-    const int n = a.ctl[row].n_prop;
-    const int e0 = blockIdx.x * C::kTile;
-    if (e0 >= n) return;
+    const int j0 = blockIdx.x * C::kEntries;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = row / a.Hkv, h = row % a.Hkv;
-    const int slice = lane % C::kNL, sub = lane / C::kNL;
-    const int Hq = a.Hkv * a.G;
+    const int L = load_len(a.len, b, a.Lmax, a.st, kWhereRescore);
+    const int32_t *src = a.src + (size_t)row * a.kappa;
 
-    for (int i = tid; i < kHistBins; i += C::kThreads) hist_s[i] = 0;
-
-    const int32_t *cpos = a.cpos + (size_t)row * a.Lmax;
-    const uint16_t *kb = static_cast<const uint16_t *>(a.k) +
-                                  (size_t)row * a.Lmax * D;
-    uint4 kv[C::kSteps];
-    const int ebase = e0 + warp * C::kRowsPerWarp + sub;
+    if (warp == 0) {
+        int lo = 0, cnt = 0;
+        if (lane < C::kEntries && j0 + lane < a.kappa)
+            cnt = owned_range(src, j0 + lane, a.radius, L, &lo, a.st, kWhereRescore);
+        int incl = cnt;
 #pragma unroll
-    for (int st = 0; st < C::kSteps; ++st) {
-        const int e = ebase + st * C::kRPI;
-        if (e < n) {
-            const int p = __ldg(cpos + e);
-            kv[st] = ld_nc_v4(kb + (size_t)p * D + slice * 8);
-        } else {
-            kv[st] = make_uint4(0u, 0u, 0u, 0u);
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane < C::kEntries) {
+            lo_s[lane] = lo;
+            cnt_s[lane] = cnt;
+            off_s[lane] = incl - cnt;
+        }
+        if (lane == C::kEntries - 1) off_s[C::kEntries] = incl;
+        if (lane == 0) {
+            fail_s = 0;
+            mbar_init(&bar, 1);
+            fence_mbar_init();
         }
     }
+    for (int i = tid; i < kHistBins; i += C::kThreads) hist_s[i] = 0;
+    __syncthreads();
+    const int total = off_s[C::kEntries];
+    if (total == 0) return;
+    if (tid == 0) atomicAdd(&a.ctl[row].n_prop, total);
+
+    const int slice = lane % C::kNL, sub = lane / C::kNL;
     float qreg[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) qreg[e] = 0.f;
     const uint16_t *qb = static_cast<const uint16_t *>(a.q);
+    const int Hq = a.Hkv * a.G;
     for (int g = 0; g < a.G; ++g) {
         const uint4 w = *reinterpret_cast<const uint4 *>(
             qb + ((size_t)b * Hq + (size_t)h * a.G + g) * D + slice * 8);
@@ -322,19 +349,69 @@ k_refine_rescore(ScoreArgs a) {
         qreg[4] += bf16_lo(w.z); qreg[5] += bf16_hi(w.z);
         qreg[6] += bf16_lo(w.w); qreg[7] += bf16_hi(w.w);
     }
-    float part[C::kSteps];
+    const uint16_t *kb = static_cast<const uint16_t *>(a.k) + (size_t)row * a.Lmax * D;
+    float *S = a.S + (size_t)row * a.Lmax;
+
+    int round = 0;
+    bool pending = false;      // warp 0 lane 0: a round's copies may still be in flight
+    for (int e0 = 0; e0 < total; e0 += C::kCapRows, ++round) {
+        const int nr = min(C::kCapRows, total - e0);
+        for (int i = tid; i < nr; i += C::kThreads) {
+            int t = 0;                                  // entry owning index e0 + i
 #pragma unroll
-    for (int st = 0; st < C::kSteps; ++st) part[st] = dot8(kv[st], qreg);
-    transpose_reduce<C::kSteps, C::kNL>(part, lane);
-    __syncthreads();   // hist_s zeroed
-    const int item = transpose_item<C::kSteps, C::kNL>(lane);
-    const int e = ebase + item * C::kRPI;
-    if (transpose_writer<C::kSteps, C::kNL>(lane) && e < n) {
-        const float sc = part[0] * a.scale;
-        a.S[(size_t)row * a.Lmax + e] = sc;
-        atomicAdd(&hist_s[score_key(sc) >> (32 - kHistBits)], 1u);
+            for (int m = 8; m >= 1; m >>= 1)
+                if (t + m < C::kEntries && off_s[t + m] <= e0 + i) t += m;
+            pos_s[i] = lo_s[t] + (e0 + i - off_s[t]);
+        }
+        if (warp == 0) {
+            if (lane == 0) mbar_arrive_expect_tx(&bar, (uint32_t)nr * C::kRowBytes);
+            __syncwarp();
+            if (lane < C::kEntries) {
+                const int s0 = max(off_s[lane], e0);
+                const int s1 = min(off_s[lane] + cnt_s[lane], e0 + nr);
+                if (s0 < s1) {
+                    const uint64_t pol = l2_evict_first_policy();
+                    bulk_load(rows_s + (size_t)(s0 - e0) * C::kRowBytes,
+                              kb + (size_t)(lo_s[lane] + s0 - off_s[lane]) * D,
+                              (uint32_t)(s1 - s0) * C::kRowBytes, &bar, pol);
+                }
+            }
+            pending = true;
+        }
+        __syncthreads();                                 // pos_s ready
+        const bool ok = mbar_wait(&bar, (uint32_t)round & 1u, a.wait_ns);
+        if (!ok) {
+            report(a.st, kDevErrTimeout, kWhereRescore, (uint32_t)round);
+            fail_s = 1;
+        } else {
+            if (warp == 0) pending = false;
+            for (int r0 = warp * C::kRowsPerWarp; r0 < nr; r0 += C::kWarps * C::kRowsPerWarp) {
+                float part[C::kSteps];
+#pragma unroll
+                for (int st = 0; st < C::kSteps; ++st) {
+                    const int r = r0 + st * C::kRPI + sub;
+                    const uint4 kv = *reinterpret_cast<const uint4 *>(
+                        rows_s + (size_t)r * C::kRowBytes + slice * 16);
+                    part[st] = dot8(kv, qreg);
+                }
+                transpose_reduce<C::kSteps, C::kNL>(part, lane);
+                const int r = r0 + transpose_item<C::kSteps, C::kNL>(lane) * C::kRPI + sub;
+                if (r < nr) {
+                    const float sc = part[0] * a.scale;
+                    S[pos_s[r]] = sc;
+                    atomicAdd(&hist_s[score_key(sc) >> (32 - kHistBits)], 1u);
+                }
+            }
+        }
+        __syncthreads();                                 // buffer and pos_s free again
+        if (fail_s) break;
     }
-    __syncthreads();
+    if (fail_s) {
+        // Let any copy still in flight land before the CTA's shared memory goes.
+        if (tid == 0 && pending && !mbar_wait(&bar, (uint32_t)round & 1u, a.wait_ns))
+            report(a.st, kDevErrTimeout, kWhereRescore, 0x80000000u | (uint32_t)round);
+        return;
+    }
     for (int i = tid; i < kHistBins; i += C::kThreads) {
         const uint32_t v = hist_s[i];
         if (v) atomicAdd(a.hist + (size_t)row * kHistBins + i, v);
@@ -362,20 +439,19 @@ cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s)
 }
 
 template <int D>
-static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, long long max_prop,
-                                           cudaStream_t s) {
+static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, cudaStream_t s) {
     using C = RescoreCfg<D>;
-    const long long tiles = (max_prop + C::kTile - 1) / C::kTile;
-    if (tiles <= 0) return cudaSuccess;
-    dim3 grid((unsigned)tiles, (unsigned)(a.B * a.Hkv));
-    k_refine_rescore<D><<<grid, C::kThreads, 0, s>>>(a);
+    cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((a.kappa + C::kEntries - 1) / C::kEntries), (unsigned)(a.B * a.Hkv));
+    k_refine_rescore<D><<<grid, C::kThreads, C::kSmemBytes, s>>>(a);
     count_launches(1);
     return cudaGetLastError();
 }
 
-cudaError_t launch_refine_rescore(const ScoreArgs &a, long long max_prop, cudaStream_t s) {
-    return a.d == 128 ? launch_refine_rescore_d<128>(a, max_prop, s)
-                      : launch_refine_rescore_d<64>(a, max_prop, s);
+cudaError_t launch_refine_rescore(const ScoreArgs &a, cudaStream_t s) {
+    return a.d == 128 ? launch_refine_rescore_d<128>(a, s) : launch_refine_rescore_d<64>(a, s);
 }
 
 }  // namespace prism

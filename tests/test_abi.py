@@ -65,6 +65,7 @@ def test_workspace_size_monotone(L):
     (dict(max_len=(1 << 20) + 1), 2), (dict(batch=0), 1), (dict(mode=3), 1), (dict(chain=2), 1),
     (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1), (dict(batch=70000, n_kv_heads=1,
                                                                   n_q_heads=1), 2),
+    (dict(flags=2), 1), (dict(n_layers=-1), 1), (dict(n_layers=5000), 2),
 ])
 def test_invalid_config_rejected(L, bad, status):
     c = _cfg(**bad)

@@ -159,3 +159,26 @@ def test_invariants_on_gpu(oracle):
                              np.arange(w.max_len), 1.0 / math.sqrt(w.head_dim))
             got = out[l, 0, h * G:(h + 1) * G].float().cpu().numpy()
             assert np.all(np.abs(got - ref) <= 2e-2 + 1e-2 * np.abs(ref))
+
+
+def test_dag_schedule_matches_serial_and_graph(oracle):
+    """The multi-stream schedule, the single-stream schedule and a CUDA-graph
+    replay of the step give bit-identical selections and outputs."""
+    from long_context_decoding_anchor_b200.runner import DecodeStepGraph
+    w = synth.WORKLOADS[2].replace(max_len=9000, n_layers=9, anchor_every=3, kappa=512)
+    inp = _inputs(w)
+    cfg = prism.Config.from_workload(w)
+    out_d, idx_d = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                           want_idx=True)
+    cfg_s = prism.Config.from_workload(w, flags=prism.FLAG_SERIAL)
+    out_s, idx_s = prism.prism_decode_step(cfg_s, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                           want_idx=True)
+    assert torch.equal(idx_d, idx_s) and torch.equal(out_d, out_s)
+    idx_g = torch.empty_like(idx_d)
+    g = DecodeStepGraph(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], idx_out=idx_g)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(idx_g, idx_d) and torch.equal(g.out, out_d)
+    st, detail = prism.prism_check_device_status(g.ws)
+    assert st == 0, detail
