@@ -122,6 +122,10 @@ k_sparse_attn(AttnArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int L = load_len(a.len, b, a.Lmax, a.st, kWhereAttn);
     const int t0 = chunk * C::kC;
+    // The selection may come from the preceding kernel of this stream, and the
+    // partials buffer is shared with the preceding attention kernel.
+    pdl_wait();
+    pdl_launch_dependents();
 
     if (tid < C::kC) {
         int i = -1;
@@ -273,9 +277,7 @@ template <int D, int G>
 static cudaError_t launch_attn_dg(const AttnArgs &a, cudaStream_t s) {
     const int rows = a.B * a.Hkv;
     const int nsplit = (a.n_idx + kAttnChunk - 1) / kAttnChunk;
-    k_sparse_attn<D, G><<<dim3(nsplit, rows), 128, 0, s>>>(a);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_kernel(k_sparse_attn<D, G>, dim3(nsplit, rows), dim3(128), 0, s, a);
 }
 
 template <int D>

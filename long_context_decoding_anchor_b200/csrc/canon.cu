@@ -8,7 +8,8 @@
 // a caller's selection may come in any order, with duplicates.  One CTA per
 // (batch, KV head) marks the selected positions in a shared-memory bitmap
 // (duplicates vanish there) and a block-wide popcount scan writes them back in
-// ascending order.
+// ascending order, followed by the enumeration offsets of the proposal around
+// them.
 #include "prism_internal.cuh"
 
 namespace prism {
@@ -24,6 +25,7 @@ k_canonicalize(CanonArgs a) {
     const int tid = threadIdx.x;
     const int L = load_len(a.len, b, a.Lmax, a.st, kWhereCanon);
     const int words = (L + 31) >> 5;
+    pdl_wait();
 
     for (int w = tid; w < words; w += blockDim.x) bitmap[w] = 0u;
     __syncthreads();
@@ -56,6 +58,9 @@ k_canonicalize(CanonArgs a) {
         }
     }
     for (int e = total + tid; e < a.kappa; e += blockDim.x) out[e] = -1;
+    __syncthreads();
+    proposal_offsets(out, a.kappa, a.radius, L, a.out_off + (size_t)row * (a.kappa + 1), scratch,
+                     a.st);
 }
 
 cudaError_t launch_canonicalize(const CanonArgs &a, cudaStream_t s) {
@@ -63,9 +68,7 @@ cudaError_t launch_canonicalize(const CanonArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(k_canonicalize,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    k_canonicalize<<<a.B * a.Hkv, kCanonThreads, smem, s>>>(a);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_kernel(k_canonicalize, dim3(a.B * a.Hkv), dim3(kCanonThreads), smem, s, a);
 }
 
 }  // namespace prism

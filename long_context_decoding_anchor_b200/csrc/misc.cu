@@ -4,44 +4,30 @@
 
 namespace prism {
 
-// The proposal of a refined layer in ascending order, with its scores: the
-// owned ranges of the canonical source selection, enumerated by one CTA per
-// row.
-__global__ void __launch_bounds__(512)
-k_export_candidates(const float *S, const int32_t *src, const int32_t *len, int Hkv, int Lmax,
-                    int kappa, int radius, int32_t *cand_pos, float *cand_score,
-                    int32_t *cand_count, int cand_cap, DevStatus *st) {
-    __shared__ int scratch[40];
-    const int row = blockIdx.x, tid = threadIdx.x;
-    const int L = load_len(len, row / Hkv, Lmax, st, kWhereCanon);
-    const int32_t *s = src + (size_t)row * kappa;
-    int running = 0;
-    for (int jb = 0; jb < kappa; jb += blockDim.x) {
-        int lo = 0, cnt = 0;
-        if (jb + tid < kappa) cnt = owned_range(s, jb + tid, radius, L, &lo, st, kWhereCanon);
-        int tot;
-        const int ex = block_exclusive_scan(cnt, scratch, &tot);
-        for (int i = 0; i < cnt; ++i) {
-            const int o = running + ex + i;
-            if (o < cand_cap) {
-                cand_pos[(size_t)row * cand_cap + o] = lo + i;
-                cand_score[(size_t)row * cand_cap + o] = S[(size_t)row * Lmax + lo + i];
-            }
-        }
-        running += tot;
+// Diagnostic copy of a refined layer's candidates (ascending positions and
+// their scores) into caller buffers of capacity cand_cap per row.
+__global__ void __launch_bounds__(256)
+k_export_candidates(const float *cscore, const int32_t *cpos, const int32_t *src_off, int Lmax,
+                    int kappa, int32_t *cand_pos, float *cand_score, int32_t *cand_count,
+                    int cand_cap) {
+    pdl_wait();
+    const int row = blockIdx.y;
+    const int n = min(src_off[(size_t)row * (kappa + 1) + kappa], Lmax);
+    if (blockIdx.x == 0 && threadIdx.x == 0) cand_count[row] = n;
+    const int lim = min(n, cand_cap);
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < lim; e += gridDim.x * blockDim.x) {
+        cand_pos[(size_t)row * cand_cap + e] = cpos[(size_t)row * Lmax + e];
+        cand_score[(size_t)row * cand_cap + e] = cscore[(size_t)row * Lmax + e];
     }
-    if (tid == 0) cand_count[row] = running;
 }
 
-cudaError_t launch_export_candidates(const float *S, const int32_t *src, const RowCtl *,
-                                     const int32_t *len, int B, int Hkv, int Lmax, int kappa,
-                                     int radius, int32_t *cand_pos, float *cand_score,
-                                     int32_t *cand_count, int cand_cap, DevStatus *st,
-                                     cudaStream_t s) {
-    k_export_candidates<<<B * Hkv, 512, 0, s>>>(S, src, len, Hkv, Lmax, kappa, radius, cand_pos,
-                                                cand_score, cand_count, cand_cap, st);
-    count_launches(1);
-    return cudaGetLastError();
+cudaError_t launch_export_candidates(const float *cscore, const int32_t *cpos,
+                                     const int32_t *src_off, int rows, int Lmax, int kappa,
+                                     int32_t *cand_pos, float *cand_score, int32_t *cand_count,
+                                     int cand_cap, cudaStream_t s) {
+    const int blocks = max(1, min(64, (cand_cap + 255) / 256));
+    return launch_kernel(k_export_candidates, dim3(blocks, rows), dim3(256), 0, s, cscore, cpos,
+                         src_off, Lmax, kappa, cand_pos, cand_score, cand_count, cand_cap);
 }
 
 // Waits on an mbarrier that nothing will ever complete, for at most limit_ns,
@@ -62,9 +48,7 @@ __global__ void k_debug_wait(DevStatus *st, uint64_t limit_ns) {
 }
 
 cudaError_t launch_debug_wait(DevStatus *st, uint64_t limit_ns, cudaStream_t s) {
-    k_debug_wait<<<1, 32, 0, s>>>(st, limit_ns);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_kernel(k_debug_wait, dim3(1), dim3(32), 0, s, st, limit_ns);
 }
 
 }  // namespace prism

@@ -33,24 +33,34 @@ thread_local uint64_t g_launches = 0;
 
 void prism::count_launches(int n) { g_launches += (uint64_t)n; }
 
+bool prism::use_pdl() {
+    static int v = -1;
+    if (v < 0) {
+        const char *e = std::getenv("PRISM_NO_PDL");
+        v = (e && e[0] == '1') ? 0 : 1;
+    }
+    return v == 1;
+}
+
 namespace {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-constexpr int kSlots = 3;           // selection slots: 0, 1 anchors (ring), 2 refined layers
-constexpr int kRefineSlot = 2;
+constexpr int kAnchorAhead = 2;     // anchors indexed ahead of the chain (ring of anchor slots)
+constexpr int kSlots = kAnchorAhead + 1;   // selection slots: the anchor ring, then refined layers
+constexpr int kRefineSlot = kAnchorAhead;
 
 // Buffers of one selection slot.
 struct SlotLayout {
-    size_t hist, ctl, S, tie, sel;
+    size_t hist, S, cpos, cspill;
 };
 
 struct Layout {
     size_t status;
-    size_t ctl_begin, ctl_end;      // [ctl_begin, ctl_end): histograms and counters, zeroed per call
+    size_t ctl_begin, ctl_end;      // [ctl_begin, ctl_end): histograms and counters; zeroed per call
     SlotLayout slot[kSlots];
     size_t attn_ctl;
-    size_t canon, idx_all, pacc, pml, total;
+    size_t canon, canon_off, idx_all, off_all, pacc, pml, total;
 };
 
 int n_layers_of(const prism_config_t &c) { return c.n_layers > 0 ? c.n_layers : 1; }
@@ -60,25 +70,27 @@ Layout make_layout(const prism_config_t &c) {
     const size_t G = (size_t)(c.n_q_heads / c.n_kv_heads);
     const size_t nsplit = ((size_t)c.kappa + kAttnChunk - 1) / kAttnChunk;
     const size_t sel_elems = rows * (size_t)c.kappa;
+    const size_t off_elems = rows * ((size_t)c.kappa + 1);
     Layout l{};
     size_t off = 0;
     l.status = off; off = align256(off + sizeof(DevStatus));
     l.ctl_begin = off;
     for (int s = 0; s < kSlots; ++s) {
-        l.slot[s].hist = off; off = align256(off + rows * kHistBins * sizeof(uint32_t));
-        l.slot[s].ctl = off;  off = align256(off + rows * sizeof(RowCtl));
+        l.slot[s].hist = off;   off = align256(off + rows * kHistBins * sizeof(uint32_t));
     }
     l.attn_ctl = off; off = align256(off + rows * sizeof(RowCtl));
     l.ctl_end = off;
     for (int s = 0; s < kSlots; ++s) {
-        l.slot[s].S = off;   off = align256(off + rows * (size_t)c.max_len * sizeof(float));
-        l.slot[s].tie = off; off = align256(off + rows * (size_t)c.max_len * sizeof(uint64_t));
-        l.slot[s].sel = off; off = align256(off + sel_elems * sizeof(int32_t));
+        l.slot[s].S = off;    off = align256(off + rows * (size_t)c.max_len * sizeof(float));
+        l.slot[s].cpos = off; off = align256(off + (s == kRefineSlot ? rows * (size_t)c.max_len : 1) * sizeof(int32_t));
+        l.slot[s].cspill = off; off = align256(off + rows * 2 * (size_t)c.max_len * sizeof(uint64_t));
     }
-    l.canon = off;   off = align256(off + sel_elems * sizeof(int32_t));
-    l.idx_all = off; off = align256(off + (size_t)n_layers_of(c) * sel_elems * sizeof(int32_t));
-    l.pacc = off;    off = align256(off + rows * nsplit * G * (size_t)c.head_dim * sizeof(float));
-    l.pml = off;     off = align256(off + rows * nsplit * G * 2 * sizeof(float));
+    l.canon = off;     off = align256(off + sel_elems * sizeof(int32_t));
+    l.canon_off = off; off = align256(off + off_elems * sizeof(int32_t));
+    l.idx_all = off;   off = align256(off + (size_t)n_layers_of(c) * sel_elems * sizeof(int32_t));
+    l.off_all = off;   off = align256(off + (size_t)n_layers_of(c) * off_elems * sizeof(int32_t));
+    l.pacc = off;      off = align256(off + rows * nsplit * G * (size_t)c.head_dim * sizeof(float));
+    l.pml = off;       off = align256(off + rows * nsplit * G * 2 * sizeof(float));
     l.total = off;
     return l;
 }
@@ -170,18 +182,17 @@ prism_status_t helpers_for_current_device(size_t n_events, DeviceHelpers **out) 
 
 struct Slot {
     uint32_t *hist;
-    RowCtl *ctl;
     float *S;
-    uint64_t *tie;
-    int32_t *sel;
+    int32_t *cpos;
+    uint64_t *cspill;
 };
 
 struct Ws {
     DevStatus *st;
     Slot slot[kSlots];
     RowCtl *attn_ctl;
-    int32_t *canon;
-    int32_t *idx_all;
+    int32_t *canon, *canon_off;
+    int32_t *idx_all, *off_all;
     float *pacc, *pml;
     uint8_t *base;
     Layout l;
@@ -196,14 +207,15 @@ prism_status_t carve(const prism_config_t &c, void *ws, size_t ws_bytes, Ws *w) 
     w->st = reinterpret_cast<DevStatus *>(b + w->l.status);
     for (int s = 0; s < kSlots; ++s) {
         w->slot[s].hist = reinterpret_cast<uint32_t *>(b + w->l.slot[s].hist);
-        w->slot[s].ctl = reinterpret_cast<RowCtl *>(b + w->l.slot[s].ctl);
         w->slot[s].S = reinterpret_cast<float *>(b + w->l.slot[s].S);
-        w->slot[s].tie = reinterpret_cast<uint64_t *>(b + w->l.slot[s].tie);
-        w->slot[s].sel = reinterpret_cast<int32_t *>(b + w->l.slot[s].sel);
+        w->slot[s].cpos = reinterpret_cast<int32_t *>(b + w->l.slot[s].cpos);
+        w->slot[s].cspill = reinterpret_cast<uint64_t *>(b + w->l.slot[s].cspill);
     }
     w->attn_ctl = reinterpret_cast<RowCtl *>(b + w->l.attn_ctl);
     w->canon = reinterpret_cast<int32_t *>(b + w->l.canon);
+    w->canon_off = reinterpret_cast<int32_t *>(b + w->l.canon_off);
     w->idx_all = reinterpret_cast<int32_t *>(b + w->l.idx_all);
+    w->off_all = reinterpret_cast<int32_t *>(b + w->l.off_all);
     w->pacc = reinterpret_cast<float *>(b + w->l.pacc);
     w->pml = reinterpret_cast<float *>(b + w->l.pml);
     return PRISM_OK;
@@ -228,19 +240,20 @@ ScoreArgs score_args(const prism_config_t &c, const Ws &w, const Slot &sl, const
     sa.q = q; sa.k = k; sa.len = len;
     sa.B = c.batch; sa.Hkv = c.n_kv_heads; sa.G = c.n_q_heads / c.n_kv_heads;
     sa.d = c.head_dim; sa.Lmax = c.max_len; sa.scale = eff_scale(c);
-    sa.S = sl.S; sa.hist = sl.hist; sa.src = nullptr; sa.kappa = c.kappa; sa.radius = c.radius;
-    sa.ctl = sl.ctl; sa.st = w.st; sa.wait_ns = wait_limit_ns();
+    sa.S = sl.S; sa.cpos = sl.cpos; sa.hist = sl.hist; sa.src = nullptr; sa.src_off = nullptr;
+    sa.kappa = c.kappa; sa.radius = c.radius; sa.st = w.st; sa.wait_ns = wait_limit_ns();
     return sa;
 }
 
 SelectArgs select_args(const prism_config_t &c, const Ws &w, const Slot &sl, const float *S,
-                       const int32_t *src, const int32_t *len, int32_t *idx_out) {
+                       const int32_t *cpos, const int32_t *src_off, const int32_t *len,
+                       int32_t *idx_out, int32_t *prop_off) {
     SelectArgs se{};
-    se.S = S; se.src = src; se.len = len;
+    se.S = S; se.cpos = cpos; se.src_off = src_off; se.len = len;
     se.B = c.batch; se.Hkv = c.n_kv_heads; se.Lmax = c.max_len; se.kappa = c.kappa;
     se.radius = c.radius;
-    se.hist = sl.hist; se.ctl = sl.ctl; se.sel = sl.sel; se.tie = sl.tie; se.idx_out = idx_out;
-    se.st = w.st;
+    se.hist = sl.hist; se.cspill = sl.cspill;
+    se.idx_out = idx_out; se.prop_off = prop_off; se.st = w.st; se.wait_ns = wait_limit_ns();
     return se;
 }
 
@@ -253,25 +266,28 @@ prism_status_t run_anchor_score(const prism_config_t &c, const Ws &w, int slot, 
     return cuda_status(launch_anchor_score(sa, num_sms(), s));
 }
 
-// Anchor top-kappa (Eq. (2)) from slot `slot`.
+// Anchor top-kappa (Eq. (2)) from slot `slot`; prop_off (nullable) receives
+// the offsets of the proposal around the selection.
 prism_status_t run_anchor_select(const prism_config_t &c, const Ws &w, int slot,
-                                 const int32_t *len, int32_t *idx_out, const float *scores,
+                                 const int32_t *len, int32_t *idx_out, int32_t *prop_off,
                                  cudaStream_t s) {
     const Slot &sl = w.slot[slot];
-    return cuda_status(launch_select(select_args(c, w, sl, scores ? scores : sl.S, nullptr, len,
-                                                 idx_out), s));
+    return cuda_status(launch_select(select_args(c, w, sl, sl.S, nullptr, nullptr, len, idx_out,
+                                                 prop_off), s));
 }
 
-// Refined layer: +-r proposal around the canonical source selection `src`,
-// Eq. (5) on it, Eq. (6).
+// Refined layer: +-r proposal around the canonical source selection `src`
+// (with its offsets `src_off`), Eq. (5) on it, Eq. (6).
 prism_status_t run_refine(const prism_config_t &c, const Ws &w, const void *q, const void *k,
-                          const int32_t *len, const int32_t *src, int32_t *idx_out,
-                          cudaStream_t s) {
+                          const int32_t *len, const int32_t *src, const int32_t *src_off,
+                          int32_t *idx_out, int32_t *prop_off, cudaStream_t s) {
     const Slot &sl = w.slot[kRefineSlot];
     ScoreArgs sa = score_args(c, w, sl, q, k, len);
     sa.src = src;
-    PRISM_CUDA(launch_refine_rescore(sa, s));
-    return cuda_status(launch_select(select_args(c, w, sl, sl.S, src, len, idx_out), s));
+    sa.src_off = src_off;
+    PRISM_CUDA(launch_refine_rescore(sa, num_sms(), s));
+    return cuda_status(launch_select(select_args(c, w, sl, sl.S, sl.cpos, src_off, len, idx_out,
+                                                 prop_off), s));
 }
 
 prism_status_t run_attn(const prism_config_t &c, const Ws &w, const void *q, const void *k,
@@ -299,6 +315,9 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     const uint16_t *qb = static_cast<const uint16_t *>(q);
     uint16_t *ob = static_cast<uint16_t *>(out);
     int32_t *idx_base = idx_out ? idx_out : w.idx_all;
+    const size_t off_elems = rows * ((size_t)c.kappa + 1);
+    // A layer's proposal offsets are needed when a later layer refines from it.
+    const bool refining = c.mode == PRISM_MODE_REFINE;
     auto is_anchor = [&](int l) { return c.mode == PRISM_MODE_DENSE_ANCHOR || c.anchor_mask[l] != 0; };
     std::vector<int> anchors;
     for (int l = 0; l < N; ++l)
@@ -306,17 +325,18 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     const int NA = (int)anchors.size();
 
     cudaStream_t sA = hp ? hp->anchor : s0, sM = hp ? hp->chain : s0, sC = hp ? hp->attn : s0;
-    // Events: fork, two joins, per anchor "scored" and "slot free", per layer "selected".
+    // Events: fork, two joins, per anchor "indexed" and "reached by the chain",
+    // per layer "selected".
     cudaEvent_t ev_fork = nullptr, ev_join_m = nullptr, ev_join_c = nullptr;
-    const cudaEvent_t *ev_scored = nullptr, *ev_free = nullptr, *ev_sel = nullptr;
+    const cudaEvent_t *ev_indexed = nullptr, *ev_reached = nullptr, *ev_sel = nullptr;
     if (hp) {
         const cudaEvent_t *e = hp->events.data();
         ev_fork = e[0];
         ev_join_m = e[1];
         ev_join_c = e[2];
-        ev_scored = e + 3;
-        ev_free = ev_scored + NA;
-        ev_sel = ev_free + NA;
+        ev_indexed = e + 3;
+        ev_reached = ev_indexed + NA;
+        ev_sel = ev_reached + NA;
     }
 
     PRISM_TRY(zero_control(w, s0));
@@ -326,37 +346,45 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         PRISM_CUDA(cudaStreamWaitEvent(sM, ev_fork, 0));
         PRISM_CUDA(cudaStreamWaitEvent(sC, ev_fork, 0));
     }
-    auto score_anchor = [&](int g) -> prism_status_t {
+    // An anchor's scoring and selection depend on nothing but its own q and K,
+    // so both run on the anchor stream, kAnchorAhead anchors ahead of the
+    // chain of refined layers (the anchor slots form a ring of that size).
+    auto index_anchor = [&](int g) -> prism_status_t {
         const int l = anchors[g];
-        if (hp && g >= 2) PRISM_CUDA(cudaStreamWaitEvent(sA, ev_free[g - 2], 0));
-        PRISM_TRY(run_anchor_score(c, w, g % 2, qb + (size_t)l * q_elems, k[l], len, nullptr, sA));
-        if (hp) PRISM_CUDA(cudaEventRecord(ev_scored[g], sA));
+        const bool next_refines = refining && l + 1 < N && !is_anchor(l + 1);
+        if (hp && g >= kAnchorAhead) PRISM_CUDA(cudaStreamWaitEvent(sA, ev_reached[g - kAnchorAhead], 0));
+        PRISM_TRY(run_anchor_score(c, w, g % kAnchorAhead, qb + (size_t)l * q_elems, k[l], len,
+                                   nullptr, sA));
+        PRISM_TRY(run_anchor_select(c, w, g % kAnchorAhead, len, idx_base + (size_t)l * sel_elems,
+                                    next_refines ? w.off_all + (size_t)l * off_elems : nullptr,
+                                    sA));
+        if (hp) PRISM_CUDA(cudaEventRecord(ev_indexed[g], sA));
         return PRISM_OK;
     };
-    // The anchor stream starts up to two anchors ahead.
     if (hp) {
-        for (int g = 0; g < NA && g < 2; ++g) PRISM_TRY(score_anchor(g));
+        for (int g = 0; g < NA && g < kAnchorAhead; ++g) PRISM_TRY(index_anchor(g));
     }
 
-    const int32_t *anchor_sel = nullptr;
-    const int32_t *prev_sel = nullptr;
+    const int32_t *anchor_sel = nullptr, *anchor_off = nullptr;
+    const int32_t *prev_sel = nullptr, *prev_off = nullptr;
     int g = 0;
     for (int l = 0; l < N; ++l) {
         const void *ql = qb + (size_t)l * q_elems;
         const int32_t *src = c.chain == PRISM_CHAIN_ANCHOR ? anchor_sel : prev_sel;
+        const int32_t *src_off = c.chain == PRISM_CHAIN_ANCHOR ? anchor_off : prev_off;
         int32_t *dst = idx_base + (size_t)l * sel_elems;
-        const int32_t *cur = dst;
+        int32_t *dst_off = w.off_all + (size_t)l * off_elems;
+        const bool next_refines = refining && l + 1 < N && !is_anchor(l + 1);
+        const int32_t *cur = dst, *cur_off = dst_off;
         if (is_anchor(l)) {
             if (hp) {
-                PRISM_CUDA(cudaStreamWaitEvent(sM, ev_scored[g], 0));
+                PRISM_CUDA(cudaStreamWaitEvent(sM, ev_indexed[g], 0));
+                PRISM_CUDA(cudaEventRecord(ev_reached[g], sM));
+                if (g + kAnchorAhead < NA) PRISM_TRY(index_anchor(g + kAnchorAhead));
             } else {
-                PRISM_TRY(score_anchor(g));
+                PRISM_TRY(index_anchor(g));
             }
-            PRISM_TRY(run_anchor_select(c, w, g % 2, len, dst, nullptr, sM));
-            if (hp) {
-                PRISM_CUDA(cudaEventRecord(ev_free[g], sM));
-                if (g + 2 < NA) PRISM_TRY(score_anchor(g + 2));
-            }
+            anchor_off = dst_off;
             anchor_sel = dst;
             ++g;
         } else if (c.mode == PRISM_MODE_STATIC_REUSE) {
@@ -366,8 +394,11 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
             } else {
                 cur = src;
             }
+            cur_off = nullptr;
         } else {
-            PRISM_TRY(run_refine(c, w, ql, k[l], len, src, dst, sM));
+            const bool need_off = c.chain == PRISM_CHAIN_PREV && next_refines;
+            PRISM_TRY(run_refine(c, w, ql, k[l], len, src, src_off, dst, need_off ? dst_off : nullptr,
+                                 sM));
         }
         if (hp) {
             PRISM_CUDA(cudaEventRecord(ev_sel[l], sM));
@@ -376,6 +407,7 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         PRISM_TRY(run_attn(c, w, ql, k[l], v[l], len, cur, c.kappa, c.kappa,
                            ob + (size_t)l * q_elems, sC));
         prev_sel = cur;
+        prev_off = cur_off;
     }
     if (hp) {
         // Every anchor score was waited on by M; join M and C into the caller's stream.
@@ -410,8 +442,15 @@ prism_status_t prism_index_anchor(const prism_config_t *cfg, const void *q, cons
     PRISM_TRY(carve(*cfg, ws, ws_bytes, &w));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     PRISM_TRY(zero_control(w, s));
-    PRISM_TRY(run_anchor_score(*cfg, w, 0, q, k, len, scores_out, s));
-    return run_anchor_select(*cfg, w, 0, len, idx_out, scores_out, s);
+    PRISM_TRY(run_anchor_score(*cfg, w, 0, q, k, len, nullptr, s));
+    PRISM_TRY(run_anchor_select(*cfg, w, 0, len, idx_out, nullptr, s));
+    if (scores_out) {
+        // The selection reads the workspace copy (its staged copies may round
+        // a row's end up to 16 bytes); the caller gets the scores afterwards.
+        const size_t bytes = (size_t)cfg->batch * cfg->n_kv_heads * cfg->max_len * sizeof(float);
+        PRISM_CUDA(cudaMemcpyAsync(scores_out, w.slot[0].S, bytes, cudaMemcpyDeviceToDevice, s));
+    }
+    return PRISM_OK;
 }
 
 prism_status_t prism_score_anchor(const prism_config_t *cfg, const void *q, const void *k,
@@ -447,14 +486,15 @@ prism_status_t prism_index_refine(const prism_config_t *cfg, const void *q, cons
     PRISM_TRY(zero_control(w, s));
     CanonArgs ca{};
     ca.idx = idx_prev; ca.len = len; ca.B = cfg->batch; ca.Hkv = cfg->n_kv_heads;
-    ca.Lmax = cfg->max_len; ca.kappa = cfg->kappa; ca.out = w.canon; ca.st = w.st;
+    ca.Lmax = cfg->max_len; ca.kappa = cfg->kappa; ca.radius = cfg->radius;
+    ca.out = w.canon; ca.out_off = w.canon_off; ca.st = w.st;
     PRISM_CUDA(launch_canonicalize(ca, s));
-    PRISM_TRY(run_refine(*cfg, w, q, k, len, w.canon, idx_out, s));
+    PRISM_TRY(run_refine(*cfg, w, q, k, len, w.canon, w.canon_off, idx_out, nullptr, s));
     if (all)
-        PRISM_CUDA(launch_export_candidates(w.slot[kRefineSlot].S, w.canon, nullptr, len,
-                                            cfg->batch, cfg->n_kv_heads, cfg->max_len,
-                                            cfg->kappa, cfg->radius, cand_pos, cand_score,
-                                            cand_count, cand_cap, w.st, s));
+        PRISM_CUDA(launch_export_candidates(w.slot[kRefineSlot].S, w.slot[kRefineSlot].cpos,
+                                            w.canon_off, cfg->batch * cfg->n_kv_heads,
+                                            cfg->max_len, cfg->kappa, cand_pos, cand_score,
+                                            cand_count, cand_cap, s));
     return PRISM_OK;
 }
 

@@ -36,15 +36,11 @@ enum : uint32_t {
     kWhereDebugWait = 7,
 };
 
-// Per (batch, KV head) row counters; zeroed at the start of every public call
-// that uses them and left zeroed by the kernels that consume them.
+// Per (batch, KV head) row counter of the attention kernel's split-K merge;
+// zeroed at the start of every public call that uses it and left zeroed.
 struct RowCtl {
-    int32_t n_sel;         // items strictly above the threshold digit (select)
-    int32_t n_tie;         // items on the threshold digit (select)
-    int32_t n_prop;        // |P| of the refine proposal (rescore)
-    uint32_t done_select;  // select CTAs of this row that have finished
     uint32_t done_attn;    // attention CTAs of this row that have finished
-    int32_t pad[3];
+    uint32_t pad[7];
 };
 
 __device__ __forceinline__ void report(DevStatus *st, uint32_t code, uint32_t where,
@@ -94,6 +90,14 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+// Programmatic dependent launch: wait for the preceding kernel of the stream
+// (and the visibility of its writes); let the next kernel start its prologue.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Transposing butterfly reduction.  Each lane of an NL-lane group holds NV
@@ -156,7 +160,7 @@ __device__ __forceinline__ int owned_range(const int32_t *src, int j, long long 
     if (i < 0) return 0;
     const int prev = j > 0 ? src[j - 1] : -1;
     if (i >= L || (prev >= 0 && i <= prev)) {
-        report(st, kDevErrBadIndex, where, (uint32_t)i);
+        if (st) report(st, kDevErrBadIndex, where, (uint32_t)i);
         return 0;
     }
     long long lo = (long long)i - r;
@@ -343,9 +347,58 @@ __device__ __forceinline__ int slice_position(const int *lo_s, const int *off_s,
     return lo_s[a] + (e - off_s[a]);
 }
 
+// Enumeration offsets of the proposal around a canonical selection sel[0..kappa):
+// off[j] = number of proposal positions owned by entries before j, off[kappa]
+// = |P|.  Whole-CTA cooperative; sel may have been written by this CTA
+// (call after a barrier).  Contains __syncthreads().
+__device__ __forceinline__ void proposal_offsets(const int32_t *sel, int kappa, int radius, int L,
+                                                 int32_t *off, int *scratch, DevStatus *st) {
+    const int NT = blockDim.x, tid = threadIdx.x;
+    const int per = (kappa + NT - 1) / NT;
+    const int j0 = min(kappa, tid * per), j1 = min(kappa, j0 + per);
+    int cnt = 0;
+    for (int j = j0; j < j1; ++j) {
+        int lo;
+        cnt += owned_range(sel, j, radius, L, &lo, st, kWhereFinalize);
+    }
+    int total;
+    int run = block_exclusive_scan(cnt, scratch, &total);
+    for (int j = j0; j < j1; ++j) {
+        off[j] = run;
+        int lo;
+        run += owned_range(sel, j, radius, L, &lo, nullptr, 0);
+    }
+    if (tid == 0) off[kappa] = total;
+}
+
 // ---- launch interfaces (host side, defined in the .cu files) -------------
 // Kernels launched by the calling host thread (see prism_launch_count()).
 void count_launches(int n);
+
+// Whether kernels are launched with programmatic dependent launch (on unless
+// the environment sets PRISM_NO_PDL=1).
+bool use_pdl();
+
+// Launch with the programmatic-stream-serialization attribute, so that the
+// kernel may begin while its predecessor in the stream finishes (the kernel
+// calls pdl_wait() before it touches the predecessor's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = use_pdl() ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+    count_launches(1);
+    return e;
+}
 
 struct ScoreArgs {
     const void *q;          // bf16 [B][Hq][d]
@@ -353,38 +406,42 @@ struct ScoreArgs {
     const int32_t *len;     // [B]
     int B, Hkv, G, d, Lmax;
     float scale;
-    float *S;               // fp32 [rows][Lmax], indexed by position
+    float *S;               // fp32 [rows][Lmax]: anchor scores by position; refine
+                            // candidate scores in enumeration (= ascending position) order
+    int32_t *cpos;          // refine: [rows][Lmax] candidate positions
     uint32_t *hist;         // [rows][kHistBins]
     const int32_t *src;     // refine: canonical source selection [rows][kappa]
+    const int32_t *src_off; // refine: its proposal enumeration offsets [rows][kappa + 1]
     int kappa, radius;      // refine
-    RowCtl *ctl;            // [rows]
     DevStatus *st;
     uint64_t wait_ns;
 };
 
 cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s);
-cudaError_t launch_refine_rescore(const ScoreArgs &a, cudaStream_t s);
+cudaError_t launch_refine_rescore(const ScoreArgs &a, int num_sms, cudaStream_t s);
 
 struct CanonArgs {
     const int32_t *idx;        // [rows][kappa], any order, duplicates, -1 padding
     const int32_t *len;
-    int B, Hkv, Lmax, kappa;
+    int B, Hkv, Lmax, kappa, radius;
     int32_t *out;              // [rows][kappa] canonical: ascending, distinct, -1 padded
+    int32_t *out_off;          // [rows][kappa + 1] its proposal enumeration offsets
     DevStatus *st;
 };
 cudaError_t launch_canonicalize(const CanonArgs &a, cudaStream_t s);
 
 struct SelectArgs {
-    const float *S;            // [rows][Lmax] scores indexed by position
-    const int32_t *src;        // refine: canonical source selection; nullptr for the anchor
+    const float *S;            // anchor: [rows][Lmax] scores by position; refine: candidate scores
+    const int32_t *cpos;       // refine: [rows][Lmax] candidate positions; nullptr for the anchor
+    const int32_t *src_off;    // refine: [rows][kappa + 1]; src_off[kappa] = number of candidates
     const int32_t *len;
     int B, Hkv, Lmax, kappa, radius;
-    uint32_t *hist;            // [rows][kHistBins]
-    RowCtl *ctl;
-    int32_t *sel;              // [rows][kappa] positions above the threshold digit
-    uint64_t *tie;             // [rows][Lmax] (key << 32 | position) on the threshold digit
+    uint32_t *hist;            // [rows][kHistBins], left zeroed
+    uint64_t *cspill;          // [rows][2][Lmax] overflow of the CTAs' candidate and tie lists
     int32_t *idx_out;          // [rows][kappa]
+    int32_t *prop_off;         // nullable: [rows][kappa + 1] offsets of the next proposal
     DevStatus *st;
+    uint64_t wait_ns;          // bound on the wait for the slice copies
 };
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
 
@@ -405,11 +462,10 @@ struct AttnArgs {
 constexpr int kAttnChunk = 64;
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s);
 
-cudaError_t launch_export_candidates(const float *S, const int32_t *src, const RowCtl *ctl,
-                                     const int32_t *len, int B, int Hkv, int Lmax, int kappa,
-                                     int radius, int32_t *cand_pos, float *cand_score,
-                                     int32_t *cand_count, int cand_cap, DevStatus *st,
-                                     cudaStream_t s);
+cudaError_t launch_export_candidates(const float *cscore, const int32_t *cpos,
+                                     const int32_t *src_off, int rows, int Lmax, int kappa,
+                                     int32_t *cand_pos, float *cand_score, int32_t *cand_count,
+                                     int cand_cap, cudaStream_t s);
 
 cudaError_t launch_debug_wait(DevStatus *st, uint64_t limit_ns, cudaStream_t s);
 

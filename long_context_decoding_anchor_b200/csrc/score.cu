@@ -9,7 +9,7 @@
 // k_anchor_score streams the whole key cache of the anchor layer: a
 // persistent grid (one CTA per SM) walks a contiguous range of 128-token
 // tiles; one producer thread moves each tile (contiguous in memory) into a
-// 4-stage shared-memory ring with a 1-D bulk copy (TMA, cp.async.bulk) that
+// 3-stage shared-memory ring with a 1-D bulk copy (TMA, cp.async.bulk) that
 // completes on an mbarrier, and eight consumer warps form the dot products
 // from shared memory.  Scores go to global memory (they stay L2-resident for
 // the selection) and their top 11 key bits into a per-row histogram, the
@@ -17,7 +17,9 @@
 //
 // k_refine_rescore scores only the proposal positions of a refined layer
 // (Eq. (5)), enumerated from the owned ranges of the source selection; each
-// owned range is one bulk copy, and scores are stored by position.
+// owned range (or its piece of a 128-slot window) is one bulk copy into the
+// same kind of ring, and the (score, position) candidates are stored
+// contiguously at their enumeration index.
 #include "prism_internal.cuh"
 
 namespace prism {
@@ -25,7 +27,7 @@ namespace prism {
 template <int D>
 struct AnchorCfg {
     static constexpr int kTileRows = 128;
-    static constexpr int kStages = 4;
+    static constexpr int kStages = 3;
     static constexpr int kConsumerWarps = 8;
     static constexpr int kThreads = 32 * (kConsumerWarps + 1);
     static constexpr int kNL = D / 8;                     // lanes per key row (16 B each)
@@ -122,6 +124,7 @@ k_anchor_score(ScoreArgs a) {
     int *scratch = reinterpret_cast<int *>(hist_s + kHistBins);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_launch_dependents();
 
     for (int i = tid; i < kHistBins; i += blockDim.x) hist_s[i] = 0;
     if (tid == 0) {
@@ -143,12 +146,19 @@ k_anchor_score(ScoreArgs a) {
     }
     const long long t_begin = total * blockIdx.x / gridDim.x;
     const long long t_end = total * (blockIdx.x + 1) / gridDim.x;
-    if (t_begin >= t_end) return;
+    if (t_begin >= t_end) {
+        pdl_wait();
+        return;
+    }
     {
         long long tot2;
         locate_tile<TILE>(a.len, a.B, a.Hkv, a.Lmax, t_begin, &cur0, &tot2, scratch, a.st);
     }
     const int ntiles = (int)(t_end - t_begin);
+    if (ntiles <= 0) {
+        pdl_wait();
+        return;
+    }
 
     if (warp == C::kConsumerWarps) {
         // ---------------- producer: one thread issues the bulk copies -------------
@@ -190,6 +200,9 @@ k_anchor_score(ScoreArgs a) {
     }
 
     // ---------------- consumers ------------------------------------------------
+    // The key cache is an input: the producer streams it at once.  Scores and
+    // the histogram are written only after the preceding kernel has finished.
+    pdl_wait();
     const int slice = lane % C::kNL;            // which 8 elements of a key row
     const int sub = lane / C::kNL;              // which row of an instruction's rows
     const int row0 = warp * C::kRowsPerWarp;
@@ -268,73 +281,185 @@ k_anchor_score(ScoreArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Refined layer: score only the proposal positions (Eq. (5)).  One CTA per 16
-// entries of the (canonical) source selection.  Each entry owns a contiguous
-// run of key rows, so the gather is one 1-D bulk copy (TMA) per run, issued by
-// 16 lanes of warp 0 into a shared-memory buffer that completes on an
-// mbarrier; nothing is held in registers while the copies fly.  The eight
-// warps then form 32 dot products per round each from shared memory, and the
-// transposing reduction leaves one score per lane, stored by position.
+// Refined layer: score only the proposal positions (Eq. (5)).  The proposal
+// of a row is enumerated slot by slot from the owned ranges of the canonical
+// source selection (the offsets src_off give each entry's first slot), so a
+// row's n slots split evenly into P contiguous parts, one CTA each.  A CTA
+// walks its part in windows of 128 slots: the producer warp finds the
+// entries overlapping a window (one coalesced load of 32 entries at a time)
+// and moves each entry's piece of the window -- consecutive key rows -- with
+// one 1-D bulk copy (TMA) into a 3-stage shared-memory ring, noting every
+// slot's position; eight consumer warps form the dot products.  Candidates
+// (score, position) are stored at their slot index.
 template <int D>
 struct RescoreCfg {
-    static constexpr int kEntries = 16;
-    static constexpr int kWarps = 8;
-    static constexpr int kThreads = 32 * kWarps;
+    static constexpr int kTileRows = 128;
+    static constexpr int kStages = 3;
+    static constexpr int kConsumerWarps = 8;
+    static constexpr int kThreads = 32 * (kConsumerWarps + 1);
     static constexpr int kNL = D / 8;
     static constexpr int kRPI = 32 / kNL;
-    static constexpr int kRowsPerWarp = 32;
-    static constexpr int kSteps = kRowsPerWarp / kRPI;       // == kNL
+    static constexpr int kRowsPerWarp = kTileRows / kConsumerWarps;   // 16
+    static constexpr int kSteps = kRowsPerWarp / kRPI;
     static constexpr int kRowBytes = D * 2;
-    static constexpr int kCapRows = 48 * 1024 / kRowBytes;    // rows staged per round
-    static constexpr int kSmemBytes = kCapRows * kRowBytes;
-    static_assert(kSteps == kNL, "one score per lane after the reduction");
+    static constexpr int kTileBytes = kTileRows * kRowBytes;
+    static constexpr int kPosOff = kStages * kTileBytes;
+    static constexpr int kBarOff = kPosOff + kStages * kTileRows * 4;
+    static constexpr int kHistOff = kBarOff + 2 * kStages * 8;
+    static constexpr int kSmemBytes = kHistOff + kHistBins * 4;
 };
 
+// One entry of the source selection as the producer lane sees it: its slots
+// [o0, o1) of the enumeration and the first key row `lo` of its owned range.
+// The raw loads are issued one batch ahead of their use.
+struct EntryRaw {
+    int o0, o1, i, prev;
+};
+struct EntryRun {
+    int o0, o1, lo;
+};
+
+__device__ __forceinline__ EntryRaw load_entry_raw(const int32_t *src, const int32_t *off,
+                                                   int kappa, int jj) {
+    EntryRaw w{-1, -1, -1, -1};
+    if (jj < kappa) {
+        w.o0 = __ldcg(off + jj);
+        w.o1 = __ldcg(off + jj + 1);
+        w.i = __ldcg(src + jj);
+        w.prev = jj > 0 ? __ldcg(src + jj - 1) : -1;
+    }
+    return w;
+}
+
+__device__ __forceinline__ EntryRun make_entry(const EntryRaw &w, int jj, int kappa, int n,
+                                               long long r, int L, DevStatus *st) {
+    EntryRun e{n, n, 0};
+    if (jj >= kappa) return e;
+    e.o0 = min(w.o0, n);
+    e.o1 = min(w.o1, n);
+    long long lo = (long long)w.i - r;
+    if (w.prev >= 0 && (long long)w.prev + r + 1 > lo) lo = (long long)w.prev + r + 1;
+    if (lo < 0) lo = 0;
+    long long hi = (long long)w.i + r;
+    if (hi > L - 1) hi = L - 1;
+    const int own = (w.i < 0 || hi < lo) ? 0 : (int)(hi - lo + 1);
+    if (e.o1 - e.o0 != own && e.o1 > e.o0) {
+        report(st, kDevErrInternal, kWhereRescore, (uint32_t)jj);   // offsets disagree
+        lo = 0;
+    }
+    e.lo = (int)lo;
+    return e;
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 template <int D>
-__global__ void __launch_bounds__(RescoreCfg<D>::kThreads)
+__global__ void __launch_bounds__(RescoreCfg<D>::kThreads, 1)
 k_refine_rescore(ScoreArgs a) {
     using C = RescoreCfg<D>;
-    extern __shared__ __align__(128) uint8_t rows_s[];
-    __shared__ uint64_t bar;
-    __shared__ uint32_t hist_s[kHistBins];
-    __shared__ int lo_s[C::kEntries], cnt_s[C::kEntries], off_s[C::kEntries + 1];
-    __shared__ int pos_s[C::kCapRows];
-    __shared__ int fail_s;
-    const int row = blockIdx.y;
-    const int j0 = blockIdx.x * C::kEntries;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *stages = smem;
+    int *pos_s = reinterpret_cast<int *>(smem + C::kPosOff);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *empty = full + C::kStages;
+    uint32_t *hist_s = reinterpret_cast<uint32_t *>(smem + C::kHistOff);
+    const int row = blockIdx.y, part = blockIdx.x, P = gridDim.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = row / a.Hkv, h = row % a.Hkv;
     const int L = load_len(a.len, b, a.Lmax, a.st, kWhereRescore);
-    const int32_t *src = a.src + (size_t)row * a.kappa;
-
-    if (warp == 0) {
-        int lo = 0, cnt = 0;
-        if (lane < C::kEntries && j0 + lane < a.kappa)
-            cnt = owned_range(src, j0 + lane, a.radius, L, &lo, a.st, kWhereRescore);
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (lane < C::kEntries) {
-            lo_s[lane] = lo;
-            cnt_s[lane] = cnt;
-            off_s[lane] = incl - cnt;
-        }
-        if (lane == C::kEntries - 1) off_s[C::kEntries] = incl;
-        if (lane == 0) {
-            fail_s = 0;
-            mbar_init(&bar, 1);
-            fence_mbar_init();
-        }
-    }
     for (int i = tid; i < kHistBins; i += C::kThreads) hist_s[i] = 0;
+    if (tid == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], C::kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
     __syncthreads();
-    const int total = off_s[C::kEntries];
-    if (total == 0) return;
-    if (tid == 0) atomicAdd(&a.ctl[row].n_prop, total);
+    // The source selection and its offsets come from the preceding kernels.
+    pdl_wait();
+    const int32_t *off = a.src_off + (size_t)row * (a.kappa + 1);
+    const int n = min(min(__ldcg(off + a.kappa), L), a.Lmax);
+    const int s_begin = (int)((long long)part * n / P);
+    const int s_end = (int)((long long)(part + 1) * n / P);
+    if (s_begin >= s_end) {
+        pdl_launch_dependents();
+        return;
+    }
 
+    if (warp == C::kConsumerWarps) {
+        // ---------------- producer warp ----------------------------------------
+        const int32_t *src = a.src + (size_t)row * a.kappa;
+        const uint16_t *kb = static_cast<const uint16_t *>(a.k) + (size_t)row * a.Lmax * D;
+        const uint64_t pol = l2_evict_first_policy();
+        // First entry to look at: the last one starting at or before s_begin,
+        // by a 64-way search over the offsets (off[0] = 0 <= s_begin).
+        int lo = 0, hi = a.kappa;
+        while (hi - lo > 32) {
+            const int st = (hi - lo + 63) / 64;
+            const int x0 = lo + 2 * lane * st, x1 = x0 + st;
+            const bool p0 = x0 < hi && __ldcg(off + x0) <= s_begin;
+            const bool p1 = x1 < hi && __ldcg(off + x1) <= s_begin;
+            const unsigned m0 = __ballot_sync(0xffffffffu, p0), m1 = __ballot_sync(0xffffffffu, p1);
+            const int k0 = m0 ? 2 * (31 - __clz(m0)) : 0;
+            const int k1 = m1 ? 2 * (31 - __clz(m1)) + 1 : 0;
+            lo += max(k0, k1) * st;
+            hi = min(hi, lo + st);
+        }
+        int jb = lo;
+        EntryRun e = make_entry(load_entry_raw(src, off, a.kappa, jb + lane), jb + lane, a.kappa, n,
+                                a.radius, L, a.st);
+        EntryRaw next = load_entry_raw(src, off, a.kappa, jb + 32 + lane);
+        bool failed = false;
+        int issued = 0;
+        for (int it = 0, w0 = s_begin; w0 < s_end; ++it, w0 += C::kTileRows) {
+            const int s = it % C::kStages;
+            const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+            if (!mbar_wait(&empty[s], ph ^ 1u, a.wait_ns)) {
+                if (lane == 0) report(a.st, kDevErrTimeout, kWhereRescore, (uint32_t)it);
+                failed = true;
+                break;
+            }
+            const int wend = min(w0 + C::kTileRows, s_end);
+            if (lane == 0) mbar_expect_tx(&full[s], (uint32_t)(wend - w0) * C::kRowBytes);
+            __syncwarp();
+            uint8_t *tile = stages + s * C::kTileBytes;
+            int *pos = pos_s + s * C::kTileRows;
+            for (;;) {
+                const int g0 = max(e.o0, w0), g1 = min(e.o1, wend);
+                if (g0 < g1) {
+                    // keep the copy inside this row of the key cache whatever the offsets say
+                    const int r0 = min(e.lo + (g0 - e.o0), a.Lmax - (g1 - g0));
+                    bulk_load(tile + (size_t)(g0 - w0) * C::kRowBytes, kb + (size_t)r0 * D,
+                              (uint32_t)(g1 - g0) * C::kRowBytes, &full[s], pol);
+                    for (int t = g0; t < g1; ++t) pos[t - w0] = r0 + (t - g0);
+                }
+                const int reach = __shfl_sync(0xffffffffu, e.o1, 31);
+                if (reach >= wend || jb + 32 >= a.kappa) break;
+                jb += 32;
+                e = make_entry(next, jb + lane, a.kappa, n, a.radius, L, a.st);
+                next = load_entry_raw(src, off, a.kappa, jb + 32 + lane);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[s]);
+            issued = it + 1;
+        }
+        // Every issued copy must land before the CTA may exit.
+        if (failed) {
+            for (int it = max(0, issued - C::kStages); it < issued; ++it) {
+                const int s = it % C::kStages;
+                if (!mbar_wait(&full[s], (uint32_t)(it / C::kStages) & 1u, a.wait_ns) && lane == 0)
+                    report(a.st, kDevErrTimeout, kWhereRescore, 0x80000000u | (uint32_t)it);
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumers ------------------------------------------------
     const int slice = lane % C::kNL, sub = lane / C::kNL;
     float qreg[8];
 #pragma unroll
@@ -349,70 +474,41 @@ k_refine_rescore(ScoreArgs a) {
         qreg[4] += bf16_lo(w.z); qreg[5] += bf16_hi(w.z);
         qreg[6] += bf16_lo(w.w); qreg[7] += bf16_hi(w.w);
     }
-    const uint16_t *kb = static_cast<const uint16_t *>(a.k) + (size_t)row * a.Lmax * D;
     float *S = a.S + (size_t)row * a.Lmax;
-
-    int round = 0;
-    bool pending = false;      // warp 0 lane 0: a round's copies may still be in flight
-    for (int e0 = 0; e0 < total; e0 += C::kCapRows, ++round) {
-        const int nr = min(C::kCapRows, total - e0);
-        for (int i = tid; i < nr; i += C::kThreads) {
-            int t = 0;                                  // entry owning index e0 + i
+    int32_t *cpos = a.cpos + (size_t)row * a.Lmax;
+    const int r_base = warp * C::kRowsPerWarp;
+    const int r_item = r_base + transpose_item<C::kSteps, C::kNL>(lane) * C::kRPI + sub;
+    const bool writer = transpose_writer<C::kSteps, C::kNL>(lane);
+    for (int it = 0, w0 = s_begin; w0 < s_end; ++it, w0 += C::kTileRows) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
+        if (!mbar_wait(&full[s], ph, a.wait_ns)) {
+            if (lane == 0) report(a.st, kDevErrTimeout, kWhereRescore, 0x40000000u | (uint32_t)it);
+            break;
+        }
+        const uint8_t *tile = stages + s * C::kTileBytes;
+        float part_[C::kSteps];
 #pragma unroll
-            for (int m = 8; m >= 1; m >>= 1)
-                if (t + m < C::kEntries && off_s[t + m] <= e0 + i) t += m;
-            pos_s[i] = lo_s[t] + (e0 + i - off_s[t]);
+        for (int st = 0; st < C::kSteps; ++st) {
+            const int r = r_base + st * C::kRPI + sub;
+            const uint4 kv = *reinterpret_cast<const uint4 *>(tile + r * C::kRowBytes + slice * 16);
+            part_[st] = dot8(kv, qreg);
         }
-        if (warp == 0) {
-            if (lane == 0) mbar_arrive_expect_tx(&bar, (uint32_t)nr * C::kRowBytes);
-            __syncwarp();
-            if (lane < C::kEntries) {
-                const int s0 = max(off_s[lane], e0);
-                const int s1 = min(off_s[lane] + cnt_s[lane], e0 + nr);
-                if (s0 < s1) {
-                    const uint64_t pol = l2_evict_first_policy();
-                    bulk_load(rows_s + (size_t)(s0 - e0) * C::kRowBytes,
-                              kb + (size_t)(lo_s[lane] + s0 - off_s[lane]) * D,
-                              (uint32_t)(s1 - s0) * C::kRowBytes, &bar, pol);
-                }
-            }
-            pending = true;
+        const int p_item = pos_s[s * C::kTileRows + r_item];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        transpose_reduce<C::kSteps, C::kNL>(part_, lane);
+        const int nrows = min(C::kTileRows, s_end - w0);
+        if (writer && r_item < nrows) {
+            const float sc = part_[0] * a.scale;
+            S[w0 + r_item] = sc;
+            cpos[w0 + r_item] = p_item;
+            atomicAdd(&hist_s[score_key(sc) >> (32 - kHistBits)], 1u);
         }
-        __syncthreads();                                 // pos_s ready
-        const bool ok = mbar_wait(&bar, (uint32_t)round & 1u, a.wait_ns);
-        if (!ok) {
-            report(a.st, kDevErrTimeout, kWhereRescore, (uint32_t)round);
-            fail_s = 1;
-        } else {
-            if (warp == 0) pending = false;
-            for (int r0 = warp * C::kRowsPerWarp; r0 < nr; r0 += C::kWarps * C::kRowsPerWarp) {
-                float part[C::kSteps];
-#pragma unroll
-                for (int st = 0; st < C::kSteps; ++st) {
-                    const int r = r0 + st * C::kRPI + sub;
-                    const uint4 kv = *reinterpret_cast<const uint4 *>(
-                        rows_s + (size_t)r * C::kRowBytes + slice * 16);
-                    part[st] = dot8(kv, qreg);
-                }
-                transpose_reduce<C::kSteps, C::kNL>(part, lane);
-                const int r = r0 + transpose_item<C::kSteps, C::kNL>(lane) * C::kRPI + sub;
-                if (r < nr) {
-                    const float sc = part[0] * a.scale;
-                    S[pos_s[r]] = sc;
-                    atomicAdd(&hist_s[score_key(sc) >> (32 - kHistBits)], 1u);
-                }
-            }
-        }
-        __syncthreads();                                 // buffer and pos_s free again
-        if (fail_s) break;
     }
-    if (fail_s) {
-        // Let any copy still in flight land before the CTA's shared memory goes.
-        if (tid == 0 && pending && !mbar_wait(&bar, (uint32_t)round & 1u, a.wait_ns))
-            report(a.st, kDevErrTimeout, kWhereRescore, 0x80000000u | (uint32_t)round);
-        return;
-    }
-    for (int i = tid; i < kHistBins; i += C::kThreads) {
+    consumer_sync();
+    pdl_launch_dependents();
+    for (int i = tid; i < kHistBins; i += 32 * C::kConsumerWarps) {
         const uint32_t v = hist_s[i];
         if (v) atomicAdd(a.hist + (size_t)row * kHistBins + i, v);
     }
@@ -428,9 +524,7 @@ static cudaError_t launch_anchor_score_d(const ScoreArgs &a, int num_sms, cudaSt
     const long long rows = (long long)a.B * a.Hkv;
     const long long max_tiles = rows * ((a.Lmax + C::kTileRows - 1) / C::kTileRows);
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
-    k_anchor_score<D><<<grid, C::kThreads, C::kSmemBytes, s>>>(a);
-    count_launches(1);
-    return cudaGetLastError();
+    return launch_kernel(k_anchor_score<D>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, s, a);
 }
 
 cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s) {
@@ -439,19 +533,21 @@ cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s)
 }
 
 template <int D>
-static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, cudaStream_t s) {
+static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, int num_sms, cudaStream_t s) {
     using C = RescoreCfg<D>;
     cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((a.kappa + C::kEntries - 1) / C::kEntries), (unsigned)(a.B * a.Hkv));
-    k_refine_rescore<D><<<grid, C::kThreads, C::kSmemBytes, s>>>(a);
-    count_launches(1);
-    return cudaGetLastError();
+    // About one CTA per SM over all rows; each row's proposal is split evenly.
+    const int rows = a.B * a.Hkv;
+    const int parts = rows >= num_sms ? 1 : num_sms / rows;
+    return launch_kernel(k_refine_rescore<D>, dim3((unsigned)parts, (unsigned)rows),
+                         dim3(C::kThreads), C::kSmemBytes, s, a);
 }
 
-cudaError_t launch_refine_rescore(const ScoreArgs &a, cudaStream_t s) {
-    return a.d == 128 ? launch_refine_rescore_d<128>(a, s) : launch_refine_rescore_d<64>(a, s);
+cudaError_t launch_refine_rescore(const ScoreArgs &a, int num_sms, cudaStream_t s) {
+    return a.d == 128 ? launch_refine_rescore_d<128>(a, num_sms, s)
+                      : launch_refine_rescore_d<64>(a, num_sms, s);
 }
 
 }  // namespace prism
