@@ -16,10 +16,9 @@
 // first radix digit of the top-kappa selection.
 //
 // k_refine_rescore scores only the proposal positions of a refined layer
-// (Eq. (5)), enumerated from the owned ranges of the source selection; each
-// owned range (or its piece of a 128-slot window) is one bulk copy into the
-// same kind of ring, and the (score, position) candidates are stored
-// contiguously at their enumeration index.
+// (Eq. (5)), enumerated from the owned ranges of the source selection and
+// gathered with 16-byte cp.async pieces; the (score, position) candidates
+// are stored contiguously at their enumeration index.
 #include "prism_internal.cuh"
 
 namespace prism {
@@ -124,7 +123,6 @@ k_anchor_score(ScoreArgs a) {
     int *scratch = reinterpret_cast<int *>(hist_s + kHistBins);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    pdl_launch_dependents();
 
     for (int i = tid; i < kHistBins; i += blockDim.x) hist_s[i] = 0;
     if (tid == 0) {
@@ -272,6 +270,9 @@ k_anchor_score(ScoreArgs a) {
         next_tile<TILE>(c, a.len, a.B, a.Hkv, a.Lmax);
     }
     consumer_sync();
+    // The dependent (the selection) may start only now: launched earlier, its
+    // CTAs would sit on SMs for the whole scan, waiting.
+    pdl_launch_dependents();
     if (cur_row >= 0) {
         for (int i = tid; i < kHistBins; i += 32 * C::kConsumerWarps) {
             uint32_t v = hist_s[i];
@@ -285,16 +286,21 @@ k_anchor_score(ScoreArgs a) {
 // of a row is enumerated slot by slot from the owned ranges of the canonical
 // source selection (the offsets src_off give each entry's first slot), so a
 // row's n slots split evenly into P contiguous parts, one CTA each.  A CTA
-// walks its part in windows of 128 slots: the producer warp finds the
-// entries overlapping a window (one coalesced load of 32 entries at a time)
-// and moves each entry's piece of the window -- consecutive key rows -- with
-// one 1-D bulk copy (TMA) into a 3-stage shared-memory ring, noting every
-// slot's position; eight consumer warps form the dot products.  Candidates
-// (score, position) are stored at their slot index.
+// walks its part in windows of 128 slots.  The producer warp finds the
+// entries overlapping each window (one coalesced load of 32 entries at a
+// time, the next batch in flight) and writes every slot's key row into a ring
+// of position tables, up to kPosDepth windows ahead.  Each consumer warp owns
+// 16 slots of every window: it gathers exactly the 16-byte pieces of those
+// key rows that its lanes will read (cp.async, a 3-stage pipeline per warp,
+// no hand-off between warps), forms the dot products and stores the
+// (score, position) candidates at their slot index.  (A run of the proposal
+// is only ~11-17 rows, 3-4 KB: issuing one bulk copy per run from a single
+// warp, not DRAM, limited an earlier version to ~25 GB/s per SM.)
 template <int D>
 struct RescoreCfg {
     static constexpr int kTileRows = 128;
-    static constexpr int kStages = 3;
+    static constexpr int kStages = 3;                  // data stages per consumer warp
+    static constexpr int kPosDepth = 8;                // position tables in the ring
     static constexpr int kConsumerWarps = 8;
     static constexpr int kThreads = 32 * (kConsumerWarps + 1);
     static constexpr int kNL = D / 8;
@@ -304,8 +310,8 @@ struct RescoreCfg {
     static constexpr int kRowBytes = D * 2;
     static constexpr int kTileBytes = kTileRows * kRowBytes;
     static constexpr int kPosOff = kStages * kTileBytes;
-    static constexpr int kBarOff = kPosOff + kStages * kTileRows * 4;
-    static constexpr int kHistOff = kBarOff + 2 * kStages * 8;
+    static constexpr int kBarOff = kPosOff + kPosDepth * kTileRows * 4;
+    static constexpr int kHistOff = kBarOff + 2 * kPosDepth * 8;
     static constexpr int kSmemBytes = kHistOff + kHistBins * 4;
 };
 
@@ -351,12 +357,6 @@ __device__ __forceinline__ EntryRun make_entry(const EntryRaw &w, int jj, int ka
     return e;
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(RescoreCfg<D>::kThreads, 1)
 k_refine_rescore(ScoreArgs a) {
@@ -364,8 +364,8 @@ k_refine_rescore(ScoreArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *stages = smem;
     int *pos_s = reinterpret_cast<int *>(smem + C::kPosOff);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
-    uint64_t *empty = full + C::kStages;
+    uint64_t *pos_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *pos_empty = pos_full + C::kPosDepth;
     uint32_t *hist_s = reinterpret_cast<uint32_t *>(smem + C::kHistOff);
     const int row = blockIdx.y, part = blockIdx.x, P = gridDim.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -373,9 +373,9 @@ k_refine_rescore(ScoreArgs a) {
     const int L = load_len(a.len, b, a.Lmax, a.st, kWhereRescore);
     for (int i = tid; i < kHistBins; i += C::kThreads) hist_s[i] = 0;
     if (tid == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], C::kConsumerWarps);
+        for (int s = 0; s < C::kPosDepth; ++s) {
+            mbar_init(&pos_full[s], 1);
+            mbar_init(&pos_empty[s], C::kConsumerWarps);
         }
         fence_mbar_init();
     }
@@ -386,16 +386,15 @@ k_refine_rescore(ScoreArgs a) {
     const int n = min(min(__ldcg(off + a.kappa), L), a.Lmax);
     const int s_begin = (int)((long long)part * n / P);
     const int s_end = (int)((long long)(part + 1) * n / P);
-    if (s_begin >= s_end) {
+    const int nwin = (s_end - s_begin + C::kTileRows - 1) / C::kTileRows;
+    if (nwin <= 0) {
         pdl_launch_dependents();
         return;
     }
 
     if (warp == C::kConsumerWarps) {
-        // ---------------- producer warp ----------------------------------------
+        // ---------------- producer warp: the position tables ---------------------
         const int32_t *src = a.src + (size_t)row * a.kappa;
-        const uint16_t *kb = static_cast<const uint16_t *>(a.k) + (size_t)row * a.Lmax * D;
-        const uint64_t pol = l2_evict_first_policy();
         // First entry to look at: the last one starting at or before s_begin,
         // by a 64-way search over the offsets (off[0] = 0 <= s_begin).
         int lo = 0, hi = a.kappa;
@@ -414,28 +413,21 @@ k_refine_rescore(ScoreArgs a) {
         EntryRun e = make_entry(load_entry_raw(src, off, a.kappa, jb + lane), jb + lane, a.kappa, n,
                                 a.radius, L, a.st);
         EntryRaw next = load_entry_raw(src, off, a.kappa, jb + 32 + lane);
-        bool failed = false;
-        int issued = 0;
-        for (int it = 0, w0 = s_begin; w0 < s_end; ++it, w0 += C::kTileRows) {
-            const int s = it % C::kStages;
-            const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
-            if (!mbar_wait(&empty[s], ph ^ 1u, a.wait_ns)) {
+        for (int it = 0; it < nwin; ++it) {
+            const int s = it % C::kPosDepth;
+            const uint32_t ph = (uint32_t)(it / C::kPosDepth) & 1u;
+            if (!mbar_wait(&pos_empty[s], ph ^ 1u, a.wait_ns)) {
                 if (lane == 0) report(a.st, kDevErrTimeout, kWhereRescore, (uint32_t)it);
-                failed = true;
                 break;
             }
+            const int w0 = s_begin + it * C::kTileRows;
             const int wend = min(w0 + C::kTileRows, s_end);
-            if (lane == 0) mbar_expect_tx(&full[s], (uint32_t)(wend - w0) * C::kRowBytes);
-            __syncwarp();
-            uint8_t *tile = stages + s * C::kTileBytes;
             int *pos = pos_s + s * C::kTileRows;
             for (;;) {
                 const int g0 = max(e.o0, w0), g1 = min(e.o1, wend);
                 if (g0 < g1) {
-                    // keep the copy inside this row of the key cache whatever the offsets say
+                    // keep the rows inside this row of the key cache whatever the offsets say
                     const int r0 = min(e.lo + (g0 - e.o0), a.Lmax - (g1 - g0));
-                    bulk_load(tile + (size_t)(g0 - w0) * C::kRowBytes, kb + (size_t)r0 * D,
-                              (uint32_t)(g1 - g0) * C::kRowBytes, &full[s], pol);
                     for (int t = g0; t < g1; ++t) pos[t - w0] = r0 + (t - g0);
                 }
                 const int reach = __shfl_sync(0xffffffffu, e.o1, 31);
@@ -445,16 +437,7 @@ k_refine_rescore(ScoreArgs a) {
                 next = load_entry_raw(src, off, a.kappa, jb + 32 + lane);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&full[s]);
-            issued = it + 1;
-        }
-        // Every issued copy must land before the CTA may exit.
-        if (failed) {
-            for (int it = max(0, issued - C::kStages); it < issued; ++it) {
-                const int s = it % C::kStages;
-                if (!mbar_wait(&full[s], (uint32_t)(it / C::kStages) & 1u, a.wait_ns) && lane == 0)
-                    report(a.st, kDevErrTimeout, kWhereRescore, 0x80000000u | (uint32_t)it);
-            }
+            if (lane == 0) mbar_arrive(&pos_full[s]);
         }
         return;
     }
@@ -474,19 +457,45 @@ k_refine_rescore(ScoreArgs a) {
         qreg[4] += bf16_lo(w.z); qreg[5] += bf16_hi(w.z);
         qreg[6] += bf16_lo(w.w); qreg[7] += bf16_hi(w.w);
     }
+    const uint16_t *kb = static_cast<const uint16_t *>(a.k) + (size_t)row * a.Lmax * D;
     float *S = a.S + (size_t)row * a.Lmax;
     int32_t *cpos = a.cpos + (size_t)row * a.Lmax;
     const int r_base = warp * C::kRowsPerWarp;
     const int r_item = r_base + transpose_item<C::kSteps, C::kNL>(lane) * C::kRPI + sub;
     const bool writer = transpose_writer<C::kSteps, C::kNL>(lane);
-    for (int it = 0, w0 = s_begin; w0 < s_end; ++it, w0 += C::kTileRows) {
-        const int s = it % C::kStages;
-        const uint32_t ph = (uint32_t)(it / C::kStages) & 1u;
-        if (!mbar_wait(&full[s], ph, a.wait_ns)) {
+    bool failed = false;
+    // Issue this lane's pieces of window `it` (rows r_base + st*kRPI + sub,
+    // bytes [16*slice, 16*slice + 16)); rows past the window are zero-filled.
+    auto gather = [&](int it) {
+        const int s = it % C::kPosDepth;
+        const uint32_t ph = (uint32_t)(it / C::kPosDepth) & 1u;
+        if (!failed && !mbar_wait(&pos_full[s], ph, a.wait_ns)) {
             if (lane == 0) report(a.st, kDevErrTimeout, kWhereRescore, 0x40000000u | (uint32_t)it);
-            break;
+            failed = true;
         }
-        const uint8_t *tile = stages + s * C::kTileBytes;
+        const int nrows = min(C::kTileRows, s_end - (s_begin + it * C::kTileRows));
+        const int *pos = pos_s + s * C::kTileRows;
+        uint8_t *tile = stages + (it % C::kStages) * C::kTileBytes;
+#pragma unroll
+        for (int st = 0; st < C::kSteps; ++st) {
+            const int r = r_base + st * C::kRPI + sub;
+            const bool ok = !failed && r < nrows;
+            const int krow = ok ? pos[r] : 0;
+            cp_async16(tile + r * C::kRowBytes + slice * 16, kb + (size_t)krow * D + slice * 8,
+                       ok ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int it = 0; it < C::kStages - 1; ++it) {
+        if (it < nwin) gather(it);
+        else cp_async_commit();
+    }
+    for (int it = 0; it < nwin; ++it) {
+        if (it + C::kStages - 1 < nwin) gather(it + C::kStages - 1);
+        else cp_async_commit();
+        cp_async_wait<C::kStages - 1>();                // this lane's pieces of window `it`
+        const uint8_t *tile = stages + (it % C::kStages) * C::kTileBytes;
         float part_[C::kSteps];
 #pragma unroll
         for (int st = 0; st < C::kSteps; ++st) {
@@ -494,18 +503,21 @@ k_refine_rescore(ScoreArgs a) {
             const uint4 kv = *reinterpret_cast<const uint4 *>(tile + r * C::kRowBytes + slice * 16);
             part_[st] = dot8(kv, qreg);
         }
+        const int s = it % C::kPosDepth;
         const int p_item = pos_s[s * C::kTileRows + r_item];
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        if (lane == 0) mbar_arrive(&pos_empty[s]);
         transpose_reduce<C::kSteps, C::kNL>(part_, lane);
+        const int w0 = s_begin + it * C::kTileRows;
         const int nrows = min(C::kTileRows, s_end - w0);
-        if (writer && r_item < nrows) {
+        if (!failed && writer && r_item < nrows) {
             const float sc = part_[0] * a.scale;
             S[w0 + r_item] = sc;
             cpos[w0 + r_item] = p_item;
             atomicAdd(&hist_s[score_key(sc) >> (32 - kHistBits)], 1u);
         }
     }
+    cp_async_wait<0>();
     consumer_sync();
     pdl_launch_dependents();
     for (int i = tid; i < kHistBins; i += 32 * C::kConsumerWarps) {
