@@ -127,6 +127,30 @@ def gpu_id_for(dev) -> str:
         return str(dev.index or 0)
 
 
+# --------------------------------------------------------------------------- ranks
+def max_over_ranks(x: float, device) -> float:
+    """The largest of every rank's x (a time); x itself with a single rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_us_per_layer(ms_per_step: float, n_layers: int, world: int) -> float:
+    """Every rank runs its own replica of the step (no collective on the data
+    path), so the job processes world * n_layers layers per step time."""
+    return ms_per_step * 1e3 / (n_layers * world)
+
+
+def barrier_if_distributed():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
 # --------------------------------------------------------------------------- helpers
 def anchor_bytes(w, lens):
     return int(sum(int(L) for L in lens)) * w.n_kv_heads * w.head_dim * 2
@@ -281,8 +305,7 @@ def run_prism(args, rank, world, dev):
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
+    barrier_if_distributed()
     clocks = ClockSampler(gpu_id_for(dev))
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -293,17 +316,13 @@ def run_prism(args, rank, world, dev):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        torch.distributed.barrier()
+    barrier_if_distributed()
     clk = clocks.stop()
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     st, detail = prism.prism_check_device_status(ws)
     if st != 0:
         raise RuntimeError(f"device status after timing {st} {detail}")
-    value = ms * 1e3 / (N * world)
+    value = whole_job_us_per_layer(ms, N, world)
     peak, peak_kind = peaks()
     step_gbs = step_bytes / (ms * 1e-3) / 1e9
 
@@ -392,12 +411,8 @@ def run_prism(args, rank, world, dev):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e2e = a.elapsed_time(b) / args.steps
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = {"value": ms_e2e * 1e3 / (N * world), "unit": UNIT,
+        ms_e2e = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
+        e2e = {"value": whole_job_us_per_layer(ms_e2e, N, world), "unit": UNIT,
                "h2d_bytes_per_step": q_h.numel() * 2 + lens_hp.numel() * 4,
                "d2h_bytes_per_step": out_h.numel() * 2,
                "path": "prism_decode_step (eager, public C ABI) with pinned host q/len in "

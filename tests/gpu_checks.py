@@ -121,17 +121,23 @@ def check_attention(o, cfg, q, k, v, lens, idx, out, rows=None, stats=None):
         stats["out_err"] = max(stats.get("out_err", 0.0), worst)
 
 
-def layerwise_step_check(o, cfg, inp, out, idx_all, rows=None, stats=None):
+def layerwise_step_check(o, cfg, inp, out, idx_all, rows=None, stats=None, layers=None):
     """Check a decode step layer by layer: every layer's selection is
     reproduced by the stage entry points on the GPU's own inputs (bit-exact),
     those stages are checked against the oracle, and every layer's output is
-    checked against the oracle's attention over that layer's selection."""
+    checked against the oracle's attention over that layer's selection.
+    `layers` restricts the check to some layers (each is checked on the
+    step's own source selection, so any subset is valid)."""
     mask = list(inp["anchor_mask"])
     N = cfg.n_layers
     ws = prism.workspace(cfg)
     last_anchor = 0
     for l in range(N):
         anchor = cfg.mode == prism.MODE_DENSE_ANCHOR or mask[l]
+        if layers is not None and l not in layers:
+            if anchor:
+                last_anchor = l
+            continue
         q, k, v, lens = inp["q"][l], inp["k"][l], inp["v"][l], inp["lens"]
         if anchor:
             S = torch.empty((cfg.batch, cfg.n_kv_heads, cfg.max_len), dtype=torch.float32,
