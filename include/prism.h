@@ -191,6 +191,25 @@ PRISM_API prism_status_t prism_sparse_decode(const prism_config_t *cfg, const vo
                                    int32_t n_idx, void *out, void *ws,
                                    size_t ws_bytes, void *stream);
 
+/* prism_sparse_decode without a caller workspace.  The paper has no
+ * counterpart: this is a library convenience for callers that cannot provide
+ * device scratch (a host holding only device pointers to its KV cache, with
+ * no device allocator of its own, or one that must not allocate once it has
+ * started).  Same computation, arguments and validation as
+ * prism_sparse_decode; the split-K scratch is a fixed device array inside the
+ * library, so nothing is allocated by this call or by the library.
+ * Limits (else PRISM_ERR_WORKSPACE, nothing launched):
+ *   B * Hkv <= 1024  and  B * Hkv * ceil(n_idx / 64) * G * head_dim <= 2^20.
+ * The first call on a device looks up the array's address; make it before any
+ * stream capture.  All calls share the one array: calls that overlap in time
+ * (other streams, other threads) race on it and must be serialised by the
+ * caller.  Device-side contract violations (len outside [0, Lmax]) are
+ * clamped as in prism_sparse_decode but not reported.                        */
+PRISM_API prism_status_t prism_sparse_decode_noalloc(const prism_config_t *cfg, const void *q,
+                                   const void *k, const void *v,
+                                   const int32_t *len, const int32_t *idx,
+                                   int32_t n_idx, void *out, void *stream);
+
 /* One decode step over cfg->n_layers layers (Algorithm 1), per cfg->mode and
  * cfg->chain, every layer ending in sparse attention over its own selection.
  * q        bf16 [N][B][Hq][d] (device)

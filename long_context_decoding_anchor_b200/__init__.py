@@ -32,7 +32,7 @@ STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED",
 EXPORTS = ("prism_workspace_size", "prism_index_anchor", "prism_index_refine",
            "prism_sparse_decode", "prism_decode_step", "prism_check_device_status",
            "prism_debug_wait_timeout", "prism_score_anchor", "prism_status_string",
-           "prism_version", "prism_launch_count")
+           "prism_version", "prism_launch_count", "prism_sparse_decode_noalloc")
 
 
 class PrismError(RuntimeError):
@@ -98,6 +98,8 @@ def lib() -> ctypes.CDLL:
         L.prism_index_refine.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
         L.prism_sparse_decode.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
         L.prism_decode_step.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_sparse_decode_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, vp, vp]
+        L.prism_sparse_decode_noalloc.restype = ctypes.c_int
         L.prism_check_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)]
         L.prism_debug_wait_timeout.argtypes = [vp, sz, u64, vp]
         L.prism_status_string.argtypes = [ctypes.c_int]
@@ -235,6 +237,26 @@ def prism_sparse_decode(cfg: Config, q, k, v, lens, idx, out=None, ws=None, stre
     return out
 
 
+def prism_sparse_decode_noalloc(cfg: Config, q, k, v, lens, idx, out=None, stream=None):
+    """prism_sparse_decode with the library's own fixed scratch (no workspace)."""
+    B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
+    _need(q, "q", torch.bfloat16, (B, Hq, d))
+    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need(v, "v", torch.bfloat16, (B, Hkv, L, d))
+    _need(lens, "lens", torch.int32, (B,))
+    if idx.dim() != 3 or tuple(idx.shape[:2]) != (B, Hkv):
+        raise ValueError("idx must be [B][Hkv][n_idx]")
+    _need(idx, "idx", torch.int32)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, d))
+    _check(lib().prism_sparse_decode_noalloc(ctypes.byref(cfg), _p(q), _p(k), _p(v), _p(lens),
+                                             _p(idx), int(idx.shape[2]), _p(out),
+                                             _stream(stream)),
+           "prism_sparse_decode_noalloc")
+    return out
+
+
 def prism_decode_step(cfg: Config, q, k_layers, v_layers, lens, out=None, idx_out=None,
                       ws=None, stream=None, want_idx=False):
     N, B, Hq, Hkv, d, L = (cfg.n_layers, cfg.batch, cfg.n_q_heads, cfg.n_kv_heads,
@@ -284,5 +306,5 @@ def raw_status(fn_name: str, *args) -> int:
 __all__ = ["Config", "PrismError", "lib", "workspace", "prism_workspace_size",
            "prism_index_anchor", "prism_index_refine", "prism_sparse_decode",
            "prism_decode_step", "prism_check_device_status", "prism_debug_wait_timeout",
-           "prism_score_anchor", "raw_status", "MODE_REFINE", "MODE_STATIC_REUSE", "MODE_DENSE_ANCHOR",
+           "prism_score_anchor", "prism_sparse_decode_noalloc", "raw_status", "MODE_REFINE", "MODE_STATIC_REUSE", "MODE_DENSE_ANCHOR",
            "CHAIN_PREV", "CHAIN_ANCHOR", "FLAG_SERIAL", "EXPORTS", "LIB_PATH"]

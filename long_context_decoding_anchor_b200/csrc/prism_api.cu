@@ -516,6 +516,38 @@ prism_status_t prism_sparse_decode(const prism_config_t *cfg, const void *q, con
     return run_attn(*cfg, w, q, k, v, len, idx, n_idx, n_idx, out, s);
 }
 
+prism_status_t prism_sparse_decode_noalloc(const prism_config_t *cfg, const void *q,
+                                           const void *k, const void *v, const int32_t *len,
+                                           const int32_t *idx, int32_t n_idx, void *out,
+                                           void *stream) {
+    PRISM_TRY(check_config(cfg));
+    if (!q || !k || !v || !len || !idx || !out) return PRISM_ERR_INVALID_ARG;
+    if (n_idx < 1 || n_idx > cfg->kappa) return PRISM_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(len, 4) || !aligned(idx, 4))
+        return PRISM_ERR_INVALID_ARG;
+    const long long rows = (long long)cfg->batch * cfg->n_kv_heads;
+    const long long nsplit = (n_idx + kAttnChunk - 1) / kAttnChunk;
+    const long long G = cfg->n_q_heads / cfg->n_kv_heads;
+    if (rows > kStaticAttnMaxRows ||
+        rows * nsplit * G * cfg->head_dim > (long long)kStaticAttnMaxAccFloats)
+        return PRISM_ERR_WORKSPACE;
+    StaticAttnScratch sc;
+    PRISM_CUDA(static_attn_scratch(&sc));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // The merge counters must start at zero (the kernel leaves them zeroed,
+    // but a call cut short would not).
+    PRISM_CUDA(cudaMemsetAsync(sc.st, 0, sizeof(DevStatus), s));
+    PRISM_CUDA(cudaMemsetAsync(sc.ctl, 0, (size_t)rows * sizeof(RowCtl), s));
+    AttnArgs aa{};
+    aa.q = q; aa.k = k; aa.v = v; aa.len = len; aa.idx = idx;
+    aa.idx_stride = n_idx; aa.n_idx = n_idx;
+    aa.B = cfg->batch; aa.Hkv = cfg->n_kv_heads; aa.G = (int)G;
+    aa.d = cfg->head_dim; aa.Lmax = cfg->max_len; aa.scale = eff_scale(*cfg);
+    aa.part_acc = sc.part_acc; aa.part_ml = sc.part_ml; aa.ctl = sc.ctl; aa.out = out; aa.st = sc.st;
+    return cuda_status(launch_sparse_attn(aa, s));
+}
+
 prism_status_t prism_decode_step(const prism_config_t *cfg, const void *q, const void *const *k,
                                  const void *const *v, const int32_t *len, void *out,
                                  int32_t *idx_out, void *ws, size_t ws_bytes, void *stream) {

@@ -462,6 +462,16 @@ struct AttnArgs {
 constexpr int kAttnChunk = 64;
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t s);
 
+// Static scratch of the no-workspace attention variant (attn_static.cu).
+constexpr int kStaticAttnMaxRows = 1024;                 // B * Hkv
+constexpr size_t kStaticAttnMaxAccFloats = (size_t)1 << 20;   // rows * splits * G * d
+struct StaticAttnScratch {
+    DevStatus *st;
+    RowCtl *ctl;
+    float *part_ml, *part_acc;
+};
+cudaError_t static_attn_scratch(StaticAttnScratch *out);
+
 cudaError_t launch_export_candidates(const float *cscore, const int32_t *cpos,
                                      const int32_t *src_off, int rows, int Lmax, int kappa,
                                      int32_t *cand_pos, float *cand_score, int32_t *cand_count,
