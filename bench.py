@@ -218,6 +218,7 @@ def run_reference(args, rank, world):
         times.append(t)
     ms = statistics.mean(times) * 1e3
     value = ms * 1e3 / len(layers)
+    n_anchor = sum(w.anchor_mask()[:len(layers)])
     cores = min(threads, w.rows)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -226,9 +227,9 @@ def run_reference(args, rank, world):
         "config": {"workload": f"{w.name}: {w.describe()}", "sample_layers": layers,
                    "kv_heads": w.n_kv_heads},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"layers {layers[0]}-{layers[-1]} (1 anchor + "
-                                   f"{len(layers) - 1} refined) x all {w.n_kv_heads} KV heads "
-                                   f"of the 128K workload, per step"},
+                         "sample": f"layers {layers[0]}-{layers[-1]} ({n_anchor} anchor + "
+                                   f"{len(layers) - n_anchor} refined) x all {w.n_kv_heads} KV "
+                                   f"heads of the 128K workload, per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -353,6 +354,37 @@ def run_prism(args, rank, world, dev):
     torch.cuda.synchronize(dev)
     t_score = statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e-3
     ach = a_bytes / t_score / 1e9
+
+    # -- refined layers alone (the second roofline target): the same step with
+    #    one anchor at layer 0 and every other layer refined, minus the step of
+    #    layer 0 alone; bytes = the measured proposals + the gathered K/V rows
+    def graph_ms(c, reps):
+        r = DecodeStepGraph(c, inp["q"][:c.n_layers], inp["k"][:c.n_layers],
+                            inp["v"][:c.n_layers], inp["lens"])
+        for _ in range(3):
+            r.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(reps):
+            r.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        del r
+        return a.elapsed_time(b) / reps
+    cfg_r = prism.Config.from_workload(w, anchor_mask=[1] + [0] * (N - 1))
+    cfg_0 = prism.Config.from_workload(w.replace(n_layers=1))
+    t_r = graph_ms(cfg_r, max(5, args.steps // 2))
+    t_0 = graph_ms(cfg_0, max(5, args.steps // 2))
+    _, idx_r = prism.prism_decode_step(cfg_r, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                       want_idx=True, ws=ws)
+    props_r = []
+    for l in range(1, N):
+        _, _, _, cc = prism.prism_index_refine(cfg_r, inp["q"][l], inp["k"][l], inp["lens"],
+                                               idx_r[l - 1].contiguous(), cand_cap=1, ws=ws)
+        props_r.append(int(cc.sum()))
+    refine_us = (t_r - t_0) * 1e3 / (N - 1)
+    refine_bytes = statistics.mean(props_r) * w.head_dim * 2 + gather
     score_src = [os.path.join(ROOT, "long_context_decoding_anchor_b200", "csrc", f)
                  for f in ("score.cu", "prism_internal.cuh")]
     traffic = kernel_traffic(score_src, os.path.join(ROOT, "profiles", "anchor_score_128k.md"))
@@ -418,17 +450,21 @@ def run_prism(args, rank, world, dev):
                "path": "prism_decode_step (eager, public C ABI) with pinned host q/len in "
                        "and out back, KV cache resident"}
 
-    # -- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only)
+    # -- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only),
+    #    repeated to about 10 s of CPU time
     cpu = None
     if not args.skip_cpu and rank == 0 and world == 1:
         layers = list(range(min(args.cpu_layers, N)))
         sample = oracle_sample(w, inp, layers, (0, w.n_kv_heads))
-        t_cpu, threads = time_oracle(w, sample)
+        t1, threads = time_oracle(w, sample)
+        reps = max(1, min(30, int(10.0 / max(t1, 1e-3))))
+        t_cpu, threads = time_oracle(w, sample, reps=reps) if reps > 1 else (t1, threads)
+        na = sum(mask[:len(layers)])
         cpu = {"value": t_cpu * 1e6 / len(layers), "unit": UNIT,
                "cores": min(threads, w.rows), "kind": "oracle",
-               "sample": f"layers 0-{layers[-1]} ({sum(mask[:len(layers)])} anchor + "
-                         f"{len(layers) - sum(mask[:len(layers)])} refined) x all "
-                         f"{w.n_kv_heads} KV heads, one pass ({t_cpu:.1f} s)"}
+               "sample": f"layers 0-{layers[-1]} ({na} anchor + {len(layers) - na} refined) x all "
+                         f"{w.n_kv_heads} KV heads of the 128K workload, mean of {reps} passes "
+                         f"({t_cpu * reps:.1f} s)"}
 
     if rank == 0:
         line = {
@@ -449,7 +485,16 @@ def run_prism(args, rank, world, dev):
             "roofline": {"kernel": "k_anchor_score", "bound": "hbm", "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "traffic": traffic,
                          "bytes_per_launch": a_bytes, "us_per_launch": t_score * 1e6,
-                         "peak_kind": peak_kind},
+                         "peak_kind": peak_kind,
+                         "share_of_step": n_anchor * t_score * 1e3 / ms,
+                         "why": "largest HBM consumer of the step (anchor K: "
+                                f"{n_anchor * a_bytes / step_bytes:.0%} of its bytes)"},
+            "refine_attn": {"bytes_per_layer": refine_bytes, "us_per_layer": refine_us,
+                            "gbs": refine_bytes / (refine_us * 1e-6) / 1e9,
+                            "frac": refine_bytes / (refine_us * 1e-6) / 1e9 / peak,
+                            "how": "one anchor then 31 refined layers, graph-timed, minus the "
+                                   "anchor layer alone, per refined layer; bytes = measured "
+                                   "proposal K rows + gathered K/V rows"},
             "breakdown_us": br,
             "gpu_launches": launches_per_step * args.steps,
             "launches_per_step": launches_per_step,
