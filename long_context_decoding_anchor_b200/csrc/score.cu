@@ -315,48 +315,6 @@ struct RescoreCfg {
     static constexpr int kSmemBytes = kHistOff + kHistBins * 4;
 };
 
-// One entry of the source selection as the producer lane sees it: its slots
-// [o0, o1) of the enumeration and the first key row `lo` of its owned range.
-// The raw loads are issued one batch ahead of their use.
-struct EntryRaw {
-    int o0, o1, i, prev;
-};
-struct EntryRun {
-    int o0, o1, lo;
-};
-
-__device__ __forceinline__ EntryRaw load_entry_raw(const int32_t *src, const int32_t *off,
-                                                   int kappa, int jj) {
-    EntryRaw w{-1, -1, -1, -1};
-    if (jj < kappa) {
-        w.o0 = __ldcg(off + jj);
-        w.o1 = __ldcg(off + jj + 1);
-        w.i = __ldcg(src + jj);
-        w.prev = jj > 0 ? __ldcg(src + jj - 1) : -1;
-    }
-    return w;
-}
-
-__device__ __forceinline__ EntryRun make_entry(const EntryRaw &w, int jj, int kappa, int n,
-                                               long long r, int L, DevStatus *st) {
-    EntryRun e{n, n, 0};
-    if (jj >= kappa) return e;
-    e.o0 = min(w.o0, n);
-    e.o1 = min(w.o1, n);
-    long long lo = (long long)w.i - r;
-    if (w.prev >= 0 && (long long)w.prev + r + 1 > lo) lo = (long long)w.prev + r + 1;
-    if (lo < 0) lo = 0;
-    long long hi = (long long)w.i + r;
-    if (hi > L - 1) hi = L - 1;
-    const int own = (w.i < 0 || hi < lo) ? 0 : (int)(hi - lo + 1);
-    if (e.o1 - e.o0 != own && e.o1 > e.o0) {
-        report(st, kDevErrInternal, kWhereRescore, (uint32_t)jj);   // offsets disagree
-        lo = 0;
-    }
-    e.lo = (int)lo;
-    return e;
-}
-
 template <int D>
 __global__ void __launch_bounds__(RescoreCfg<D>::kThreads, 1)
 k_refine_rescore(ScoreArgs a) {
@@ -543,6 +501,7 @@ cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s)
     return a.d == 128 ? launch_anchor_score_d<128>(a, num_sms, s)
                       : launch_anchor_score_d<64>(a, num_sms, s);
 }
+
 
 template <int D>
 static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, int num_sms, cudaStream_t s) {
