@@ -11,12 +11,14 @@
 // position) in position order.  select_finish then:
 //   1. picks the ties (first digit == b1) out of the candidates;
 //   2. after one cluster barrier, gathers the ties of all CTAs through
-//      distributed shared memory and resolves the remaining 21 bits on them
-//      (an 11-bit, then a 10-bit histogram) into the exact kappa-th key T and,
-//      if more items equal T than places remain, the cutoff position (a radix
-//      select on position).  Every CTA computes the same T, so each knows how
-//      many items every CTA selects: its output offset and the last selected
-//      position before its slice need no further exchange;
+//      distributed shared memory, histogramming their next 11 bits on the
+//      way; the bin b2 holding the kappa-th key usually has a handful of
+//      items, which one warp ranks directly (key descending, position
+//      ascending) into the exact kappa-th key T and the cutoff position (a
+//      crowded bin falls back to a 10-bit histogram and a radix select on
+//      position).  Every CTA computes the same T, so each knows how many items
+//      every CTA selects: its output offset and the last selected position
+//      before its slice need no further exchange;
 //   3. writes the CTA's selected candidates in order -- the selection comes
 //      out in ascending position order -- and, when asked, the enumeration
 //      offsets of the +-r proposal around the new selection.
@@ -35,6 +37,7 @@ namespace cg = cooperative_groups;
 
 constexpr int kSelMaxWarps = 32;
 constexpr int kMaxCluster = 16;
+constexpr int kSmallCap = 128;     // items of the second-level bin ranked directly
 
 struct SelShared {
     uint32_t hist[kHistBins];
@@ -54,6 +57,9 @@ struct SelShared {
     int warp_cnt[kSelMaxWarps];
     int owned[kMaxCluster];        // proposal positions owned by each CTA's entries
     int fail;
+    int n_small;                   // items in the threshold's second-level bin
+    uint64_t small[kSmallCap];
+    int small_owner[kSmallCap];
 };
 
 // Float value of the smallest key whose first digit is d: the inverse of
@@ -247,6 +253,7 @@ static __device__ void select_finish(SelShared &sm, cg::cluster_group &cluster, 
         sm.ntie = ntie;
         sm.nsure = ncand - ntie;
     }
+    for (int i = tid; i < kHistBins; i += nthreads) sm.hist[i] = 0;   // for the ties' next digit
     cluster.sync();     // every CTA's candidates, ties and summary are in place
 
     // 2. every CTA: all ties of the row -> T, cutoff; its offset and predecessor
@@ -286,26 +293,86 @@ static __device__ void select_finish(SelShared &sm, cg::cluster_group &cluster, 
                                : __ldcg(x.tie_g + slice_begin_of(r, x.n, C) + t);
     };
     const bool local_ok = m <= x.tie_cache;
-    if (local_ok) {
-        for (int e = tid; e < m; e += nthreads) x.tie_all[e] = tie_src(e);
-        __syncthreads();
-    }
     uint32_t T = 0;
     int cutoff = 0x7fffffff;
     if (!x.all) {
-        if (local_ok) resolve_threshold(sm, [&](int e) { return x.tie_all[e]; }, m, x.b1, x.need1, &T, &cutoff);
-        else resolve_threshold(sm, tie_src, m, x.b1, x.need1, &T, &cutoff);   // very many ties
-        // selected ties per CTA, and the last selected tie position per CTA
-        for (int e0 = 0; e0 < m; e0 += nthreads) {
-            const int e = e0 + tid;
-            const uint64_t it = e < m ? (local_ok ? x.tie_all[e] : tie_src(e)) : 0;
-            const uint32_t k_ = (uint32_t)(it >> 32);
-            const int p = (int)(uint32_t)it;
-            const bool f = e < m && (k_ > T || (k_ == T && p <= cutoff));
-            const int r = e < m ? owner(e) : -1;
-            const unsigned grp = __match_any_sync(0xffffffffu, r) & __ballot_sync(0xffffffffu, f);
-            if (f && lane == __ffs(grp) - 1) atomicAdd(&sm.chosen[r], __popc(grp));
-            if (f && lane == 31 - __clz(grp)) atomicMax(&sm.last_chosen[r], p);
+        // The ties' next 11 bits are histogrammed while they are gathered
+        // (the histogram was zeroed before the cluster barrier).
+        for (int e = tid; e < m; e += nthreads) {
+            const uint64_t it = tie_src(e);
+            if (local_ok) x.tie_all[e] = it;
+            atomicAdd(&sm.hist[((uint32_t)(it >> 32) >> 10) & 0x7ffu], 1u);
+        }
+        if (tid == 0) sm.n_small = 0;
+        __syncthreads();
+        auto tie_at = [&](int e) -> uint64_t { return local_ok ? x.tie_all[e] : tie_src(e); };
+        int b2, above2;
+        threshold_bin(sm, kHistBins, x.need1, &b2, &above2);
+        const int need2 = x.need1 - above2;
+        const uint32_t hi21 = (x.b1 << 21) | ((uint32_t)b2 << 10);
+        const int in_b2 = (int)sm.hist[b2];
+        if (in_b2 <= kSmallCap) {
+            // One pass: per CTA, the ties certainly selected (above the bin)
+            // and the last of their positions; the few items of the bin are
+            // listed and ranked directly by one warp.
+            for (int e0 = 0; e0 < m; e0 += nthreads) {
+                const int e = e0 + tid;
+                const uint64_t it = e < m ? tie_at(e) : 0;
+                const uint32_t k21 = (uint32_t)(it >> 32) & 0xfffffc00u;
+                const int p = (int)(uint32_t)it;
+                const bool f = e < m && k21 > hi21;
+                const int r = e < m ? owner(e) : -1;
+                const unsigned grp = __match_any_sync(0xffffffffu, r) & __ballot_sync(0xffffffffu, f);
+                if (f && lane == __ffs(grp) - 1) atomicAdd(&sm.chosen[r], __popc(grp));
+                if (f && lane == 31 - __clz(grp)) atomicMax(&sm.last_chosen[r], p);
+                if (e < m && k21 == hi21) {
+                    const int slot = atomicAdd(&sm.n_small, 1);
+                    sm.small[slot] = it;
+                    sm.small_owner[slot] = r;
+                }
+            }
+            __syncthreads();
+            if (warp == 0) {
+                // rank = items ahead in (key descending, position ascending);
+                // the first need2 are selected, the need2-th gives (T, cutoff)
+                const int ns = sm.n_small;
+                for (int i = lane; i < ns; i += 32) {
+                    const uint64_t u = sm.small[i];
+                    const uint32_t ku = (uint32_t)(u >> 32);
+                    const int pu = (int)(uint32_t)u;
+                    int rk = 0;
+                    for (int j = 0; j < ns; ++j) {
+                        const uint64_t v = sm.small[j];
+                        const uint32_t kv = (uint32_t)(v >> 32);
+                        rk += kv > ku || (kv == ku && (int)(uint32_t)v < pu);
+                    }
+                    if (rk < need2) {
+                        atomicAdd(&sm.chosen[sm.small_owner[i]], 1);
+                        atomicMax(&sm.last_chosen[sm.small_owner[i]], pu);
+                    }
+                    if (rk == need2 - 1) {
+                        sm.thr[0] = (int)ku;
+                        sm.thr[1] = pu;
+                    }
+                }
+            }
+            __syncthreads();
+            T = (uint32_t)sm.thr[0];
+            cutoff = sm.thr[1];
+        } else {
+            // many items share the bin: resolve the remaining bits by histograms
+            resolve_threshold(sm, tie_at, m, x.b1, x.need1, &T, &cutoff);
+            for (int e0 = 0; e0 < m; e0 += nthreads) {
+                const int e = e0 + tid;
+                const uint64_t it = e < m ? tie_at(e) : 0;
+                const uint32_t k_ = (uint32_t)(it >> 32);
+                const int p = (int)(uint32_t)it;
+                const bool f = e < m && (k_ > T || (k_ == T && p <= cutoff));
+                const int r = e < m ? owner(e) : -1;
+                const unsigned grp = __match_any_sync(0xffffffffu, r) & __ballot_sync(0xffffffffu, f);
+                if (f && lane == __ffs(grp) - 1) atomicAdd(&sm.chosen[r], __popc(grp));
+                if (f && lane == 31 - __clz(grp)) atomicMax(&sm.last_chosen[r], p);
+            }
         }
     }
     __syncthreads();
