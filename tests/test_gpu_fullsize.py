@@ -1,8 +1,9 @@
-"""The 128K and 512K workloads at full size, in the benchmark's launch
-configuration (one CUDA-graph replay of the whole decode step), checked
-against the oracle on sampled (batch, KV head) rows and layers: selections
-bit-exact on the GPU's own scores, scores within 1e-2, recall >= 0.999 per
-layer and along the whole chain, outputs within 2e-2 + 1e-2 |ref|."""
+"""The 128K, 512K and batched ragged (16 x 8K-32K) workloads at full size, in
+the benchmark's launch configuration (one CUDA-graph replay of the whole
+decode step), checked against the oracle on sampled (batch, KV head) rows
+and layers: selections bit-exact on the GPU's own scores, scores within
+1e-2, recall >= 0.999 per layer and along the whole chain, outputs within
+2e-2 + 1e-2 |ref|."""
 import gc
 
 import numpy as np
@@ -47,6 +48,7 @@ def _chain_check(oracle, w, inp, out, idx, b, h):
 @pytest.mark.parametrize("wkey,rows,layers", [
     (3, [(0, 0), (0, 5)], [0, 1, 2, 3, 4, 5, 29, 30, 31]),
     (5, [(0, 2), (0, 7)], [0, 1, 2, 6, 7]),
+    (4, [(0, 0), (7, 3), (15, 6)], [0, 1, 2, 3, 4, 13, 14, 15]),
 ])
 def test_full_size_sampled_rows(oracle, wkey, rows, layers):
     w = synth.WORKLOADS[wkey]
