@@ -7,10 +7,10 @@
 // attention reads only its own selection, so it can trail behind.  The step
 // therefore runs on three streams forked from the caller's stream and joined
 // back into it (events, so a CUDA-graph capture records the same DAG):
-//   A (low priority):  anchor scoring, at most two anchor layers ahead
-//                      (two workspace slots);
-//   M (high priority): selections in layer order -- each anchor layer's
-//                      top-kappa, each refined layer's rescoring + top-kappa;
+//   A (low priority):  each anchor layer's scoring and top-kappa, at most two
+//                      anchors ahead of the chain (two workspace slots);
+//   M (high priority): the refined layers in order -- rescoring, top-kappa --
+//                      each anchor's group waiting for that anchor's selection;
 //   C (high priority): each layer's sparse attention once its selection is
 //                      done.
 // PRISM_FLAG_SERIAL runs everything on the caller's stream instead.
