@@ -20,7 +20,14 @@
  *     +-r of a previously selected index, clipped to [0, L) (Eq. (5) over the
  *     positional proposal), and reselects its own top-kappa (Eq. (6));
  *   - sparse attention over the selected rows with an exact softmax (the
- *     SparseAttn step of Algorithm 1).
+ *     SparseAttn step of Algorithm 1);
+ *   - the pool variant (mode 3) of section 4.1-4.2 as the paper states it:
+ *     the relevance score is the maximum over the GQA group (Eq. (9), on the
+ *     bf16 keys), an anchor layer keeps a pool of the rho*kappa best tokens
+ *     (Eq. (4)) and attends to the first kappa of that pool in score order
+ *     (Algorithm 1, proposal-layer branch), and every refined layer rescores
+ *     the most recent anchor's pool with its own q and K (Eq. (5)) and keeps
+ *     its top-kappa (Eq. (6)).
  *
  * Inputs are raw bf16 bit patterns (uint16); every product and sum is formed
  * in double precision.  There is no blocking, fusion or reordering beyond the
@@ -100,6 +107,35 @@ void prism_ref_score(int d, int G, const uint16_t *q_group,
             }
         }
         s_out[e] = scale * acc;
+    }
+}
+
+/*
+ * Proposal score of Eq. (9) on the bf16 key cache:
+ *   s(i) = scale * max over the query heads j of the GQA group of <q_j, k_i>.
+ * (Eq. (9) has no scale; a positive scale does not change any selection and
+ * keeps the values comparable with Eq. (1).)  Arguments as prism_ref_score.
+ */
+void prism_ref_score_max(int d, int G, const uint16_t *q_group,
+                         const uint16_t *k_rows, int n, const int32_t *pos,
+                         double scale, double *s_out)
+{
+    for (int e = 0; e < n; ++e) {
+        long i = pos ? (long)pos[e] : (long)e;
+        const uint16_t *kr = k_rows + (size_t)i * (size_t)d;
+        double best = -INFINITY;
+        for (int j = 0; j < G; ++j) {
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c)
+                dot += bf16_to_double(q_group[(size_t)j * (size_t)d + (size_t)c]) *
+                       bf16_to_double(kr[c]);
+#if PRISM_REF_PLANT == 12
+            best = (j == 0) ? dot : best + dot;    /* planted: sum instead of max */
+#else
+            if (dot > best) best = dot;
+#endif
+        }
+        s_out[e] = scale * best;
     }
 }
 
@@ -262,6 +298,14 @@ void prism_ref_attention(int d, int G, const uint16_t *q_group,
  * mode 1 (static reuse):  a non-anchor layer copies the source selection
  *                         (Eq. (3)).
  * mode 2 (dense anchor):  every layer is an anchor layer.
+ * mode 3 (pool):          scores are the group maximum of Eq. (9); an anchor
+ *                         layer keeps the pool C = TopK(s, rho*kappa) of
+ *                         Eq. (4) and selects the first kappa tokens of C in
+ *                         score order; any other layer rescores the most
+ *                         recent anchor's pool with its own q and K (Eq. (5))
+ *                         and keeps its top-kappa (Eq. (6)).  r and chain are
+ *                         not used: the association f(S) of Algorithm 1 is
+ *                         the nearest preceding anchor.
  * chain 0: the source selection is the previous layer's final selection.
  * chain 1: the source selection is the most recent anchor layer's selection
  *          (the anchor-rooted association f(S) of Algorithm 1).
@@ -269,21 +313,26 @@ void prism_ref_attention(int d, int G, const uint16_t *q_group,
  *
  * q      : [N][B][Hq][d] bf16 bits;  k[l], v[l]: [B][Hkv][Lmax][d] bf16 bits
  * len    : [B] context lengths (<= Lmax)
+ * rho    : pool expansion factor (mode 3 only; >= 1)
  * out    : [N][B][Hq][d] fp64;       idx_out: [N][B][Hkv][kappa] int32
+ * pool_out (nullable, mode 3): [N][B][Hkv][rho*kappa] int32, the pool in
+ *          effect at each layer (an anchor's own pool, a refined layer's
+ *          inherited pool), ascending positions, -1 padded.
  * Query head j uses KV head j / (Hq / Hkv).
  * Returns 0, or -1 on an invalid argument (checked before any work).
  */
 int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
                           int r, int n_layers, const uint8_t *anchor_mask,
-                          int mode, int chain, double scale,
+                          int mode, int chain, double scale, int rho,
                           const uint16_t *q, const uint16_t *const *k,
                           const uint16_t *const *v, const int32_t *len,
-                          double *out, int32_t *idx_out)
+                          double *out, int32_t *idx_out, int32_t *pool_out)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || d < 1 || Lmax < 1 ||
-        kappa < 1 || r < 0 || n_layers < 1 || mode < 0 || mode > 2 ||
+        kappa < 1 || r < 0 || n_layers < 1 || mode < 0 || mode > 3 ||
         chain < 0 || chain > 1)
         return -1;
+    if (mode == 3 && (rho < 1 || (long long)rho * kappa > 0x7fffffffLL)) return -1;
     if (mode != 2 && !anchor_mask[0]) return -1;
     for (int b = 0; b < B; ++b)
         if (len[b] < 0 || len[b] > Lmax) return -1;
@@ -292,6 +341,17 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
     const int rows = B * Hkv;
     const size_t row_sel = (size_t)kappa;
     int last_anchor = 0;
+    /* mode 3: the most recent anchor's pool, [rows][n_pool] */
+#if PRISM_REF_PLANT == 13
+    const int n_pool = kappa;                  /* planted: pool of kappa, not rho*kappa */
+#else
+    const int n_pool = (mode == 3) ? rho * kappa : 0;
+#endif
+    int32_t *pool = NULL;
+    if (mode == 3) {
+        pool = (int32_t *)malloc(sizeof(int32_t) * (size_t)rows * (size_t)n_pool);
+        if (!pool) return -1;
+    }
 
     for (int l = 0; l < n_layers; ++l) {
         const int is_anchor = (mode == 2) || anchor_mask[l];
@@ -313,7 +373,45 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
             const uint16_t *vr = v[l] + ((size_t)b * Hkv + h) * (size_t)Lmax * (size_t)d;
             int32_t *sel = sel_l + (size_t)row * row_sel;
 
-            if (is_anchor) {
+            if (mode == 3) {
+                int32_t *C = pool + (size_t)row * (size_t)n_pool;
+                if (is_anchor) {
+                    /* Eq. (9) over the whole cache, then the pool of Eq. (4) */
+                    double *s = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+                    prism_ref_score_max(d, G, qg, kr, L, NULL, scale, s);
+                    int nc = prism_ref_topk(L, s, NULL, n_pool, C);
+                    /* the first kappa of C in score order: the top-kappa of
+                       the pool's own scores */
+                    double *sc = (double *)malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1));
+                    for (int e = 0; e < nc; ++e) sc[e] = s[C[e]];
+#if PRISM_REF_PLANT == 15
+                    /* planted: the first kappa pool entries in position order */
+                    for (int e = 0; e < nc; ++e) sc[e] = -(double)C[e];
+#endif
+                    prism_ref_topk(nc, sc, C, kappa, sel);
+                    free(sc);
+                    free(s);
+                } else {
+                    /* Eq. (5) on the inherited pool, then Eq. (6) */
+                    const int32_t *cand = C;
+                    int nc = 0;
+#if PRISM_REF_PLANT == 14
+                    /* planted: rescoring the previous layer's selection */
+                    cand = sel_src + (size_t)row * row_sel;
+                    while (nc < kappa && cand[nc] >= 0) ++nc;
+#else
+                    while (nc < n_pool && C[nc] >= 0) ++nc;
+#endif
+                    double *s = (double *)malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1));
+                    prism_ref_score_max(d, G, qg, kr, nc, cand, scale, s);
+                    prism_ref_topk(nc, s, cand, kappa, sel);
+                    free(s);
+                }
+                if (pool_out) {
+                    int32_t *po = pool_out + ((size_t)l * rows + row) * (size_t)rho * (size_t)kappa;
+                    for (long e = 0; e < (long)rho * kappa; ++e) po[e] = e < n_pool ? C[e] : -1;
+                }
+            } else if (is_anchor) {
                 double *s = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
                 prism_ref_score(d, G, qg, kr, L, NULL, scale, s);
                 prism_ref_topk(L, s, NULL, kappa, sel);
@@ -340,5 +438,6 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
         }
         if (is_anchor) last_anchor = l;
     }
+    free(pool);
     return 0;
 }

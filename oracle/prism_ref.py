@@ -18,7 +18,7 @@ _i32 = ctypes.c_int
 _dbl = ctypes.c_double
 _vp = ctypes.c_void_p
 
-MODE_REFINE, MODE_STATIC_REUSE, MODE_DENSE_ANCHOR = 0, 1, 2
+MODE_REFINE, MODE_STATIC_REUSE, MODE_DENSE_ANCHOR, MODE_POOL = 0, 1, 2, 3
 CHAIN_PREV, CHAIN_ANCHOR = 0, 1
 
 
@@ -41,6 +41,8 @@ class Oracle:
         lib = ctypes.CDLL(path)
         lib.prism_ref_score.argtypes = [_i32, _i32, _vp, _vp, _i32, _vp, _dbl, _vp]
         lib.prism_ref_score.restype = None
+        lib.prism_ref_score_max.argtypes = [_i32, _i32, _vp, _vp, _i32, _vp, _dbl, _vp]
+        lib.prism_ref_score_max.restype = None
         lib.prism_ref_topk.argtypes = [_i32, _vp, _vp, _i32, _vp]
         lib.prism_ref_topk.restype = _i32
         lib.prism_ref_expand.argtypes = [_i32, _i32, _vp, _i32, _vp]
@@ -48,8 +50,8 @@ class Oracle:
         lib.prism_ref_attention.argtypes = [_i32, _i32, _vp, _vp, _vp, _i32, _vp, _dbl, _vp, _vp]
         lib.prism_ref_attention.restype = None
         lib.prism_ref_decode_step.argtypes = [
-            _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _dbl,
-            _vp, _vp, _vp, _vp, _vp, _vp]
+            _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _dbl, _i32,
+            _vp, _vp, _vp, _vp, _vp, _vp, _vp]
         lib.prism_ref_decode_step.restype = _i32
         lib.prism_ref_num_threads.restype = _i32
         lib.prism_ref_plant.restype = _i32
@@ -63,8 +65,12 @@ class Oracle:
         return self.lib.prism_ref_num_threads()
 
     # -- single (batch, KV head) row ----------------------------------------
-    def score(self, q_group, k_rows, pos=None, scale=None, n=None):
-        """Eq. (1): scores of positions ``pos`` (or 0..n-1) for one KV head."""
+    def score(self, q_group, k_rows, pos=None, scale=None, n=None, agg="sum"):
+        """Scores of positions ``pos`` (or 0..n-1) for one KV head: Eq. (1)
+        with the group sum (``agg="sum"``) or Eq. (9)'s group maximum
+        (``agg="max"``)."""
+        if agg not in ("sum", "max"):
+            raise ValueError(f"unknown aggregation {agg!r}")
         q_group = _u16(q_group)
         k_rows = _u16(k_rows)
         G, d = q_group.shape
@@ -78,9 +84,9 @@ class Oracle:
         if scale is None:
             scale = 1.0 / np.sqrt(d)
         out = np.empty(n, dtype=np.float64)
-        self.lib.prism_ref_score(d, G, _ptr(q_group), _ptr(k_rows), n,
-                                 _ptr(pos) if pos is not None else None,
-                                 float(scale), _ptr(out))
+        fn = self.lib.prism_ref_score if agg == "sum" else self.lib.prism_ref_score_max
+        fn(d, G, _ptr(q_group), _ptr(k_rows), n, _ptr(pos) if pos is not None else None,
+           float(scale), _ptr(out))
         return out
 
     def topk(self, s, kappa, pos=None):
@@ -119,12 +125,13 @@ class Oracle:
 
     # -- whole decode step ----------------------------------------------------
     def decode_step(self, q, k_layers, v_layers, lens, kappa, radius, anchor_mask,
-                    mode=MODE_REFINE, chain=CHAIN_PREV, scale=None):
+                    mode=MODE_REFINE, chain=CHAIN_PREV, scale=None, rho=1, want_pool=False):
         """Algorithm 1 over all layers.
 
         q: [N][B][Hq][d] uint16; k_layers/v_layers: N arrays [B][Hkv][Lmax][d]
         uint16; lens: [B].  Returns (out [N][B][Hq][d] fp64,
-        idx [N][B][Hkv][kappa] int32).
+        idx [N][B][Hkv][kappa] int32), plus, with ``want_pool`` (MODE_POOL),
+        the pool in effect at each layer [N][B][Hkv][rho*kappa] int32.
         """
         q = _u16(q)
         N, B, Hq, d = q.shape
@@ -144,13 +151,19 @@ class Oracle:
         vp = (ctypes.c_void_p * N)(*[_ptr(t) for t in vs])
         out = np.empty((N, B, Hq, d), dtype=np.float64)
         idx = np.empty((N, B, Hkv, kappa), dtype=np.int32)
+        pool = None
+        if want_pool:
+            if mode != MODE_POOL:
+                raise ValueError("pools exist only in MODE_POOL")
+            pool = np.empty((N, B, Hkv, int(rho) * int(kappa)), dtype=np.int32)
         rc = self.lib.prism_ref_decode_step(B, Hq, Hkv, d, Lmax, int(kappa), int(radius), N,
                                             _ptr(mask), int(mode), int(chain), float(scale),
-                                            _ptr(q), ctypes.cast(kp, _vp), ctypes.cast(vp, _vp),
-                                            _ptr(lens), _ptr(out), _ptr(idx))
+                                            int(rho), _ptr(q), ctypes.cast(kp, _vp),
+                                            ctypes.cast(vp, _vp), _ptr(lens), _ptr(out),
+                                            _ptr(idx), _ptr(pool) if pool is not None else None)
         if rc != 0:
             raise ValueError("oracle rejected the decode-step arguments")
-        return out, idx
+        return (out, idx, pool) if want_pool else (out, idx)
 
 
 _cache: dict[tuple[int, str | None], Oracle] = {}
@@ -183,7 +196,11 @@ PLANTS = {
     9: "bf16 widening uses the wrong bit position",
     10: "refined layers always start from the anchor's selection",
     11: "refined layers rescore with the previous layer's keys",
+    12: "the group maximum of Eq. (9) is replaced by the group sum",
+    13: "the anchor's pool holds kappa tokens instead of rho*kappa",
+    14: "pool-mode refined layers rescore the previous selection, not the pool",
+    15: "the anchor attends to the pool's first kappa positions, not its best kappa",
 }
 
 __all__ = ["Oracle", "load", "bf16_bits", "PLANTS", "MODE_REFINE", "MODE_STATIC_REUSE",
-           "MODE_DENSE_ANCHOR", "CHAIN_PREV", "CHAIN_ANCHOR"]
+           "MODE_DENSE_ANCHOR", "MODE_POOL", "CHAIN_PREV", "CHAIN_ANCHOR"]

@@ -89,6 +89,18 @@ def numpy_scores(q_bits, k_bits, scale, pos=None):
     return scale * np.einsum("gd,ld->l", q, k)
 
 
+def numpy_scores_max(q_bits, k_bits, scale, pos=None):
+    """Eq. (9): per-head dot products by numpy.einsum, then numpy's maximum
+    over the group."""
+    q = bf16_bits_to_f64(q_bits)
+    k = bf16_bits_to_f64(k_bits)
+    if pos is not None:
+        k = k[np.asarray(pos, dtype=np.int64)]
+    if k.shape[0] == 0:
+        return np.zeros(0)
+    return scale * np.einsum("gd,ld->gl", q, k).max(axis=0)
+
+
 def sdpa_group(q_bits, k_bits, v_bits, idx, scale):
     """Reference attention of one GQA group over a position set, by
     torch.nn.functional.scaled_dot_product_attention in fp64 with a boolean

@@ -15,9 +15,9 @@ import numpy as np
 import torch
 
 from helpers import (bf16_bits_to_f64, brute_expand, f32_to_bf16_bits, golden, lexsort_topk,
-                     numpy_scores, rand_bf16, sdpa_group, subset_topk)
+                     numpy_scores, numpy_scores_max, rand_bf16, sdpa_group, subset_topk)
 from long_context_decoding_anchor_b200 import synth
-from oracle import (CHAIN_ANCHOR, CHAIN_PREV, MODE_DENSE_ANCHOR, MODE_REFINE,
+from oracle import (CHAIN_ANCHOR, CHAIN_PREV, MODE_DENSE_ANCHOR, MODE_POOL, MODE_REFINE,
                     MODE_STATIC_REUSE, bf16_bits)
 
 
@@ -296,10 +296,162 @@ def pin_decode_invariants(o):
                     "kappa = L equals dense attention"
 
 
+# -- pool variant: Eq. (9) group maximum, Eq. (4) pool, Algorithm 1 -------------
+def pin_score_max_bruteforce(o):
+    """Group-maximum scores equal numpy.einsum per head followed by numpy max."""
+    rng = np.random.default_rng(21)
+    for G, d, L in [(4, 64, 64), (2, 128, 256), (1, 16, 100), (8, 64, 128), (16, 128, 70)]:
+        q = rand_bf16(rng, (G, d))
+        k = rand_bf16(rng, (L, d))
+        scale = 1.0 / math.sqrt(d)
+        ref = numpy_scores_max(q, k, scale)
+        got = o.score(q, k, scale=scale, agg="max")
+        assert np.allclose(got, ref, rtol=1e-12, atol=1e-12), "max score vs einsum+max"
+        pos = np.sort(rng.choice(L, size=L // 3, replace=False)).astype(np.int32)
+        got = o.score(q, k, pos=pos, scale=scale, agg="max")
+        assert np.allclose(got, ref[pos], rtol=1e-12, atol=1e-12), "max score on a position list"
+        if G == 1:
+            assert np.allclose(got, numpy_scores(q, k, scale, pos), rtol=1e-12, atol=1e-12), \
+                "one head: maximum = sum"
+
+
+def _pool_hand_inputs():
+    g = golden("pool_hand_case")
+    L, N = g["L"], len(g["keys"])
+    q = np.array(g["queries"], np.float32)[None, None].repeat(N, 0)      # [N][1][2][2]
+    ks, vs = [], []
+    for l in range(N):
+        ks.append(f32_to_bf16_bits(np.array(g["keys"][l], np.float32).reshape(1, 1, L, 2)))
+        vs.append(f32_to_bf16_bits(np.stack([np.arange(L), np.ones(L)], 1)
+                                   .astype(np.float32).reshape(1, 1, L, 2)))
+    return g, f32_to_bf16_bits(q), ks, vs, np.array([L], np.int32)
+
+
+def pin_score_max_hand(o):
+    """Hand case of two heads where the group maximum and the group sum order
+    the tokens differently."""
+    g, q, ks, _, _ = _pool_hand_inputs()
+    k0 = ks[0][0, 0]
+    assert list(o.score(q[0, 0], k0, scale=1.0, agg="max")) == g["layer0_max_scores"], "hand max"
+    assert list(o.score(q[0, 0], k0, scale=1.0)) == g["layer0_sum_scores"], "hand sum"
+
+
+def pin_pool_hand(o):
+    g, q, ks, vs, lens = _pool_hand_inputs()
+    kw = dict(mode=MODE_POOL, scale=g["scale"], want_pool=True)
+    _, idx, pool = o.decode_step(q, ks, vs, lens, g["kappa"], 0, g["anchor_mask"], rho=g["rho"], **kw)
+    assert idx[:, 0, 0].tolist() == g["expected"]["selection"], "hand pool selections"
+    assert pool[:, 0, 0].tolist() == g["expected"]["pool"], "hand pools"
+    _, idx, _ = o.decode_step(q, ks, vs, lens, g["kappa"], 0, g["anchor_mask"], rho=1, **kw)
+    assert idx[:, 0, 0].tolist() == g["expected"]["selection_rho1"], "hand pool, rho = 1"
+    _, idx, _ = o.decode_step(q, ks, vs, lens, g["kappa"], 0, [1, 1, 1], rho=g["rho"], **kw)
+    assert idx[:, 0, 0].tolist() == g["expected"]["selection_all_anchors"], "hand pool, all anchors"
+
+
+def _numpy_pool_chain(w, q, ks, lens, rho, mask=None):
+    """The pool variant recomputed with numpy: einsum+max scores, lexsort
+    top-(rho*kappa) pool, the anchor's selection as the lexsort top-kappa of the
+    pool's scores, refined layers as the lexsort top-kappa of their own scores
+    over the nearest preceding anchor's pool."""
+    N, B, Hq, d = q.shape
+    H, G = w.n_kv_heads, w.group
+    scale = 1.0 / math.sqrt(d)
+    mask = w.anchor_mask() if mask is None else mask
+    n = rho * w.kappa
+    idx = np.zeros((N, B, H, w.kappa), dtype=np.int64)
+    pool = np.zeros((N, B, H, n), dtype=np.int64)
+    for l in range(N):
+        for b in range(B):
+            L = int(lens[b])
+            for h in range(H):
+                qg = q[l, b, h * G:(h + 1) * G]
+                kr = ks[l][b, h, :L]
+                if mask[l]:
+                    s = numpy_scores_max(qg, kr, scale)
+                    pool[l, b, h] = lexsort_topk(s, n)
+                    C = pool[l, b, h][pool[l, b, h] >= 0]
+                    idx[l, b, h] = lexsort_topk(s[C], w.kappa, C)
+                else:
+                    pool[l, b, h] = pool[l - 1, b, h]
+                    C = pool[l, b, h][pool[l, b, h] >= 0]
+                    idx[l, b, h] = lexsort_topk(numpy_scores_max(qg, kr, scale, C), w.kappa, C)
+    return idx, pool
+
+
+def pin_pool_numpy_chain(o):
+    """The pool variant's selections and pools equal the numpy recomputation."""
+    for w in small_workloads():
+        q, ks, vs, lens = _bits(synth.make_inputs(w))
+        for rho in (1, 2, 4):
+            _, idx, pool = o.decode_step(q, ks, vs, lens, w.kappa, w.radius, w.anchor_mask(),
+                                         mode=MODE_POOL, rho=rho, want_pool=True)
+            ref_idx, ref_pool = _numpy_pool_chain(w, q, ks, lens, rho)
+            assert np.array_equal(pool, ref_pool), f"pools vs numpy ({w.name}, rho {rho})"
+            assert np.array_equal(idx, ref_idx), f"pool selections vs numpy ({w.name}, rho {rho})"
+
+
+def pin_pool_invariants(o):
+    """Invariants of the pool variant:
+    rho*kappa >= L: every refined layer selects its exact per-layer top-kappa;
+    rho = 1: every refined layer keeps its anchor's selection (static reuse);
+    an anchor's selection lies inside its pool, which lies inside [0, L);
+    one query head per KV head: the pool variant with every layer an anchor is
+    the dense-anchor mode (maximum = sum);
+    every output is SDPA over its layer's selection."""
+    w = small_workloads()[1]
+    q, ks, vs, lens = _bits(synth.make_inputs(w))
+    mask = w.anchor_mask()
+    N = len(mask)
+    everywhere = [1] * N
+    rho_all = -(-w.max_len // w.kappa)
+    _, exact, _ = o.decode_step(q, ks, vs, lens, w.kappa, 0, everywhere, mode=MODE_POOL, rho=2,
+                                want_pool=True)
+    _, wide, _ = o.decode_step(q, ks, vs, lens, w.kappa, 0, mask, mode=MODE_POOL, rho=rho_all,
+                               want_pool=True)
+    assert np.array_equal(wide, exact), "rho*kappa >= L equals per-layer exact selection"
+    out, r1, pool1 = o.decode_step(q, ks, vs, lens, w.kappa, 0, mask, mode=MODE_POOL, rho=1,
+                                   want_pool=True)
+    last = 0
+    for l in range(N):
+        if mask[l]:
+            last = l
+        assert np.array_equal(r1[l], r1[last]), "rho = 1 keeps the anchor's selection"
+    _, idx, pool = o.decode_step(q, ks, vs, lens, w.kappa, 0, mask, mode=MODE_POOL, rho=3,
+                                 want_pool=True)
+    B, H = w.batch, w.n_kv_heads
+    for l in range(N):
+        for b in range(B):
+            L = int(lens[b])
+            for h in range(H):
+                P = pool[l, b, h]
+                P = P[P >= 0]
+                assert len(P) == min(L, 3 * w.kappa) and np.all(P < L), "pool size and range"
+                S = idx[l, b, h]
+                assert set(S[S >= 0].tolist()) <= set(P.tolist()), "selection inside the pool"
+    # one query head per KV head: group maximum = group sum
+    w1 = w.replace(n_q_heads=w.n_kv_heads)
+    q1 = q[:, :, ::w.group].copy()
+    _, dense = o.decode_step(q1, ks, vs, lens, w1.kappa, 0, mask, mode=MODE_DENSE_ANCHOR)
+    _, pooled = o.decode_step(q1, ks, vs, lens, w1.kappa, 0, everywhere, mode=MODE_POOL, rho=2)
+    assert np.array_equal(dense, pooled), "G = 1: pool variant with anchors everywhere = dense"
+    d = q.shape[-1]
+    G = w.group
+    for l in range(N):
+        for b in range(B):
+            L = int(lens[b])
+            for h in range(H):
+                ref = sdpa_group(q[l, b, h * G:(h + 1) * G], ks[l][b, h, :L], vs[l][b, h, :L],
+                                 r1[l, b, h], 1.0 / math.sqrt(d))
+                assert np.allclose(out[l, b, h * G:(h + 1) * G], ref, rtol=1e-10, atol=1e-12), \
+                    "pool-mode output vs SDPA"
+
+
 ALL_PINS = [pin_score_bruteforce, pin_score_hand, pin_topk_golden, pin_topk_lexsort,
             pin_topk_all_equal, pin_topk_subsets, pin_expand_golden, pin_expand_bruteforce,
             pin_attention_sdpa, pin_attention_closed_forms, pin_decode_hand,
-            pin_decode_numpy_chain, pin_decode_outputs_sdpa, pin_decode_invariants]
+            pin_decode_numpy_chain, pin_decode_outputs_sdpa, pin_decode_invariants,
+            pin_score_max_bruteforce, pin_score_max_hand, pin_pool_hand, pin_pool_numpy_chain,
+            pin_pool_invariants]
 
 __all__ = ["ALL_PINS", "small_workloads"] + [p.__name__ for p in ALL_PINS]
 _ = torch  # torch is used through helpers.sdpa_group and synth
