@@ -77,11 +77,21 @@ typedef enum {
  * REFINE:        anchor layers select exactly (Eq. (1)-(2)); other layers
  *                expand +-radius, rescore (Eq. (5)) and reselect (Eq. (6)).
  * STATIC_REUSE:  other layers reuse the source selection unchanged (Eq. (3)).
- * DENSE_ANCHOR:  every layer is an anchor layer (per-layer exact top-kappa). */
+ * DENSE_ANCHOR:  every layer is an anchor layer (per-layer exact top-kappa).
+ * POOL:          the paper's proposal-refined sharing as section 4 states it:
+ *                every score is the group maximum of Eq. (9),
+ *                  s(i) = scale * max_{j in G(h)} <q_j, k_i>  (bf16 keys);
+ *                an anchor layer keeps the pool C = TopK(s, rho * kappa) of
+ *                Eq. (4) and attends to its own top-kappa (the first kappa of
+ *                C in score order, Algorithm 1); every other layer rescores
+ *                the nearest preceding anchor's pool with its own q and K
+ *                (Eq. (5)) and keeps its top-kappa (Eq. (6)).  rho is
+ *                cfg->pool_factor; radius and chain are not used. */
 typedef enum {
     PRISM_MODE_REFINE = 0,
     PRISM_MODE_STATIC_REUSE = 1,
-    PRISM_MODE_DENSE_ANCHOR = 2
+    PRISM_MODE_DENSE_ANCHOR = 2,
+    PRISM_MODE_POOL = 3
 } prism_mode_t;
 
 /* Source selection of a refined layer.
@@ -112,6 +122,8 @@ typedef struct {
     int32_t chain;          /* prism_chain_t                                  */
     float scale;            /* score/logit scale; 0 means 1/sqrt(d)           */
     int32_t flags;          /* PRISM_FLAG_* bits, 0 by default                */
+    int32_t pool_factor;    /* rho >= 1 with rho * kappa <= PRISM_MAX_LEN in
+                               PRISM_MODE_POOL; ignored by the other modes    */
 } prism_config_t;
 
 /* prism_decode_step schedules anchor scoring, selections and attention as a
@@ -138,6 +150,8 @@ PRISM_API prism_status_t prism_workspace_size(const prism_config_t *cfg, size_t 
 /* Anchor layer index construction: Eq. (1) over every cached token, then the
  * exact top-kappa of Eq. (2).
  *   s[b][h][i] = scale * sum_{j in G(h)} <q[b][j], k[b][h][i]>, i < len[b]
+ *                (PRISM_MODE_POOL: scale * max_{j in G(h)} <q[b][j], k[b][h][i]>,
+ *                Eq. (9))
  *   idx_out[b][h] = the min(kappa, len[b]) positions with the largest s,
  *                   ties to the lower position, ascending, -1 padded.
  * q          bf16 [B][Hq][d]           k bf16 [B][Hkv][Lmax][d]
@@ -148,6 +162,25 @@ PRISM_API prism_status_t prism_index_anchor(const prism_config_t *cfg, const voi
                                   const void *k, const int32_t *len,
                                   int32_t *idx_out, float *scores_out,
                                   void *ws, size_t ws_bytes, void *stream);
+
+/* Proposal layer of PRISM_MODE_POOL (cfg->mode must be PRISM_MODE_POOL):
+ * the group-maximum scores of Eq. (9) over every cached token, the candidate
+ * pool of Eq. (4) and the layer's own selection (Algorithm 1, proposal
+ * branch).
+ *   s[b][h][i]     = scale * max_{j in G(h)} <q[b][j], k[b][h][i]>, i < len[b]
+ *   pool_out[b][h] = the min(rho*kappa, len[b]) positions with the largest s
+ *                    (Eq. (4), rho = cfg->pool_factor), ascending, -1 padded
+ *   idx_out[b][h]  = the first kappa of the pool in score order, i.e. the
+ *                    min(kappa, len[b]) largest s, ascending, -1 padded
+ * Ties go to the lower position in both.
+ * pool_out   int32 [B][Hkv][rho*kappa] (written)
+ * idx_out    int32 [B][Hkv][kappa] (written)
+ * scores_out fp32 [B][Hkv][Lmax] or NULL (as for prism_index_anchor).        */
+PRISM_API prism_status_t prism_index_pool(const prism_config_t *cfg, const void *q,
+                                  const void *k, const int32_t *len,
+                                  int32_t *pool_out, int32_t *idx_out,
+                                  float *scores_out, void *ws, size_t ws_bytes,
+                                  void *stream);
 
 /* Anchor scoring only: Eq. (1) over every cached token, exactly one kernel
  * launch (the streaming kernel that prism_index_anchor starts with).  Meant
@@ -167,6 +200,10 @@ PRISM_API prism_status_t prism_score_anchor(const prism_config_t *cfg, const voi
  * idx_prev   int32 [B][Hkv][kappa]: entries < 0 are padding and skipped; any
  *            order is accepted.
  * idx_out    int32 [B][Hkv][kappa] (written; may not alias idx_prev).
+ * In PRISM_MODE_POOL the candidate set is the pool itself (Eq. (5)) and the
+ * scores are the group maximum of Eq. (9): idx_prev is then a pool, int32
+ * [B][Hkv][rho*kappa] (any order, duplicates and -1 padding allowed), and
+ * radius is not used.
  * cand_pos, cand_score, cand_count: optional diagnostic copies of P (all
  *            three NULL, or all three given): cand_pos int32 [B][Hkv][cand_cap]
  *            ascending positions, cand_score fp32 [B][Hkv][cand_cap] their

@@ -7,9 +7,9 @@ kernels of the library.  There is no fallback: if the library is missing or
 cannot be loaded, every call raises.
 
 Functions carry the C names:
-  prism_workspace_size, prism_index_anchor, prism_index_refine,
-  prism_sparse_decode, prism_decode_step, prism_check_device_status,
-  prism_debug_wait_timeout
+  prism_workspace_size, prism_index_anchor, prism_index_pool,
+  prism_index_refine, prism_sparse_decode, prism_decode_step,
+  prism_check_device_status, prism_debug_wait_timeout
 plus ``Config`` (the prism_config_t struct) and ``workspace()``.
 """
 from __future__ import annotations
@@ -23,7 +23,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libprism.so")
 
-MODE_REFINE, MODE_STATIC_REUSE, MODE_DENSE_ANCHOR = 0, 1, 2
+MODE_REFINE, MODE_STATIC_REUSE, MODE_DENSE_ANCHOR, MODE_POOL = 0, 1, 2, 3
 CHAIN_PREV, CHAIN_ANCHOR = 0, 1
 FLAG_SERIAL = 1
 STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED",
@@ -32,7 +32,8 @@ STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED",
 EXPORTS = ("prism_workspace_size", "prism_index_anchor", "prism_index_refine",
            "prism_sparse_decode", "prism_decode_step", "prism_check_device_status",
            "prism_debug_wait_timeout", "prism_score_anchor", "prism_status_string",
-           "prism_version", "prism_launch_count", "prism_sparse_decode_noalloc")
+           "prism_version", "prism_launch_count", "prism_sparse_decode_noalloc",
+           "prism_index_pool")
 
 
 class PrismError(RuntimeError):
@@ -49,14 +50,15 @@ class Config(ctypes.Structure):
                 ("radius", ctypes.c_int32), ("n_layers", ctypes.c_int32),
                 ("anchor_mask", ctypes.POINTER(ctypes.c_uint8)),
                 ("mode", ctypes.c_int32), ("chain", ctypes.c_int32),
-                ("scale", ctypes.c_float), ("flags", ctypes.c_int32)]
+                ("scale", ctypes.c_float), ("flags", ctypes.c_int32),
+                ("pool_factor", ctypes.c_int32)]
 
     @classmethod
     def make(cls, batch, n_q_heads, n_kv_heads, head_dim, max_len, kappa, radius=0,
              n_layers=1, anchor_mask: Optional[Sequence[int]] = None, mode=MODE_REFINE,
-             chain=CHAIN_PREV, scale=0.0, flags=0) -> "Config":
+             chain=CHAIN_PREV, scale=0.0, flags=0, pool_factor=1) -> "Config":
         c = cls(batch, n_q_heads, n_kv_heads, head_dim, max_len, kappa, radius, n_layers,
-                None, mode, chain, scale, flags)
+                None, mode, chain, scale, flags, pool_factor)
         if anchor_mask is not None:
             arr = (ctypes.c_uint8 * len(anchor_mask))(*[1 if x else 0 for x in anchor_mask])
             c._mask_keepalive = arr
@@ -75,6 +77,12 @@ class Config(ctypes.Structure):
     def rows(self) -> int:
         return self.batch * self.n_kv_heads
 
+    @property
+    def src_kappa(self) -> int:
+        """Entries of a refined layer's source: the pool (rho * kappa) in pool
+        mode, a selection (kappa) otherwise."""
+        return self.pool_factor * self.kappa if self.mode == MODE_POOL else self.kappa
+
 
 _lib = None
 
@@ -91,6 +99,8 @@ def lib() -> ctypes.CDLL:
         cfgp = ctypes.POINTER(Config)
         L.prism_workspace_size.argtypes = [cfgp, ctypes.POINTER(sz)]
         L.prism_index_anchor.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_index_pool.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_index_pool.restype = ctypes.c_int
         L.prism_score_anchor.argtypes = [cfgp, vp, vp, vp, vp, vp, sz, vp]
         L.prism_score_anchor.restype = ctypes.c_int
         L.prism_launch_count.restype = ctypes.c_uint64
@@ -177,6 +187,30 @@ def prism_index_anchor(cfg: Config, q, k, lens, idx_out=None, scores_out=None, w
     return idx_out
 
 
+def prism_index_pool(cfg: Config, q, k, lens, pool_out=None, idx_out=None, scores_out=None,
+                     ws=None, stream=None):
+    """Pool mode proposal layer: returns (pool [B][Hkv][rho*kappa], idx [B][Hkv][kappa])."""
+    B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
+    _need(q, "q", torch.bfloat16, (B, Hq, d))
+    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need(lens, "lens", torch.int32, (B,))
+    n = cfg.pool_factor * cfg.kappa
+    if pool_out is None:
+        pool_out = torch.empty((B, Hkv, n), dtype=torch.int32, device=q.device)
+    if idx_out is None:
+        idx_out = torch.empty((B, Hkv, cfg.kappa), dtype=torch.int32, device=q.device)
+    _need(pool_out, "pool_out", torch.int32, (B, Hkv, n))
+    _need(idx_out, "idx_out", torch.int32, (B, Hkv, cfg.kappa))
+    if scores_out is not None:
+        _need(scores_out, "scores_out", torch.float32, (B, Hkv, L))
+    ws = workspace(cfg, q.device) if ws is None else ws
+    _check(lib().prism_index_pool(ctypes.byref(cfg), _p(q), _p(k), _p(lens), _p(pool_out),
+                                  _p(idx_out), _p(scores_out), _p(ws), ws.numel(),
+                                  _stream(stream)),
+           "prism_index_pool")
+    return pool_out, idx_out
+
+
 def prism_score_anchor(cfg: Config, q, k, lens, scores_out=None, ws=None, stream=None):
     """Eq. (1) only: one launch of the anchor scoring kernel."""
     B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
@@ -195,12 +229,13 @@ def prism_score_anchor(cfg: Config, q, k, lens, scores_out=None, ws=None, stream
 
 def prism_index_refine(cfg: Config, q, k, lens, idx_prev, idx_out=None, cand_cap=0, ws=None,
                        stream=None):
-    """Returns idx_out, or (idx_out, cand_pos, cand_score, cand_count) when cand_cap > 0."""
+    """Returns idx_out, or (idx_out, cand_pos, cand_score, cand_count) when cand_cap > 0.
+    In pool mode idx_prev is a pool [B][Hkv][rho*kappa]."""
     B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
     _need(q, "q", torch.bfloat16, (B, Hq, d))
     _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
     _need(lens, "lens", torch.int32, (B,))
-    _need(idx_prev, "idx_prev", torch.int32, (B, Hkv, cfg.kappa))
+    _need(idx_prev, "idx_prev", torch.int32, (B, Hkv, cfg.src_kappa))
     if idx_out is None:
         idx_out = torch.empty((B, Hkv, cfg.kappa), dtype=torch.int32, device=q.device)
     _need(idx_out, "idx_out", torch.int32, (B, Hkv, cfg.kappa))
@@ -304,7 +339,7 @@ def raw_status(fn_name: str, *args) -> int:
 
 
 __all__ = ["Config", "PrismError", "lib", "workspace", "prism_workspace_size",
-           "prism_index_anchor", "prism_index_refine", "prism_sparse_decode",
+           "prism_index_anchor", "prism_index_pool", "prism_index_refine", "prism_sparse_decode",
            "prism_decode_step", "prism_check_device_status", "prism_debug_wait_timeout",
-           "prism_score_anchor", "prism_sparse_decode_noalloc", "raw_status", "MODE_REFINE", "MODE_STATIC_REUSE", "MODE_DENSE_ANCHOR",
+           "prism_score_anchor", "prism_sparse_decode_noalloc", "raw_status", "MODE_REFINE", "MODE_STATIC_REUSE", "MODE_DENSE_ANCHOR", "MODE_POOL",
            "CHAIN_PREV", "CHAIN_ANCHOR", "FLAG_SERIAL", "EXPORTS", "LIB_PATH"]

@@ -13,6 +13,8 @@
 //                      each anchor's group waiting for that anchor's selection;
 //   C (high priority): each layer's sparse attention once its selection is
 //                      done.
+// In pool mode the anchor stream also selects each anchor's pool, and every
+// refined layer rescores its anchor's pool instead of a +-r proposal.
 // PRISM_FLAG_SERIAL runs everything on the caller's stream instead.
 #include <cuda_runtime.h>
 
@@ -60,10 +62,18 @@ struct Layout {
     size_t ctl_begin, ctl_end;      // [ctl_begin, ctl_end): histograms and counters; zeroed per call
     SlotLayout slot[kSlots];
     size_t attn_ctl;
-    size_t canon, canon_off, idx_all, off_all, pacc, pml, total;
+    size_t canon, canon_off, idx_all, off_all, pool_all, pool_off_all, pacc, pml, total;
 };
 
 int n_layers_of(const prism_config_t &c) { return c.n_layers > 0 ? c.n_layers : 1; }
+
+bool pool_mode(const prism_config_t &c) { return c.mode == PRISM_MODE_POOL; }
+
+// Entries of the selection a refined layer starts from: the anchor's pool of
+// rho * kappa tokens in pool mode, a selection of kappa tokens otherwise.
+int src_kappa_of(const prism_config_t &c) {
+    return pool_mode(c) ? c.pool_factor * c.kappa : c.kappa;
+}
 
 Layout make_layout(const prism_config_t &c) {
     const size_t rows = (size_t)c.batch * c.n_kv_heads;
@@ -71,6 +81,9 @@ Layout make_layout(const prism_config_t &c) {
     const size_t nsplit = ((size_t)c.kappa + kAttnChunk - 1) / kAttnChunk;
     const size_t sel_elems = rows * (size_t)c.kappa;
     const size_t off_elems = rows * ((size_t)c.kappa + 1);
+    const size_t src_elems = rows * (size_t)src_kappa_of(c);
+    const size_t src_off_elems = rows * ((size_t)src_kappa_of(c) + 1);
+    const size_t n_pools = pool_mode(c) ? (size_t)n_layers_of(c) : 0;
     Layout l{};
     size_t off = 0;
     l.status = off; off = align256(off + sizeof(DevStatus));
@@ -85,10 +98,12 @@ Layout make_layout(const prism_config_t &c) {
         l.slot[s].cpos = off; off = align256(off + (s == kRefineSlot ? rows * (size_t)c.max_len : 1) * sizeof(int32_t));
         l.slot[s].cspill = off; off = align256(off + rows * 2 * (size_t)c.max_len * sizeof(uint64_t));
     }
-    l.canon = off;     off = align256(off + sel_elems * sizeof(int32_t));
-    l.canon_off = off; off = align256(off + off_elems * sizeof(int32_t));
+    l.canon = off;     off = align256(off + src_elems * sizeof(int32_t));
+    l.canon_off = off; off = align256(off + src_off_elems * sizeof(int32_t));
     l.idx_all = off;   off = align256(off + (size_t)n_layers_of(c) * sel_elems * sizeof(int32_t));
     l.off_all = off;   off = align256(off + (size_t)n_layers_of(c) * off_elems * sizeof(int32_t));
+    l.pool_all = off;  off = align256(off + n_pools * src_elems * sizeof(int32_t));
+    l.pool_off_all = off; off = align256(off + n_pools * src_off_elems * sizeof(int32_t));
     l.pacc = off;      off = align256(off + rows * nsplit * G * (size_t)c.head_dim * sizeof(float));
     l.pml = off;       off = align256(off + rows * nsplit * G * 2 * sizeof(float));
     l.total = off;
@@ -104,7 +119,8 @@ prism_status_t check_config(const prism_config_t *c) {
         return PRISM_ERR_INVALID_ARG;
     if (c->n_q_heads % c->n_kv_heads != 0) return PRISM_ERR_INVALID_ARG;
     if (!(c->scale >= 0.f) || std::isinf(c->scale)) return PRISM_ERR_INVALID_ARG;
-    if (c->mode < PRISM_MODE_REFINE || c->mode > PRISM_MODE_DENSE_ANCHOR) return PRISM_ERR_INVALID_ARG;
+    if (c->mode < PRISM_MODE_REFINE || c->mode > PRISM_MODE_POOL) return PRISM_ERR_INVALID_ARG;
+    if (c->mode == PRISM_MODE_POOL && c->pool_factor < 1) return PRISM_ERR_INVALID_ARG;
     if (c->chain < PRISM_CHAIN_PREV || c->chain > PRISM_CHAIN_ANCHOR) return PRISM_ERR_INVALID_ARG;
     if (c->flags & ~PRISM_FLAG_SERIAL) return PRISM_ERR_INVALID_ARG;
     if (c->head_dim != 64 && c->head_dim != 128) return PRISM_ERR_UNSUPPORTED;
@@ -112,6 +128,8 @@ prism_status_t check_config(const prism_config_t *c) {
     if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return PRISM_ERR_UNSUPPORTED;
     if (G > c->head_dim / 8) return PRISM_ERR_UNSUPPORTED;
     if (c->max_len > PRISM_MAX_LEN || c->kappa > PRISM_MAX_LEN) return PRISM_ERR_UNSUPPORTED;
+    if (c->mode == PRISM_MODE_POOL && (long long)c->pool_factor * c->kappa > PRISM_MAX_LEN)
+        return PRISM_ERR_UNSUPPORTED;
     if ((long long)c->batch * c->n_kv_heads > PRISM_MAX_BATCH_ROWS) return PRISM_ERR_UNSUPPORTED;
     if (c->n_layers > PRISM_MAX_LAYERS) return PRISM_ERR_UNSUPPORTED;
     return PRISM_OK;
@@ -193,6 +211,7 @@ struct Ws {
     RowCtl *attn_ctl;
     int32_t *canon, *canon_off;
     int32_t *idx_all, *off_all;
+    int32_t *pool_all, *pool_off_all;     // pool mode: [N][rows][rho*kappa], [N][rows][rho*kappa + 1]
     float *pacc, *pml;
     uint8_t *base;
     Layout l;
@@ -216,6 +235,8 @@ prism_status_t carve(const prism_config_t &c, void *ws, size_t ws_bytes, Ws *w) 
     w->canon_off = reinterpret_cast<int32_t *>(b + w->l.canon_off);
     w->idx_all = reinterpret_cast<int32_t *>(b + w->l.idx_all);
     w->off_all = reinterpret_cast<int32_t *>(b + w->l.off_all);
+    w->pool_all = reinterpret_cast<int32_t *>(b + w->l.pool_all);
+    w->pool_off_all = reinterpret_cast<int32_t *>(b + w->l.pool_off_all);
     w->pacc = reinterpret_cast<float *>(b + w->l.pacc);
     w->pml = reinterpret_cast<float *>(b + w->l.pml);
     return PRISM_OK;
@@ -242,6 +263,7 @@ ScoreArgs score_args(const prism_config_t &c, const Ws &w, const Slot &sl, const
     sa.d = c.head_dim; sa.Lmax = c.max_len; sa.scale = eff_scale(c);
     sa.S = sl.S; sa.cpos = sl.cpos; sa.hist = sl.hist; sa.src = nullptr; sa.src_off = nullptr;
     sa.kappa = c.kappa; sa.radius = c.radius; sa.st = w.st; sa.wait_ns = wait_limit_ns();
+    sa.agg = pool_mode(c) ? kAggMax : kAggSum;
     return sa;
 }
 
@@ -276,18 +298,44 @@ prism_status_t run_anchor_select(const prism_config_t &c, const Ws &w, int slot,
                                                  prop_off), s));
 }
 
-// Refined layer: +-r proposal around the canonical source selection `src`
-// (with its offsets `src_off`), Eq. (5) on it, Eq. (6).
+// Pool mode, proposal layer: from the scores and histogram in slot `slot`,
+// the pool of Eq. (4) (rho * kappa tokens, with its enumeration offsets at
+// radius 0 when pool_off is given) and the layer's own top-kappa.  The first
+// selection leaves the histogram for the second, which clears it.
+prism_status_t run_pool_select(const prism_config_t &c, const Ws &w, int slot, const int32_t *len,
+                               int32_t *pool_out, int32_t *pool_off, int32_t *idx_out,
+                               cudaStream_t s) {
+    const Slot &sl = w.slot[slot];
+    SelectArgs p = select_args(c, w, sl, sl.S, nullptr, nullptr, len, pool_out, pool_off);
+    p.kappa = src_kappa_of(c);
+    p.radius = 0;
+    p.keep_hist = 1;
+    PRISM_CUDA(launch_select(p, s));
+    return cuda_status(launch_select(select_args(c, w, sl, sl.S, nullptr, nullptr, len, idx_out,
+                                                 nullptr), s));
+}
+
+// Refined layer: the candidates of the canonical source selection `src` (with
+// its enumeration offsets `src_off`) -- its +-r proposal, or in pool mode the
+// pool itself -- rescored (Eq. (5)), then Eq. (6).
 prism_status_t run_refine(const prism_config_t &c, const Ws &w, const void *q, const void *k,
                           const int32_t *len, const int32_t *src, const int32_t *src_off,
                           int32_t *idx_out, int32_t *prop_off, cudaStream_t s) {
     const Slot &sl = w.slot[kRefineSlot];
+    const bool pool = pool_mode(c);
     ScoreArgs sa = score_args(c, w, sl, q, k, len);
     sa.src = src;
     sa.src_off = src_off;
+    sa.kappa = src_kappa_of(c);
+    sa.radius = pool ? 0 : c.radius;
     PRISM_CUDA(launch_refine_rescore(sa, num_sms(), s));
-    return cuda_status(launch_select(select_args(c, w, sl, sl.S, sl.cpos, src_off, len, idx_out,
-                                                 prop_off), s));
+    SelectArgs se = select_args(c, w, sl, sl.S, sl.cpos, src_off, len, idx_out, pool ? nullptr : prop_off);
+    se.src_kappa = src_kappa_of(c);
+    if (pool) {
+        se.radius = 0;
+        se.n_bound = src_kappa_of(c) < c.max_len ? src_kappa_of(c) : c.max_len;
+    }
+    return cuda_status(launch_select(se, s));
 }
 
 prism_status_t run_attn(const prism_config_t &c, const Ws &w, const void *q, const void *k,
@@ -318,6 +366,10 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     const size_t off_elems = rows * ((size_t)c.kappa + 1);
     // A layer's proposal offsets are needed when a later layer refines from it.
     const bool refining = c.mode == PRISM_MODE_REFINE;
+    // Pool mode: each anchor's pool and its offsets, by layer.
+    const bool pool = pool_mode(c);
+    const size_t pool_elems = rows * (size_t)src_kappa_of(c);
+    const size_t pool_off_elems = rows * ((size_t)src_kappa_of(c) + 1);
     auto is_anchor = [&](int l) { return c.mode == PRISM_MODE_DENSE_ANCHOR || c.anchor_mask[l] != 0; };
     std::vector<int> anchors;
     for (int l = 0; l < N; ++l)
@@ -355,9 +407,15 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         if (hp && g >= kAnchorAhead) PRISM_CUDA(cudaStreamWaitEvent(sA, ev_reached[g - kAnchorAhead], 0));
         PRISM_TRY(run_anchor_score(c, w, g % kAnchorAhead, qb + (size_t)l * q_elems, k[l], len,
                                    nullptr, sA));
-        PRISM_TRY(run_anchor_select(c, w, g % kAnchorAhead, len, idx_base + (size_t)l * sel_elems,
-                                    next_refines ? w.off_all + (size_t)l * off_elems : nullptr,
-                                    sA));
+        if (pool) {
+            PRISM_TRY(run_pool_select(c, w, g % kAnchorAhead, len, w.pool_all + (size_t)l * pool_elems,
+                                      w.pool_off_all + (size_t)l * pool_off_elems,
+                                      idx_base + (size_t)l * sel_elems, sA));
+        } else {
+            PRISM_TRY(run_anchor_select(c, w, g % kAnchorAhead, len, idx_base + (size_t)l * sel_elems,
+                                        next_refines ? w.off_all + (size_t)l * off_elems : nullptr,
+                                        sA));
+        }
         if (hp) PRISM_CUDA(cudaEventRecord(ev_indexed[g], sA));
         return PRISM_OK;
     };
@@ -367,6 +425,7 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
 
     const int32_t *anchor_sel = nullptr, *anchor_off = nullptr;
     const int32_t *prev_sel = nullptr, *prev_off = nullptr;
+    int anchor_layer = 0;
     int g = 0;
     for (int l = 0; l < N; ++l) {
         const void *ql = qb + (size_t)l * q_elems;
@@ -386,7 +445,13 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
             }
             anchor_off = dst_off;
             anchor_sel = dst;
+            anchor_layer = l;
             ++g;
+        } else if (pool) {
+            // Eq. (5)-(6) over the nearest preceding anchor's pool.
+            PRISM_TRY(run_refine(c, w, ql, k[l], len, w.pool_all + (size_t)anchor_layer * pool_elems,
+                                 w.pool_off_all + (size_t)anchor_layer * pool_off_elems, dst, nullptr,
+                                 sM));
         } else if (c.mode == PRISM_MODE_STATIC_REUSE) {
             if (idx_out) {
                 PRISM_CUDA(cudaMemcpyAsync(dst, src, sel_elems * sizeof(int32_t),
@@ -453,6 +518,28 @@ prism_status_t prism_index_anchor(const prism_config_t *cfg, const void *q, cons
     return PRISM_OK;
 }
 
+prism_status_t prism_index_pool(const prism_config_t *cfg, const void *q, const void *k,
+                                const int32_t *len, int32_t *pool_out, int32_t *idx_out,
+                                float *scores_out, void *ws, size_t ws_bytes, void *stream) {
+    PRISM_TRY(check_config(cfg));
+    if (cfg->mode != PRISM_MODE_POOL) return PRISM_ERR_INVALID_ARG;
+    if (!q || !k || !len || !pool_out || !idx_out || pool_out == idx_out) return PRISM_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(len, 4) || !aligned(pool_out, 4) ||
+        !aligned(idx_out, 4) || (scores_out && !aligned(scores_out, 4)))
+        return PRISM_ERR_INVALID_ARG;
+    Ws w;
+    PRISM_TRY(carve(*cfg, ws, ws_bytes, &w));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    PRISM_TRY(zero_control(w, s));
+    PRISM_TRY(run_anchor_score(*cfg, w, 0, q, k, len, nullptr, s));
+    PRISM_TRY(run_pool_select(*cfg, w, 0, len, pool_out, nullptr, idx_out, s));
+    if (scores_out) {
+        const size_t bytes = (size_t)cfg->batch * cfg->n_kv_heads * cfg->max_len * sizeof(float);
+        PRISM_CUDA(cudaMemcpyAsync(scores_out, w.slot[0].S, bytes, cudaMemcpyDeviceToDevice, s));
+    }
+    return PRISM_OK;
+}
+
 prism_status_t prism_score_anchor(const prism_config_t *cfg, const void *q, const void *k,
                                   const int32_t *len, float *scores_out, void *ws,
                                   size_t ws_bytes, void *stream) {
@@ -486,14 +573,15 @@ prism_status_t prism_index_refine(const prism_config_t *cfg, const void *q, cons
     PRISM_TRY(zero_control(w, s));
     CanonArgs ca{};
     ca.idx = idx_prev; ca.len = len; ca.B = cfg->batch; ca.Hkv = cfg->n_kv_heads;
-    ca.Lmax = cfg->max_len; ca.kappa = cfg->kappa; ca.radius = cfg->radius;
+    ca.Lmax = cfg->max_len; ca.kappa = src_kappa_of(*cfg);
+    ca.radius = pool_mode(*cfg) ? 0 : cfg->radius;
     ca.out = w.canon; ca.out_off = w.canon_off; ca.st = w.st;
     PRISM_CUDA(launch_canonicalize(ca, s));
     PRISM_TRY(run_refine(*cfg, w, q, k, len, w.canon, w.canon_off, idx_out, nullptr, s));
     if (all)
         PRISM_CUDA(launch_export_candidates(w.slot[kRefineSlot].S, w.slot[kRefineSlot].cpos,
                                             w.canon_off, cfg->batch * cfg->n_kv_heads,
-                                            cfg->max_len, cfg->kappa, cand_pos, cand_score,
+                                            cfg->max_len, src_kappa_of(*cfg), cand_pos, cand_score,
                                             cand_count, cand_cap, s));
     return PRISM_OK;
 }
@@ -618,6 +706,6 @@ const char *prism_status_string(prism_status_t st) {
 
 uint64_t prism_launch_count(void) { return g_launches; }
 
-int32_t prism_version(void) { return 10100; }
+int32_t prism_version(void) { return 10200; }
 
 }  // extern "C"

@@ -454,12 +454,16 @@ struct ScoreArgs {
     uint32_t *hist;         // [rows][kHistBins]
     const int32_t *src;     // refine: canonical source selection [rows][kappa]
     const int32_t *src_off; // refine: its proposal enumeration offsets [rows][kappa + 1]
-    int kappa, radius;      // refine
+    int kappa, radius;      // refine: entries of the source selection, proposal radius
+    int agg;                // kAggSum: Eq. (1) group sum; kAggMax: Eq. (9) group maximum
     DevStatus *st;
     uint64_t wait_ns;
 };
+enum : int { kAggSum = 0, kAggMax = 1 };
 
 cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s);
+// The group-maximum form of the full-cache scan (tensor cores; score_max.cu).
+cudaError_t launch_anchor_score_max(const ScoreArgs &a, int num_sms, cudaStream_t s);
 
 cudaError_t launch_refine_rescore(const ScoreArgs &a, int num_sms, cudaStream_t s);
 
@@ -476,10 +480,13 @@ cudaError_t launch_canonicalize(const CanonArgs &a, cudaStream_t s);
 struct SelectArgs {
     const float *S;            // anchor: [rows][Lmax] scores by position; refine: candidate scores
     const int32_t *cpos;       // refine: [rows][Lmax] candidate positions; nullptr for the anchor
-    const int32_t *src_off;    // refine: [rows][kappa + 1]; src_off[kappa] = number of candidates
+    const int32_t *src_off;    // refine: [rows][src_kappa + 1]; its last entry = number of candidates
     const int32_t *len;
     int B, Hkv, Lmax, kappa, radius;
-    uint32_t *hist;            // [rows][kHistBins], left zeroed
+    int src_kappa;             // refine: entries of the source selection (0: kappa)
+    int n_bound;               // bound on a row's items, sizes the cluster (0: from kappa, radius)
+    int keep_hist;             // nonzero: leave the histogram for another selection of the same scores
+    uint32_t *hist;            // [rows][kHistBins], left zeroed (unless keep_hist)
     uint64_t *cspill;          // [rows][2][Lmax] overflow of the CTAs' candidate and tie lists
     int32_t *idx_out;          // [rows][kappa]
     int32_t *prop_off;         // nullable: [rows][kappa + 1] offsets of the next proposal

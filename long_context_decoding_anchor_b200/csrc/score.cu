@@ -20,6 +20,7 @@
 // gathered with 16-byte cp.async pieces; the (score, position) candidates
 // are stored contiguously at their enumeration index.
 #include "prism_internal.cuh"
+#include "tiles.cuh"
 
 namespace prism {
 
@@ -36,75 +37,6 @@ struct AnchorCfg {
     static constexpr int kTileBytes = kTileRows * D * 2;
     static constexpr int kSmemBytes = kStages * kTileBytes + 2 * kStages * 8 + kHistBins * 4 + 64 * 4;
 };
-
-// Position of tile `t` of the global tile order (row-major over (b, h), then
-// tile j) given tiles_b = ceil(len[b] / TILE).  Found by a block-wide scan over
-// the batch; every thread of the block gets the result.
-struct TileCursor {
-    int b, h, j, tiles_b;
-};
-
-template <int TILE>
-__device__ void locate_tile(const int32_t *len, int B, int Hkv, int Lmax, long long t,
-                            TileCursor *cur, long long *total, int *scratch, DevStatus *st) {
-    long long base = 0;  // tiles of all (b, h) before the current batch chunk
-    __shared__ long long s_found_base;
-    __shared__ int s_found_b;
-    __syncthreads();   // earlier readers of s_found_b are done
-    if (threadIdx.x == 0) s_found_b = -1;
-    __syncthreads();
-    for (int b0 = 0; b0 < B; b0 += blockDim.x) {
-        const int b = b0 + threadIdx.x;
-        int tb = 0;
-        if (b < B) {
-            int L = load_len(len, b, Lmax, st, kWhereScore);
-            tb = (L + TILE - 1) / TILE;
-        }
-        int tot;
-        int ex = block_exclusive_scan(tb, scratch, &tot);
-        long long my0 = base + (long long)ex * Hkv;
-        long long my1 = my0 + (long long)tb * Hkv;
-        if (b < B && tb > 0 && t >= my0 && t < my1) {
-            s_found_b = b;
-            s_found_base = my0;
-        }
-        base += (long long)tot * Hkv;
-    }
-    __syncthreads();
-    *total = base;
-    if (s_found_b >= 0) {
-        const int b = s_found_b;
-        int L = __ldg(len + b);
-        L = L < 0 ? 0 : (L > Lmax ? Lmax : L);
-        const int tb = (L + TILE - 1) / TILE;
-        const long long rem = t - s_found_base;
-        cur->b = b;
-        cur->h = (int)(rem / tb);
-        cur->j = (int)(rem % tb);
-        cur->tiles_b = tb;
-    } else {
-        cur->b = B;
-        cur->h = 0;
-        cur->j = 0;
-        cur->tiles_b = 0;
-    }
-}
-
-// Advance to the next tile (skipping empty sequences).
-template <int TILE>
-__device__ __forceinline__ void next_tile(TileCursor &c, const int32_t *len, int B, int Hkv,
-                                          int Lmax) {
-    if (++c.j < c.tiles_b) return;
-    c.j = 0;
-    if (++c.h < Hkv) return;
-    c.h = 0;
-    for (++c.b; c.b < B; ++c.b) {
-        int L = __ldg(len + c.b);
-        L = L < 0 ? 0 : (L > Lmax ? Lmax : L);
-        c.tiles_b = (L + TILE - 1) / TILE;
-        if (c.tiles_b > 0) return;
-    }
-}
 
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -315,7 +247,55 @@ struct RescoreCfg {
     static constexpr int kSmemBytes = kHistOff + kHistBins * 4;
 };
 
+// Group maximum (Eq. (9) form) of a warp's 16 gathered rows: the [16 x d] x
+// [d x 8] products of mma.sync m16n8k16 (bf16 in, fp32 accumulate; one or two
+// n-tiles of 8 heads), A fragments by ldmatrix from rows whose 16-byte chunk c
+// sits at chunk c ^ (row % 8) (conflict-free), B fragments (the group's
+// queries, head n % G in column n) held in registers.  Returns the maxima of
+// rows lane/4 (.x) and lane/4 + 8 (.y) of the warp's block, in every lane of
+// the quad.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1,
+                                            uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 template <int D>
+__device__ __forceinline__ float2 group_max_16rows(const uint8_t *rows16, const uint32_t (&qf)[2][D / 16][2],
+                                                   bool two_tiles, int lane) {
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+    const int r = (lane & 7) + ((lane >> 3) & 1) * 8;       // row this lane addresses
+    const uint32_t base = smem_addr(rows16 + r * (D * 2));
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const int chunk = 2 * kk + (lane >> 4);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(base + (uint32_t)((chunk ^ (lane & 7)) << 4), a0, a1, a2, a3);
+        mma_bf16_16816(c0, a0, a1, a2, a3, qf[0][kk][0], qf[0][kk][1]);
+        if (two_tiles) mma_bf16_16816(c1, a0, a1, a2, a3, qf[1][kk][0], qf[1][kk][1]);
+    }
+    float lo = fmaxf(c0[0], c0[1]), hi = fmaxf(c0[2], c0[3]);
+    if (two_tiles) {
+        lo = fmaxf(lo, fmaxf(c1[0], c1[1]));
+        hi = fmaxf(hi, fmaxf(c1[2], c1[3]));
+    }
+    lo = fmaxf(lo, __shfl_xor_sync(0xffffffffu, lo, 1));
+    lo = fmaxf(lo, __shfl_xor_sync(0xffffffffu, lo, 2));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, 1));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, 2));
+    return make_float2(lo, hi);
+}
+
+template <int D, bool MAXAGG>
 __global__ void __launch_bounds__(RescoreCfg<D>::kThreads, 1)
 k_refine_rescore(ScoreArgs a) {
     using C = RescoreCfg<D>;
@@ -402,25 +382,45 @@ k_refine_rescore(ScoreArgs a) {
 
     // ---------------- consumers ------------------------------------------------
     const int slice = lane % C::kNL, sub = lane / C::kNL;
-    float qreg[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) qreg[e] = 0.f;
     const uint16_t *qb = static_cast<const uint16_t *>(a.q);
     const int Hq = a.Hkv * a.G;
-    for (int g = 0; g < a.G; ++g) {
-        const uint4 w = *reinterpret_cast<const uint4 *>(
-            qb + ((size_t)b * Hq + (size_t)h * a.G + g) * D + slice * 8);
-        qreg[0] += bf16_lo(w.x); qreg[1] += bf16_hi(w.x);
-        qreg[2] += bf16_lo(w.y); qreg[3] += bf16_hi(w.y);
-        qreg[4] += bf16_lo(w.z); qreg[5] += bf16_hi(w.z);
-        qreg[6] += bf16_lo(w.w); qreg[7] += bf16_hi(w.w);
+    // Group sum: qbar, this lane's 8 elements.  Group maximum: the B fragments
+    // of the group's queries (column n of n-tile t is head (8t + n) % G; k
+    // pairs 2*(lane%4) and +8 of each 16-wide k step).
+    float qreg[8];
+    uint32_t qf[2][D / 16][2];
+    if constexpr (!MAXAGG) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qreg[e] = 0.f;
+        for (int g = 0; g < a.G; ++g) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(
+                qb + ((size_t)b * Hq + (size_t)h * a.G + g) * D + slice * 8);
+            qreg[0] += bf16_lo(w.x); qreg[1] += bf16_hi(w.x);
+            qreg[2] += bf16_lo(w.y); qreg[3] += bf16_hi(w.y);
+            qreg[4] += bf16_lo(w.z); qreg[5] += bf16_hi(w.z);
+            qreg[6] += bf16_lo(w.w); qreg[7] += bf16_hi(w.w);
+        }
+    } else {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const int head = (8 * t + (lane >> 2)) % a.G;
+            const uint16_t *qh = qb + ((size_t)b * Hq + (size_t)h * a.G + head) * D + 2 * (lane & 3);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                qf[t][kk][0] = *reinterpret_cast<const uint32_t *>(qh + 16 * kk);
+                qf[t][kk][1] = *reinterpret_cast<const uint32_t *>(qh + 16 * kk + 8);
+            }
+        }
     }
+    const bool two_tiles = a.G > 8;
     const uint16_t *kb = static_cast<const uint16_t *>(a.k) + (size_t)row * a.Lmax * D;
     float *S = a.S + (size_t)row * a.Lmax;
     int32_t *cpos = a.cpos + (size_t)row * a.Lmax;
     const int r_base = warp * C::kRowsPerWarp;
-    const int r_item = r_base + transpose_item<C::kSteps, C::kNL>(lane) * C::kRPI + sub;
-    const bool writer = transpose_writer<C::kSteps, C::kNL>(lane);
+    // The row whose score this lane stores, if it is a writer.
+    const int r_item = MAXAGG ? r_base + (lane >> 2) + ((lane & 3) == 1 ? 8 : 0)
+                              : r_base + transpose_item<C::kSteps, C::kNL>(lane) * C::kRPI + sub;
+    const bool writer = MAXAGG ? (lane & 3) < 2 : transpose_writer<C::kSteps, C::kNL>(lane);
     bool failed = false;
     // Issue this lane's pieces of window `it` (rows r_base + st*kRPI + sub,
     // bytes [16*slice, 16*slice + 16)); rows past the window are zero-filled.
@@ -439,7 +439,9 @@ k_refine_rescore(ScoreArgs a) {
             const int r = r_base + st * C::kRPI + sub;
             const bool ok = !failed && r < nrows;
             const int krow = ok ? pos[r] : 0;
-            cp_async16(tile + r * C::kRowBytes + slice * 16, kb + (size_t)krow * D + slice * 8,
+            // the group-maximum path reads the rows by ldmatrix: swizzled chunks
+            const int chunk = MAXAGG ? (slice ^ (r & 7)) : slice;
+            cp_async16(tile + r * C::kRowBytes + chunk * 16, kb + (size_t)krow * D + slice * 8,
                        ok ? 16u : 0u);
         }
         cp_async_commit();
@@ -455,17 +457,24 @@ k_refine_rescore(ScoreArgs a) {
         cp_async_wait<C::kStages - 1>();                // this lane's pieces of window `it`
         const uint8_t *tile = stages + (it % C::kStages) * C::kTileBytes;
         float part_[C::kSteps];
+        if constexpr (MAXAGG) {
+            // The warp reads rows gathered by all of its lanes.
+            __syncwarp();
+            const float2 m = group_max_16rows<D>(tile + r_base * C::kRowBytes, qf, two_tiles, lane);
+            part_[0] = (lane & 3) == 1 ? m.y : m.x;
+        } else {
 #pragma unroll
-        for (int st = 0; st < C::kSteps; ++st) {
-            const int r = r_base + st * C::kRPI + sub;
-            const uint4 kv = *reinterpret_cast<const uint4 *>(tile + r * C::kRowBytes + slice * 16);
-            part_[st] = dot8(kv, qreg);
+            for (int st = 0; st < C::kSteps; ++st) {
+                const int r = r_base + st * C::kRPI + sub;
+                const uint4 kv = *reinterpret_cast<const uint4 *>(tile + r * C::kRowBytes + slice * 16);
+                part_[st] = dot8(kv, qreg);
+            }
         }
         const int s = it % C::kPosDepth;
         const int p_item = pos_s[s * C::kTileRows + r_item];
         __syncwarp();
         if (lane == 0) mbar_arrive(&pos_empty[s]);
-        transpose_reduce<C::kSteps, C::kNL>(part_, lane);
+        if constexpr (!MAXAGG) transpose_reduce<C::kSteps, C::kNL>(part_, lane);
         const int w0 = s_begin + it * C::kTileRows;
         const int nrows = min(C::kTileRows, s_end - w0);
         if (!failed && writer && r_item < nrows) {
@@ -498,27 +507,31 @@ static cudaError_t launch_anchor_score_d(const ScoreArgs &a, int num_sms, cudaSt
 }
 
 cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s) {
+    if (a.agg == kAggMax) return launch_anchor_score_max(a, num_sms, s);
     return a.d == 128 ? launch_anchor_score_d<128>(a, num_sms, s)
                       : launch_anchor_score_d<64>(a, num_sms, s);
 }
 
 
-template <int D>
+template <int D, bool MAXAGG>
 static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, int num_sms, cudaStream_t s) {
     using C = RescoreCfg<D>;
-    cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D>,
+    cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D, MAXAGG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // About one CTA per SM over all rows; each row's proposal is split evenly.
     const int rows = a.B * a.Hkv;
     const int parts = rows >= num_sms ? 1 : num_sms / rows;
-    return launch_kernel(k_refine_rescore<D>, dim3((unsigned)parts, (unsigned)rows),
+    return launch_kernel(k_refine_rescore<D, MAXAGG>, dim3((unsigned)parts, (unsigned)rows),
                          dim3(C::kThreads), C::kSmemBytes, s, a);
 }
 
 cudaError_t launch_refine_rescore(const ScoreArgs &a, int num_sms, cudaStream_t s) {
-    return a.d == 128 ? launch_refine_rescore_d<128>(a, num_sms, s)
-                      : launch_refine_rescore_d<64>(a, num_sms, s);
+    if (a.agg == kAggMax)
+        return a.d == 128 ? launch_refine_rescore_d<128, true>(a, num_sms, s)
+                          : launch_refine_rescore_d<64, true>(a, num_sms, s);
+    return a.d == 128 ? launch_refine_rescore_d<128, false>(a, num_sms, s)
+                      : launch_refine_rescore_d<64, false>(a, num_sms, s);
 }
 
 }  // namespace prism

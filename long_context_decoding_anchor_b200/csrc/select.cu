@@ -75,7 +75,8 @@ k_select(SelectArgs a) {
     // A refined row's candidate count was written by the selection two
     // kernels back (the rescoring kernel in between waited for it before
     // letting this grid start), so it may be read before the wait.
-    const int n = refine ? min(min(__ldcg(a.src_off + (size_t)row * (a.kappa + 1) + a.kappa), L), a.Lmax) : L;
+    const int src_kappa = a.src_kappa > 0 ? a.src_kappa : a.kappa;
+    const int n = refine ? min(min(__ldcg(a.src_off + (size_t)row * (src_kappa + 1) + src_kappa), L), a.Lmax) : L;
     const float *S = a.S + (size_t)row * a.Lmax;
     const int32_t *cpos = refine ? a.cpos + (size_t)row * a.Lmax : nullptr;
     int32_t *out = a.idx_out + (size_t)row * a.kappa;
@@ -179,7 +180,8 @@ k_select(SelectArgs a) {
     x.cand_cap = kCandCap; x.mytie_cap = kMyTieCap; x.tie_cache = kTieCache; x.sel_cache = kSelCache;
     x.spill = spill; x.tie_g = tie_g; x.out = out;
     x.prop_off = a.prop_off ? a.prop_off + (size_t)row * (a.kappa + 1) : nullptr;
-    x.hist_g = a.hist + (size_t)row * kHistBins;    // zeroed for the next use even if unread
+    // zeroed for the next use even if unread, unless another selection reads it too
+    x.hist_g = a.keep_hist ? nullptr : a.hist + (size_t)row * kHistBins;
     x.st = a.st; x.where = kWhereFinalize;
     select_finish(sm, cluster, x, ncand);
     pdl_launch_dependents();
@@ -207,7 +209,8 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t s) {
     }
     const int rows = a.B * a.Hkv;
     const bool refine = a.cpos != nullptr;
-    const long long bound = refine ? (long long)a.kappa * (2LL * a.radius + 1) : (long long)a.Lmax;
+    const long long bound = a.n_bound > 0 ? (long long)a.n_bound
+                            : refine ? (long long)a.kappa * (2LL * a.radius + 1) : (long long)a.Lmax;
     const int items = (int)(bound < a.Lmax ? bound : a.Lmax);
     const int C = select_cluster_size(items, refine);
     cudaLaunchConfig_t cfg = {};

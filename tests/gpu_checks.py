@@ -97,6 +97,69 @@ def check_refine(o, cfg, q, k, lens, idx_prev, idx, cpos, cscore, ccount, rows=N
         stats["score_err"] = max(stats.get("score_err", 0.0), worst)
 
 
+def check_pool_anchor(o, cfg, q, k, lens, pool, idx, S, rows=None, stats=None):
+    """Pool mode proposal layer: Eq. (9) scores within 1e-2 of fp64; the pool
+    (Eq. (4)) and the layer's own top-kappa bit-exact against the oracle's
+    TopK on the GPU's own scores; recall of both against the fp64 scores."""
+    G = cfg.n_q_heads // cfg.n_kv_heads
+    n_pool = cfg.pool_factor * cfg.kappa
+    qh = bf16_bits(q)
+    Sh, Ph, Ih = S.cpu().numpy(), pool.cpu().numpy(), idx.cpu().numpy()
+    lh = lens.cpu().numpy()
+    worst = 0.0
+    for b, h in rows_of(cfg, rows):
+        L = int(lh[b])
+        kh = bf16_bits(k[b, h, :L]) if L > 0 else np.zeros((0, cfg.head_dim), np.uint16)
+        s_ref = o.score(qh[b, h * G:(h + 1) * G], kh, scale=scale_of(cfg), n=L, agg="max")
+        s_gpu = Sh[b, h, :L].astype(np.float64)
+        if L:
+            err = float(np.max(np.abs(s_gpu - s_ref)))
+            worst = max(worst, err)
+            assert err <= SCORE_ATOL, f"pool scores row {(b, h)}: max err {err}"
+        for got, budget, what in ((Ph[b, h], n_pool, "pool"), (Ih[b, h], cfg.kappa, "selection")):
+            sel, _ = o.topk(s_gpu, budget)
+            assert np.array_equal(sel, got), f"anchor {what} row {(b, h)} not bit-exact"
+            ref, _ = o.topk(s_ref, budget)
+            rc = recall(got, ref)
+            assert rc >= RECALL_MIN, f"anchor {what} recall row {(b, h)}: {rc}"
+        valid = Ih[b, h][Ih[b, h] >= 0]
+        assert set(valid.tolist()) <= set(Ph[b, h].tolist()), "selection outside the pool"
+    if stats is not None:
+        stats["score_err"] = max(stats.get("score_err", 0.0), worst)
+
+
+def check_pool_refine(o, cfg, q, k, lens, pool, idx, cpos, cscore, ccount, rows=None, stats=None):
+    """Pool mode refined layer: the candidates are the pool's distinct valid
+    positions (ascending), Eq. (9) scores within 1e-2, Eq. (6) bit-exact on
+    the GPU's own candidate scores, recall against fp64."""
+    G = cfg.n_q_heads // cfg.n_kv_heads
+    qh = bf16_bits(q)
+    Ph, Ih = pool.cpu().numpy(), idx.cpu().numpy()
+    cp, cs, cc = cpos.cpu().numpy(), cscore.cpu().numpy(), ccount.cpu().numpy()
+    lh = lens.cpu().numpy()
+    worst = 0.0
+    for b, h in rows_of(cfg, rows):
+        L = int(lh[b])
+        P = np.unique(Ph[b, h][(Ph[b, h] >= 0) & (Ph[b, h] < L)]).astype(np.int32)
+        n = int(cc[b, h])
+        assert n == len(P), f"pool candidates row {(b, h)}: {n} vs {len(P)}"
+        assert np.array_equal(cp[b, h, :n], P), f"pool candidate positions row {(b, h)}"
+        kh = bf16_bits(k[b, h, :max(L, 1)])
+        s_ref = o.score(qh[b, h * G:(h + 1) * G], kh, pos=P, scale=scale_of(cfg), agg="max")
+        s_gpu = cs[b, h, :n].astype(np.float64)
+        if n:
+            err = float(np.max(np.abs(s_gpu - s_ref)))
+            worst = max(worst, err)
+            assert err <= SCORE_ATOL, f"pool rescoring row {(b, h)}: max err {err}"
+        sel, _ = o.topk(s_gpu, cfg.kappa, pos=P)
+        assert np.array_equal(sel, Ih[b, h]), f"pool refine selection row {(b, h)} not bit-exact"
+        ref, _ = o.topk(s_ref, cfg.kappa, pos=P)
+        rc = recall(Ih[b, h], ref)
+        assert rc >= RECALL_MIN, f"pool refine recall row {(b, h)}: {rc}"
+    if stats is not None:
+        stats["score_err"] = max(stats.get("score_err", 0.0), worst)
+
+
 def check_attention(o, cfg, q, k, v, lens, idx, out, rows=None, stats=None):
     G = cfg.n_q_heads // cfg.n_kv_heads
     qh = bf16_bits(q)
@@ -132,13 +195,32 @@ def layerwise_step_check(o, cfg, inp, out, idx_all, rows=None, stats=None, layer
     N = cfg.n_layers
     ws = prism.workspace(cfg)
     last_anchor = 0
+    pool = None
     for l in range(N):
         anchor = cfg.mode == prism.MODE_DENSE_ANCHOR or mask[l]
+        q, k, v, lens = inp["q"][l], inp["k"][l], inp["v"][l], inp["lens"]
+        if cfg.mode == prism.MODE_POOL:
+            # The pool of an anchor is not an output of the step: the stage
+            # call reproduces it (bit-exact, as the selections show).
+            if anchor:
+                S = torch.empty((cfg.batch, cfg.n_kv_heads, cfg.max_len), dtype=torch.float32,
+                                device=q.device)
+                pool, idx = prism.prism_index_pool(cfg, q, k, lens, scores_out=S, ws=ws)
+                assert torch.equal(idx, idx_all[l]), f"layer {l}: step selection != stage selection"
+                if layers is None or l in layers:
+                    check_pool_anchor(o, cfg, q, k, lens, pool, idx, S, rows, stats)
+            elif layers is None or l in layers:
+                idx, cp, cs, cc = prism.prism_index_refine(cfg, q, k, lens, pool,
+                                                           cand_cap=cfg.max_len, ws=ws)
+                assert torch.equal(idx, idx_all[l]), f"layer {l}: step selection != stage selection"
+                check_pool_refine(o, cfg, q, k, lens, pool, idx, cp, cs, cc, rows, stats)
+            if layers is None or l in layers:
+                check_attention(o, cfg, q, k, v, lens, idx_all[l], out[l], rows, stats)
+            continue
         if layers is not None and l not in layers:
             if anchor:
                 last_anchor = l
             continue
-        q, k, v, lens = inp["q"][l], inp["k"][l], inp["v"][l], inp["lens"]
         if anchor:
             S = torch.empty((cfg.batch, cfg.n_kv_heads, cfg.max_len), dtype=torch.float32,
                             device=q.device)

@@ -62,7 +62,9 @@ def test_workspace_size_monotone(L):
     (dict(head_dim=96), 2), (dict(head_dim=32), 2), (dict(n_q_heads=12, n_kv_heads=8), 1),
     (dict(n_q_heads=24, n_kv_heads=8), 2), (dict(n_q_heads=32, n_kv_heads=2, head_dim=64), 2),
     (dict(kappa=0), 1), (dict(radius=-1), 1), (dict(max_len=0), 1),
-    (dict(max_len=(1 << 20) + 1), 2), (dict(batch=0), 1), (dict(mode=3), 1), (dict(chain=2), 1),
+    (dict(max_len=(1 << 20) + 1), 2), (dict(batch=0), 1), (dict(mode=4), 1), (dict(chain=2), 1),
+    (dict(mode=3, pool_factor=0), 1), (dict(mode=3, pool_factor=-2), 1),
+    (dict(mode=3, kappa=1 << 19, pool_factor=4), 2),
     (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1), (dict(batch=70000, n_kv_heads=1,
                                                                   n_q_heads=1), 2),
     (dict(flags=2), 1), (dict(n_layers=-1), 1), (dict(n_layers=5000), 2),
@@ -94,6 +96,24 @@ def test_anchor_argument_validation(L):
     assert f(cp, A16, A16, A4, A4, None, ctypes.c_void_p(0x100010), ws_n, None) == 1  # ws align
     assert f(cp, A16, A16, A4, A4, None, ws, ws_n - 1, None) == 3       # short workspace
     assert f(cp, A16, A16, A4, A4, None, None, ws_n, None) == 1         # null workspace
+
+
+def test_pool_argument_validation(L):
+    c = _cfg(mode=prism.MODE_POOL, pool_factor=4)
+    ws_n = prism.prism_workspace_size(c)
+    assert ws_n > prism.prism_workspace_size(_cfg())            # room for the pools
+    ws = ctypes.c_void_p(0x100000)
+    f = L.prism_index_pool
+    cp = ctypes.byref(c)
+    P = ctypes.c_void_p(0x50000)
+    assert f(cp, None, A16, A4, P, A4, None, ws, ws_n, None) == 1          # null q
+    assert f(cp, A16, A16, A4, None, A4, None, ws, ws_n, None) == 1        # null pool_out
+    assert f(cp, A16, A16, A4, P, None, None, ws, ws_n, None) == 1         # null idx_out
+    assert f(cp, A16, A16, A4, P, P, None, ws, ws_n, None) == 1            # pool aliases idx
+    assert f(cp, A16, MIS, A4, P, A4, None, ws, ws_n, None) == 1           # k misaligned
+    assert f(cp, A16, A16, A4, P, A4, None, ws, ws_n - 1, None) == 3       # short workspace
+    other = _cfg()                                                          # not pool mode
+    assert f(ctypes.byref(other), A16, A16, A4, P, A4, None, ws, ws_n, None) == 1
 
 
 def test_refine_argument_validation(L):

@@ -25,16 +25,18 @@ def _gpu():
     prism.lib()
 
 
-def _chain_check(oracle, w, inp, out, idx, b, h):
+def _chain_check(oracle, w, inp, out, idx, b, h, rho=0):
     """The oracle's fp64 chain on one row: recall of every layer's GPU
-    selection, and the outputs against the oracle's own chain."""
-    from oracle import bf16_bits
+    selection, and the outputs against the oracle's own chain (pool mode
+    when rho > 0)."""
+    from oracle import MODE_POOL, MODE_REFINE, bf16_bits
     G = w.group
     q = bf16_bits(inp["q"][:, b:b + 1, h * G:(h + 1) * G])
     ks = [bf16_bits(t[b:b + 1, h:h + 1]) for t in inp["k"]]
     vs = [bf16_bits(t[b:b + 1, h:h + 1]) for t in inp["v"]]
     lens = inp["lens"][b:b + 1].cpu().numpy()
-    ref_out, ref_idx = oracle.decode_step(q, ks, vs, lens, w.kappa, w.radius, w.anchor_mask())
+    ref_out, ref_idx = oracle.decode_step(q, ks, vs, lens, w.kappa, w.radius, w.anchor_mask(),
+                                          mode=MODE_POOL if rho else MODE_REFINE, rho=max(rho, 1))
     gi = idx[:, b, h].cpu().numpy()
     worst = min(recall(gi[l], ref_idx[l, 0, 0]) for l in range(w.n_layers))
     assert worst >= RECALL_MIN, f"chain recall row {(b, h)}: {worst}"
@@ -50,10 +52,12 @@ def _chain_check(oracle, w, inp, out, idx, b, h):
     (5, [(0, 2), (0, 7)], [0, 1, 2, 6, 7]),
     (4, [(0, 0), (7, 3), (15, 6)], [0, 1, 2, 3, 4, 13, 14, 15]),
 ])
-def test_full_size_sampled_rows(oracle, wkey, rows, layers):
+@pytest.mark.parametrize("rho", [0, 4], ids=["refine", "pool4"])
+def test_full_size_sampled_rows(oracle, wkey, rows, layers, rho):
     w = synth.WORKLOADS[wkey]
     inp = synth.make_inputs(w, device="cuda")
-    cfg = prism.Config.from_workload(w)
+    cfg = (prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=rho) if rho
+           else prism.Config.from_workload(w))
     idx = torch.empty((w.n_layers, w.batch, w.n_kv_heads, w.kappa), dtype=torch.int32,
                       device="cuda")
     g = DecodeStepGraph(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], idx_out=idx)
@@ -65,7 +69,7 @@ def test_full_size_sampled_rows(oracle, wkey, rows, layers):
     out = g.out.clone()
     del g
     layerwise_step_check(oracle, cfg, inp, out, idx, rows=rows, layers=layers)
-    _chain_check(oracle, w, inp, out, idx, *rows[0])
+    _chain_check(oracle, w, inp, out, idx, *rows[0], rho=rho)
     del inp, out, idx
     gc.collect()
     torch.cuda.empty_cache()

@@ -182,3 +182,119 @@ def test_dag_schedule_matches_serial_and_graph(oracle):
     assert torch.equal(idx_g, idx_d) and torch.equal(g.out, out_d)
     st, detail = prism.prism_check_device_status(g.ws)
     assert st == 0, detail
+
+
+# -- pool mode: Eq. (9) group maximum, Eq. (4) pool, refined layers on the pool --
+POOL_SHAPES = ["tiny-full", "d128-g4", "d128-g8-ragged", "d128-g16", "d64-g1", "d64-g2-batch"]
+
+
+@pytest.mark.parametrize("name", POOL_SHAPES)
+@pytest.mark.parametrize("rho", [2, 4])
+def test_pool_stages(oracle, name, rho):
+    w = SHAPES[name]
+    inp = _inputs(w, layers=[0, 1])
+    cfg = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=rho)
+    from gpu_checks import check_pool_anchor, check_pool_refine
+    q0, k0, v0, lens = inp["q"][0], inp["k"][0], inp["v"][0], inp["lens"]
+    S = torch.empty((w.batch, w.n_kv_heads, w.max_len), dtype=torch.float32, device="cuda")
+    ws = prism.workspace(cfg)
+    pool, idx0 = prism.prism_index_pool(cfg, q0, k0, lens, scores_out=S, ws=ws)
+    check_pool_anchor(oracle, cfg, q0, k0, lens, pool, idx0, S)
+    # the anchor entry point of pool mode scores with the group maximum too
+    idx_a = prism.prism_index_anchor(cfg, q0, k0, lens, ws=ws)
+    assert torch.equal(idx_a, idx0)
+    q1, k1, v1 = inp["q"][1], inp["k"][1], inp["v"][1]
+    idx1, cp, cs, cc = prism.prism_index_refine(cfg, q1, k1, lens, pool, cand_cap=w.max_len, ws=ws)
+    check_pool_refine(oracle, cfg, q1, k1, lens, pool, idx1, cp, cs, cc)
+    out1 = prism.prism_sparse_decode(cfg, q1, k1, v1, lens, idx1, ws=ws)
+    check_attention(oracle, cfg, q1, k1, v1, lens, idx1, out1)
+    # a shuffled pool with duplicates and padding is the same candidate set
+    perm = torch.randperm(pool.shape[-1], device="cuda")
+    messy = pool[..., perm].clone()
+    messy[..., : pool.shape[-1] // 8] = messy[..., pool.shape[-1] // 8: pool.shape[-1] // 4]
+    messy[..., -3:] = -1
+    uniq = [[torch.unique(messy[b, h][messy[b, h] >= 0]) for h in range(w.n_kv_heads)]
+            for b in range(w.batch)]
+    idx_m, cp_m, cs_m, cc_m = prism.prism_index_refine(cfg, q1, k1, lens, messy,
+                                                       cand_cap=w.max_len, ws=ws)
+    for b in range(w.batch):
+        for h in range(w.n_kv_heads):
+            n = int(cc_m[b, h])
+            assert torch.equal(cp_m[b, h, :n], uniq[b][h].to(torch.int32))
+    check_pool_refine(oracle, cfg, q1, k1, lens, messy, idx_m, cp_m, cs_m, cc_m)
+    st, detail = prism.prism_check_device_status(ws)
+    assert st == 0, detail
+
+
+@pytest.mark.parametrize("wkey,rho", [(1, 2), (1, 4), (2, 4)])
+def test_pool_decode_step(oracle, wkey, rho):
+    """The tiny (4K) and 32K workloads at full size in pool mode, every layer
+    checked stage by stage, and the whole chain against the oracle's."""
+    w = synth.WORKLOADS[wkey]
+    inp = _inputs(w)
+    cfg = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=rho)
+    out, idx = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                       want_idx=True)
+    layerwise_step_check(oracle, cfg, inp, out, idx)
+    from oracle import MODE_POOL, bf16_bits
+    ref_out, ref_idx = oracle.decode_step(bf16_bits(inp["q"]), [bf16_bits(t) for t in inp["k"]],
+                                          [bf16_bits(t) for t in inp["v"]],
+                                          inp["lens"].cpu().numpy(), w.kappa, 0,
+                                          w.anchor_mask(), mode=MODE_POOL, rho=rho)
+    gi = idx.cpu().numpy()
+    for l in range(w.n_layers):
+        for b in range(w.batch):
+            for h in range(w.n_kv_heads):
+                assert recall(gi[l, b, h], ref_idx[l, b, h]) >= 0.999, (l, b, h)
+    assert np.max(np.abs(out.float().cpu().numpy() - ref_out)) < 5e-2
+
+
+def test_pool_decode_step_batched_ragged(oracle):
+    w = synth.WORKLOADS[4].replace(batch=4, max_len=6000, ragged=(1500, 6000), n_layers=6,
+                                   kappa=256, n_clusters=16)
+    inp = _inputs(w)
+    cfg = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=4)
+    out, idx = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                       want_idx=True)
+    layerwise_step_check(oracle, cfg, inp, out, idx)
+
+
+def test_pool_invariants_on_gpu(oracle):
+    """rho * kappa >= L: every refined layer selects exactly (= anchors
+    everywhere); rho = 1: every refined layer keeps its anchor's selection."""
+    w = synth.WORKLOADS[1].replace(max_len=1200, n_layers=5, kappa=64, anchor_every=3)
+    inp = _inputs(w)
+    run = lambda **kw: prism.prism_decode_step(
+        prism.Config.from_workload(w, mode=prism.MODE_POOL, **kw), inp["q"], inp["k"], inp["v"],
+        inp["lens"], want_idx=True)
+    _, wide = run(pool_factor=-(-w.max_len // w.kappa))
+    _, exact = run(pool_factor=2, anchor_mask=[1] * w.n_layers)
+    assert torch.equal(wide, exact)
+    _, r1 = run(pool_factor=1)
+    mask = w.anchor_mask()
+    last = 0
+    for l in range(w.n_layers):
+        last = l if mask[l] else last
+        assert torch.equal(r1[l], r1[last]), l
+
+
+def test_pool_dag_matches_serial_and_graph(oracle):
+    from long_context_decoding_anchor_b200.runner import DecodeStepGraph
+    w = synth.WORKLOADS[2].replace(max_len=9000, n_layers=9, anchor_every=3, kappa=512)
+    inp = _inputs(w)
+    cfg = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=4)
+    out_d, idx_d = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                           want_idx=True)
+    cfg_s = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=4,
+                                       flags=prism.FLAG_SERIAL)
+    out_s, idx_s = prism.prism_decode_step(cfg_s, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                           want_idx=True)
+    assert torch.equal(idx_d, idx_s) and torch.equal(out_d, out_s)
+    idx_g = torch.empty_like(idx_d)
+    g = DecodeStepGraph(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], idx_out=idx_g)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(idx_g, idx_d) and torch.equal(g.out, out_d)
+    st, detail = prism.prism_check_device_status(g.ws)
+    assert st == 0, detail
