@@ -56,6 +56,10 @@ def parse_args():
                     help="only run --steps eager decode steps (for ncu captures)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (profiling a smaller case)")
+    ap.add_argument("--pool", type=int, default=4,
+                    help="rho of the pool-mode measurement (0: skip it)")
+    ap.add_argument("--mode", choices=["refine", "pool"], default="refine",
+                    help="decode-step mode of a --profile run (pool uses --pool as rho)")
     return ap.parse_args()
 
 
@@ -249,7 +253,9 @@ def run_prism(args, rank, world, dev):
         w = w.replace(n_layers=args.layers)
     inp = synth.make_inputs(w, device=dev)
     if args.profile:
-        cfg = prism.Config.from_workload(w)
+        pool_run = args.mode == "pool"
+        cfg = (prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=args.pool)
+               if pool_run else prism.Config.from_workload(w))
         ws = prism.workspace(cfg, dev)
         for _ in range(args.steps):
             prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], ws=ws)
@@ -257,7 +263,8 @@ def run_prism(args, rank, world, dev):
         st, detail = prism.prism_check_device_status(ws)
         if st != 0:
             raise RuntimeError(f"device status {st} {detail}")
-        print(f"profile run: {args.steps} eager steps of {w.name} ({w.n_layers} layers)")
+        print(f"profile run: {args.steps} eager steps of {w.name} ({w.n_layers} layers, "
+              f"{'pool rho %d' % args.pool if pool_run else 'refine'})")
         return
     cfg = prism.Config.from_workload(w)
     ws = prism.workspace(cfg, dev)
@@ -389,6 +396,80 @@ def run_prism(args, rank, world, dev):
                  for f in ("score.cu", "prism_internal.cuh")]
     traffic = kernel_traffic(score_src, os.path.join(ROOT, "profiles", "anchor_score_128k.md"))
 
+    # -- pool mode (the paper's own proposal: Eq. (9) group maximum, Eq. (4)
+    #    pool of rho*kappa tokens, refined layers rescore the anchor's pool)
+    pool = None
+    if args.pool > 0:
+        rho = args.pool
+        cfg_p = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=rho)
+        ws_p = prism.workspace(cfg_p, dev)
+        rp = DecodeStepGraph(cfg_p, inp["q"], inp["k"], inp["v"], inp["lens"], ws=ws_p)
+        for _ in range(max(3, args.warmup)):
+            rp.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(args.steps):
+            rp.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_p = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
+        launches_p = rp.launches
+        del rp
+        st, detail = prism.prism_check_device_status(ws_p)
+        if st != 0:
+            raise RuntimeError(f"device status after the pool-mode step {st} {detail}")
+        cfgpp = ctypes.byref(cfg_p)
+
+        def score_max_launch(l):
+            rc = L.prism_score_anchor(cfgpp, ctypes.c_void_p(inp["q"][l].data_ptr()),
+                                      ctypes.c_void_p(inp["k"][l].data_ptr()),
+                                      ctypes.c_void_p(inp["lens"].data_ptr()),
+                                      ctypes.c_void_p(S.data_ptr()),
+                                      ctypes.c_void_p(ws_p.data_ptr()), ws_p.numel(),
+                                      ctypes.c_void_p(stream.cuda_stream))
+            if rc != 0:
+                raise RuntimeError(f"prism_score_anchor (pool mode): {rc}")
+        for i in range(3):
+            score_max_launch(anchors[i % len(anchors)])
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_k)]
+        for i in range(n_k):
+            evs[i][0].record(stream)
+            score_max_launch(anchors[i % len(anchors)])
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        t_max = statistics.mean(x.elapsed_time(y) for x, y in evs) * 1e-3
+        # MMA work per launch: every key row against the 16 padded head columns
+        tc_flops = 2.0 * sum(int(x) for x in lens_h) * w.n_kv_heads * 16 * w.head_dim
+        cfg_pr = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=rho,
+                                            anchor_mask=[1] + [0] * (N - 1))
+        cfg_p0 = prism.Config.from_workload(w.replace(n_layers=1), mode=prism.MODE_POOL,
+                                            pool_factor=rho)
+        t_pr = graph_ms(cfg_pr, max(5, args.steps // 2))
+        t_p0 = graph_ms(cfg_p0, max(5, args.steps // 2))
+        pool_rows = sum(min(rho * w.kappa, int(x)) for x in lens_h) * w.n_kv_heads
+        p_refine_bytes = pool_rows * w.head_dim * 2 + gather
+        p_refine_us = (t_pr - t_p0) * 1e3 / (N - 1)
+        p_step_bytes = n_anchor * a_bytes + (N - n_anchor) * pool_rows * w.head_dim * 2 + N * gather
+        pool = {
+            "rho": rho, "value": whole_job_us_per_layer(ms_p, N, world), "unit": UNIT,
+            "ms_per_step": ms_p, "launches_per_step": launches_p,
+            "step_hbm": {"algorithmic_bytes": p_step_bytes,
+                         "gbs": p_step_bytes / (ms_p * 1e-3) / 1e9,
+                         "frac": p_step_bytes / (ms_p * 1e-3) / 1e9 / peak},
+            "anchor_kernel": {"kernel": "k_anchor_score_max (tcgen05)", "bound": "hbm",
+                              "achieved": a_bytes / t_max / 1e9, "peak": peak, "unit": "GB/s",
+                              "frac": a_bytes / t_max / 1e9 / peak,
+                              "us_per_launch": t_max * 1e6, "bytes_per_launch": a_bytes,
+                              "tensor_tflops": tc_flops / t_max / 1e12},
+            "refine_attn": {"bytes_per_layer": p_refine_bytes, "us_per_layer": p_refine_us,
+                            "gbs": p_refine_bytes / (p_refine_us * 1e-6) / 1e9,
+                            "frac": p_refine_bytes / (p_refine_us * 1e-6) / 1e9 / peak},
+            "how": "pool mode (Eq. (9) group maximum, rho*kappa pool) on the same workload "
+                   "and inputs, graph-timed like the headline step",
+        }
+
     # -- per-stage breakdown (events around each public stage call)
     def timed(fn, reps=8):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -496,6 +577,7 @@ def run_prism(args, rank, world, dev):
                                    "anchor layer alone, per refined layer; bytes = measured "
                                    "proposal K rows + gathered K/V rows"},
             "breakdown_us": br,
+            "pool_mode": pool,
             "gpu_launches": launches_per_step * args.steps,
             "launches_per_step": launches_per_step,
             "clocks": clk,

@@ -62,6 +62,9 @@ struct Layout {
     size_t ctl_begin, ctl_end;      // [ctl_begin, ctl_end): histograms and counters; zeroed per call
     SlotLayout slot[kSlots];
     size_t attn_ctl;
+    // pool mode: kMaxZ candidate slots of refined layers scored together
+    size_t phist, pS, pcpos, pspill;
+    int cstride;                    // their row stride: rho*kappa (at most Lmax), 4-aligned
     size_t canon, canon_off, idx_all, off_all, pool_all, pool_off_all, pacc, pml, total;
 };
 
@@ -92,7 +95,16 @@ Layout make_layout(const prism_config_t &c) {
         l.slot[s].hist = off;   off = align256(off + rows * kHistBins * sizeof(uint32_t));
     }
     l.attn_ctl = off; off = align256(off + rows * sizeof(RowCtl));
+    const size_t nzs = pool_mode(c) ? (size_t)kMaxZ : 0;
+    l.phist = off;    off = align256(off + nzs * rows * kHistBins * sizeof(uint32_t));
     l.ctl_end = off;
+    {
+        const long long n = (long long)src_kappa_of(c) < c.max_len ? src_kappa_of(c) : c.max_len;
+        l.cstride = (int)((n + 3) & ~3LL);
+    }
+    l.pS = off;       off = align256(off + nzs * rows * (size_t)l.cstride * sizeof(float));
+    l.pcpos = off;    off = align256(off + nzs * rows * (size_t)l.cstride * sizeof(int32_t));
+    l.pspill = off;   off = align256(off + nzs * rows * 2 * (size_t)l.cstride * sizeof(uint64_t));
     for (int s = 0; s < kSlots; ++s) {
         l.slot[s].S = off;    off = align256(off + rows * (size_t)c.max_len * sizeof(float));
         l.slot[s].cpos = off; off = align256(off + (s == kRefineSlot ? rows * (size_t)c.max_len : 1) * sizeof(int32_t));
@@ -171,6 +183,7 @@ int num_sms() {
 // kept until the process exits.
 struct DeviceHelpers {
     cudaStream_t anchor = nullptr, chain = nullptr, attn = nullptr;
+    cudaStream_t aux = nullptr;     // pool mode: the anchors' two selections
     std::vector<cudaEvent_t> events;
 };
 std::mutex g_helpers_mu;
@@ -186,7 +199,8 @@ prism_status_t helpers_for_current_device(size_t n_events, DeviceHelpers **out) 
         // lo is the least urgent priority, hi the most urgent.
         if (cudaStreamCreateWithPriority(&h.anchor, cudaStreamNonBlocking, lo) != cudaSuccess ||
             cudaStreamCreateWithPriority(&h.chain, cudaStreamNonBlocking, hi) != cudaSuccess ||
-            cudaStreamCreateWithPriority(&h.attn, cudaStreamNonBlocking, hi) != cudaSuccess)
+            cudaStreamCreateWithPriority(&h.attn, cudaStreamNonBlocking, hi) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&h.aux, cudaStreamNonBlocking, hi) != cudaSuccess)
             return PRISM_ERR_CUDA;
     }
     while (h.events.size() < n_events) {
@@ -212,6 +226,10 @@ struct Ws {
     int32_t *canon, *canon_off;
     int32_t *idx_all, *off_all;
     int32_t *pool_all, *pool_off_all;     // pool mode: [N][rows][rho*kappa], [N][rows][rho*kappa + 1]
+    uint32_t *phist;                      // pool mode: [kMaxZ][rows][kHistBins]
+    float *pS;                            // pool mode: [kMaxZ][rows][cstride]
+    int32_t *pcpos;                       // pool mode: [kMaxZ][rows][cstride]
+    uint64_t *pspill;                     // pool mode: [kMaxZ][rows][2][cstride]
     float *pacc, *pml;
     uint8_t *base;
     Layout l;
@@ -237,6 +255,10 @@ prism_status_t carve(const prism_config_t &c, void *ws, size_t ws_bytes, Ws *w) 
     w->off_all = reinterpret_cast<int32_t *>(b + w->l.off_all);
     w->pool_all = reinterpret_cast<int32_t *>(b + w->l.pool_all);
     w->pool_off_all = reinterpret_cast<int32_t *>(b + w->l.pool_off_all);
+    w->phist = reinterpret_cast<uint32_t *>(b + w->l.phist);
+    w->pS = reinterpret_cast<float *>(b + w->l.pS);
+    w->pcpos = reinterpret_cast<int32_t *>(b + w->l.pcpos);
+    w->pspill = reinterpret_cast<uint64_t *>(b + w->l.pspill);
     w->pacc = reinterpret_cast<float *>(b + w->l.pacc);
     w->pml = reinterpret_cast<float *>(b + w->l.pml);
     return PRISM_OK;
@@ -315,26 +337,51 @@ prism_status_t run_pool_select(const prism_config_t &c, const Ws &w, int slot, c
                                                  nullptr), s));
 }
 
-// Refined layer: the candidates of the canonical source selection `src` (with
-// its enumeration offsets `src_off`) -- its +-r proposal, or in pool mode the
-// pool itself -- rescored (Eq. (5)), then Eq. (6).
+// Refined layer: +-r proposal around the canonical source selection `src`
+// (with its offsets `src_off`), Eq. (5) on it, Eq. (6).
 prism_status_t run_refine(const prism_config_t &c, const Ws &w, const void *q, const void *k,
                           const int32_t *len, const int32_t *src, const int32_t *src_off,
                           int32_t *idx_out, int32_t *prop_off, cudaStream_t s) {
     const Slot &sl = w.slot[kRefineSlot];
-    const bool pool = pool_mode(c);
     ScoreArgs sa = score_args(c, w, sl, q, k, len);
     sa.src = src;
     sa.src_off = src_off;
-    sa.kappa = src_kappa_of(c);
-    sa.radius = pool ? 0 : c.radius;
     PRISM_CUDA(launch_refine_rescore(sa, num_sms(), s));
-    SelectArgs se = select_args(c, w, sl, sl.S, sl.cpos, src_off, len, idx_out, pool ? nullptr : prop_off);
-    se.src_kappa = src_kappa_of(c);
-    if (pool) {
-        se.radius = 0;
-        se.n_bound = src_kappa_of(c) < c.max_len ? src_kappa_of(c) : c.max_len;
+    return cuda_status(launch_select(select_args(c, w, sl, sl.S, sl.cpos, src_off, len, idx_out,
+                                                 prop_off), s));
+}
+
+// Pool mode: nz (<= kMaxZ) refined layers that share one anchor's pool
+// (`pool`, with its radius-0 enumeration offsets `pool_off`): Eq. (5) on the
+// pool with each layer's own q and K, then Eq. (6), one launch of each kernel
+// for all of them (layer z in grid z).  Selections go to idx_out + z * rows
+// * kappa; the candidates of layer z stay in candidate slot z.
+prism_status_t run_refine_pool(const prism_config_t &c, const Ws &w, const void *const *qs,
+                               const void *const *ks, int nz, const int32_t *len,
+                               const int32_t *pool, const int32_t *pool_off, int32_t *idx_out,
+                               cudaStream_t s) {
+    if (nz < 1 || nz > kMaxZ) return PRISM_ERR_INVALID_ARG;
+    const size_t rows = (size_t)c.batch * c.n_kv_heads;
+    const int cs = w.l.cstride;
+    ScoreArgs sa = score_args(c, w, w.slot[kRefineSlot], qs[0], ks[0], len);
+    sa.S = w.pS; sa.cpos = w.pcpos; sa.hist = w.phist;
+    sa.src = pool; sa.src_off = pool_off;
+    sa.kappa = src_kappa_of(c); sa.radius = 0;
+    sa.nz = nz; sa.cstride = cs;
+    sa.zS = rows * (size_t)cs; sa.zhist = rows * kHistBins;
+    for (int z = 0; z < nz; ++z) {
+        sa.qz[z] = qs[z];
+        sa.kz[z] = ks[z];
     }
+    PRISM_CUDA(launch_refine_rescore(sa, num_sms(), s));
+    SelectArgs se = select_args(c, w, w.slot[kRefineSlot], w.pS, w.pcpos, pool_off, len, idx_out,
+                                nullptr);
+    se.hist = w.phist; se.cspill = w.pspill;
+    se.src_kappa = src_kappa_of(c); se.radius = 0;
+    se.n_bound = cs;
+    se.nz = nz; se.cstride = cs;
+    se.zS = rows * (size_t)cs; se.zhist = rows * kHistBins; se.zspill = rows * 2 * (size_t)cs;
+    se.zout = rows * (size_t)c.kappa;
     return cuda_status(launch_select(se, s));
 }
 
@@ -377,18 +424,26 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     const int NA = (int)anchors.size();
 
     cudaStream_t sA = hp ? hp->anchor : s0, sM = hp ? hp->chain : s0, sC = hp ? hp->attn : s0;
+    cudaStream_t sX = hp ? hp->aux : s0;
     // Events: fork, two joins, per anchor "indexed" and "reached by the chain",
     // per layer "selected".
     cudaEvent_t ev_fork = nullptr, ev_join_m = nullptr, ev_join_c = nullptr;
     const cudaEvent_t *ev_indexed = nullptr, *ev_reached = nullptr, *ev_sel = nullptr;
+    // pool mode: an anchor's scores done, its pool selected, its own top-kappa selected
+    const cudaEvent_t *ev_scored = nullptr, *ev_pool = nullptr, *ev_kdone = nullptr;
+    cudaEvent_t ev_join_x = nullptr;
     if (hp) {
         const cudaEvent_t *e = hp->events.data();
         ev_fork = e[0];
         ev_join_m = e[1];
         ev_join_c = e[2];
-        ev_indexed = e + 3;
+        ev_join_x = e[3];
+        ev_indexed = e + 4;
         ev_reached = ev_indexed + NA;
         ev_sel = ev_reached + NA;
+        ev_scored = ev_sel + N;
+        ev_pool = ev_scored + NA;
+        ev_kdone = ev_pool + NA;
     }
 
     PRISM_TRY(zero_control(w, s0));
@@ -397,11 +452,45 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         PRISM_CUDA(cudaStreamWaitEvent(sA, ev_fork, 0));
         PRISM_CUDA(cudaStreamWaitEvent(sM, ev_fork, 0));
         PRISM_CUDA(cudaStreamWaitEvent(sC, ev_fork, 0));
+        PRISM_CUDA(cudaStreamWaitEvent(sX, ev_fork, 0));
     }
+    // Pool mode with helper streams: the anchor stream only scans (Eq. (9));
+    // the pool and the anchor's own top-kappa are selected on the aux stream,
+    // so that they overlap the next anchor's scan.  Neither selection clears
+    // the slot's histogram; the anchor stream clears it before the slot's
+    // next scan, once both selections of the slot's previous anchor are done.
+    auto index_anchor_pool = [&](int g) -> prism_status_t {
+        const int l = anchors[g];
+        const int slot = g % kAnchorAhead;
+        if (g >= kAnchorAhead) {
+            PRISM_CUDA(cudaStreamWaitEvent(sA, ev_reached[g - kAnchorAhead], 0));
+            PRISM_CUDA(cudaStreamWaitEvent(sA, ev_kdone[g - kAnchorAhead], 0));
+            PRISM_CUDA(cudaMemsetAsync(w.slot[slot].hist, 0, rows * kHistBins * sizeof(uint32_t), sA));
+        }
+        PRISM_TRY(run_anchor_score(c, w, slot, qb + (size_t)l * q_elems, k[l], len, nullptr, sA));
+        PRISM_CUDA(cudaEventRecord(ev_scored[g], sA));
+        PRISM_CUDA(cudaStreamWaitEvent(sX, ev_scored[g], 0));
+        const Slot &sl = w.slot[slot];
+        SelectArgs p = select_args(c, w, sl, sl.S, nullptr, nullptr, len,
+                                   w.pool_all + (size_t)l * pool_elems,
+                                   w.pool_off_all + (size_t)l * pool_off_elems);
+        p.kappa = src_kappa_of(c);
+        p.radius = 0;
+        p.keep_hist = 1;
+        PRISM_CUDA(launch_select(p, sX));
+        PRISM_CUDA(cudaEventRecord(ev_pool[g], sX));
+        SelectArgs t = select_args(c, w, sl, sl.S, nullptr, nullptr, len,
+                                   idx_base + (size_t)l * sel_elems, nullptr);
+        t.keep_hist = 1;
+        PRISM_CUDA(launch_select(t, sX));
+        PRISM_CUDA(cudaEventRecord(ev_kdone[g], sX));
+        return PRISM_OK;
+    };
     // An anchor's scoring and selection depend on nothing but its own q and K,
     // so both run on the anchor stream, kAnchorAhead anchors ahead of the
     // chain of refined layers (the anchor slots form a ring of that size).
     auto index_anchor = [&](int g) -> prism_status_t {
+        if (pool && hp) return index_anchor_pool(g);
         const int l = anchors[g];
         const bool next_refines = refining && l + 1 < N && !is_anchor(l + 1);
         if (hp && g >= kAnchorAhead) PRISM_CUDA(cudaStreamWaitEvent(sA, ev_reached[g - kAnchorAhead], 0));
@@ -426,6 +515,7 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     const int32_t *anchor_sel = nullptr, *anchor_off = nullptr;
     const int32_t *prev_sel = nullptr, *prev_off = nullptr;
     int anchor_layer = 0;
+    int pool_batch_end = 0;     // pool mode: first layer after the batch enqueued last
     int g = 0;
     for (int l = 0; l < N; ++l) {
         const void *ql = qb + (size_t)l * q_elems;
@@ -437,7 +527,7 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         const int32_t *cur = dst, *cur_off = dst_off;
         if (is_anchor(l)) {
             if (hp) {
-                PRISM_CUDA(cudaStreamWaitEvent(sM, ev_indexed[g], 0));
+                PRISM_CUDA(cudaStreamWaitEvent(sM, pool ? ev_pool[g] : ev_indexed[g], 0));
                 PRISM_CUDA(cudaEventRecord(ev_reached[g], sM));
                 if (g + kAnchorAhead < NA) PRISM_TRY(index_anchor(g + kAnchorAhead));
             } else {
@@ -446,12 +536,28 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
             anchor_off = dst_off;
             anchor_sel = dst;
             anchor_layer = l;
+            pool_batch_end = l + 1;
             ++g;
         } else if (pool) {
-            // Eq. (5)-(6) over the nearest preceding anchor's pool.
-            PRISM_TRY(run_refine(c, w, ql, k[l], len, w.pool_all + (size_t)anchor_layer * pool_elems,
-                                 w.pool_off_all + (size_t)anchor_layer * pool_off_elems, dst, nullptr,
-                                 sM));
+            // Eq. (5)-(6) over the nearest preceding anchor's pool.  The
+            // refined layers of a group depend on that pool alone, so up to
+            // kMaxZ of them are rescored and selected by one launch each: the
+            // first layer of a batch enqueues it for the run that follows.
+            if (l == pool_batch_end) {
+                int e = l;
+                while (e < N && !is_anchor(e) && e - l < kMaxZ) ++e;
+                const void *qs[kMaxZ];
+                const void *ks[kMaxZ];
+                for (int z = 0; z < e - l; ++z) {
+                    qs[z] = qb + (size_t)(l + z) * q_elems;
+                    ks[z] = k[l + z];
+                }
+                PRISM_TRY(run_refine_pool(c, w, qs, ks, e - l, len,
+                                          w.pool_all + (size_t)anchor_layer * pool_elems,
+                                          w.pool_off_all + (size_t)anchor_layer * pool_off_elems,
+                                          dst, sM));
+                pool_batch_end = e;
+            }
         } else if (c.mode == PRISM_MODE_STATIC_REUSE) {
             if (idx_out) {
                 PRISM_CUDA(cudaMemcpyAsync(dst, src, sel_elems * sizeof(int32_t),
@@ -468,6 +574,8 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         if (hp) {
             PRISM_CUDA(cudaEventRecord(ev_sel[l], sM));
             PRISM_CUDA(cudaStreamWaitEvent(sC, ev_sel[l], 0));
+            // a pool-mode anchor's own selection comes from the aux stream
+            if (pool && is_anchor(l)) PRISM_CUDA(cudaStreamWaitEvent(sC, ev_kdone[g - 1], 0));
         }
         PRISM_TRY(run_attn(c, w, ql, k[l], v[l], len, cur, c.kappa, c.kappa,
                            ob + (size_t)l * q_elems, sC));
@@ -478,8 +586,10 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         // Every anchor score was waited on by M; join M and C into the caller's stream.
         PRISM_CUDA(cudaEventRecord(ev_join_m, sM));
         PRISM_CUDA(cudaEventRecord(ev_join_c, sC));
+        PRISM_CUDA(cudaEventRecord(ev_join_x, sX));
         PRISM_CUDA(cudaStreamWaitEvent(s0, ev_join_m, 0));
         PRISM_CUDA(cudaStreamWaitEvent(s0, ev_join_c, 0));
+        PRISM_CUDA(cudaStreamWaitEvent(s0, ev_join_x, 0));
     }
     return PRISM_OK;
 }
@@ -577,11 +687,22 @@ prism_status_t prism_index_refine(const prism_config_t *cfg, const void *q, cons
     ca.radius = pool_mode(*cfg) ? 0 : cfg->radius;
     ca.out = w.canon; ca.out_off = w.canon_off; ca.st = w.st;
     PRISM_CUDA(launch_canonicalize(ca, s));
+    if (pool_mode(*cfg)) {
+        const void *qs[1] = {q};
+        const void *ks[1] = {k};
+        PRISM_TRY(run_refine_pool(*cfg, w, qs, ks, 1, len, w.canon, w.canon_off, idx_out, s));
+        if (all)
+            PRISM_CUDA(launch_export_candidates(w.pS, w.pcpos, w.canon_off,
+                                                cfg->batch * cfg->n_kv_heads, w.l.cstride,
+                                                src_kappa_of(*cfg), cand_pos, cand_score,
+                                                cand_count, cand_cap, s));
+        return PRISM_OK;
+    }
     PRISM_TRY(run_refine(*cfg, w, q, k, len, w.canon, w.canon_off, idx_out, nullptr, s));
     if (all)
         PRISM_CUDA(launch_export_candidates(w.slot[kRefineSlot].S, w.slot[kRefineSlot].cpos,
                                             w.canon_off, cfg->batch * cfg->n_kv_heads,
-                                            cfg->max_len, src_kappa_of(*cfg), cand_pos, cand_score,
+                                            cfg->max_len, cfg->kappa, cand_pos, cand_score,
                                             cand_count, cand_cap, s));
     return PRISM_OK;
 }
@@ -657,7 +778,7 @@ prism_status_t prism_decode_step(const prism_config_t *cfg, const void *q, const
     if (c.flags & PRISM_FLAG_SERIAL) return enqueue_step(c, w, q, k, v, len, out, idx_out, s, nullptr);
     std::lock_guard<std::mutex> lock(g_helpers_mu);
     DeviceHelpers *hp = nullptr;
-    PRISM_TRY(helpers_for_current_device(3 + 3 * (size_t)c.n_layers, &hp));
+    PRISM_TRY(helpers_for_current_device(4 + 6 * (size_t)c.n_layers, &hp));
     return enqueue_step(c, w, q, k, v, len, out, idx_out, s, hp);
 }
 

@@ -456,10 +456,20 @@ struct ScoreArgs {
     const int32_t *src_off; // refine: its proposal enumeration offsets [rows][kappa + 1]
     int kappa, radius;      // refine: entries of the source selection, proposal radius
     int agg;                // kAggSum: Eq. (1) group sum; kAggMax: Eq. (9) group maximum
+    // refine: several layers rescoring the same source in one launch (grid z);
+    // layer z reads qz[z] / kz[z] (z = 0: q / k) and writes S, cpos, hist
+    // shifted by z * zS, z * zS, z * zhist.  cstride is the row stride of S
+    // and cpos (0: Lmax).
+    int nz;
+    const void *qz[8];
+    const void *kz[8];
+    int cstride;
+    size_t zS, zhist;
     DevStatus *st;
     uint64_t wait_ns;
 };
 enum : int { kAggSum = 0, kAggMax = 1 };
+constexpr int kMaxZ = 8;           // refined layers batched into one launch
 
 cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s);
 // The group-maximum form of the full-cache scan (tensor cores; score_max.cu).
@@ -486,6 +496,12 @@ struct SelectArgs {
     int src_kappa;             // refine: entries of the source selection (0: kappa)
     int n_bound;               // bound on a row's items, sizes the cluster (0: from kappa, radius)
     int keep_hist;             // nonzero: leave the histogram for another selection of the same scores
+    // refine: nz selections in one launch (grid z), selection z reading S, cpos,
+    // hist, cspill and writing idx_out shifted by z times the strides below;
+    // cstride is the row stride of S, cpos and the two halves of cspill (0: Lmax)
+    int nz;
+    int cstride;
+    size_t zS, zhist, zspill, zout;
     uint32_t *hist;            // [rows][kHistBins], left zeroed (unless keep_hist)
     uint64_t *cspill;          // [rows][2][Lmax] overflow of the CTAs' candidate and tie lists
     int32_t *idx_out;          // [rows][kappa]

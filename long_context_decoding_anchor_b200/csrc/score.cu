@@ -305,9 +305,10 @@ k_refine_rescore(ScoreArgs a) {
     uint64_t *pos_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *pos_empty = pos_full + C::kPosDepth;
     uint32_t *hist_s = reinterpret_cast<uint32_t *>(smem + C::kHistOff);
-    const int row = blockIdx.y, part = blockIdx.x, P = gridDim.x;
+    const int row = blockIdx.y, part = blockIdx.x, P = gridDim.x, z = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = row / a.Hkv, h = row % a.Hkv;
+    const int cstride = a.cstride > 0 ? a.cstride : a.Lmax;
     const int L = load_len(a.len, b, a.Lmax, a.st, kWhereRescore);
     for (int i = tid; i < kHistBins; i += C::kThreads) hist_s[i] = 0;
     if (tid == 0) {
@@ -382,7 +383,7 @@ k_refine_rescore(ScoreArgs a) {
 
     // ---------------- consumers ------------------------------------------------
     const int slice = lane % C::kNL, sub = lane / C::kNL;
-    const uint16_t *qb = static_cast<const uint16_t *>(a.q);
+    const uint16_t *qb = static_cast<const uint16_t *>(z == 0 ? a.q : a.qz[z]);
     const int Hq = a.Hkv * a.G;
     // Group sum: qbar, this lane's 8 elements.  Group maximum: the B fragments
     // of the group's queries (column n of n-tile t is head (8t + n) % G; k
@@ -413,9 +414,9 @@ k_refine_rescore(ScoreArgs a) {
         }
     }
     const bool two_tiles = a.G > 8;
-    const uint16_t *kb = static_cast<const uint16_t *>(a.k) + (size_t)row * a.Lmax * D;
-    float *S = a.S + (size_t)row * a.Lmax;
-    int32_t *cpos = a.cpos + (size_t)row * a.Lmax;
+    const uint16_t *kb = static_cast<const uint16_t *>(z == 0 ? a.k : a.kz[z]) + (size_t)row * a.Lmax * D;
+    float *S = a.S + (size_t)z * a.zS + (size_t)row * cstride;
+    int32_t *cpos = a.cpos + (size_t)z * a.zS + (size_t)row * cstride;
     const int r_base = warp * C::kRowsPerWarp;
     // The row whose score this lane stores, if it is a writer.
     const int r_item = MAXAGG ? r_base + (lane >> 2) + ((lane & 3) == 1 ? 8 : 0)
@@ -487,9 +488,10 @@ k_refine_rescore(ScoreArgs a) {
     cp_async_wait<0>();
     consumer_sync();
     pdl_launch_dependents();
+    uint32_t *hist_g = a.hist + (size_t)z * a.zhist + (size_t)row * kHistBins;
     for (int i = tid; i < kHistBins; i += 32 * C::kConsumerWarps) {
         const uint32_t v = hist_s[i];
-        if (v) atomicAdd(a.hist + (size_t)row * kHistBins + i, v);
+        if (v) atomicAdd(hist_g + i, v);
     }
 }
 
@@ -519,10 +521,12 @@ static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, int num_sms, cuda
     cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D, MAXAGG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    // About one CTA per SM over all rows; each row's proposal is split evenly.
+    // About one CTA per SM over all rows (of all batched layers); each row's
+    // proposal is split evenly.
+    const int nz = a.nz > 1 ? a.nz : 1;
     const int rows = a.B * a.Hkv;
-    const int parts = rows >= num_sms ? 1 : num_sms / rows;
-    return launch_kernel(k_refine_rescore<D, MAXAGG>, dim3((unsigned)parts, (unsigned)rows),
+    const int parts = rows * nz >= num_sms ? 1 : num_sms / (rows * nz);
+    return launch_kernel(k_refine_rescore<D, MAXAGG>, dim3((unsigned)parts, (unsigned)rows, (unsigned)nz),
                          dim3(C::kThreads), C::kSmemBytes, s, a);
 }
 

@@ -10,7 +10,7 @@
 // Persistent grid, one CTA per SM, over the same contiguous tile ranges as the
 // group-sum scan (tiles.cuh).  Warp roles:
 //   warp 0    TMA producer: per tile, two (d = 128) or one 128-row x 64-column
-//             boxes of the key cache with 128-byte swizzle into a 4-stage
+//             boxes of the key cache with 128-byte swizzle into a 3-stage
 //             ring; when the tile's row differs from the stage's last one,
 //             the lanes first write the group's queries (B operand, 16 rows:
 //             the G heads, repeated to fill 16) in the same swizzled layout;
@@ -36,7 +36,10 @@ namespace prism {
 template <int D>
 struct MaxCfg {
     static constexpr int kTileRows = 128;
-    static constexpr int kStages = 4;
+    // Three stages keep the CTA at ~118 KB of shared memory, so that a CTA of
+    // the selection kernel (~107 KB) fits on the same SM: the selections of
+    // one anchor overlap the scan of the next.
+    static constexpr int kStages = 3;
     static constexpr int kBoxes = D / 64;                     // 64 bf16 = one 128-byte row
     static constexpr int kBoxBytes = kTileRows * 128;
     static constexpr int kKBytes = kBoxes * kBoxBytes;

@@ -64,8 +64,10 @@ k_select(SelectArgs a) {
     const int C = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
     const int row = blockIdx.y;
+    const size_t z = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int L = load_len(a.len, row / a.Hkv, a.Lmax, a.st, kWhereFinalize);
+    const int cstride = a.cstride > 0 ? a.cstride : a.Lmax;
     if (tid == 0) {
         sm.fail = 0;
         mbar_init(&sm.bar, 1);
@@ -77,13 +79,14 @@ k_select(SelectArgs a) {
     // letting this grid start), so it may be read before the wait.
     const int src_kappa = a.src_kappa > 0 ? a.src_kappa : a.kappa;
     const int n = refine ? min(min(__ldcg(a.src_off + (size_t)row * (src_kappa + 1) + src_kappa), L), a.Lmax) : L;
-    const float *S = a.S + (size_t)row * a.Lmax;
-    const int32_t *cpos = refine ? a.cpos + (size_t)row * a.Lmax : nullptr;
-    int32_t *out = a.idx_out + (size_t)row * a.kappa;
-    // Overflow areas of the row: candidates beyond kCandCap in the first Lmax
-    // entries, ties beyond kMyTieCap in the second, each at the slice's offset.
-    uint64_t *spill = a.cspill + (size_t)row * 2 * a.Lmax;
-    uint64_t *tie_g = spill + a.Lmax;
+    const float *S = a.S + z * a.zS + (size_t)row * cstride;
+    const int32_t *cpos = refine ? a.cpos + z * a.zS + (size_t)row * cstride : nullptr;
+    int32_t *out = a.idx_out + z * a.zout + (size_t)row * a.kappa;
+    // Overflow areas of the row: candidates beyond kCandCap in the first
+    // cstride entries, ties beyond kMyTieCap in the second, each at the
+    // slice's offset.
+    uint64_t *spill = a.cspill + z * a.zspill + (size_t)row * 2 * cstride;
+    uint64_t *tie_g = spill + cstride;
     const bool all = n <= a.kappa;
     const int i_begin = slice_begin_of(rank, n, C), i_end = slice_begin_of(rank + 1, n, C);
     const int chunk = refine ? kChunkPairs : kChunkScores;
@@ -103,7 +106,7 @@ k_select(SelectArgs a) {
     // 1. the first digit b1 while the slice is in flight
     int b1i = 0, above1 = 0;
     if (!all) {
-        const uint32_t *hg = a.hist + (size_t)row * kHistBins;
+        const uint32_t *hg = a.hist + z * a.zhist + (size_t)row * kHistBins;
         for (int i = tid; i < kHistBins; i += kSelThreads) sm.hist[i] = __ldcg(hg + i);
         __syncthreads();
         threshold_bin(sm, kHistBins, a.kappa, &b1i, &above1);
@@ -179,9 +182,9 @@ k_select(SelectArgs a) {
     x.cand_s = cand_s; x.mytie = mytie; x.tie_all = tie_all; x.sel_s = sel_s;
     x.cand_cap = kCandCap; x.mytie_cap = kMyTieCap; x.tie_cache = kTieCache; x.sel_cache = kSelCache;
     x.spill = spill; x.tie_g = tie_g; x.out = out;
-    x.prop_off = a.prop_off ? a.prop_off + (size_t)row * (a.kappa + 1) : nullptr;
+    x.prop_off = a.prop_off ? a.prop_off + (size_t)row * (a.kappa + 1) : nullptr;   // single layer
     // zeroed for the next use even if unread, unless another selection reads it too
-    x.hist_g = a.keep_hist ? nullptr : a.hist + (size_t)row * kHistBins;
+    x.hist_g = a.keep_hist ? nullptr : a.hist + z * a.zhist + (size_t)row * kHistBins;
     x.st = a.st; x.where = kWhereFinalize;
     select_finish(sm, cluster, x, ncand);
     pdl_launch_dependents();
@@ -214,7 +217,7 @@ cudaError_t launch_select(const SelectArgs &a, cudaStream_t s) {
     const int items = (int)(bound < a.Lmax ? bound : a.Lmax);
     const int C = select_cluster_size(items, refine);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(C, rows);
+    cfg.gridDim = dim3(C, rows, a.nz > 1 ? a.nz : 1);
     cfg.blockDim = dim3(kSelThreads);
     cfg.dynamicSmemBytes = kSelDynSmem;
     cfg.stream = s;

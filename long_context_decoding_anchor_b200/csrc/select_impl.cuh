@@ -292,20 +292,21 @@ static __device__ void select_finish(SelShared &sm, cg::cluster_group &cluster, 
         return t < x.mytie_cap ? cluster.map_shared_rank(x.mytie, r)[t]
                                : __ldcg(x.tie_g + slice_begin_of(r, x.n, C) + t);
     };
-    const bool local_ok = m <= x.tie_cache;
     uint32_t T = 0;
     int cutoff = 0x7fffffff;
     if (!x.all) {
         // The ties' next 11 bits are histogrammed while they are gathered
-        // (the histogram was zeroed before the cluster barrier).
+        // (the histogram was zeroed before the cluster barrier).  The first
+        // tie_cache ties are kept in shared memory; the rest, if any, are
+        // read from their owners again when needed.
         for (int e = tid; e < m; e += nthreads) {
             const uint64_t it = tie_src(e);
-            if (local_ok) x.tie_all[e] = it;
+            if (e < x.tie_cache) x.tie_all[e] = it;
             atomicAdd(&sm.hist[((uint32_t)(it >> 32) >> 10) & 0x7ffu], 1u);
         }
         if (tid == 0) sm.n_small = 0;
         __syncthreads();
-        auto tie_at = [&](int e) -> uint64_t { return local_ok ? x.tie_all[e] : tie_src(e); };
+        auto tie_at = [&](int e) -> uint64_t { return e < x.tie_cache ? x.tie_all[e] : tie_src(e); };
         int b2, above2;
         threshold_bin(sm, kHistBins, x.need1, &b2, &above2);
         const int need2 = x.need1 - above2;
