@@ -452,6 +452,9 @@ def run_prism(args, rank, world, dev):
         p_refine_bytes = pool_rows * w.head_dim * 2 + gather
         p_refine_us = (t_pr - t_p0) * 1e3 / (N - 1)
         p_step_bytes = n_anchor * a_bytes + (N - n_anchor) * pool_rows * w.head_dim * 2 + N * gather
+        max_src = [os.path.join(ROOT, "long_context_decoding_anchor_b200", "csrc", f)
+                   for f in ("score_max.cu", "tc_sm100.cuh", "tiles.cuh", "prism_internal.cuh")]
+        traffic_max = kernel_traffic(max_src, os.path.join(ROOT, "profiles", "anchor_score_max_128k.md"))
         pool = {
             "rho": rho, "value": whole_job_us_per_layer(ms_p, N, world), "unit": UNIT,
             "ms_per_step": ms_p, "launches_per_step": launches_p,
@@ -462,6 +465,7 @@ def run_prism(args, rank, world, dev):
                               "achieved": a_bytes / t_max / 1e9, "peak": peak, "unit": "GB/s",
                               "frac": a_bytes / t_max / 1e9 / peak,
                               "us_per_launch": t_max * 1e6, "bytes_per_launch": a_bytes,
+                              "traffic": traffic_max,
                               "tensor_tflops": tc_flops / t_max / 1e12},
             "refine_attn": {"bytes_per_layer": p_refine_bytes, "us_per_layer": p_refine_us,
                             "gbs": p_refine_bytes / (p_refine_us * 1e-6) / 1e9,
