@@ -17,7 +17,7 @@
  *  - Pointers named q, k, v, out, idx*, cand*, len, ws are DEVICE pointers on
  *    the current CUDA device; the caller owns every buffer.  The library
  *    allocates no device memory.  Between calls it keeps only per-device
- *    caches: the SM count, and (for prism_decode_step) three helper streams
+ *    caches: the SM count, and (for prism_decode_step) four helper streams
  *    and a pool of events, created on first use and kept until exit.
  *  - Layouts (row-major, no padding between rows):
  *      q    bf16 [B][Hq][d]            one decode query per sequence

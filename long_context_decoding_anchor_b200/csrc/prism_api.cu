@@ -13,8 +13,10 @@
 //                      each anchor's group waiting for that anchor's selection;
 //   C (high priority): each layer's sparse attention once its selection is
 //                      done.
-// In pool mode the anchor stream also selects each anchor's pool, and every
-// refined layer rescores its anchor's pool instead of a +-r proposal.
+// In pool mode a fourth stream X (high priority) selects each anchor's pool
+// and its own top-kappa while A scans the next anchor, and the refined layers
+// of each group rescore their anchor's pool together (one launch of each
+// kernel per group) once the pool is selected.
 // PRISM_FLAG_SERIAL runs everything on the caller's stream instead.
 #include <cuda_runtime.h>
 
