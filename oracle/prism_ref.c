@@ -309,6 +309,10 @@ void prism_ref_attention(int d, int G, const uint16_t *q_group,
  * chain 0: the source selection is the previous layer's final selection.
  * chain 1: the source selection is the most recent anchor layer's selection
  *          (the anchor-rooted association f(S) of Algorithm 1).
+ * Layer kinds (anchor_mask[l], ignored in mode 2): 1 = anchor (F), 0 = the
+ * mode's other layer (R: refined; static reuse in mode 1), 2 = shared (S,
+ * Table 9): the layer keeps the previous layer's final selection, i.e. the
+ * selection of its nearest preceding F or R layer, with no rescoring.
  * Every layer then attends over its own selection (SparseAttn).
  *
  * q      : [N][B][Hq][d] bf16 bits;  k[l], v[l]: [B][Hkv][Lmax][d] bf16 bits
@@ -333,7 +337,11 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
         chain < 0 || chain > 1)
         return -1;
     if (mode == 3 && (rho < 1 || (long long)rho * kappa > 0x7fffffffLL)) return -1;
-    if (mode != 2 && !anchor_mask[0]) return -1;
+    if (mode != 2) {
+        if (anchor_mask[0] != 1) return -1;
+        for (int l = 0; l < n_layers; ++l)
+            if (anchor_mask[l] > 2) return -1;
+    }
     for (int b = 0; b < B; ++b)
         if (len[b] < 0 || len[b] > Lmax) return -1;
 
@@ -354,7 +362,8 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
     }
 
     for (int l = 0; l < n_layers; ++l) {
-        const int is_anchor = (mode == 2) || anchor_mask[l];
+        const int is_anchor = (mode == 2) || anchor_mask[l] == 1;
+        const int is_shared = (mode != 2) && anchor_mask[l] == 2;
         int src_layer = l - 1;
 #if PRISM_REF_PLANT == 10
         src_layer = last_anchor;               /* planted: ignores the chain choice */
@@ -363,6 +372,12 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
 #endif
         int32_t *sel_l = idx_out + (size_t)l * (size_t)rows * row_sel;
         const int32_t *sel_src = (l > 0) ? idx_out + (size_t)src_layer * (size_t)rows * row_sel : NULL;
+        /* the previous layer's final selection (what a shared layer keeps) */
+#if PRISM_REF_PLANT == 16
+        const int32_t *sel_prev = (l > 0) ? idx_out + (size_t)last_anchor * (size_t)rows * row_sel : NULL;   /* planted: the anchor's */
+#else
+        const int32_t *sel_prev = (l > 0) ? idx_out + (size_t)(l - 1) * (size_t)rows * row_sel : NULL;
+#endif
 
 #pragma omp parallel for schedule(dynamic, 1)
         for (int row = 0; row < rows; ++row) {
@@ -373,7 +388,14 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
             const uint16_t *vr = v[l] + ((size_t)b * Hkv + h) * (size_t)Lmax * (size_t)d;
             int32_t *sel = sel_l + (size_t)row * row_sel;
 
-            if (mode == 3) {
+            if (is_shared) {
+                memcpy(sel, sel_prev + (size_t)row * row_sel, sizeof(int32_t) * row_sel);
+                if (mode == 3 && pool_out) {
+                    int32_t *po = pool_out + ((size_t)l * rows + row) * (size_t)rho * (size_t)kappa;
+                    const int32_t *C = pool + (size_t)row * (size_t)n_pool;
+                    for (long e = 0; e < (long)rho * kappa; ++e) po[e] = e < n_pool ? C[e] : -1;
+                }
+            } else if (mode == 3) {
                 int32_t *C = pool + (size_t)row * (size_t)n_pool;
                 if (is_anchor) {
                     /* Eq. (9) over the whole cache, then the pool of Eq. (4) */

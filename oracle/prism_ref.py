@@ -143,6 +143,7 @@ class Oracle:
         for t in ks + vs:
             assert t.shape == (B, Hkv, Lmax, d)
         lens = np.ascontiguousarray(lens, dtype=np.int32)
+        # layer kinds: 1 anchor (F), 0 refined (R), 2 shared (S)
         mask = np.ascontiguousarray(np.asarray(anchor_mask, dtype=np.uint8))
         assert mask.shape[0] == N
         if scale is None:
@@ -200,6 +201,7 @@ PLANTS = {
     13: "the anchor's pool holds kappa tokens instead of rho*kappa",
     14: "pool-mode refined layers rescore the previous selection, not the pool",
     15: "the anchor attends to the pool's first kappa positions, not its best kappa",
+    16: "shared layers keep the anchor's selection, not the previous layer's",
 }
 
 __all__ = ["Oracle", "load", "bf16_bits", "PLANTS", "MODE_REFINE", "MODE_STATIC_REUSE",

@@ -180,6 +180,10 @@ def pin_decode_hand(o):
         _, idx = o.decode_step(q, ks, vs, lens, g["kappa"], g["r"], g["anchor_mask"],
                                mode=mode, chain=chain, scale=g["scale"])
         assert idx[:, 0, 0, :].tolist() == g["expected"][name], f"hand decode {name}"
+    # shared (S) layers, Table 9: mask value 2
+    for name, kinds in (("refine_prev_FSR", [1, 2, 0]), ("refine_prev_FRS", [1, 0, 2])):
+        _, idx = o.decode_step(q, ks, vs, lens, g["kappa"], g["r"], kinds, scale=g["scale"])
+        assert idx[:, 0, 0, :].tolist() == g["expected"][name], f"hand decode {name}"
 
 
 def small_workloads():
@@ -202,24 +206,28 @@ def _bits(inp):
     return q, ks, vs, inp["lens"].cpu().numpy().astype(np.int32)
 
 
-def _numpy_chain(w, q, ks, lens, mode, chain, r):
+def _numpy_chain(w, q, ks, lens, mode, chain, r, mask=None):
     """The decode step's selections recomputed with numpy: einsum scores,
-    lexsort top-kappa, set-based proposal."""
+    lexsort top-kappa, set-based proposal.  Layer kinds: 1 anchor, 0 refined,
+    2 shared (keeps the previous layer's selection)."""
     N, B, Hq, d = q.shape
     H, G = w.n_kv_heads, w.group
     scale = 1.0 / math.sqrt(d)
-    mask = w.anchor_mask()
+    mask = w.anchor_mask() if mask is None else mask
     idx = np.zeros((N, B, H, w.kappa), dtype=np.int64)
     last_anchor = 0
     for l in range(N):
-        anchor = mode == MODE_DENSE_ANCHOR or mask[l]
+        anchor = mode == MODE_DENSE_ANCHOR or mask[l] == 1
+        shared = mode != MODE_DENSE_ANCHOR and mask[l] == 2
         src = last_anchor if chain == CHAIN_ANCHOR else l - 1
         for b in range(B):
             L = int(lens[b])
             for h in range(H):
                 qg = q[l, b, h * G:(h + 1) * G]
                 kr = ks[l][b, h, :L]
-                if anchor:
+                if shared:
+                    idx[l, b, h] = idx[l - 1, b, h]
+                elif anchor:
                     idx[l, b, h] = lexsort_topk(numpy_scores(qg, kr, scale), w.kappa)
                 elif mode == MODE_STATIC_REUSE:
                     idx[l, b, h] = idx[src, b, h]
@@ -346,6 +354,10 @@ def pin_pool_hand(o):
     assert idx[:, 0, 0].tolist() == g["expected"]["selection_rho1"], "hand pool, rho = 1"
     _, idx, _ = o.decode_step(q, ks, vs, lens, g["kappa"], 0, [1, 1, 1], rho=g["rho"], **kw)
     assert idx[:, 0, 0].tolist() == g["expected"]["selection_all_anchors"], "hand pool, all anchors"
+    for name, kinds in (("selection_FRS", [1, 0, 2]), ("selection_FSR", [1, 2, 0])):
+        _, idx, pool = o.decode_step(q, ks, vs, lens, g["kappa"], 0, kinds, rho=g["rho"], **kw)
+        assert idx[:, 0, 0].tolist() == g["expected"][name], f"hand pool {name}"
+        assert pool[:, 0, 0].tolist() == g["expected"]["pool"], f"hand pool {name}: pools"
 
 
 def _numpy_pool_chain(w, q, ks, lens, rho, mask=None):
@@ -366,7 +378,10 @@ def _numpy_pool_chain(w, q, ks, lens, rho, mask=None):
             for h in range(H):
                 qg = q[l, b, h * G:(h + 1) * G]
                 kr = ks[l][b, h, :L]
-                if mask[l]:
+                if mask[l] == 2:
+                    pool[l, b, h] = pool[l - 1, b, h]
+                    idx[l, b, h] = idx[l - 1, b, h]
+                elif mask[l] == 1:
                     s = numpy_scores_max(qg, kr, scale)
                     pool[l, b, h] = lexsort_topk(s, n)
                     C = pool[l, b, h][pool[l, b, h] >= 0]
@@ -446,12 +461,66 @@ def pin_pool_invariants(o):
                     "pool-mode output vs SDPA"
 
 
+# Table 9 layer kinds -- 'F' anchor (1), 'R' refined (0), 'S' shared (2) --
+# the 10F11R57S hybrid pattern of the paper's GLM experiment (78 layers)
+TABLE9_10F11R57S = ("FFRSSSRSSSRSSSFSSSFSSSRSSSFSSSRSSSFSSSRSSSFSSSRSSSRSSSRSSSRSSSFSSSRSSSFSSSFSSS")
+KIND = {"F": 1, "R": 0, "S": 2}
+
+
+def kinds_of(pattern):
+    return [KIND[c] for c in pattern]
+
+
+def pin_shared_numpy(o):
+    """Patterns mixing F, R and S layers, in refine and pool modes, equal the
+    numpy recomputations; Table 9's 78-layer hybrid pattern on a small row."""
+    rng = np.random.default_rng(22)
+    w = small_workloads()[1].replace(n_layers=8)
+    q, ks, vs, lens = _bits(synth.make_inputs(w))
+    for trial in range(3):
+        kinds = [1] + [int(x) for x in rng.integers(0, 3, w.n_layers - 1)]
+        for chain in (CHAIN_PREV, CHAIN_ANCHOR):
+            _, idx = o.decode_step(q, ks, vs, lens, w.kappa, w.radius, kinds, chain=chain)
+            ref = _numpy_chain(w, q, ks, lens, MODE_REFINE, chain, w.radius, mask=kinds)
+            assert np.array_equal(idx, ref), f"refine F/R/S chain vs numpy {kinds}"
+        _, idx, pool = o.decode_step(q, ks, vs, lens, w.kappa, 0, kinds, mode=MODE_POOL, rho=2,
+                                     want_pool=True)
+        ref_idx, ref_pool = _numpy_pool_chain(w, q, ks, lens, 2, mask=kinds)
+        assert np.array_equal(idx, ref_idx) and np.array_equal(pool, ref_pool), \
+            f"pool F/R/S chain vs numpy {kinds}"
+    # the paper's hybrid pattern, 78 layers, on a tiny row
+    wt = small_workloads()[2].replace(n_layers=len(TABLE9_10F11R57S), max_len=48, kappa=4)
+    q, ks, vs, lens = _bits(synth.make_inputs(wt))
+    kinds = kinds_of(TABLE9_10F11R57S)
+    _, idx, _ = o.decode_step(q, ks, vs, lens, wt.kappa, 0, kinds, mode=MODE_POOL, rho=4,
+                              want_pool=True)
+    ref_idx, _ = _numpy_pool_chain(wt, q, ks, lens, 4, mask=kinds)
+    assert np.array_equal(idx, ref_idx), "Table 9 pattern vs numpy"
+
+
+def pin_shared_invariants(o):
+    """An anchor followed only by shared layers is static reuse (Eq. (3)); a
+    shared layer never changes the selection it follows."""
+    w = small_workloads()[1]
+    q, ks, vs, lens = _bits(synth.make_inputs(w))
+    N = w.n_layers
+    mask = w.anchor_mask()
+    shared = [1 if m else 2 for m in mask]
+    _, st = o.decode_step(q, ks, vs, lens, w.kappa, w.radius, mask, mode=MODE_STATIC_REUSE)
+    _, idx = o.decode_step(q, ks, vs, lens, w.kappa, w.radius, shared)
+    assert np.array_equal(idx, st), "F then S equals static reuse"
+    # pool mode scores by the group maximum: its static reuse is rho = 1
+    _, st_max = o.decode_step(q, ks, vs, lens, w.kappa, 0, mask, mode=MODE_POOL, rho=1)
+    _, idx = o.decode_step(q, ks, vs, lens, w.kappa, 0, shared, mode=MODE_POOL, rho=2)
+    assert np.array_equal(idx, st_max), "F then S equals rho = 1 in pool mode"
+
+
 ALL_PINS = [pin_score_bruteforce, pin_score_hand, pin_topk_golden, pin_topk_lexsort,
             pin_topk_all_equal, pin_topk_subsets, pin_expand_golden, pin_expand_bruteforce,
             pin_attention_sdpa, pin_attention_closed_forms, pin_decode_hand,
             pin_decode_numpy_chain, pin_decode_outputs_sdpa, pin_decode_invariants,
             pin_score_max_bruteforce, pin_score_max_hand, pin_pool_hand, pin_pool_numpy_chain,
-            pin_pool_invariants]
+            pin_pool_invariants, pin_shared_numpy, pin_shared_invariants]
 
 __all__ = ["ALL_PINS", "small_workloads"] + [p.__name__ for p in ALL_PINS]
 _ = torch  # torch is used through helpers.sdpa_group and synth

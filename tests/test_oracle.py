@@ -43,6 +43,10 @@ def test_decode_step_rejects_bad_arguments(oracle):
         oracle.decode_step(q, k, k, np.array([17], np.int32), 4, 1, [1, 0])   # len > Lmax
     with pytest.raises(ValueError):
         oracle.decode_step(q, k, k, lens, 4, -1, [1, 0])         # negative radius
+    with pytest.raises(ValueError):
+        oracle.decode_step(q, k, k, lens, 4, 1, [2, 0])          # layer 0 shared
+    with pytest.raises(ValueError):
+        oracle.decode_step(q, k, k, lens, 4, 1, [1, 3])          # unknown layer kind
     out, idx = oracle.decode_step(q, k, k, np.array([0], np.int32), 4, 1, [1, 0])
     assert np.all(idx == -1) and np.all(out == 0.0), "empty context: nothing selected"
 
