@@ -114,10 +114,15 @@ typedef struct {
     int32_t kappa;          /* sparse budget, 1 <= kappa <= PRISM_MAX_LEN     */
     int32_t radius;         /* proposal radius r >= 0                         */
     int32_t n_layers;       /* N >= 1 for prism_decode_step, <= PRISM_MAX_LAYERS */
-    const uint8_t *anchor_mask; /* HOST array [N]; nonzero = anchor layer;
-                                   mask[0] must be nonzero unless DENSE_ANCHOR
-                                   (prism_decode_step only; may be NULL for the
-                                   single-stage calls)                        */
+    const uint8_t *anchor_mask; /* HOST array [N] of layer kinds (Table 9's F/R/S):
+                                   1 = anchor (F), 0 = refined (R; a reuse layer
+                                   in STATIC_REUSE), 2 = shared (S: keeps the
+                                   previous layer's selection, i.e. that of the
+                                   nearest preceding F or R layer, with no
+                                   rescoring); other values are invalid.
+                                   mask[0] must be 1 unless DENSE_ANCHOR, which
+                                   ignores the array.  prism_decode_step only;
+                                   may be NULL for the single-stage calls.    */
     int32_t mode;           /* prism_mode_t                                   */
     int32_t chain;          /* prism_chain_t                                  */
     float scale;            /* score/logit scale; 0 means 1/sqrt(d)           */

@@ -25,6 +25,7 @@ LIB_PATH = os.path.join(_PKG, "libprism.so")
 
 MODE_REFINE, MODE_STATIC_REUSE, MODE_DENSE_ANCHOR, MODE_POOL = 0, 1, 2, 3
 CHAIN_PREV, CHAIN_ANCHOR = 0, 1
+LAYER_REFINED, LAYER_ANCHOR, LAYER_SHARED = 0, 1, 2
 FLAG_SERIAL = 1
 STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED",
           3: "PRISM_ERR_WORKSPACE", 4: "PRISM_ERR_CUDA", 5: "PRISM_ERR_TIMEOUT",
@@ -60,7 +61,8 @@ class Config(ctypes.Structure):
         c = cls(batch, n_q_heads, n_kv_heads, head_dim, max_len, kappa, radius, n_layers,
                 None, mode, chain, scale, flags, pool_factor)
         if anchor_mask is not None:
-            arr = (ctypes.c_uint8 * len(anchor_mask))(*[1 if x else 0 for x in anchor_mask])
+            # layer kinds: 1 anchor (F), 0 refined (R), 2 shared (S)
+            arr = (ctypes.c_uint8 * len(anchor_mask))(*[int(x) for x in anchor_mask])
             c._mask_keepalive = arr
             c.anchor_mask = ctypes.cast(arr, ctypes.POINTER(ctypes.c_uint8))
         return c
@@ -342,4 +344,4 @@ __all__ = ["Config", "PrismError", "lib", "workspace", "prism_workspace_size",
            "prism_index_anchor", "prism_index_pool", "prism_index_refine", "prism_sparse_decode",
            "prism_decode_step", "prism_check_device_status", "prism_debug_wait_timeout",
            "prism_score_anchor", "prism_sparse_decode_noalloc", "raw_status", "MODE_REFINE", "MODE_STATIC_REUSE", "MODE_DENSE_ANCHOR", "MODE_POOL",
-           "CHAIN_PREV", "CHAIN_ANCHOR", "FLAG_SERIAL", "EXPORTS", "LIB_PATH"]
+           "CHAIN_PREV", "CHAIN_ANCHOR", "LAYER_REFINED", "LAYER_ANCHOR", "LAYER_SHARED", "FLAG_SERIAL", "EXPORTS", "LIB_PATH"]

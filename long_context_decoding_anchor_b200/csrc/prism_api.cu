@@ -356,11 +356,11 @@ prism_status_t run_refine(const prism_config_t &c, const Ws &w, const void *q, c
 // Pool mode: nz (<= kMaxZ) refined layers that share one anchor's pool
 // (`pool`, with its radius-0 enumeration offsets `pool_off`): Eq. (5) on the
 // pool with each layer's own q and K, then Eq. (6), one launch of each kernel
-// for all of them (layer z in grid z).  Selections go to idx_out + z * rows
-// * kappa; the candidates of layer z stay in candidate slot z.
+// for all of them (layer z in grid z).  Layer z's selection goes to outs[z];
+// its candidates stay in candidate slot z.
 prism_status_t run_refine_pool(const prism_config_t &c, const Ws &w, const void *const *qs,
-                               const void *const *ks, int nz, const int32_t *len,
-                               const int32_t *pool, const int32_t *pool_off, int32_t *idx_out,
+                               const void *const *ks, int32_t *const *outs, int nz,
+                               const int32_t *len, const int32_t *pool, const int32_t *pool_off,
                                cudaStream_t s) {
     if (nz < 1 || nz > kMaxZ) return PRISM_ERR_INVALID_ARG;
     const size_t rows = (size_t)c.batch * c.n_kv_heads;
@@ -376,14 +376,14 @@ prism_status_t run_refine_pool(const prism_config_t &c, const Ws &w, const void 
         sa.kz[z] = ks[z];
     }
     PRISM_CUDA(launch_refine_rescore(sa, num_sms(), s));
-    SelectArgs se = select_args(c, w, w.slot[kRefineSlot], w.pS, w.pcpos, pool_off, len, idx_out,
+    SelectArgs se = select_args(c, w, w.slot[kRefineSlot], w.pS, w.pcpos, pool_off, len, outs[0],
                                 nullptr);
     se.hist = w.phist; se.cspill = w.pspill;
     se.src_kappa = src_kappa_of(c); se.radius = 0;
     se.n_bound = cs;
     se.nz = nz; se.cstride = cs;
     se.zS = rows * (size_t)cs; se.zhist = rows * kHistBins; se.zspill = rows * 2 * (size_t)cs;
-    se.zout = rows * (size_t)c.kappa;
+    for (int z = 0; z < nz; ++z) se.outz[z] = outs[z];
     return cuda_status(launch_select(se, s));
 }
 
@@ -419,7 +419,11 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     const bool pool = pool_mode(c);
     const size_t pool_elems = rows * (size_t)src_kappa_of(c);
     const size_t pool_off_elems = rows * ((size_t)src_kappa_of(c) + 1);
-    auto is_anchor = [&](int l) { return c.mode == PRISM_MODE_DENSE_ANCHOR || c.anchor_mask[l] != 0; };
+    // Layer kinds: 1 anchor (F), 0 the mode's other layer (R), 2 shared (S,
+    // Table 9: keeps the previous layer's selection).
+    auto kind_of = [&](int l) { return c.mode == PRISM_MODE_DENSE_ANCHOR ? 1 : (int)c.anchor_mask[l]; };
+    auto is_anchor = [&](int l) { return kind_of(l) == 1; };
+    auto is_shared = [&](int l) { return kind_of(l) == 2; };
     std::vector<int> anchors;
     for (int l = 0; l < N; ++l)
         if (is_anchor(l)) anchors.push_back(l);
@@ -517,7 +521,7 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     const int32_t *anchor_sel = nullptr, *anchor_off = nullptr;
     const int32_t *prev_sel = nullptr, *prev_off = nullptr;
     int anchor_layer = 0;
-    int pool_batch_end = 0;     // pool mode: first layer after the batch enqueued last
+    std::vector<char> batched(pool ? (size_t)N : 0, 0);   // pool mode: refined layers enqueued
     int g = 0;
     for (int l = 0; l < N; ++l) {
         const void *ql = qb + (size_t)l * q_elems;
@@ -538,27 +542,39 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
             anchor_off = dst_off;
             anchor_sel = dst;
             anchor_layer = l;
-            pool_batch_end = l + 1;
             ++g;
+        } else if (is_shared(l)) {
+            // Table 9's shared layer: the previous layer's selection, unchanged
+            // (and still described by the previous layer's proposal offsets).
+            if (idx_out) {
+                PRISM_CUDA(cudaMemcpyAsync(dst, prev_sel, sel_elems * sizeof(int32_t),
+                                           cudaMemcpyDeviceToDevice, sM));
+            } else {
+                cur = prev_sel;
+            }
+            cur_off = prev_off;
         } else if (pool) {
             // Eq. (5)-(6) over the nearest preceding anchor's pool.  The
             // refined layers of a group depend on that pool alone, so up to
-            // kMaxZ of them are rescored and selected by one launch each: the
-            // first layer of a batch enqueues it for the run that follows.
-            if (l == pool_batch_end) {
-                int e = l;
-                while (e < N && !is_anchor(e) && e - l < kMaxZ) ++e;
+            // kMaxZ of them (skipping shared layers) are rescored and selected
+            // by one launch each, enqueued at the first of them.
+            if (!batched[l]) {
                 const void *qs[kMaxZ];
                 const void *ks[kMaxZ];
-                for (int z = 0; z < e - l; ++z) {
-                    qs[z] = qb + (size_t)(l + z) * q_elems;
-                    ks[z] = k[l + z];
+                int32_t *outs[kMaxZ];
+                int nz = 0;
+                for (int e = l; e < N && !is_anchor(e) && nz < kMaxZ; ++e) {
+                    if (is_shared(e)) continue;
+                    qs[nz] = qb + (size_t)e * q_elems;
+                    ks[nz] = k[e];
+                    outs[nz] = idx_base + (size_t)e * sel_elems;
+                    batched[e] = 1;
+                    ++nz;
                 }
-                PRISM_TRY(run_refine_pool(c, w, qs, ks, e - l, len,
+                PRISM_TRY(run_refine_pool(c, w, qs, ks, outs, nz, len,
                                           w.pool_all + (size_t)anchor_layer * pool_elems,
                                           w.pool_off_all + (size_t)anchor_layer * pool_off_elems,
-                                          dst, sM));
-                pool_batch_end = e;
+                                          sM));
             }
         } else if (c.mode == PRISM_MODE_STATIC_REUSE) {
             if (idx_out) {
@@ -692,7 +708,8 @@ prism_status_t prism_index_refine(const prism_config_t *cfg, const void *q, cons
     if (pool_mode(*cfg)) {
         const void *qs[1] = {q};
         const void *ks[1] = {k};
-        PRISM_TRY(run_refine_pool(*cfg, w, qs, ks, 1, len, w.canon, w.canon_off, idx_out, s));
+        int32_t *outs[1] = {idx_out};
+        PRISM_TRY(run_refine_pool(*cfg, w, qs, ks, outs, 1, len, w.canon, w.canon_off, s));
         if (all)
             PRISM_CUDA(launch_export_candidates(w.pS, w.pcpos, w.canon_off,
                                                 cfg->batch * cfg->n_kv_heads, w.l.cstride,
@@ -766,7 +783,10 @@ prism_status_t prism_decode_step(const prism_config_t *cfg, const void *q, const
     const prism_config_t &c = *cfg;
     if (c.n_layers < 1 || !q || !k || !v || !len || !out) return PRISM_ERR_INVALID_ARG;
     if (c.mode != PRISM_MODE_DENSE_ANCHOR) {
-        if (!c.anchor_mask || !c.anchor_mask[0]) return PRISM_ERR_INVALID_ARG;
+        // layer kinds: 0 refined, 1 anchor, 2 shared; layer 0 is an anchor
+        if (!c.anchor_mask || c.anchor_mask[0] != 1) return PRISM_ERR_INVALID_ARG;
+        for (int l = 0; l < c.n_layers; ++l)
+            if (c.anchor_mask[l] > 2) return PRISM_ERR_INVALID_ARG;
     }
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(len, 4) ||
         (idx_out && !aligned(idx_out, 4)))

@@ -497,11 +497,13 @@ struct SelectArgs {
     int n_bound;               // bound on a row's items, sizes the cluster (0: from kappa, radius)
     int keep_hist;             // nonzero: leave the histogram for another selection of the same scores
     // refine: nz selections in one launch (grid z), selection z reading S, cpos,
-    // hist, cspill and writing idx_out shifted by z times the strides below;
-    // cstride is the row stride of S, cpos and the two halves of cspill (0: Lmax)
+    // hist, cspill shifted by z times the strides below and writing outz[z]
+    // (nz > 1; idx_out otherwise); cstride is the row stride of S, cpos and
+    // the two halves of cspill (0: Lmax)
     int nz;
     int cstride;
-    size_t zS, zhist, zspill, zout;
+    size_t zS, zhist, zspill;
+    int32_t *outz[8];
     uint32_t *hist;            // [rows][kHistBins], left zeroed (unless keep_hist)
     uint64_t *cspill;          // [rows][2][Lmax] overflow of the CTAs' candidate and tie lists
     int32_t *idx_out;          // [rows][kappa]

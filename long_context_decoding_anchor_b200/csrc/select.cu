@@ -81,7 +81,7 @@ k_select(SelectArgs a) {
     const int n = refine ? min(min(__ldcg(a.src_off + (size_t)row * (src_kappa + 1) + src_kappa), L), a.Lmax) : L;
     const float *S = a.S + z * a.zS + (size_t)row * cstride;
     const int32_t *cpos = refine ? a.cpos + z * a.zS + (size_t)row * cstride : nullptr;
-    int32_t *out = a.idx_out + z * a.zout + (size_t)row * a.kappa;
+    int32_t *out = (a.nz > 1 ? a.outz[z] : a.idx_out) + (size_t)row * a.kappa;
     // Overflow areas of the row: candidates beyond kCandCap in the first
     // cstride entries, ties beyond kMyTieCap in the second, each at the
     // slice's offset.

@@ -197,8 +197,15 @@ def layerwise_step_check(o, cfg, inp, out, idx_all, rows=None, stats=None, layer
     last_anchor = 0
     pool = None
     for l in range(N):
-        anchor = cfg.mode == prism.MODE_DENSE_ANCHOR or mask[l]
+        anchor = cfg.mode == prism.MODE_DENSE_ANCHOR or mask[l] == 1
+        shared = cfg.mode != prism.MODE_DENSE_ANCHOR and mask[l] == 2
         q, k, v, lens = inp["q"][l], inp["k"][l], inp["v"][l], inp["lens"]
+        if shared:
+            # Table 9's shared layer keeps the previous layer's selection
+            assert torch.equal(idx_all[l], idx_all[l - 1]), f"layer {l}: shared layer changed"
+            if layers is None or l in layers:
+                check_attention(o, cfg, q, k, v, lens, idx_all[l], out[l], rows, stats)
+            continue
         if cfg.mode == prism.MODE_POOL:
             # The pool of an anchor is not an output of the step: the stage
             # call reproduces it (bit-exact, as the selections show).

@@ -159,6 +159,10 @@ def test_decode_step_argument_validation(L):
     assert f(ctypes.byref(c), A16, kp, kp, A4, A16, None, ws, ws_n, None) == 1
     c = _cfg(anchor_mask=None)
     assert f(ctypes.byref(c), A16, kp, kp, A4, A16, None, ws, ws_n, None) == 1  # mask required
+    c = _cfg(anchor_mask=[2, 0, 0, 0])
+    assert f(ctypes.byref(c), A16, kp, kp, A4, A16, None, ws, ws_n, None) == 1  # layer 0 shared
+    c = _cfg(anchor_mask=[1, 0, 3, 0])
+    assert f(ctypes.byref(c), A16, kp, kp, A4, A16, None, ws, ws_n, None) == 1  # unknown kind
 
 
 def test_debug_wait_validation(L):

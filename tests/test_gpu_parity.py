@@ -298,3 +298,54 @@ def test_pool_dag_matches_serial_and_graph(oracle):
     assert torch.equal(idx_g, idx_d) and torch.equal(g.out, out_d)
     st, detail = prism.prism_check_device_status(g.ws)
     assert st == 0, detail
+
+
+# -- Table 9's F/R/S layer kinds (shared layers keep the previous selection) --
+from pins import TABLE9_10F11R57S, kinds_of   # noqa: E402
+
+
+@pytest.mark.parametrize("mode", [prism.MODE_REFINE, prism.MODE_POOL])
+def test_frs_pattern(oracle, mode):
+    pattern = "FRSSRSFSRSRR"
+    w = synth.WORKLOADS[2].replace(max_len=6000, n_layers=len(pattern), kappa=256, n_clusters=16)
+    inp = _inputs(w)
+    inp["anchor_mask"] = kinds_of(pattern)
+    cfg = prism.Config.from_workload(w, mode=mode, pool_factor=4, anchor_mask=kinds_of(pattern))
+    out, idx = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                       want_idx=True)
+    layerwise_step_check(oracle, cfg, inp, out, idx)
+    from oracle import bf16_bits
+    _, ref_idx = oracle.decode_step(bf16_bits(inp["q"]), [bf16_bits(t) for t in inp["k"]],
+                                    [bf16_bits(t) for t in inp["v"]], inp["lens"].cpu().numpy(),
+                                    w.kappa, w.radius, kinds_of(pattern), mode=mode, rho=4)
+    gi = idx.cpu().numpy()
+    for l in range(w.n_layers):
+        for h in range(w.n_kv_heads):
+            assert recall(gi[l, 0, h], ref_idx[l, 0, h]) >= 0.999, (l, h)
+    # the same selections without idx_out (shared layers then alias their source)
+    out_b = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"])
+    assert torch.equal(out, out_b)
+
+
+def test_table9_hybrid_pattern_pool(oracle):
+    """The paper's 78-layer 10F11R57S pattern in pool mode (rho 4) on a short
+    context: every layer checked against the oracle, DAG = serial = graph."""
+    from long_context_decoding_anchor_b200.runner import DecodeStepGraph
+    kinds = kinds_of(TABLE9_10F11R57S)
+    w = synth.WORKLOADS[2].replace(max_len=2048, n_layers=len(kinds), kappa=64, n_clusters=8)
+    inp = _inputs(w)
+    inp["anchor_mask"] = kinds
+    cfg = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=4, anchor_mask=kinds)
+    out, idx = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                       want_idx=True)
+    layerwise_step_check(oracle, cfg, inp, out, idx)
+    cfg_s = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=4, anchor_mask=kinds,
+                                       flags=prism.FLAG_SERIAL)
+    out_s, idx_s = prism.prism_decode_step(cfg_s, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                           want_idx=True)
+    assert torch.equal(idx, idx_s) and torch.equal(out, out_s)
+    idx_g = torch.empty_like(idx)
+    g = DecodeStepGraph(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], idx_out=idx_g)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(idx_g, idx) and torch.equal(g.out, out)
