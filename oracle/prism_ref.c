@@ -21,6 +21,7 @@
  *     positional proposal), and reselects its own top-kappa (Eq. (6));
  *   - sparse attention over the selected rows with an exact softmax (the
  *     SparseAttn step of Algorithm 1);
+ *   - the 2-bit proposal keys of section 4.2 (Eq. (7)-(9)) for mode 3;
  *   - the pool variant (mode 3) of section 4.1-4.2 as the paper states it:
  *     the relevance score is the maximum over the GQA group (Eq. (9), on the
  *     bf16 keys), an anchor layer keeps a pool of the rho*kappa best tokens
@@ -50,6 +51,9 @@
 #ifndef PRISM_REF_PLANT
 #define PRISM_REF_PLANT 0
 #endif
+
+/* Group size g of the 2-bit proposal keys (Eq. (7); the paper leaves g open). */
+#define PRISM_REF_QGROUP 32
 
 /* bf16 is the top half of an IEEE-754 binary32; widening to double is exact. */
 static double bf16_to_double(uint16_t h)
@@ -134,6 +138,83 @@ void prism_ref_score_max(int d, int G, const uint16_t *q_group,
 #else
             if (dot > best) best = dot;
 #endif
+        }
+        s_out[e] = scale * best;
+    }
+}
+
+/*
+ * Group-wise asymmetric b = 2 bit quantization of one key row, Eq. (7)-(8):
+ * the d elements split into d/g groups of g; group m keeps
+ *   alpha_m = (max - min) / (2^b - 1),  beta_m = min,
+ *   code_e  = clip(round((k_e - beta_m) / alpha_m), 0, 3)  (round half up),
+ * and alpha_m = 0 (all codes 0) when max == min.  Every step is an IEEE
+ * binary32 operation (the codes are decided in the kernel's precision).
+ * codes: [d] one code per element; alpha, beta: [d/g].
+ */
+void prism_ref_quantize_row(int d, int g, const uint16_t *k_row, uint8_t *codes, float *alpha,
+                            float *beta)
+{
+    for (int m = 0; m < d / g; ++m) {
+        float lo = (float)bf16_to_double(k_row[m * g]), hi = lo;
+        for (int e = 1; e < g; ++e) {
+            const float x = (float)bf16_to_double(k_row[m * g + e]);
+            if (x < lo) lo = x;
+            if (x > hi) hi = x;
+        }
+#if PRISM_REF_PLANT == 17
+        volatile float a = (hi - lo) / 4.0f;        /* planted: 2^b levels, not 2^b - 1 */
+#else
+        volatile float a = (hi - lo) / 3.0f;
+#endif
+        alpha[m] = a;
+        beta[m] = lo;
+        for (int e = 0; e < g; ++e) {
+            int c = 0;
+            if (a > 0.0f) {
+                volatile float t = (float)bf16_to_double(k_row[m * g + e]) - lo;
+                volatile float x = t / a;
+#if PRISM_REF_PLANT == 18
+                c = (int)floorf(x);                     /* planted: truncation, not rounding */
+#else
+                volatile float xr = x + 0.5f;
+                c = (int)floorf(xr);
+#endif
+                if (c < 0) c = 0;
+                if (c > 3) c = 3;
+            }
+            codes[m * g + e] = (uint8_t)c;
+        }
+    }
+}
+
+/*
+ * Proposal score of Eq. (9) on the 2-bit keys: the group maximum of
+ * <q_j, khat_i> with khat_i,e = alpha_m * code_e + beta_m (the dequantized
+ * key; group m holds element e), times scale, in fp64.
+ * codes: [*][d] (one per element), alpha/beta: [*][d/g]; pos as prism_ref_score.
+ */
+void prism_ref_score_max_q2(int d, int g, int G, const uint16_t *q_group, const uint8_t *codes,
+                            const float *alpha, const float *beta, int n, const int32_t *pos,
+                            double scale, double *s_out)
+{
+    const int M = d / g;
+    for (int e = 0; e < n; ++e) {
+        long i = pos ? (long)pos[e] : (long)e;
+        double best = -INFINITY;
+        for (int j = 0; j < G; ++j) {
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) {
+                const int m = c / g;
+#if PRISM_REF_PLANT == 19
+                const double kh = (double)alpha[i * M + m] * codes[(size_t)i * d + c];   /* planted: beta dropped */
+#else
+                const double kh = (double)alpha[i * M + m] * codes[(size_t)i * d + c] +
+                                  (double)beta[i * M + m];
+#endif
+                dot += bf16_to_double(q_group[(size_t)j * (size_t)d + (size_t)c]) * kh;
+            }
+            if (dot > best) best = dot;
         }
         s_out[e] = scale * best;
     }
@@ -318,6 +399,9 @@ void prism_ref_attention(int d, int G, const uint16_t *q_group,
  * q      : [N][B][Hq][d] bf16 bits;  k[l], v[l]: [B][Hkv][Lmax][d] bf16 bits
  * len    : [B] context lengths (<= Lmax)
  * rho    : pool expansion factor (mode 3 only; >= 1)
+ * qbits  : 0, or 2 (mode 3 only): the scores of Eq. (9) use the keys
+ *          quantized by Eq. (7)-(8) (prism_ref_quantize_row, groups of
+ *          PRISM_REF_QGROUP), dequantized; attention keeps the bf16 keys
  * out    : [N][B][Hq][d] fp64;       idx_out: [N][B][Hkv][kappa] int32
  * pool_out (nullable, mode 3): [N][B][Hkv][rho*kappa] int32, the pool in
  *          effect at each layer (an anchor's own pool, a refined layer's
@@ -327,7 +411,7 @@ void prism_ref_attention(int d, int G, const uint16_t *q_group,
  */
 int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
                           int r, int n_layers, const uint8_t *anchor_mask,
-                          int mode, int chain, double scale, int rho,
+                          int mode, int chain, double scale, int rho, int qbits,
                           const uint16_t *q, const uint16_t *const *k,
                           const uint16_t *const *v, const int32_t *len,
                           double *out, int32_t *idx_out, int32_t *pool_out)
@@ -337,6 +421,7 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
         chain < 0 || chain > 1)
         return -1;
     if (mode == 3 && (rho < 1 || (long long)rho * kappa > 0x7fffffffLL)) return -1;
+    if (qbits != 0 && (qbits != 2 || mode != 3 || d % PRISM_REF_QGROUP != 0)) return -1;
     if (mode != 2) {
         if (anchor_mask[0] != 1) return -1;
         for (int l = 0; l < n_layers; ++l)
@@ -397,10 +482,34 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
                 }
             } else if (mode == 3) {
                 int32_t *C = pool + (size_t)row * (size_t)n_pool;
+                /* qbits == 2: this layer's keys quantized by Eq. (7)-(8); the
+                   scores of Eq. (9) use them (Algorithm 1: INT2 keys at the
+                   proposal layer and in the refinement) */
+                uint8_t *qc = NULL;
+                float *qa = NULL, *qb = NULL;
+                if (qbits == 2) {
+                    const int M = d / PRISM_REF_QGROUP;
+                    const size_t nrow = (size_t)(L > 0 ? L : 1);
+                    qc = (uint8_t *)malloc(nrow * (size_t)d);
+                    qa = (float *)malloc(nrow * (size_t)M * sizeof(float));
+                    qb = (float *)malloc(nrow * (size_t)M * sizeof(float));
+                    for (int i = 0; i < L; ++i)
+                        prism_ref_quantize_row(d, PRISM_REF_QGROUP, kr + (size_t)i * d,
+                                               qc + (size_t)i * d, qa + (size_t)i * M,
+                                               qb + (size_t)i * M);
+                }
+#define POOL_SCORE(n_, pos_, s_)                                                          \
+    do {                                                                                  \
+        if (qbits == 2)                                                                   \
+            prism_ref_score_max_q2(d, PRISM_REF_QGROUP, G, qg, qc, qa, qb, (n_), (pos_),  \
+                                   scale, (s_));                                          \
+        else                                                                              \
+            prism_ref_score_max(d, G, qg, kr, (n_), (pos_), scale, (s_));                 \
+    } while (0)
                 if (is_anchor) {
                     /* Eq. (9) over the whole cache, then the pool of Eq. (4) */
                     double *s = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
-                    prism_ref_score_max(d, G, qg, kr, L, NULL, scale, s);
+                    POOL_SCORE(L, NULL, s);
                     int nc = prism_ref_topk(L, s, NULL, n_pool, C);
                     /* the first kappa of C in score order: the top-kappa of
                        the pool's own scores */
@@ -425,10 +534,14 @@ int prism_ref_decode_step(int B, int Hq, int Hkv, int d, int Lmax, int kappa,
                     while (nc < n_pool && C[nc] >= 0) ++nc;
 #endif
                     double *s = (double *)malloc(sizeof(double) * (size_t)(nc > 0 ? nc : 1));
-                    prism_ref_score_max(d, G, qg, kr, nc, cand, scale, s);
+                    POOL_SCORE(nc, cand, s);
                     prism_ref_topk(nc, s, cand, kappa, sel);
                     free(s);
                 }
+#undef POOL_SCORE
+                free(qc);
+                free(qa);
+                free(qb);
                 if (pool_out) {
                     int32_t *po = pool_out + ((size_t)l * rows + row) * (size_t)rho * (size_t)kappa;
                     for (long e = 0; e < (long)rho * kappa; ++e) po[e] = e < n_pool ? C[e] : -1;

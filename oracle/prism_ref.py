@@ -19,6 +19,7 @@ _dbl = ctypes.c_double
 _vp = ctypes.c_void_p
 
 MODE_REFINE, MODE_STATIC_REUSE, MODE_DENSE_ANCHOR, MODE_POOL = 0, 1, 2, 3
+QGROUP = 32          # group size g of the 2-bit proposal keys (Eq. (7))
 CHAIN_PREV, CHAIN_ANCHOR = 0, 1
 
 
@@ -43,6 +44,11 @@ class Oracle:
         lib.prism_ref_score.restype = None
         lib.prism_ref_score_max.argtypes = [_i32, _i32, _vp, _vp, _i32, _vp, _dbl, _vp]
         lib.prism_ref_score_max.restype = None
+        lib.prism_ref_quantize_row.argtypes = [_i32, _i32, _vp, _vp, _vp, _vp]
+        lib.prism_ref_quantize_row.restype = None
+        lib.prism_ref_score_max_q2.argtypes = [_i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp,
+                                               _dbl, _vp]
+        lib.prism_ref_score_max_q2.restype = None
         lib.prism_ref_topk.argtypes = [_i32, _vp, _vp, _i32, _vp]
         lib.prism_ref_topk.restype = _i32
         lib.prism_ref_expand.argtypes = [_i32, _i32, _vp, _i32, _vp]
@@ -50,7 +56,7 @@ class Oracle:
         lib.prism_ref_attention.argtypes = [_i32, _i32, _vp, _vp, _vp, _i32, _vp, _dbl, _vp, _vp]
         lib.prism_ref_attention.restype = None
         lib.prism_ref_decode_step.argtypes = [
-            _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _dbl, _i32,
+            _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _dbl, _i32, _i32,
             _vp, _vp, _vp, _vp, _vp, _vp, _vp]
         lib.prism_ref_decode_step.restype = _i32
         lib.prism_ref_num_threads.restype = _i32
@@ -89,6 +95,37 @@ class Oracle:
            float(scale), _ptr(out))
         return out
 
+    def quantize(self, k_rows, g=QGROUP):
+        """Eq. (7)-(8) on key rows [n][d] (uint16 bf16 bits): codes [n][d]
+        uint8 (one per element), alpha and beta [n][d/g] float32."""
+        k_rows = _u16(k_rows)
+        n, d = k_rows.shape
+        codes = np.empty((n, d), np.uint8)
+        alpha = np.empty((n, d // g), np.float32)
+        beta = np.empty((n, d // g), np.float32)
+        for i in range(n):
+            self.lib.prism_ref_quantize_row(d, g, _ptr(k_rows[i]), _ptr(codes[i]), _ptr(alpha[i]),
+                                            _ptr(beta[i]))
+        return codes, alpha, beta
+
+    def score_q2(self, q_group, codes, alpha, beta, pos=None, scale=None, g=QGROUP):
+        """Eq. (9) group maximum on dequantized 2-bit keys (fp64)."""
+        q_group = _u16(q_group)
+        codes = np.ascontiguousarray(codes, np.uint8)
+        alpha = np.ascontiguousarray(alpha, np.float32)
+        beta = np.ascontiguousarray(beta, np.float32)
+        G, d = q_group.shape
+        n = codes.shape[0] if pos is None else len(pos)
+        if pos is not None:
+            pos = np.ascontiguousarray(pos, dtype=np.int32)
+        if scale is None:
+            scale = 1.0 / np.sqrt(d)
+        out = np.empty(n, np.float64)
+        self.lib.prism_ref_score_max_q2(d, g, G, _ptr(q_group), _ptr(codes), _ptr(alpha),
+                                        _ptr(beta), n, _ptr(pos) if pos is not None else None,
+                                        float(scale), _ptr(out))
+        return out
+
     def topk(self, s, kappa, pos=None):
         """Eqs. (2)/(6): top-kappa positions, ascending, -1 padded; and kappa_eff."""
         s = np.ascontiguousarray(s, dtype=np.float64)
@@ -125,7 +162,8 @@ class Oracle:
 
     # -- whole decode step ----------------------------------------------------
     def decode_step(self, q, k_layers, v_layers, lens, kappa, radius, anchor_mask,
-                    mode=MODE_REFINE, chain=CHAIN_PREV, scale=None, rho=1, want_pool=False):
+                    mode=MODE_REFINE, chain=CHAIN_PREV, scale=None, rho=1, want_pool=False,
+                    qbits=0):
         """Algorithm 1 over all layers.
 
         q: [N][B][Hq][d] uint16; k_layers/v_layers: N arrays [B][Hkv][Lmax][d]
@@ -159,7 +197,7 @@ class Oracle:
             pool = np.empty((N, B, Hkv, int(rho) * int(kappa)), dtype=np.int32)
         rc = self.lib.prism_ref_decode_step(B, Hq, Hkv, d, Lmax, int(kappa), int(radius), N,
                                             _ptr(mask), int(mode), int(chain), float(scale),
-                                            int(rho), _ptr(q), ctypes.cast(kp, _vp),
+                                            int(rho), int(qbits), _ptr(q), ctypes.cast(kp, _vp),
                                             ctypes.cast(vp, _vp), _ptr(lens), _ptr(out),
                                             _ptr(idx), _ptr(pool) if pool is not None else None)
         if rc != 0:
@@ -202,6 +240,9 @@ PLANTS = {
     14: "pool-mode refined layers rescore the previous selection, not the pool",
     15: "the anchor attends to the pool's first kappa positions, not its best kappa",
     16: "shared layers keep the anchor's selection, not the previous layer's",
+    17: "the 2-bit scale divides by 2^b instead of 2^b - 1",
+    18: "the 2-bit codes truncate instead of rounding",
+    19: "the dequantized key drops the zero-point beta",
 }
 
 __all__ = ["Oracle", "load", "bf16_bits", "PLANTS", "MODE_REFINE", "MODE_STATIC_REUSE",

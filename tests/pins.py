@@ -515,12 +515,123 @@ def pin_shared_invariants(o):
     assert np.array_equal(idx, st_max), "F then S equals rho = 1 in pool mode"
 
 
+# -- 2-bit proposal keys: Eq. (7)-(8) quantizer, Eq. (9) on dequantized keys --
+def pin_quantize_hand(o):
+    g = golden("quantize_cases")
+    for r in g["rows"]:
+        k = f32_to_bf16_bits(np.array([r["values"]], np.float32))
+        codes, alpha, beta = o.quantize(k, g=g["g"])
+        assert codes[0].tolist() == r["codes"], f"hand codes: {r['note']}"
+        assert float(alpha[0, 0]) == r["alpha"] and float(beta[0, 0]) == r["beta"], r["note"]
+
+
+def _numpy_quantize(k_bits, g=32):
+    """Eq. (7)-(8) in numpy float32 (IEEE binary32 like the oracle and the
+    kernel): per group alpha = (max - min) / 3, beta = min, codes =
+    clip(floor((k - beta) / alpha + 0.5), 0, 3), alpha = 0 -> code 0."""
+    k = bf16_bits_to_f64(k_bits).astype(np.float32)
+    n, d = k.shape
+    kg = k.reshape(n, d // g, g)
+    lo = kg.min(axis=2)
+    hi = kg.max(axis=2)
+    a = ((hi - lo) / np.float32(3.0)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        x = ((kg - lo[..., None]) / a[..., None]).astype(np.float32)
+        c = np.floor((x + np.float32(0.5)).astype(np.float32))
+    c = np.where(a[..., None] > 0, np.clip(c, 0, 3), 0).astype(np.uint8)
+    return c.reshape(n, d), a, lo
+
+
+def pin_quantize_numpy_and_bound(o):
+    """The codes equal a numpy float32 recomputation; every element is
+    reconstructed within alpha / 2 (round to nearest), the group's minimum
+    codes to 0 and its maximum to 3."""
+    rng = np.random.default_rng(23)
+    for d, scale in ((128, 1.0), (64, 3.0), (128, 0.01)):
+        k = rand_bf16(rng, (300, d), scale)
+        codes, alpha, beta = o.quantize(k)
+        c2, a2, b2 = _numpy_quantize(k)
+        assert np.array_equal(codes, c2), "codes vs numpy"
+        assert np.array_equal(alpha, a2) and np.array_equal(beta, b2), "alpha/beta vs numpy"
+        kf = bf16_bits_to_f64(k).reshape(300, d // 32, 32)
+        rec = alpha.astype(np.float64)[..., None] * codes.reshape(300, d // 32, 32) + \
+            beta.astype(np.float64)[..., None]
+        assert np.all(np.abs(rec - kf) <= alpha.astype(np.float64)[..., None] * (0.5 + 1e-6) + 1e-12), \
+            "reconstruction within alpha/2"
+        cg = codes.reshape(300, d // 32, 32)
+        assert np.all(cg.min(axis=2) == 0) and np.all(cg.max(axis=2) == 3), "min -> 0, max -> 3"
+
+
+def pin_score_q2_numpy(o):
+    """Eq. (9) on 2-bit keys equals numpy einsum on the dequantized matrix,
+    then numpy max over the group."""
+    rng = np.random.default_rng(24)
+    for G, d, n in ((4, 128, 200), (8, 64, 100), (1, 128, 64)):
+        q = rand_bf16(rng, (G, d))
+        k = rand_bf16(rng, (n, d))
+        codes, alpha, beta = o.quantize(k)
+        khat = np.repeat(alpha.astype(np.float64), 32, axis=1) * codes + \
+            np.repeat(beta.astype(np.float64), 32, axis=1)
+        ref = (np.einsum("gd,ld->gl", bf16_bits_to_f64(q), khat) / math.sqrt(d)).max(axis=0)
+        got = o.score_q2(q, codes, alpha, beta)
+        assert np.allclose(got, ref, rtol=1e-12, atol=1e-12), "q2 score vs numpy"
+        pos = np.sort(rng.choice(n, n // 3, replace=False)).astype(np.int32)
+        assert np.allclose(o.score_q2(q, codes, alpha, beta, pos=pos), ref[pos], rtol=1e-12,
+                           atol=1e-12), "q2 score on a position list"
+
+
+def pin_q2_decode(o):
+    """The pool-mode step on 2-bit keys equals a numpy recomputation; with
+    keys that the quantizer represents exactly it equals the bf16 step."""
+    w = small_workloads()[1]
+    q, ks, vs, lens = _bits(synth.make_inputs(w))
+    N, B, Hq, d = q.shape
+    H, G = w.n_kv_heads, w.group
+    mask = w.anchor_mask()
+    _, idx = o.decode_step(q, ks, vs, lens, w.kappa, 0, mask, mode=MODE_POOL, rho=2, qbits=2)
+    n = 2 * w.kappa
+    ref = np.zeros_like(idx, dtype=np.int64)
+    pool = np.zeros((B, H, n), np.int64)
+    for l in range(N):
+        for b in range(B):
+            L = int(lens[b])
+            for h in range(H):
+                c, a, bt = _numpy_quantize(ks[l][b, h, :L])
+                khat = np.repeat(a.astype(np.float64), 32, axis=1) * c + \
+                    np.repeat(bt.astype(np.float64), 32, axis=1)
+                s = (np.einsum("gd,ld->gl", bf16_bits_to_f64(q[l, b, h * G:(h + 1) * G]), khat)
+                     / math.sqrt(d)).max(axis=0)
+                if mask[l]:
+                    pool[b, h] = lexsort_topk(s, n)
+                    C = pool[b, h][pool[b, h] >= 0]
+                    ref[l, b, h] = lexsort_topk(s[C], w.kappa, C)
+                else:
+                    C = pool[b, h][pool[b, h] >= 0]
+                    ref[l, b, h] = lexsort_topk(s[C], w.kappa, C)
+    assert np.array_equal(idx, ref), "2-bit pool step vs numpy"
+    # keys the quantizer represents exactly: every group holds beta + alpha*{0..3}
+    rng = np.random.default_rng(25)
+    ex = []
+    for l in range(N):
+        c = rng.integers(0, 4, ks[l].shape)
+        c[..., 0::32] = 0
+        c[..., 1::32] = 3
+        a = 2.0 ** rng.integers(-3, 1, ks[l].shape[:-1] + (d // 32,))
+        bt = -2.0 * a
+        kv = np.repeat(a, 32, axis=-1) * c + np.repeat(bt, 32, axis=-1)
+        ex.append(f32_to_bf16_bits(kv.astype(np.float32)))
+    _, i16 = o.decode_step(q, ex, vs, lens, w.kappa, 0, mask, mode=MODE_POOL, rho=2)
+    _, i2 = o.decode_step(q, ex, vs, lens, w.kappa, 0, mask, mode=MODE_POOL, rho=2, qbits=2)
+    assert np.array_equal(i16, i2), "exactly representable keys: 2-bit step = bf16 step"
+
+
 ALL_PINS = [pin_score_bruteforce, pin_score_hand, pin_topk_golden, pin_topk_lexsort,
             pin_topk_all_equal, pin_topk_subsets, pin_expand_golden, pin_expand_bruteforce,
             pin_attention_sdpa, pin_attention_closed_forms, pin_decode_hand,
             pin_decode_numpy_chain, pin_decode_outputs_sdpa, pin_decode_invariants,
             pin_score_max_bruteforce, pin_score_max_hand, pin_pool_hand, pin_pool_numpy_chain,
-            pin_pool_invariants, pin_shared_numpy, pin_shared_invariants]
+            pin_pool_invariants, pin_shared_numpy, pin_shared_invariants, pin_quantize_hand,
+            pin_quantize_numpy_and_bound, pin_score_q2_numpy, pin_q2_decode]
 
 __all__ = ["ALL_PINS", "small_workloads"] + [p.__name__ for p in ALL_PINS]
 _ = torch  # torch is used through helpers.sdpa_group and synth
