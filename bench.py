@@ -52,14 +52,16 @@ def parse_args():
                     help="layers per step of the reference (oracle) arm")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-q2", action="store_true", help="skip the 2-bit key measurement")
     ap.add_argument("--profile", action="store_true",
                     help="only run --steps eager decode steps (for ncu captures)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (profiling a smaller case)")
     ap.add_argument("--pool", type=int, default=4,
                     help="rho of the pool-mode measurement (0: skip it)")
-    ap.add_argument("--mode", choices=["refine", "pool"], default="refine",
-                    help="decode-step mode of a --profile run (pool uses --pool as rho)")
+    ap.add_argument("--mode", choices=["refine", "pool", "pool-int2"], default="refine",
+                    help="decode-step mode of a --profile run (pool uses --pool as rho; "
+                         "pool-int2 scores on 2-bit keys)")
     return ap.parse_args()
 
 
@@ -253,18 +255,26 @@ def run_prism(args, rank, world, dev):
         w = w.replace(n_layers=args.layers)
     inp = synth.make_inputs(w, device=dev)
     if args.profile:
-        pool_run = args.mode == "pool"
-        cfg = (prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=args.pool)
+        pool_run = args.mode in ("pool", "pool-int2")
+        q2_run = args.mode == "pool-int2"
+        cfg = (prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=args.pool,
+                                          flags=prism.FLAG_INT2_KEYS if q2_run else 0)
                if pool_run else prism.Config.from_workload(w))
         ws = prism.workspace(cfg, dev)
+        kq = [prism.prism_quantize_keys(cfg, kk, inp["lens"], ws=ws) for kk in inp["k"]] \
+            if q2_run else None
         for _ in range(args.steps):
-            prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], ws=ws)
+            if q2_run:
+                prism.prism_decode_step_kq(cfg, inp["q"], inp["k"], inp["v"], kq, inp["lens"],
+                                           ws=ws)
+            else:
+                prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], ws=ws)
         torch.cuda.synchronize(dev)
         st, detail = prism.prism_check_device_status(ws)
         if st != 0:
             raise RuntimeError(f"device status {st} {detail}")
         print(f"profile run: {args.steps} eager steps of {w.name} ({w.n_layers} layers, "
-              f"{'pool rho %d' % args.pool if pool_run else 'refine'})")
+              f"{args.mode}, rho {args.pool})")
         return
     cfg = prism.Config.from_workload(w)
     ws = prism.workspace(cfg, dev)
@@ -474,6 +484,81 @@ def run_prism(args, rank, world, dev):
                    "and inputs, graph-timed like the headline step",
         }
 
+    # -- pool mode on 2-bit proposal keys (Eq. (7)-(9)): the anchor scans and
+    #    the pool rescoring read the 2-bit cache, attention the bf16 keys
+    pool_q2 = None
+    if args.pool > 0 and not args.skip_q2:
+        rho = args.pool
+        cfg_q = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=rho,
+                                           flags=prism.FLAG_INT2_KEYS)
+        ws_q = prism.workspace(cfg_q, dev)
+        kq = [prism.prism_quantize_keys(cfg_q, kk, inp["lens"], ws=ws_q) for kk in inp["k"]]
+        # the append-time quantizer, timed per layer (not part of a decode step)
+        qa, qb_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        qa.record(stream)
+        for kk, kqq in zip(inp["k"], kq):
+            prism.prism_quantize_keys(cfg_q, kk, inp["lens"], kq=kqq, ws=ws_q, stream=stream)
+        qb_.record(stream)
+        torch.cuda.synchronize(dev)
+        t_quant = qa.elapsed_time(qb_) * 1e3 / N
+        rq = DecodeStepGraph(cfg_q, inp["q"], inp["k"], inp["v"], inp["lens"], ws=ws_q,
+                             kq_layers=kq)
+        for _ in range(max(3, args.warmup)):
+            rq.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(args.steps):
+            rq.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_q = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
+        launches_q = rq.launches
+        del rq
+        st, detail = prism.prism_check_device_status(ws_q)
+        if st != 0:
+            raise RuntimeError(f"device status after the 2-bit pool step {st} {detail}")
+        cfgqp = ctypes.byref(cfg_q)
+
+        def score_q2_launch(l):
+            rc = L.prism_score_anchor(cfgqp, ctypes.c_void_p(inp["q"][l].data_ptr()),
+                                      ctypes.c_void_p(kq[l].data_ptr()),
+                                      ctypes.c_void_p(inp["lens"].data_ptr()),
+                                      ctypes.c_void_p(S.data_ptr()),
+                                      ctypes.c_void_p(ws_q.data_ptr()), ws_q.numel(),
+                                      ctypes.c_void_p(stream.cuda_stream))
+            if rc != 0:
+                raise RuntimeError(f"prism_score_anchor (2-bit keys): {rc}")
+        for i in range(3):
+            score_q2_launch(anchors[i % len(anchors)])
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_k)]
+        for i in range(n_k):
+            evs[i][0].record(stream)
+            score_q2_launch(anchors[i % len(anchors)])
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        t_q2 = statistics.mean(x.elapsed_time(y) for x, y in evs) * 1e-3
+        q2_bytes = sum(int(x) for x in lens_h) * w.n_kv_heads * (w.head_dim // 2)
+        pool_rows_q = sum(min(rho * w.kappa, int(x)) for x in lens_h) * w.n_kv_heads
+        q2_step_bytes = (n_anchor * q2_bytes + (N - n_anchor) * pool_rows_q * (w.head_dim // 2)
+                         + N * gather)
+        pool_q2 = {
+            "rho": rho, "value": whole_job_us_per_layer(ms_q, N, world), "unit": UNIT,
+            "ms_per_step": ms_q, "launches_per_step": launches_q,
+            "step_hbm": {"algorithmic_bytes": q2_step_bytes,
+                         "gbs": q2_step_bytes / (ms_q * 1e-3) / 1e9,
+                         "frac": q2_step_bytes / (ms_q * 1e-3) / 1e9 / peak},
+            "anchor_kernel": {"kernel": "k_anchor_score_q2 (mma.sync on 2-bit codes)",
+                              "bound": "hbm", "achieved": q2_bytes / t_q2 / 1e9, "peak": peak,
+                              "unit": "GB/s", "frac": q2_bytes / t_q2 / 1e9 / peak,
+                              "us_per_launch": t_q2 * 1e6, "bytes_per_launch": q2_bytes},
+            "quantize_us_per_layer": t_quant,
+            "how": "pool mode on the 2-bit cache (64 B a key: codes + fp32 alpha/beta per 32), "
+                   "same inputs; the quantizer runs when keys are appended, timed apart",
+        }
+        del kq
+
     # -- per-stage breakdown (events around each public stage call)
     def timed(fn, reps=8):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -582,6 +667,7 @@ def run_prism(args, rank, world, dev):
                                    "proposal K rows + gathered K/V rows"},
             "breakdown_us": br,
             "pool_mode": pool,
+            "pool_mode_int2": pool_q2,
             "gpu_launches": launches_per_step * args.steps,
             "launches_per_step": launches_per_step,
             "clocks": clk,

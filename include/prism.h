@@ -135,6 +135,13 @@ typedef struct {
  * DAG over helper streams; this flag enqueues everything, in layer order, on
  * the caller's stream instead (same results, bit for bit). */
 #define PRISM_FLAG_SERIAL 1
+/* PRISM_MODE_POOL only: the proposal scores (Eq. (9)) use 2-bit keys
+ * (section 4.2, Eq. (7)-(8)).  With this flag the `k` argument of
+ * prism_index_anchor, prism_index_pool, prism_score_anchor and
+ * prism_index_refine is a 2-bit key cache written by prism_quantize_keys,
+ * and the decode step is prism_decode_step_kq (bf16 keys for attention, the
+ * 2-bit cache for scoring); prism_decode_step rejects the flag. */
+#define PRISM_FLAG_INT2_KEYS 2
 
 #define PRISM_MAX_LEN (1 << 20)
 #define PRISM_MAX_BATCH_ROWS 65535   /* B * Hkv */
@@ -264,6 +271,36 @@ PRISM_API prism_status_t prism_decode_step(const prism_config_t *cfg, const void
                                  const int32_t *len, void *out,
                                  int32_t *idx_out, void *ws, size_t ws_bytes,
                                  void *stream);
+
+/* The 2-bit proposal key cache of one layer (section 4.2, Eq. (7)-(8)):
+ * every key row is split into groups of 32 elements; group m keeps
+ *   alpha_m = (max - min) / 3,  beta_m = min  (fp32),
+ *   code_e  = clip(round half up((k_e - beta_m) / alpha_m), 0, 3),
+ * alpha_m = 0 giving code 0, each an IEEE binary32 operation.  Positions
+ * [start, len[b]) of every (batch, KV head) are (re)written -- the
+ * append-time use quantizes the newly appended tokens -- the rest of kq is
+ * left untouched.
+ * k   bf16 [B][Hkv][Lmax][d] (d in {64, 128})
+ * kq  uint8 [B][Hkv][Lmax][d/2]: per row, d/4 bytes of codes (byte
+ *     t*(d/16) + kk holds the codes of elements 16kk + 2t, 16kk + 2t + 1,
+ *     16kk + 2t + 8, 16kk + 2t + 9 in bits 0-1, 2-3, 4-5, 6-7; t = 0..3,
+ *     kk = 0..d/16-1), then alpha_m, beta_m (fp32) for each group m.
+ * ws  only its status word is used (a len[b] outside [0, Lmax] is
+ *     recorded there).  No other field of cfg than its shape is read. */
+PRISM_API prism_status_t prism_quantize_keys(const prism_config_t *cfg, const void *k,
+                                   const int32_t *len, int32_t start, void *kq,
+                                   void *ws, size_t ws_bytes, void *stream);
+
+/* prism_decode_step with 2-bit proposal keys: cfg->mode == PRISM_MODE_POOL
+ * and cfg->flags has PRISM_FLAG_INT2_KEYS.  kq: HOST array of N device
+ * pointers, each layer's 2-bit cache (prism_quantize_keys); the anchor scans
+ * and the pool rescoring read kq (Algorithm 1: INT2 keys in proposal and
+ * refinement), the sparse attention reads k and v. */
+PRISM_API prism_status_t prism_decode_step_kq(const prism_config_t *cfg, const void *q,
+                                    const void *const *k, const void *const *v,
+                                    const void *const *kq, const int32_t *len,
+                                    void *out, int32_t *idx_out, void *ws,
+                                    size_t ws_bytes, void *stream);
 
 /* Synchronises `stream`, reads the workspace status word and clears it.
  * Returns PRISM_OK, PRISM_ERR_TIMEOUT (a bounded wait ran out) or

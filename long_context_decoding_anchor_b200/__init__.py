@@ -27,6 +27,7 @@ MODE_REFINE, MODE_STATIC_REUSE, MODE_DENSE_ANCHOR, MODE_POOL = 0, 1, 2, 3
 CHAIN_PREV, CHAIN_ANCHOR = 0, 1
 LAYER_REFINED, LAYER_ANCHOR, LAYER_SHARED = 0, 1, 2
 FLAG_SERIAL = 1
+FLAG_INT2_KEYS = 2
 STATUS = {0: "PRISM_OK", 1: "PRISM_ERR_INVALID_ARG", 2: "PRISM_ERR_UNSUPPORTED",
           3: "PRISM_ERR_WORKSPACE", 4: "PRISM_ERR_CUDA", 5: "PRISM_ERR_TIMEOUT",
           6: "PRISM_ERR_DEVICE"}
@@ -34,7 +35,7 @@ EXPORTS = ("prism_workspace_size", "prism_index_anchor", "prism_index_refine",
            "prism_sparse_decode", "prism_decode_step", "prism_check_device_status",
            "prism_debug_wait_timeout", "prism_score_anchor", "prism_status_string",
            "prism_version", "prism_launch_count", "prism_sparse_decode_noalloc",
-           "prism_index_pool")
+           "prism_index_pool", "prism_quantize_keys", "prism_decode_step_kq")
 
 
 class PrismError(RuntimeError):
@@ -110,6 +111,10 @@ def lib() -> ctypes.CDLL:
         L.prism_index_refine.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
         L.prism_sparse_decode.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, vp, vp, sz, vp]
         L.prism_decode_step.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_decode_step_kq.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_decode_step_kq.restype = ctypes.c_int
+        L.prism_quantize_keys.argtypes = [cfgp, vp, vp, i32, vp, vp, sz, vp]
+        L.prism_quantize_keys.restype = ctypes.c_int
         L.prism_sparse_decode_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, i32, vp, vp]
         L.prism_sparse_decode_noalloc.restype = ctypes.c_int
         L.prism_check_device_status.argtypes = [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -158,6 +163,16 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None):
         raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def _need_keys(cfg: Config, k, name="k"):
+    """bf16 keys [B][Hkv][Lmax][d], or with FLAG_INT2_KEYS the 2-bit cache
+    uint8 [B][Hkv][Lmax][d/2] (prism_quantize_keys)."""
+    B, Hkv, d, L = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
+    if cfg.flags & FLAG_INT2_KEYS:
+        _need(k, name, torch.uint8, (B, Hkv, L, d // 2))
+    else:
+        _need(k, name, torch.bfloat16, (B, Hkv, L, d))
+
+
 def prism_workspace_size(cfg: Config) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().prism_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "prism_workspace_size")
@@ -175,7 +190,7 @@ def prism_index_anchor(cfg: Config, q, k, lens, idx_out=None, scores_out=None, w
                        stream=None):
     B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
     _need(q, "q", torch.bfloat16, (B, Hq, d))
-    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need_keys(cfg, k)
     _need(lens, "lens", torch.int32, (B,))
     if idx_out is None:
         idx_out = torch.empty((B, Hkv, cfg.kappa), dtype=torch.int32, device=q.device)
@@ -194,7 +209,7 @@ def prism_index_pool(cfg: Config, q, k, lens, pool_out=None, idx_out=None, score
     """Pool mode proposal layer: returns (pool [B][Hkv][rho*kappa], idx [B][Hkv][kappa])."""
     B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
     _need(q, "q", torch.bfloat16, (B, Hq, d))
-    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need_keys(cfg, k)
     _need(lens, "lens", torch.int32, (B,))
     n = cfg.pool_factor * cfg.kappa
     if pool_out is None:
@@ -217,7 +232,7 @@ def prism_score_anchor(cfg: Config, q, k, lens, scores_out=None, ws=None, stream
     """Eq. (1) only: one launch of the anchor scoring kernel."""
     B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
     _need(q, "q", torch.bfloat16, (B, Hq, d))
-    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need_keys(cfg, k)
     _need(lens, "lens", torch.int32, (B,))
     if scores_out is None:
         scores_out = torch.empty((B, Hkv, L), dtype=torch.float32, device=q.device)
@@ -235,7 +250,7 @@ def prism_index_refine(cfg: Config, q, k, lens, idx_prev, idx_out=None, cand_cap
     In pool mode idx_prev is a pool [B][Hkv][rho*kappa]."""
     B, Hq, Hkv, d, L = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
     _need(q, "q", torch.bfloat16, (B, Hq, d))
-    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need_keys(cfg, k)
     _need(lens, "lens", torch.int32, (B,))
     _need(idx_prev, "idx_prev", torch.int32, (B, Hkv, cfg.src_kappa))
     if idx_out is None:
@@ -322,6 +337,53 @@ def prism_decode_step(cfg: Config, q, k_layers, v_layers, lens, out=None, idx_ou
     return (out, idx_out) if idx_out is not None else out
 
 
+def prism_quantize_keys(cfg: Config, k, lens, start=0, kq=None, ws=None, stream=None):
+    """Eq. (7)-(8): the 2-bit proposal key cache of one layer (uint8
+    [B][Hkv][Lmax][d/2]); positions [start, len[b]) are written."""
+    B, Hkv, d, L = cfg.batch, cfg.n_kv_heads, cfg.head_dim, cfg.max_len
+    _need(k, "k", torch.bfloat16, (B, Hkv, L, d))
+    _need(lens, "lens", torch.int32, (B,))
+    if kq is None:
+        kq = torch.zeros((B, Hkv, L, d // 2), dtype=torch.uint8, device=k.device)
+    _need(kq, "kq", torch.uint8, (B, Hkv, L, d // 2))
+    ws = workspace(cfg, k.device) if ws is None else ws
+    _check(lib().prism_quantize_keys(ctypes.byref(cfg), _p(k), _p(lens), int(start), _p(kq),
+                                     _p(ws), ws.numel(), _stream(stream)),
+           "prism_quantize_keys")
+    return kq
+
+
+def prism_decode_step_kq(cfg: Config, q, k_layers, v_layers, kq_layers, lens, out=None,
+                         idx_out=None, ws=None, stream=None, want_idx=False):
+    """prism_decode_step with 2-bit proposal keys (pool mode, FLAG_INT2_KEYS)."""
+    N, B, Hq, Hkv, d, L = (cfg.n_layers, cfg.batch, cfg.n_q_heads, cfg.n_kv_heads,
+                           cfg.head_dim, cfg.max_len)
+    _need(q, "q", torch.bfloat16, (N, B, Hq, d))
+    if len(k_layers) != N or len(v_layers) != N or len(kq_layers) != N:
+        raise ValueError("need one K, one V and one 2-bit K tensor per layer")
+    for i in range(N):
+        _need(k_layers[i], f"k[{i}]", torch.bfloat16, (B, Hkv, L, d))
+        _need(v_layers[i], f"v[{i}]", torch.bfloat16, (B, Hkv, L, d))
+        _need(kq_layers[i], f"kq[{i}]", torch.uint8, (B, Hkv, L, d // 2))
+    _need(lens, "lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((N, B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _need(out, "out", torch.bfloat16, (N, B, Hq, d))
+    if idx_out is None and want_idx:
+        idx_out = torch.empty((N, B, Hkv, cfg.kappa), dtype=torch.int32, device=q.device)
+    if idx_out is not None:
+        _need(idx_out, "idx_out", torch.int32, (N, B, Hkv, cfg.kappa))
+    arr = lambda ts: (ctypes.c_void_p * N)(*[t.data_ptr() for t in ts])
+    kp, vp, kqp = arr(k_layers), arr(v_layers), arr(kq_layers)
+    ws = workspace(cfg, q.device) if ws is None else ws
+    _check(lib().prism_decode_step_kq(ctypes.byref(cfg), _p(q), ctypes.cast(kp, ctypes.c_void_p),
+                                      ctypes.cast(vp, ctypes.c_void_p),
+                                      ctypes.cast(kqp, ctypes.c_void_p), _p(lens), _p(out),
+                                      _p(idx_out), _p(ws), ws.numel(), _stream(stream)),
+           "prism_decode_step_kq")
+    return (out, idx_out) if idx_out is not None else out
+
+
 def prism_check_device_status(ws: torch.Tensor, stream=None):
     """Synchronises; returns (status, [code, where, value, 0]) and clears the word."""
     detail = (ctypes.c_uint32 * 4)()
@@ -344,4 +406,5 @@ __all__ = ["Config", "PrismError", "lib", "workspace", "prism_workspace_size",
            "prism_index_anchor", "prism_index_pool", "prism_index_refine", "prism_sparse_decode",
            "prism_decode_step", "prism_check_device_status", "prism_debug_wait_timeout",
            "prism_score_anchor", "prism_sparse_decode_noalloc", "raw_status", "MODE_REFINE", "MODE_STATIC_REUSE", "MODE_DENSE_ANCHOR", "MODE_POOL",
-           "CHAIN_PREV", "CHAIN_ANCHOR", "LAYER_REFINED", "LAYER_ANCHOR", "LAYER_SHARED", "FLAG_SERIAL", "EXPORTS", "LIB_PATH"]
+           "CHAIN_PREV", "CHAIN_ANCHOR", "LAYER_REFINED", "LAYER_ANCHOR", "LAYER_SHARED", "FLAG_SERIAL",
+           "FLAG_INT2_KEYS", "prism_quantize_keys", "prism_decode_step_kq", "EXPORTS", "LIB_PATH"]

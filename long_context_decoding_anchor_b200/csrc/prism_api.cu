@@ -136,7 +136,9 @@ prism_status_t check_config(const prism_config_t *c) {
     if (c->mode < PRISM_MODE_REFINE || c->mode > PRISM_MODE_POOL) return PRISM_ERR_INVALID_ARG;
     if (c->mode == PRISM_MODE_POOL && c->pool_factor < 1) return PRISM_ERR_INVALID_ARG;
     if (c->chain < PRISM_CHAIN_PREV || c->chain > PRISM_CHAIN_ANCHOR) return PRISM_ERR_INVALID_ARG;
-    if (c->flags & ~PRISM_FLAG_SERIAL) return PRISM_ERR_INVALID_ARG;
+    if (c->flags & ~(PRISM_FLAG_SERIAL | PRISM_FLAG_INT2_KEYS)) return PRISM_ERR_INVALID_ARG;
+    // 2-bit proposal keys belong to the pool mode (Eq. (9) scores)
+    if ((c->flags & PRISM_FLAG_INT2_KEYS) && c->mode != PRISM_MODE_POOL) return PRISM_ERR_INVALID_ARG;
     if (c->head_dim != 64 && c->head_dim != 128) return PRISM_ERR_UNSUPPORTED;
     const int G = c->n_q_heads / c->n_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return PRISM_ERR_UNSUPPORTED;
@@ -288,6 +290,7 @@ ScoreArgs score_args(const prism_config_t &c, const Ws &w, const Slot &sl, const
     sa.S = sl.S; sa.cpos = sl.cpos; sa.hist = sl.hist; sa.src = nullptr; sa.src_off = nullptr;
     sa.kappa = c.kappa; sa.radius = c.radius; sa.st = w.st; sa.wait_ns = wait_limit_ns();
     sa.agg = pool_mode(c) ? kAggMax : kAggSum;
+    sa.q2 = (c.flags & PRISM_FLAG_INT2_KEYS) ? 1 : 0;
     return sa;
 }
 
@@ -403,7 +406,8 @@ prism_status_t run_attn(const prism_config_t &c, const Ws &w, const void *q, con
 // `s0`; otherwise the three streams of the DAG described at the top.  Every
 // event is recorded (on the host) before any wait on it is enqueued.
 prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
-                            const void *const *k, const void *const *v, const int32_t *len,
+                            const void *const *k, const void *const *v,
+                            const void *const *kq, const int32_t *len,
                             void *out, int32_t *idx_out, cudaStream_t s0, DeviceHelpers *hp) {
     const int N = c.n_layers;
     const size_t rows = (size_t)c.batch * c.n_kv_heads;
@@ -473,7 +477,8 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
             PRISM_CUDA(cudaStreamWaitEvent(sA, ev_kdone[g - kAnchorAhead], 0));
             PRISM_CUDA(cudaMemsetAsync(w.slot[slot].hist, 0, rows * kHistBins * sizeof(uint32_t), sA));
         }
-        PRISM_TRY(run_anchor_score(c, w, slot, qb + (size_t)l * q_elems, k[l], len, nullptr, sA));
+        PRISM_TRY(run_anchor_score(c, w, slot, qb + (size_t)l * q_elems, kq ? kq[l] : k[l], len,
+                                   nullptr, sA));
         PRISM_CUDA(cudaEventRecord(ev_scored[g], sA));
         PRISM_CUDA(cudaStreamWaitEvent(sX, ev_scored[g], 0));
         const Slot &sl = w.slot[slot];
@@ -500,7 +505,8 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         const int l = anchors[g];
         const bool next_refines = refining && l + 1 < N && !is_anchor(l + 1);
         if (hp && g >= kAnchorAhead) PRISM_CUDA(cudaStreamWaitEvent(sA, ev_reached[g - kAnchorAhead], 0));
-        PRISM_TRY(run_anchor_score(c, w, g % kAnchorAhead, qb + (size_t)l * q_elems, k[l], len,
+        PRISM_TRY(run_anchor_score(c, w, g % kAnchorAhead, qb + (size_t)l * q_elems,
+                                   kq ? kq[l] : k[l], len,
                                    nullptr, sA));
         if (pool) {
             PRISM_TRY(run_pool_select(c, w, g % kAnchorAhead, len, w.pool_all + (size_t)l * pool_elems,
@@ -522,6 +528,7 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     const int32_t *prev_sel = nullptr, *prev_off = nullptr;
     int anchor_layer = 0;
     std::vector<char> batched(pool ? (size_t)N : 0, 0);   // pool mode: refined layers enqueued
+    bool prev_is_anchor_sel = false;     // the previous layer's selection is an anchor's own
     int g = 0;
     for (int l = 0; l < N; ++l) {
         const void *ql = qb + (size_t)l * q_elems;
@@ -546,6 +553,9 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         } else if (is_shared(l)) {
             // Table 9's shared layer: the previous layer's selection, unchanged
             // (and still described by the previous layer's proposal offsets).
+            // In pool mode an anchor's own selection comes from the aux
+            // stream, so a copy of it waits for that selection.
+            if (pool && hp && prev_is_anchor_sel) PRISM_CUDA(cudaStreamWaitEvent(sM, ev_kdone[g - 1], 0));
             if (idx_out) {
                 PRISM_CUDA(cudaMemcpyAsync(dst, prev_sel, sel_elems * sizeof(int32_t),
                                            cudaMemcpyDeviceToDevice, sM));
@@ -566,7 +576,7 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
                 for (int e = l; e < N && !is_anchor(e) && nz < kMaxZ; ++e) {
                     if (is_shared(e)) continue;
                     qs[nz] = qb + (size_t)e * q_elems;
-                    ks[nz] = k[e];
+                    ks[nz] = kq ? kq[e] : k[e];
                     outs[nz] = idx_base + (size_t)e * sel_elems;
                     batched[e] = 1;
                     ++nz;
@@ -599,6 +609,7 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
                            ob + (size_t)l * q_elems, sC));
         prev_sel = cur;
         prev_off = cur_off;
+        if (!is_shared(l)) prev_is_anchor_sel = is_anchor(l);
     }
     if (hp) {
         // Every anchor score was waited on by M; join M and C into the caller's stream.
@@ -776,12 +787,15 @@ prism_status_t prism_sparse_decode_noalloc(const prism_config_t *cfg, const void
     return cuda_status(launch_sparse_attn(aa, s));
 }
 
-prism_status_t prism_decode_step(const prism_config_t *cfg, const void *q, const void *const *k,
-                                 const void *const *v, const int32_t *len, void *out,
-                                 int32_t *idx_out, void *ws, size_t ws_bytes, void *stream) {
+static prism_status_t decode_step_impl(const prism_config_t *cfg, const void *q,
+                                       const void *const *k, const void *const *v,
+                                       const void *const *kq, const int32_t *len, void *out,
+                                       int32_t *idx_out, void *ws, size_t ws_bytes, void *stream) {
     PRISM_TRY(check_config(cfg));
     const prism_config_t &c = *cfg;
     if (c.n_layers < 1 || !q || !k || !v || !len || !out) return PRISM_ERR_INVALID_ARG;
+    // the 2-bit keys come with their own call (the step needs both caches)
+    if (((c.flags & PRISM_FLAG_INT2_KEYS) != 0) != (kq != nullptr)) return PRISM_ERR_INVALID_ARG;
     if (c.mode != PRISM_MODE_DENSE_ANCHOR) {
         // layer kinds: 0 refined, 1 anchor, 2 shared; layer 0 is an anchor
         if (!c.anchor_mask || c.anchor_mask[0] != 1) return PRISM_ERR_INVALID_ARG;
@@ -793,15 +807,43 @@ prism_status_t prism_decode_step(const prism_config_t *cfg, const void *q, const
         return PRISM_ERR_INVALID_ARG;
     for (int l = 0; l < c.n_layers; ++l) {
         if (!k[l] || !v[l] || !aligned(k[l], 16) || !aligned(v[l], 16)) return PRISM_ERR_INVALID_ARG;
+        if (kq && (!kq[l] || !aligned(kq[l], 16))) return PRISM_ERR_INVALID_ARG;
     }
     Ws w;
     PRISM_TRY(carve(c, ws, ws_bytes, &w));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (c.flags & PRISM_FLAG_SERIAL) return enqueue_step(c, w, q, k, v, len, out, idx_out, s, nullptr);
+    if (c.flags & PRISM_FLAG_SERIAL)
+        return enqueue_step(c, w, q, k, v, kq, len, out, idx_out, s, nullptr);
     std::lock_guard<std::mutex> lock(g_helpers_mu);
     DeviceHelpers *hp = nullptr;
     PRISM_TRY(helpers_for_current_device(4 + 6 * (size_t)c.n_layers, &hp));
-    return enqueue_step(c, w, q, k, v, len, out, idx_out, s, hp);
+    return enqueue_step(c, w, q, k, v, kq, len, out, idx_out, s, hp);
+}
+
+prism_status_t prism_decode_step(const prism_config_t *cfg, const void *q, const void *const *k,
+                                 const void *const *v, const int32_t *len, void *out,
+                                 int32_t *idx_out, void *ws, size_t ws_bytes, void *stream) {
+    return decode_step_impl(cfg, q, k, v, nullptr, len, out, idx_out, ws, ws_bytes, stream);
+}
+
+prism_status_t prism_decode_step_kq(const prism_config_t *cfg, const void *q,
+                                    const void *const *k, const void *const *v,
+                                    const void *const *kq, const int32_t *len, void *out,
+                                    int32_t *idx_out, void *ws, size_t ws_bytes, void *stream) {
+    if (!kq) return PRISM_ERR_INVALID_ARG;
+    return decode_step_impl(cfg, q, k, v, kq, len, out, idx_out, ws, ws_bytes, stream);
+}
+
+prism_status_t prism_quantize_keys(const prism_config_t *cfg, const void *k, const int32_t *len,
+                                   int32_t start, void *kq, void *ws, size_t ws_bytes,
+                                   void *stream) {
+    PRISM_TRY(check_config(cfg));
+    if (!k || !len || !kq || start < 0) return PRISM_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(kq, 16) || !aligned(len, 4)) return PRISM_ERR_INVALID_ARG;
+    if (!ws || !aligned(ws, 256) || ws_bytes < sizeof(DevStatus)) return PRISM_ERR_INVALID_ARG;
+    return cuda_status(launch_quantize_keys(k, len, cfg->batch, cfg->n_kv_heads, cfg->head_dim,
+                                            cfg->max_len, start, kq, static_cast<DevStatus *>(ws),
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 prism_status_t prism_check_device_status(void *ws, size_t ws_bytes, void *stream,

@@ -456,6 +456,8 @@ struct ScoreArgs {
     const int32_t *src_off; // refine: its proposal enumeration offsets [rows][kappa + 1]
     int kappa, radius;      // refine: entries of the source selection, proposal radius
     int agg;                // kAggSum: Eq. (1) group sum; kAggMax: Eq. (9) group maximum
+    int q2;                 // nonzero: k (and kz) are 2-bit key caches (Eq. (7)-(8),
+                            // rows of d/2 bytes, q2_impl.cuh), scored by Eq. (9)
     // refine: several layers rescoring the same source in one launch (grid z);
     // layer z reads qz[z] / kz[z] (z = 0: q / k) and writes S, cpos, hist
     // shifted by z * zS, z * zS, z * zhist.  cstride is the row stride of S
@@ -474,6 +476,10 @@ constexpr int kMaxZ = 8;           // refined layers batched into one launch
 cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s);
 // The group-maximum form of the full-cache scan (tensor cores; score_max.cu).
 cudaError_t launch_anchor_score_max(const ScoreArgs &a, int num_sms, cudaStream_t s);
+// The same on the 2-bit key cache, and its quantizer (score_q2.cu).
+cudaError_t launch_anchor_score_q2(const ScoreArgs &a, int num_sms, cudaStream_t s);
+cudaError_t launch_quantize_keys(const void *k, const int32_t *len, int B, int Hkv, int d, int Lmax,
+                                 int start, void *kq, DevStatus *st, cudaStream_t s);
 
 cudaError_t launch_refine_rescore(const ScoreArgs &a, int num_sms, cudaStream_t s);
 

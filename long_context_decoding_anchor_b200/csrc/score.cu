@@ -20,6 +20,7 @@
 // gathered with 16-byte cp.async pieces; the (score, position) candidates
 // are stored contiguously at their enumeration index.
 #include "prism_internal.cuh"
+#include "q2_impl.cuh"
 #include "tiles.cuh"
 
 namespace prism {
@@ -228,18 +229,23 @@ k_anchor_score(ScoreArgs a) {
 // (score, position) candidates at their slot index.  (A run of the proposal
 // is only ~11-17 rows, 3-4 KB: issuing one bulk copy per run from a single
 // warp, not DRAM, limited an earlier version to ~25 GB/s per SM.)
-template <int D>
+// Key formats of the rescoring kernel: bf16 keys with the group sum
+// (Eq. (1)), bf16 keys with the group maximum (Eq. (9)), 2-bit keys with the
+// group maximum (Eq. (7)-(9), row format of q2_impl.cuh).
+enum : int { kFmtSum = 0, kFmtMax = 1, kFmtQ2 = 2 };
+
+template <int D, int FMT = kFmtSum>
 struct RescoreCfg {
     static constexpr int kTileRows = 128;
     static constexpr int kStages = 3;                  // data stages per consumer warp
     static constexpr int kPosDepth = 8;                // position tables in the ring
     static constexpr int kConsumerWarps = 8;
     static constexpr int kThreads = 32 * (kConsumerWarps + 1);
-    static constexpr int kNL = D / 8;
+    static constexpr int kRowBytes = FMT == kFmtQ2 ? q2_row_bytes(D) : D * 2;
+    static constexpr int kNL = kRowBytes / 16;         // lanes (16-byte pieces) per key row
     static constexpr int kRPI = 32 / kNL;
     static constexpr int kRowsPerWarp = kTileRows / kConsumerWarps;   // 16
     static constexpr int kSteps = kRowsPerWarp / kRPI;
-    static constexpr int kRowBytes = D * 2;
     static constexpr int kTileBytes = kTileRows * kRowBytes;
     static constexpr int kPosOff = kStages * kTileBytes;
     static constexpr int kBarOff = kPosOff + kPosDepth * kTileRows * 4;
@@ -295,10 +301,11 @@ __device__ __forceinline__ float2 group_max_16rows(const uint8_t *rows16, const 
     return make_float2(lo, hi);
 }
 
-template <int D, bool MAXAGG>
-__global__ void __launch_bounds__(RescoreCfg<D>::kThreads, 1)
+template <int D, int FMT>
+__global__ void __launch_bounds__(RescoreCfg<D, FMT>::kThreads, 1)
 k_refine_rescore(ScoreArgs a) {
-    using C = RescoreCfg<D>;
+    using C = RescoreCfg<D, FMT>;
+    constexpr bool MAXAGG = FMT != kFmtSum;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *stages = smem;
     int *pos_s = reinterpret_cast<int *>(smem + C::kPosOff);
@@ -390,7 +397,10 @@ k_refine_rescore(ScoreArgs a) {
     // pairs 2*(lane%4) and +8 of each 16-wide k step).
     float qreg[8];
     uint32_t qf[2][D / 16][2];
-    if constexpr (!MAXAGG) {
+    Q2Query<D> Q;
+    if constexpr (FMT == kFmtQ2) {
+        q2_load_query<D>(Q, qb + ((size_t)b * Hq + (size_t)h * a.G) * D, a.G, lane);
+    } else if constexpr (!MAXAGG) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) qreg[e] = 0.f;
         for (int g = 0; g < a.G; ++g) {
@@ -414,7 +424,8 @@ k_refine_rescore(ScoreArgs a) {
         }
     }
     const bool two_tiles = a.G > 8;
-    const uint16_t *kb = static_cast<const uint16_t *>(z == 0 ? a.k : a.kz[z]) + (size_t)row * a.Lmax * D;
+    const uint8_t *kb = static_cast<const uint8_t *>(z == 0 ? a.k : a.kz[z]) +
+                        (size_t)row * a.Lmax * C::kRowBytes;
     float *S = a.S + (size_t)z * a.zS + (size_t)row * cstride;
     int32_t *cpos = a.cpos + (size_t)z * a.zS + (size_t)row * cstride;
     const int r_base = warp * C::kRowsPerWarp;
@@ -440,10 +451,10 @@ k_refine_rescore(ScoreArgs a) {
             const int r = r_base + st * C::kRPI + sub;
             const bool ok = !failed && r < nrows;
             const int krow = ok ? pos[r] : 0;
-            // the group-maximum path reads the rows by ldmatrix: swizzled chunks
-            const int chunk = MAXAGG ? (slice ^ (r & 7)) : slice;
-            cp_async16(tile + r * C::kRowBytes + chunk * 16, kb + (size_t)krow * D + slice * 8,
-                       ok ? 16u : 0u);
+            // the bf16 group-maximum path reads the rows by ldmatrix: swizzled chunks
+            const int chunk = FMT == kFmtMax ? (slice ^ (r & 7)) : slice;
+            cp_async16(tile + r * C::kRowBytes + chunk * 16,
+                       kb + (size_t)krow * C::kRowBytes + slice * 16, ok ? 16u : 0u);
         }
         cp_async_commit();
     };
@@ -458,7 +469,12 @@ k_refine_rescore(ScoreArgs a) {
         cp_async_wait<C::kStages - 1>();                // this lane's pieces of window `it`
         const uint8_t *tile = stages + (it % C::kStages) * C::kTileBytes;
         float part_[C::kSteps];
-        if constexpr (MAXAGG) {
+        if constexpr (FMT == kFmtQ2) {
+            // The warp reads rows gathered by all of its lanes.
+            __syncwarp();
+            const float2 m = q2_group_max_16rows<D>(tile + r_base * C::kRowBytes, Q, two_tiles, lane);
+            part_[0] = (lane & 3) == 1 ? m.y : m.x;
+        } else if constexpr (MAXAGG) {
             // The warp reads rows gathered by all of its lanes.
             __syncwarp();
             const float2 m = group_max_16rows<D>(tile + r_base * C::kRowBytes, qf, two_tiles, lane);
@@ -509,16 +525,17 @@ static cudaError_t launch_anchor_score_d(const ScoreArgs &a, int num_sms, cudaSt
 }
 
 cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s) {
+    if (a.agg == kAggMax && a.q2) return launch_anchor_score_q2(a, num_sms, s);
     if (a.agg == kAggMax) return launch_anchor_score_max(a, num_sms, s);
     return a.d == 128 ? launch_anchor_score_d<128>(a, num_sms, s)
                       : launch_anchor_score_d<64>(a, num_sms, s);
 }
 
 
-template <int D, bool MAXAGG>
+template <int D, int FMT>
 static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, int num_sms, cudaStream_t s) {
-    using C = RescoreCfg<D>;
-    cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D, MAXAGG>,
+    using C = RescoreCfg<D, FMT>;
+    cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D, FMT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // About one CTA per SM over all rows (of all batched layers); each row's
@@ -526,16 +543,19 @@ static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, int num_sms, cuda
     const int nz = a.nz > 1 ? a.nz : 1;
     const int rows = a.B * a.Hkv;
     const int parts = rows * nz >= num_sms ? 1 : num_sms / (rows * nz);
-    return launch_kernel(k_refine_rescore<D, MAXAGG>, dim3((unsigned)parts, (unsigned)rows, (unsigned)nz),
+    return launch_kernel(k_refine_rescore<D, FMT>, dim3((unsigned)parts, (unsigned)rows, (unsigned)nz),
                          dim3(C::kThreads), C::kSmemBytes, s, a);
 }
 
 cudaError_t launch_refine_rescore(const ScoreArgs &a, int num_sms, cudaStream_t s) {
+    if (a.agg == kAggMax && a.q2)
+        return a.d == 128 ? launch_refine_rescore_d<128, kFmtQ2>(a, num_sms, s)
+                          : launch_refine_rescore_d<64, kFmtQ2>(a, num_sms, s);
     if (a.agg == kAggMax)
-        return a.d == 128 ? launch_refine_rescore_d<128, true>(a, num_sms, s)
-                          : launch_refine_rescore_d<64, true>(a, num_sms, s);
-    return a.d == 128 ? launch_refine_rescore_d<128, false>(a, num_sms, s)
-                      : launch_refine_rescore_d<64, false>(a, num_sms, s);
+        return a.d == 128 ? launch_refine_rescore_d<128, kFmtMax>(a, num_sms, s)
+                          : launch_refine_rescore_d<64, kFmtMax>(a, num_sms, s);
+    return a.d == 128 ? launch_refine_rescore_d<128, kFmtSum>(a, num_sms, s)
+                      : launch_refine_rescore_d<64, kFmtSum>(a, num_sms, s);
 }
 
 }  // namespace prism

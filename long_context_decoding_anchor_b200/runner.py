@@ -10,14 +10,15 @@ from __future__ import annotations
 
 import torch
 
-from . import Config, lib, prism_decode_step, workspace
+from . import Config, lib, prism_decode_step, prism_decode_step_kq, workspace
 
 
 class DecodeStepGraph:
     def __init__(self, cfg: Config, q, k_layers, v_layers, lens, out=None, idx_out=None,
-                 ws=None):
+                 ws=None, kq_layers=None):
         self.cfg = cfg
         self.q, self.k, self.v, self.lens = q, list(k_layers), list(v_layers), lens
+        self.kq = list(kq_layers) if kq_layers is not None else None
         self.out = out if out is not None else torch.empty(
             (cfg.n_layers, cfg.batch, cfg.n_q_heads, cfg.head_dim), dtype=torch.bfloat16,
             device=q.device)
@@ -36,8 +37,12 @@ class DecodeStepGraph:
         self.launches = int(lib().prism_launch_count() - n0)
 
     def _call(self, stream):
-        prism_decode_step(self.cfg, self.q, self.k, self.v, self.lens, out=self.out,
-                          idx_out=self.idx_out, ws=self.ws, stream=stream)
+        if self.kq is not None:
+            prism_decode_step_kq(self.cfg, self.q, self.k, self.v, self.kq, self.lens,
+                                 out=self.out, idx_out=self.idx_out, ws=self.ws, stream=stream)
+        else:
+            prism_decode_step(self.cfg, self.q, self.k, self.v, self.lens, out=self.out,
+                              idx_out=self.idx_out, ws=self.ws, stream=stream)
 
     def replay(self):
         self.graph.replay()

@@ -97,7 +97,18 @@ def check_refine(o, cfg, q, k, lens, idx_prev, idx, cpos, cscore, ccount, rows=N
         stats["score_err"] = max(stats.get("score_err", 0.0), worst)
 
 
-def check_pool_anchor(o, cfg, q, k, lens, pool, idx, S, rows=None, stats=None):
+def _pool_ref_scores(o, cfg, qg, k_rows, pos, q2):
+    """Eq. (9) scores in fp64: on the bf16 keys, or (q2) on the oracle's own
+    2-bit quantization of them (Eq. (7)-(8))."""
+    if q2:
+        codes, al, be = o.quantize(k_rows)
+        return o.score_q2(qg, codes, al, be, pos=pos, scale=scale_of(cfg))
+    if pos is None:
+        return o.score(qg, k_rows, scale=scale_of(cfg), n=k_rows.shape[0], agg="max")
+    return o.score(qg, k_rows, pos=pos, scale=scale_of(cfg), agg="max")
+
+
+def check_pool_anchor(o, cfg, q, k, lens, pool, idx, S, rows=None, stats=None, q2=False):
     """Pool mode proposal layer: Eq. (9) scores within 1e-2 of fp64; the pool
     (Eq. (4)) and the layer's own top-kappa bit-exact against the oracle's
     TopK on the GPU's own scores; recall of both against the fp64 scores."""
@@ -110,7 +121,7 @@ def check_pool_anchor(o, cfg, q, k, lens, pool, idx, S, rows=None, stats=None):
     for b, h in rows_of(cfg, rows):
         L = int(lh[b])
         kh = bf16_bits(k[b, h, :L]) if L > 0 else np.zeros((0, cfg.head_dim), np.uint16)
-        s_ref = o.score(qh[b, h * G:(h + 1) * G], kh, scale=scale_of(cfg), n=L, agg="max")
+        s_ref = _pool_ref_scores(o, cfg, qh[b, h * G:(h + 1) * G], kh, None, q2)
         s_gpu = Sh[b, h, :L].astype(np.float64)
         if L:
             err = float(np.max(np.abs(s_gpu - s_ref)))
@@ -128,7 +139,8 @@ def check_pool_anchor(o, cfg, q, k, lens, pool, idx, S, rows=None, stats=None):
         stats["score_err"] = max(stats.get("score_err", 0.0), worst)
 
 
-def check_pool_refine(o, cfg, q, k, lens, pool, idx, cpos, cscore, ccount, rows=None, stats=None):
+def check_pool_refine(o, cfg, q, k, lens, pool, idx, cpos, cscore, ccount, rows=None, stats=None,
+                      q2=False):
     """Pool mode refined layer: the candidates are the pool's distinct valid
     positions (ascending), Eq. (9) scores within 1e-2, Eq. (6) bit-exact on
     the GPU's own candidate scores, recall against fp64."""
@@ -145,7 +157,7 @@ def check_pool_refine(o, cfg, q, k, lens, pool, idx, cpos, cscore, ccount, rows=
         assert n == len(P), f"pool candidates row {(b, h)}: {n} vs {len(P)}"
         assert np.array_equal(cp[b, h, :n], P), f"pool candidate positions row {(b, h)}"
         kh = bf16_bits(k[b, h, :max(L, 1)])
-        s_ref = o.score(qh[b, h * G:(h + 1) * G], kh, pos=P, scale=scale_of(cfg), agg="max")
+        s_ref = _pool_ref_scores(o, cfg, qh[b, h * G:(h + 1) * G], kh, P, q2)
         s_gpu = cs[b, h, :n].astype(np.float64)
         if n:
             err = float(np.max(np.abs(s_gpu - s_ref)))
@@ -208,19 +220,22 @@ def layerwise_step_check(o, cfg, inp, out, idx_all, rows=None, stats=None, layer
             continue
         if cfg.mode == prism.MODE_POOL:
             # The pool of an anchor is not an output of the step: the stage
-            # call reproduces it (bit-exact, as the selections show).
+            # call reproduces it (bit-exact, as the selections show).  With
+            # 2-bit keys the stage calls read the layer's 2-bit cache.
+            q2 = bool(cfg.flags & prism.FLAG_INT2_KEYS)
+            ks = inp["kq"][l] if q2 else k
             if anchor:
                 S = torch.empty((cfg.batch, cfg.n_kv_heads, cfg.max_len), dtype=torch.float32,
                                 device=q.device)
-                pool, idx = prism.prism_index_pool(cfg, q, k, lens, scores_out=S, ws=ws)
+                pool, idx = prism.prism_index_pool(cfg, q, ks, lens, scores_out=S, ws=ws)
                 assert torch.equal(idx, idx_all[l]), f"layer {l}: step selection != stage selection"
                 if layers is None or l in layers:
-                    check_pool_anchor(o, cfg, q, k, lens, pool, idx, S, rows, stats)
+                    check_pool_anchor(o, cfg, q, k, lens, pool, idx, S, rows, stats, q2=q2)
             elif layers is None or l in layers:
-                idx, cp, cs, cc = prism.prism_index_refine(cfg, q, k, lens, pool,
+                idx, cp, cs, cc = prism.prism_index_refine(cfg, q, ks, lens, pool,
                                                            cand_cap=cfg.max_len, ws=ws)
                 assert torch.equal(idx, idx_all[l]), f"layer {l}: step selection != stage selection"
-                check_pool_refine(o, cfg, q, k, lens, pool, idx, cp, cs, cc, rows, stats)
+                check_pool_refine(o, cfg, q, k, lens, pool, idx, cp, cs, cc, rows, stats, q2=q2)
             if layers is None or l in layers:
                 check_attention(o, cfg, q, k, v, lens, idx_all[l], out[l], rows, stats)
             continue

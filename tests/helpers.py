@@ -121,3 +121,19 @@ def sdpa_group(q_bits, k_bits, v_bits, idx, scale):
         q.view(1, G, 1, d), k.view(1, 1, L, d).expand(1, G, L, d),
         v.view(1, 1, L, d).expand(1, G, L, d), attn_mask=mask.expand(1, G, 1, L), scale=scale)
     return o.view(G, d).numpy()
+
+
+def unpack_q2(kq, d):
+    """The 2-bit key cache format of include/prism.h read back: kq uint8
+    [n][d/2] -> codes [n][d] (uint8), alpha and beta [n][d/32] (float32)."""
+    kq = np.ascontiguousarray(kq, dtype=np.uint8)
+    n = kq.shape[0]
+    ks = d // 16
+    codes = np.zeros((n, d), np.uint8)
+    for t in range(4):
+        for kk in range(ks):
+            byte = kq[:, t * ks + kk]
+            for i, off in enumerate((2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9)):
+                codes[:, 16 * kk + off] = (byte >> (2 * i)) & 3
+    par = kq[:, d // 4:].copy().view(np.float32).reshape(n, d // 32, 2)
+    return codes, par[..., 0].copy(), par[..., 1].copy()

@@ -67,7 +67,7 @@ def test_workspace_size_monotone(L):
     (dict(mode=3, kappa=1 << 19, pool_factor=4), 2),
     (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1), (dict(batch=70000, n_kv_heads=1,
                                                                   n_q_heads=1), 2),
-    (dict(flags=2), 1), (dict(n_layers=-1), 1), (dict(n_layers=5000), 2),
+    (dict(flags=4), 1), (dict(flags=2), 1), (dict(n_layers=-1), 1), (dict(n_layers=5000), 2),
 ])
 def test_invalid_config_rejected(L, bad, status):
     c = _cfg(**bad)
@@ -178,3 +178,26 @@ def test_binding_rejects_cpu_tensors():
         prism.prism_index_anchor(c, torch.zeros(1, 8, 64, dtype=torch.bfloat16),
                                  torch.zeros(1, 2, 4096, 64, dtype=torch.bfloat16),
                                  torch.zeros(1, dtype=torch.int32))
+
+
+def test_int2_key_validation(L):
+    """The 2-bit key flag belongs to pool mode; the plain step rejects it and
+    the kq step needs it."""
+    ws = ctypes.c_void_p(0x100000)
+    kp = (ctypes.c_void_p * 4)(*[0x40000 + 0x100 * i for i in range(4)])
+    c = _cfg(mode=prism.MODE_POOL, pool_factor=4, flags=prism.FLAG_INT2_KEYS)
+    ws_n = prism.prism_workspace_size(c)
+    assert L.prism_decode_step(ctypes.byref(c), A16, kp, kp, A4, A16, None, ws, ws_n, None) == 1
+    plain = _cfg(mode=prism.MODE_POOL, pool_factor=4)
+    assert L.prism_decode_step_kq(ctypes.byref(plain), A16, kp, kp, kp, A4, A16, None, ws, ws_n,
+                                  None) == 1
+    assert L.prism_decode_step_kq(ctypes.byref(c), A16, kp, kp, None, A4, A16, None, ws, ws_n,
+                                  None) == 1
+    bad = (ctypes.c_void_p * 4)(0x40000, 0x40108, 0x40200, 0x40300)          # kq[1] misaligned
+    assert L.prism_decode_step_kq(ctypes.byref(c), A16, kp, kp, bad, A4, A16, None, ws, ws_n,
+                                  None) == 1
+    q = L.prism_quantize_keys
+    assert q(ctypes.byref(c), None, A4, 0, A16, ws, 256, None) == 1
+    assert q(ctypes.byref(c), A16, A4, -1, A16, ws, 256, None) == 1          # negative start
+    assert q(ctypes.byref(c), A16, A4, 0, MIS, ws, 256, None) == 1           # kq misaligned
+    assert q(ctypes.byref(c), A16, A4, 0, A16, None, 256, None) == 1         # no status word

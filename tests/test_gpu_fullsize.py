@@ -25,7 +25,7 @@ def _gpu():
     prism.lib()
 
 
-def _chain_check(oracle, w, inp, out, idx, b, h, rho=0):
+def _chain_check(oracle, w, inp, out, idx, b, h, rho=0, qbits=0):
     """The oracle's fp64 chain on one row: recall of every layer's GPU
     selection, and the outputs against the oracle's own chain (pool mode
     when rho > 0)."""
@@ -36,7 +36,8 @@ def _chain_check(oracle, w, inp, out, idx, b, h, rho=0):
     vs = [bf16_bits(t[b:b + 1, h:h + 1]) for t in inp["v"]]
     lens = inp["lens"][b:b + 1].cpu().numpy()
     ref_out, ref_idx = oracle.decode_step(q, ks, vs, lens, w.kappa, w.radius, w.anchor_mask(),
-                                          mode=MODE_POOL if rho else MODE_REFINE, rho=max(rho, 1))
+                                          mode=MODE_POOL if rho else MODE_REFINE, rho=max(rho, 1),
+                                          qbits=qbits)
     gi = idx[:, b, h].cpu().numpy()
     worst = min(recall(gi[l], ref_idx[l, 0, 0]) for l in range(w.n_layers))
     assert worst >= RECALL_MIN, f"chain recall row {(b, h)}: {worst}"
@@ -52,15 +53,20 @@ def _chain_check(oracle, w, inp, out, idx, b, h, rho=0):
     (5, [(0, 2), (0, 7)], [0, 1, 2, 6, 7]),
     (4, [(0, 0), (7, 3), (15, 6)], [0, 1, 2, 3, 4, 13, 14, 15]),
 ])
-@pytest.mark.parametrize("rho", [0, 4], ids=["refine", "pool4"])
-def test_full_size_sampled_rows(oracle, wkey, rows, layers, rho):
+@pytest.mark.parametrize("rho,q2", [(0, False), (4, False), (4, True)],
+                         ids=["refine", "pool4", "pool4-int2"])
+def test_full_size_sampled_rows(oracle, wkey, rows, layers, rho, q2):
     w = synth.WORKLOADS[wkey]
     inp = synth.make_inputs(w, device="cuda")
-    cfg = (prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=rho) if rho
+    cfg = (prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=rho,
+                                      flags=prism.FLAG_INT2_KEYS if q2 else 0) if rho
            else prism.Config.from_workload(w))
+    if q2:
+        inp["kq"] = [prism.prism_quantize_keys(cfg, k, inp["lens"]) for k in inp["k"]]
     idx = torch.empty((w.n_layers, w.batch, w.n_kv_heads, w.kappa), dtype=torch.int32,
                       device="cuda")
-    g = DecodeStepGraph(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], idx_out=idx)
+    g = DecodeStepGraph(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], idx_out=idx,
+                        kq_layers=inp.get("kq"))
     for _ in range(2):
         g.replay()
     torch.cuda.synchronize()
@@ -69,7 +75,7 @@ def test_full_size_sampled_rows(oracle, wkey, rows, layers, rho):
     out = g.out.clone()
     del g
     layerwise_step_check(oracle, cfg, inp, out, idx, rows=rows, layers=layers)
-    _chain_check(oracle, w, inp, out, idx, *rows[0], rho=rho)
+    _chain_check(oracle, w, inp, out, idx, *rows[0], rho=rho, qbits=2 if q2 else 0)
     del inp, out, idx
     gc.collect()
     torch.cuda.empty_cache()

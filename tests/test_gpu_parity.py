@@ -349,3 +349,88 @@ def test_table9_hybrid_pattern_pool(oracle):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(idx_g, idx) and torch.equal(g.out, out)
+
+
+# -- 2-bit proposal keys (Eq. (7)-(9)) in pool mode ---------------------------
+from helpers import unpack_q2   # noqa: E402
+
+
+@pytest.mark.parametrize("name", ["tiny-full", "d128-g8-ragged", "d64-g2-batch"])
+def test_quantize_keys_bit_exact(oracle, name):
+    """The 2-bit cache equals the oracle's quantization of every row, codes and
+    alpha/beta bit for bit; positions outside [start, len) are left alone."""
+    from oracle import bf16_bits
+    w = SHAPES[name]
+    inp = _inputs(w, layers=[0])
+    cfg = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=4)
+    k, lens = inp["k"][0], inp["lens"]
+    sentinel = 0xA5
+    kq = torch.full((w.batch, w.n_kv_heads, w.max_len, w.head_dim // 2), sentinel,
+                    dtype=torch.uint8, device="cuda")
+    start = 5
+    prism.prism_quantize_keys(cfg, k, lens, start=start, kq=kq)
+    torch.cuda.synchronize()
+    kqh = kq.cpu().numpy()
+    lh = lens.cpu().numpy()
+    for b in range(w.batch):
+        L = int(lh[b])
+        for h in range(w.n_kv_heads):
+            codes, al, be = oracle.quantize(bf16_bits(k[b, h, start:L]))
+            gc, ga, gb = unpack_q2(kqh[b, h, start:L], w.head_dim)
+            assert np.array_equal(gc, codes), (b, h)
+            assert np.array_equal(ga.view(np.uint32), al.view(np.uint32)), (b, h)
+            assert np.array_equal(gb.view(np.uint32), be.view(np.uint32)), (b, h)
+            assert np.all(kqh[b, h, :start] == sentinel) and np.all(kqh[b, h, L:] == sentinel)
+
+
+def _q2_inputs(w, cfg, layers=None):
+    inp = _inputs(w, layers=layers)
+    inp["kq"] = [prism.prism_quantize_keys(cfg, k, inp["lens"]) for k in inp["k"]]
+    return inp
+
+
+@pytest.mark.parametrize("name", ["tiny-full", "d128-g4", "d128-g8-ragged", "d128-g16", "d64-g2-batch"])
+def test_q2_pool_stages(oracle, name):
+    from gpu_checks import check_pool_anchor, check_pool_refine
+    w = SHAPES[name]
+    cfg = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=4,
+                                     flags=prism.FLAG_INT2_KEYS)
+    inp = _q2_inputs(w, cfg, layers=[0, 1])
+    lens = inp["lens"]
+    S = torch.empty((w.batch, w.n_kv_heads, w.max_len), dtype=torch.float32, device="cuda")
+    ws = prism.workspace(cfg)
+    pool, idx0 = prism.prism_index_pool(cfg, inp["q"][0], inp["kq"][0], lens, scores_out=S, ws=ws)
+    check_pool_anchor(oracle, cfg, inp["q"][0], inp["k"][0], lens, pool, idx0, S, q2=True)
+    idx1, cp, cs, cc = prism.prism_index_refine(cfg, inp["q"][1], inp["kq"][1], lens, pool,
+                                                cand_cap=w.max_len, ws=ws)
+    check_pool_refine(oracle, cfg, inp["q"][1], inp["k"][1], lens, pool, idx1, cp, cs, cc, q2=True)
+    st, detail = prism.prism_check_device_status(ws)
+    assert st == 0, detail
+
+
+@pytest.mark.parametrize("wkey", [1, 2])
+def test_q2_decode_step(oracle, wkey):
+    """The tiny and 32K workloads in pool mode on 2-bit keys: stage-by-stage
+    checks and the chain against the oracle's (qbits = 2)."""
+    from long_context_decoding_anchor_b200.runner import DecodeStepGraph
+    w = synth.WORKLOADS[wkey]
+    cfg = prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=4,
+                                     flags=prism.FLAG_INT2_KEYS)
+    inp = _q2_inputs(w, cfg)
+    out, idx = prism.prism_decode_step_kq(cfg, inp["q"], inp["k"], inp["v"], inp["kq"],
+                                          inp["lens"], want_idx=True)
+    layerwise_step_check(oracle, cfg, inp, out, idx)
+    from oracle import MODE_POOL, bf16_bits
+    _, ref_idx = oracle.decode_step(bf16_bits(inp["q"]), [bf16_bits(t) for t in inp["k"]],
+                                    [bf16_bits(t) for t in inp["v"]], inp["lens"].cpu().numpy(),
+                                    w.kappa, 0, w.anchor_mask(), mode=MODE_POOL, rho=4, qbits=2)
+    gi = idx.cpu().numpy()
+    for l in range(w.n_layers):
+        for h in range(w.n_kv_heads):
+            assert recall(gi[l, 0, h], ref_idx[l, 0, h]) >= 0.999, (l, h)
+    idx_g = torch.empty_like(idx)
+    g = DecodeStepGraph(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], idx_out=idx_g,
+                        kq_layers=inp["kq"])
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(idx_g, idx) and torch.equal(g.out, out)
