@@ -57,16 +57,17 @@ __device__ __forceinline__ void mma16816_bf16(float (&c)[4], uint32_t a0, uint32
 // 2*(lane%4) and +8 of each k step).  S: sum over each group m of the
 // elements of the heads this lane's accumulator columns hold (heads
 // (8u + 2*(lane%4)) % G and (8u + 2*(lane%4) + 1) % G).
-template <int D>
+template <int D, int NT>
 struct Q2Query {
-    uint32_t qf[2][D / 16][2];
-    float S[2][D / kQ2Group][2];
+    uint32_t qf[NT][D / 16][2];
+    float S[NT][D / kQ2Group][2];
 };
 
-template <int D>
-__device__ __forceinline__ void q2_load_query(Q2Query<D> &Q, const uint16_t *qg, int G, int lane) {
+// NT n-tiles of 8 heads: 1 for G <= 8, 2 for G = 16.
+template <int D, int NT>
+__device__ __forceinline__ void q2_load_query(Q2Query<D, NT> &Q, const uint16_t *qg, int G, int lane) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < NT; ++u) {
         const uint16_t *qh = qg + (size_t)((8 * u + (lane >> 2)) % G) * D + 2 * (lane & 3);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -92,9 +93,9 @@ __device__ __forceinline__ void q2_load_query(Q2Query<D> &Q, const uint16_t *qg,
 // shared memory), computed side by side so that their latency chains
 // overlap: out[i].x for row lane/4 of block i, out[i].y for row lane/4 + 8,
 // in every lane of the quad.
-template <int D, int NS>
+template <int D, int NT, int NS>
 __device__ __forceinline__ void q2_group_max_rows(const uint8_t *rows16, int block_stride,
-                                                  const Q2Query<D> &Q, bool two_tiles, int lane,
+                                                  const Q2Query<D, NT> &Q, int lane,
                                                   float2 (&out)[NS]) {
     constexpr int RB = q2_row_bytes(D);
     constexpr int KS = D / 16;
@@ -111,11 +112,11 @@ __device__ __forceinline__ void q2_group_max_rows(const uint8_t *rows16, int blo
             w1[i][j] = *reinterpret_cast<const uint32_t *>(r1 + t * KS + 4 * j);
         }
     }
-    float acc[NS][2][M][4];
+    float acc[NS][NT][M][4];
 #pragma unroll
     for (int i = 0; i < NS; ++i)
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
+        for (int u = 0; u < NT; ++u)
 #pragma unroll
             for (int m = 0; m < M; ++m)
 #pragma unroll
@@ -129,9 +130,9 @@ __device__ __forceinline__ void q2_group_max_rows(const uint8_t *rows16, int blo
             const uint32_t b1 = (w1[i][kk >> 2] >> (8 * (kk & 3))) & 0xffu;
             uint32_t a0, a1, a2, a3;
             q2_afrag(b0, b1, a0, a1, a2, a3);
-            mma16816_bf16(acc[i][0][m], a0, a1, a2, a3, Q.qf[0][kk][0], Q.qf[0][kk][1]);
-            if (two_tiles)
-                mma16816_bf16(acc[i][1][m], a0, a1, a2, a3, Q.qf[1][kk][0], Q.qf[1][kk][1]);
+#pragma unroll
+            for (int u = 0; u < NT; ++u)
+                mma16816_bf16(acc[i][u][m], a0, a1, a2, a3, Q.qf[u][kk][0], Q.qf[u][kk][1]);
         }
     }
 #pragma unroll
@@ -139,8 +140,7 @@ __device__ __forceinline__ void q2_group_max_rows(const uint8_t *rows16, int blo
         const uint8_t *r0 = rows16 + i * block_stride + g * RB, *r1 = r0 + 8 * RB;
         float lo = -INFINITY, hi = -INFINITY;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (u == 1 && !two_tiles) break;
+        for (int u = 0; u < NT; ++u) {
             float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;  // (row g | g+8) x (column 2t | 2t+1)
 #pragma unroll
             for (int m = 0; m < M; ++m) {
@@ -163,11 +163,11 @@ __device__ __forceinline__ void q2_group_max_rows(const uint8_t *rows16, int blo
     }
 }
 
-template <int D>
-__device__ __forceinline__ float2 q2_group_max_16rows(const uint8_t *rows16, const Q2Query<D> &Q,
-                                                      bool two_tiles, int lane) {
+template <int D, int NT>
+__device__ __forceinline__ float2 q2_group_max_16rows(const uint8_t *rows16, const Q2Query<D, NT> &Q,
+                                                      int lane) {
     float2 o[1];
-    q2_group_max_rows<D, 1>(rows16, 0, Q, two_tiles, lane, o);
+    q2_group_max_rows<D, NT, 1>(rows16, 0, Q, lane, o);
     return o[0];
 }
 

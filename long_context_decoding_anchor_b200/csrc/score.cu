@@ -301,7 +301,7 @@ __device__ __forceinline__ float2 group_max_16rows(const uint8_t *rows16, const 
     return make_float2(lo, hi);
 }
 
-template <int D, int FMT>
+template <int D, int FMT, int NT = 1>
 __global__ void __launch_bounds__(RescoreCfg<D, FMT>::kThreads, 1)
 k_refine_rescore(ScoreArgs a) {
     using C = RescoreCfg<D, FMT>;
@@ -397,9 +397,9 @@ k_refine_rescore(ScoreArgs a) {
     // pairs 2*(lane%4) and +8 of each 16-wide k step).
     float qreg[8];
     uint32_t qf[2][D / 16][2];
-    Q2Query<D> Q;
+    Q2Query<D, NT> Q;
     if constexpr (FMT == kFmtQ2) {
-        q2_load_query<D>(Q, qb + ((size_t)b * Hq + (size_t)h * a.G) * D, a.G, lane);
+        q2_load_query<D, NT>(Q, qb + ((size_t)b * Hq + (size_t)h * a.G) * D, a.G, lane);
     } else if constexpr (!MAXAGG) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) qreg[e] = 0.f;
@@ -472,7 +472,7 @@ k_refine_rescore(ScoreArgs a) {
         if constexpr (FMT == kFmtQ2) {
             // The warp reads rows gathered by all of its lanes.
             __syncwarp();
-            const float2 m = q2_group_max_16rows<D>(tile + r_base * C::kRowBytes, Q, two_tiles, lane);
+            const float2 m = q2_group_max_16rows<D, NT>(tile + r_base * C::kRowBytes, Q, lane);
             part_[0] = (lane & 3) == 1 ? m.y : m.x;
         } else if constexpr (MAXAGG) {
             // The warp reads rows gathered by all of its lanes.
@@ -532,10 +532,10 @@ cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s)
 }
 
 
-template <int D, int FMT>
+template <int D, int FMT, int NT = 1>
 static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, int num_sms, cudaStream_t s) {
     using C = RescoreCfg<D, FMT>;
-    cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D, FMT>,
+    cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D, FMT, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     // About one CTA per SM over all rows (of all batched layers); each row's
@@ -543,14 +543,18 @@ static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, int num_sms, cuda
     const int nz = a.nz > 1 ? a.nz : 1;
     const int rows = a.B * a.Hkv;
     const int parts = rows * nz >= num_sms ? 1 : num_sms / (rows * nz);
-    return launch_kernel(k_refine_rescore<D, FMT>, dim3((unsigned)parts, (unsigned)rows, (unsigned)nz),
+    return launch_kernel(k_refine_rescore<D, FMT, NT>, dim3((unsigned)parts, (unsigned)rows, (unsigned)nz),
                          dim3(C::kThreads), C::kSmemBytes, s, a);
 }
 
 cudaError_t launch_refine_rescore(const ScoreArgs &a, int num_sms, cudaStream_t s) {
-    if (a.agg == kAggMax && a.q2)
-        return a.d == 128 ? launch_refine_rescore_d<128, kFmtQ2>(a, num_sms, s)
-                          : launch_refine_rescore_d<64, kFmtQ2>(a, num_sms, s);
+    if (a.agg == kAggMax && a.q2) {
+        if (a.G > 8)
+            return a.d == 128 ? launch_refine_rescore_d<128, kFmtQ2, 2>(a, num_sms, s)
+                              : launch_refine_rescore_d<64, kFmtQ2, 2>(a, num_sms, s);
+        return a.d == 128 ? launch_refine_rescore_d<128, kFmtQ2, 1>(a, num_sms, s)
+                          : launch_refine_rescore_d<64, kFmtQ2, 1>(a, num_sms, s);
+    }
     if (a.agg == kAggMax)
         return a.d == 128 ? launch_refine_rescore_d<128, kFmtMax>(a, num_sms, s)
                           : launch_refine_rescore_d<64, kFmtMax>(a, num_sms, s);

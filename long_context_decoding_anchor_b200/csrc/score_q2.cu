@@ -9,7 +9,7 @@
 //
 // k_anchor_score_q2: the persistent scan of k_anchor_score over 512-row tiles
 // of the quantized cache (d/2 bytes a row: 32 KB tiles at d = 128), a 4-stage
-// ring of 1-D bulk copies, eight consumer warps of 64 rows each scoring on
+// ring of 1-D bulk copies, sixteen consumer warps of 32 rows each scoring on
 // the tensor cores, scores and the first-digit histogram as in the bf16 scan.
 #include "q2_impl.cuh"
 #include "tiles.cuh"
@@ -94,12 +94,12 @@ cudaError_t launch_quantize_keys(const void *k, const int32_t *len, int B, int H
 
 template <int D>
 struct Q2ScanCfg {
-    // 512-row tiles (32 KB at d = 128): each consumer warp scores 64 rows, two
-    // 16-row blocks side by side, so the latency of its mma chain is hidden
-    // behind the other block's and amortised over a large tile.
+    // 512-row tiles (32 KB at d = 128): each of 16 consumer warps scores 32
+    // rows, two 16-row blocks side by side, so that the latency of the mma
+    // chains is hidden behind other blocks and warps.
     static constexpr int kTileRows = 512;
     static constexpr int kStages = 4;
-    static constexpr int kConsumerWarps = 8;
+    static constexpr int kConsumerWarps = 16;
     static constexpr int kRowsPerWarp = kTileRows / kConsumerWarps;
     static constexpr int kThreads = 32 * (kConsumerWarps + 1);
     static constexpr int kRowBytes = q2_row_bytes(D);
@@ -108,10 +108,10 @@ struct Q2ScanCfg {
 };
 
 __device__ __forceinline__ void q2_consumer_sync() {
-    asm volatile("bar.sync 1, 256;" ::: "memory");
+    asm volatile("bar.sync 1, 512;" ::: "memory");
 }
 
-template <int D>
+template <int D, int NT>
 __global__ void __launch_bounds__(Q2ScanCfg<D>::kThreads, 1)
 k_anchor_score_q2(ScoreArgs a) {
     using C = Q2ScanCfg<D>;
@@ -193,8 +193,7 @@ k_anchor_score_q2(ScoreArgs a) {
     pdl_wait();
     const uint16_t *qb = static_cast<const uint16_t *>(a.q);
     const int Hq = a.Hkv * a.G;
-    const bool two_tiles = a.G > 8;
-    Q2Query<D> Q;
+    Q2Query<D, NT> Q;
     int cur_row = -1;
     TileCursor c = cur0;
     bool failed = false;
@@ -215,7 +214,7 @@ k_anchor_score_q2(ScoreArgs a) {
                 }
                 q2_consumer_sync();
             }
-            q2_load_query<D>(Q, qb + ((size_t)c.b * Hq + (size_t)c.h * a.G) * D, a.G, lane);
+            q2_load_query<D, NT>(Q, qb + ((size_t)c.b * Hq + (size_t)c.h * a.G) * D, a.G, lane);
             cur_row = row;
         }
         int L = __ldg(a.len + c.b);
@@ -226,16 +225,16 @@ k_anchor_score_q2(ScoreArgs a) {
         }
         if (!failed) {
             const uint8_t *rows_w = stages + s * C::kTileBytes + warp * C::kRowsPerWarp * C::kRowBytes;
-            float2 mx[2][2];
+            float2 mx[C::kRowsPerWarp / 32][2];
 #pragma unroll
-            for (int pr = 0; pr < 2; ++pr)
-                q2_group_max_rows<D, 2>(rows_w + pr * 32 * C::kRowBytes, 16 * C::kRowBytes, Q,
-                                        two_tiles, lane, mx[pr]);
+            for (int pr = 0; pr < C::kRowsPerWarp / 32; ++pr)
+                q2_group_max_rows<D, NT, 2>(rows_w + pr * 32 * C::kRowBytes, 16 * C::kRowBytes, Q,
+                                            lane, mx[pr]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
             if (t < 2) {
 #pragma unroll
-                for (int blk = 0; blk < 4; ++blk) {
+                for (int blk = 0; blk < C::kRowsPerWarp / 16; ++blk) {
                     const float2 m2 = mx[blk >> 1][blk & 1];
                     const int pos = c.j * TILE + warp * C::kRowsPerWarp + 16 * blk + g + (t == 1 ? 8 : 0);
                     if (pos < L) {
@@ -258,21 +257,25 @@ k_anchor_score_q2(ScoreArgs a) {
     }
 }
 
-template <int D>
+template <int D, int NT>
 static cudaError_t launch_anchor_score_q2_d(const ScoreArgs &a, int num_sms, cudaStream_t s) {
     using C = Q2ScanCfg<D>;
-    cudaError_t e = cudaFuncSetAttribute(k_anchor_score_q2<D>,
+    cudaError_t e = cudaFuncSetAttribute(k_anchor_score_q2<D, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     const long long rows = (long long)a.B * a.Hkv;
     const long long max_tiles = rows * ((a.Lmax + C::kTileRows - 1) / C::kTileRows);
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
-    return launch_kernel(k_anchor_score_q2<D>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, s, a);
+    return launch_kernel(k_anchor_score_q2<D, NT>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, s,
+                         a);
 }
 
 cudaError_t launch_anchor_score_q2(const ScoreArgs &a, int num_sms, cudaStream_t s) {
-    return a.d == 128 ? launch_anchor_score_q2_d<128>(a, num_sms, s)
-                      : launch_anchor_score_q2_d<64>(a, num_sms, s);
+    if (a.G > 8)
+        return a.d == 128 ? launch_anchor_score_q2_d<128, 2>(a, num_sms, s)
+                          : launch_anchor_score_q2_d<64, 2>(a, num_sms, s);
+    return a.d == 128 ? launch_anchor_score_q2_d<128, 1>(a, num_sms, s)
+                      : launch_anchor_score_q2_d<64, 1>(a, num_sms, s);
 }
 
 }  // namespace prism
