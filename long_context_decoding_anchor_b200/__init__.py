@@ -10,7 +10,10 @@ Functions carry the C names:
   prism_workspace_size, prism_index_anchor, prism_index_pool,
   prism_index_refine, prism_sparse_decode, prism_decode_step,
   prism_check_device_status, prism_debug_wait_timeout
-plus ``Config`` (the prism_config_t struct) and ``workspace()``.
+plus ``Config`` (the prism_config_t struct) and ``workspace()``; and the
+context-parallel calls of ``include/prism_cp.h`` (prism_cp_workspace_size,
+prism_cp_index_local, prism_cp_merge, prism_cp_attn_local, prism_cp_combine,
+with ``CpShard`` and ``cp_workspace()``), which ``cp.py`` strings together.
 """
 from __future__ import annotations
 
@@ -35,7 +38,9 @@ EXPORTS = ("prism_workspace_size", "prism_index_anchor", "prism_index_refine",
            "prism_sparse_decode", "prism_decode_step", "prism_check_device_status",
            "prism_debug_wait_timeout", "prism_score_anchor", "prism_status_string",
            "prism_version", "prism_launch_count", "prism_sparse_decode_noalloc",
-           "prism_index_pool", "prism_quantize_keys", "prism_decode_step_kq")
+           "prism_index_pool", "prism_quantize_keys", "prism_decode_step_kq",
+           "prism_cp_workspace_size", "prism_cp_index_local", "prism_cp_merge",
+           "prism_cp_attn_local", "prism_cp_combine")
 
 
 class PrismError(RuntimeError):
@@ -87,6 +92,17 @@ class Config(ctypes.Structure):
         return self.pool_factor * self.kappa if self.mode == MODE_POOL else self.kappa
 
 
+class CpShard(ctypes.Structure):
+    """prism_cp_shard_t: rank `rank` of `n_ranks` holds the positions
+    [rank * shard_len, (rank + 1) * shard_len) of every sequence."""
+    _fields_ = [("n_ranks", ctypes.c_int32), ("rank", ctypes.c_int32),
+                ("shard_len", ctypes.c_int32)]
+
+    @property
+    def lo(self) -> int:
+        return self.rank * self.shard_len
+
+
 _lib = None
 
 
@@ -122,6 +138,14 @@ def lib() -> ctypes.CDLL:
         L.prism_status_string.argtypes = [ctypes.c_int]
         L.prism_status_string.restype = ctypes.c_char_p
         L.prism_version.restype = i32
+        shp = ctypes.POINTER(CpShard)
+        L.prism_cp_workspace_size.argtypes = [cfgp, shp, ctypes.POINTER(sz)]
+        L.prism_cp_index_local.argtypes = [cfgp, shp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_cp_merge.argtypes = [cfgp, shp, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_cp_attn_local.argtypes = [cfgp, shp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.prism_cp_combine.argtypes = [cfgp, i32, vp, vp, vp]
+        for name in EXPORTS[-5:]:
+            getattr(L, name).restype = ctypes.c_int
         for name in EXPORTS[:8]:
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -384,6 +408,106 @@ def prism_decode_step_kq(cfg: Config, q, k_layers, v_layers, kq_layers, lens, ou
     return (out, idx_out) if idx_out is not None else out
 
 
+# -- context parallel (include/prism_cp.h) -----------------------------------------
+def prism_cp_workspace_size(cfg: Config, shard: CpShard) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().prism_cp_workspace_size(ctypes.byref(cfg), ctypes.byref(shard), ctypes.byref(n)),
+           "prism_cp_workspace_size")
+    return n.value
+
+
+def cp_workspace(cfg: Config, shard: CpShard, device=None) -> torch.Tensor:
+    return torch.zeros(prism_cp_workspace_size(cfg, shard), dtype=torch.uint8,
+                       device=device or torch.device("cuda"))
+
+
+def _need_shard_kv(cfg: Config, shard: CpShard, t, name):
+    _need(t, name, torch.bfloat16, (cfg.batch, cfg.n_kv_heads, shard.shard_len, cfg.head_dim))
+
+
+def prism_cp_index_local(cfg: Config, shard: CpShard, q, k, lens, src=None, ws=None,
+                         stream=None):
+    """This shard's half of a selection: (cand_pos, cand_score) [B][Hkv][kappa],
+    plus (pool_pos, pool_score) [B][Hkv][rho*kappa] for a pool-mode anchor
+    (src None).  src: the canonical global source selection of a refined layer."""
+    B, Hq, Hkv, d = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    _need(q, "q", torch.bfloat16, (B, Hq, d))
+    _need_shard_kv(cfg, shard, k, "k")
+    _need(lens, "lens", torch.int32, (B,))
+    if src is not None:
+        _need(src, "src", torch.int32, (B, Hkv, cfg.src_kappa))
+    dev = q.device
+    cp = torch.empty((B, Hkv, cfg.kappa), dtype=torch.int32, device=dev)
+    cs = torch.empty((B, Hkv, cfg.kappa), dtype=torch.float32, device=dev)
+    pp = ps = None
+    if cfg.mode == MODE_POOL and src is None:
+        pp = torch.empty((B, Hkv, cfg.src_kappa), dtype=torch.int32, device=dev)
+        ps = torch.empty((B, Hkv, cfg.src_kappa), dtype=torch.float32, device=dev)
+    ws = cp_workspace(cfg, shard, dev) if ws is None else ws
+    _check(lib().prism_cp_index_local(ctypes.byref(cfg), ctypes.byref(shard), _p(q), _p(k),
+                                      _p(lens), _p(src), _p(cp), _p(cs), _p(pp), _p(ps), _p(ws),
+                                      ws.numel(), _stream(stream)),
+           "prism_cp_index_local")
+    return (cp, cs) if pp is None else (cp, cs, pp, ps)
+
+
+def prism_cp_merge(cfg: Config, shard: CpShard, cand_pos, cand_score, lens, idx_out=None,
+                   ws=None, stream=None):
+    """Exact top-n over the gathered lists [R][B][Hkv][n] (n = kappa, or rho*kappa
+    for a pool): ascending global positions [B][Hkv][n], -1 padded."""
+    R, B, Hkv = shard.n_ranks, cfg.batch, cfg.n_kv_heads
+    if cand_pos.dim() != 4:
+        raise ValueError("cand_pos must be [R][B][Hkv][n]")
+    n = int(cand_pos.shape[3])
+    _need(cand_pos, "cand_pos", torch.int32, (R, B, Hkv, n))
+    _need(cand_score, "cand_score", torch.float32, (R, B, Hkv, n))
+    _need(lens, "lens", torch.int32, (B,))
+    if idx_out is None:
+        idx_out = torch.empty((B, Hkv, n), dtype=torch.int32, device=cand_pos.device)
+    _need(idx_out, "idx_out", torch.int32, (B, Hkv, n))
+    ws = cp_workspace(cfg, shard, cand_pos.device) if ws is None else ws
+    _check(lib().prism_cp_merge(ctypes.byref(cfg), ctypes.byref(shard), n, _p(cand_pos),
+                                _p(cand_score), _p(lens), _p(idx_out), _p(ws), ws.numel(),
+                                _stream(stream)),
+           "prism_cp_merge")
+    return idx_out
+
+
+def prism_cp_attn_local(cfg: Config, shard: CpShard, q, k, v, lens, idx, part_out=None,
+                        ws=None, stream=None):
+    """This shard's split-softmax partial fp32 [B][Hq][d + 2] (acc, m, l)."""
+    B, Hq, Hkv, d = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    _need(q, "q", torch.bfloat16, (B, Hq, d))
+    _need_shard_kv(cfg, shard, k, "k")
+    _need_shard_kv(cfg, shard, v, "v")
+    _need(lens, "lens", torch.int32, (B,))
+    _need(idx, "idx", torch.int32, (B, Hkv, cfg.kappa))
+    if part_out is None:
+        part_out = torch.empty((B, Hq, d + 2), dtype=torch.float32, device=q.device)
+    _need(part_out, "part_out", torch.float32, (B, Hq, d + 2))
+    ws = cp_workspace(cfg, shard, q.device) if ws is None else ws
+    _check(lib().prism_cp_attn_local(ctypes.byref(cfg), ctypes.byref(shard), _p(q), _p(k), _p(v),
+                                     _p(lens), _p(idx), _p(part_out), _p(ws), ws.numel(),
+                                     _stream(stream)),
+           "prism_cp_attn_local")
+    return part_out
+
+
+def prism_cp_combine(cfg: Config, part_all, out=None, stream=None):
+    """Merge of the gathered partials [R][B][Hq][d + 2] into bf16 [B][Hq][d]."""
+    B, Hq, d = cfg.batch, cfg.n_q_heads, cfg.head_dim
+    if part_all.dim() != 4:
+        raise ValueError("part_all must be [R][B][Hq][d + 2]")
+    R = int(part_all.shape[0])
+    _need(part_all, "part_all", torch.float32, (R, B, Hq, d + 2))
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=part_all.device)
+    _need(out, "out", torch.bfloat16, (B, Hq, d))
+    _check(lib().prism_cp_combine(ctypes.byref(cfg), R, _p(part_all), _p(out), _stream(stream)),
+           "prism_cp_combine")
+    return out
+
+
 def prism_check_device_status(ws: torch.Tensor, stream=None):
     """Synchronises; returns (status, [code, where, value, 0]) and clears the word."""
     detail = (ctypes.c_uint32 * 4)()
@@ -407,4 +531,6 @@ __all__ = ["Config", "PrismError", "lib", "workspace", "prism_workspace_size",
            "prism_decode_step", "prism_check_device_status", "prism_debug_wait_timeout",
            "prism_score_anchor", "prism_sparse_decode_noalloc", "raw_status", "MODE_REFINE", "MODE_STATIC_REUSE", "MODE_DENSE_ANCHOR", "MODE_POOL",
            "CHAIN_PREV", "CHAIN_ANCHOR", "LAYER_REFINED", "LAYER_ANCHOR", "LAYER_SHARED", "FLAG_SERIAL",
-           "FLAG_INT2_KEYS", "prism_quantize_keys", "prism_decode_step_kq", "EXPORTS", "LIB_PATH"]
+           "FLAG_INT2_KEYS", "prism_quantize_keys", "prism_decode_step_kq", "EXPORTS", "LIB_PATH",
+           "CpShard", "cp_workspace", "prism_cp_workspace_size", "prism_cp_index_local",
+           "prism_cp_merge", "prism_cp_attn_local", "prism_cp_combine"]

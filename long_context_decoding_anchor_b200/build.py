@@ -24,7 +24,7 @@ def sources() -> list:
 
 def _inputs() -> list:
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [
-        os.path.join(INCLUDE, "prism.h")]
+        os.path.join(INCLUDE, "prism.h"), os.path.join(INCLUDE, "prism_cp.h")]
 
 
 def up_to_date() -> bool:

@@ -18,6 +18,10 @@
 // of each group rescore their anchor's pool together (one launch of each
 // kernel per group) once the pool is selected.
 // PRISM_FLAG_SERIAL runs everything on the caller's stream instead.
+//
+// The context-parallel calls (include/prism_cp.h, at the end of this file)
+// run the same kernels on one rank's shard of the positions, with the
+// helpers of cp.cu around them.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -26,7 +30,9 @@
 #include <mutex>
 #include <vector>
 
+#include "cp_internal.cuh"
 #include "prism.h"
+#include "prism_cp.h"
 #include "prism_internal.cuh"
 
 using namespace prism;
@@ -892,5 +898,267 @@ const char *prism_status_string(prism_status_t st) {
 uint64_t prism_launch_count(void) { return g_launches; }
 
 int32_t prism_version(void) { return 10200; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Context-parallel pieces (include/prism_cp.h).  A rank's workspace starts
+// with the single-GPU layout of its shard (capacity shard_len, one layer),
+// followed by the buffers of the shard-local steps and of the merge.
+namespace {
+
+prism_config_t local_config(const prism_config_t &c, const prism_cp_shard_t &sh) {
+    prism_config_t lc = c;
+    lc.max_len = sh.shard_len;
+    lc.n_layers = 1;
+    lc.anchor_mask = nullptr;
+    return lc;
+}
+
+// Radius of a refined layer's proposal: the pool is rescored as it is.
+int cp_radius(const prism_config_t &c) { return pool_mode(c) ? 0 : c.radius; }
+
+// Entries of the radius-0 source that a refined layer's proposal becomes
+// inside one shard: at most |source| * (2r + 1) positions, at most shard_len.
+int cp_local_src(const prism_config_t &c, const prism_cp_shard_t &sh) {
+    const long long n = (long long)src_kappa_of(c) * (2LL * cp_radius(c) + 1);
+    return (int)(n < sh.shard_len ? n : sh.shard_len);
+}
+
+struct CpLayout {
+    Layout l;
+    int lsrc_k, kmax, R, cs_m;
+    size_t llen, lsrc, lsrc_off, lsel, lpool, latt, lout;
+    size_t mS, mcpos, mcount, mhist, mspill, total;
+};
+
+CpLayout make_cp_layout(const prism_config_t &c, const prism_cp_shard_t &sh) {
+    CpLayout L{};
+    L.l = make_layout(local_config(c, sh));
+    const size_t rows = (size_t)c.batch * c.n_kv_heads;
+    L.lsrc_k = cp_local_src(c, sh);
+    L.kmax = src_kappa_of(c);
+    L.R = sh.n_ranks;
+    L.cs_m = (int)(((long long)L.R * L.kmax + 3) & ~3LL);
+    size_t off = L.l.total;
+    L.llen = off;     off = align256(off + (size_t)c.batch * sizeof(int32_t));
+    L.lsrc = off;     off = align256(off + rows * (size_t)L.lsrc_k * sizeof(int32_t));
+    L.lsrc_off = off; off = align256(off + rows * ((size_t)L.lsrc_k + 1) * sizeof(int32_t));
+    L.lsel = off;     off = align256(off + rows * (size_t)c.kappa * sizeof(int32_t));
+    L.lpool = off;    off = align256(off + rows * (size_t)L.kmax * sizeof(int32_t));
+    L.latt = off;     off = align256(off + rows * (size_t)c.kappa * sizeof(int32_t));
+    L.lout = off;     off = align256(off + (size_t)c.batch * c.n_q_heads * c.head_dim * 2);
+    L.mS = off;       off = align256(off + rows * (size_t)L.cs_m * sizeof(float));
+    L.mcpos = off;    off = align256(off + rows * (size_t)L.cs_m * sizeof(int32_t));
+    L.mcount = off;   off = align256(off + rows * ((size_t)L.R * L.kmax + 1) * sizeof(int32_t));
+    L.mhist = off;    off = align256(off + rows * kHistBins * sizeof(uint32_t));
+    L.mspill = off;   off = align256(off + rows * 2 * (size_t)L.cs_m * sizeof(uint64_t));
+    L.total = off;
+    return L;
+}
+
+prism_status_t check_cp(const prism_config_t *c, const prism_cp_shard_t *sh) {
+    PRISM_TRY(check_config(c));
+    if (!sh) return PRISM_ERR_INVALID_ARG;
+    if (sh->n_ranks < 1 || sh->rank < 0 || sh->rank >= sh->n_ranks || sh->shard_len < 1)
+        return PRISM_ERR_INVALID_ARG;
+    if ((long long)sh->n_ranks * sh->shard_len < c->max_len) return PRISM_ERR_INVALID_ARG;
+    if (c->flags & PRISM_FLAG_INT2_KEYS) return PRISM_ERR_UNSUPPORTED;
+    if (sh->shard_len > PRISM_MAX_LEN) return PRISM_ERR_UNSUPPORTED;
+    if ((long long)sh->n_ranks * src_kappa_of(*c) > PRISM_MAX_LEN) return PRISM_ERR_UNSUPPORTED;
+    return PRISM_OK;
+}
+
+struct CpWs {
+    Ws w;
+    CpLayout L;
+    int32_t *llen, *lsrc, *lsrc_off, *lsel, *lpool, *latt;
+    void *lout;
+    float *mS;
+    int32_t *mcpos, *mcount;
+    uint32_t *mhist;
+    uint64_t *mspill;
+};
+
+prism_status_t carve_cp(const prism_config_t &c, const prism_cp_shard_t &sh, void *ws,
+                        size_t ws_bytes, CpWs *x) {
+    if (!ws || !aligned(ws, 256)) return PRISM_ERR_INVALID_ARG;
+    x->L = make_cp_layout(c, sh);
+    if (ws_bytes < x->L.total) return PRISM_ERR_WORKSPACE;
+    PRISM_TRY(carve(local_config(c, sh), ws, ws_bytes, &x->w));
+    uint8_t *b = static_cast<uint8_t *>(ws);
+    x->llen = reinterpret_cast<int32_t *>(b + x->L.llen);
+    x->lsrc = reinterpret_cast<int32_t *>(b + x->L.lsrc);
+    x->lsrc_off = reinterpret_cast<int32_t *>(b + x->L.lsrc_off);
+    x->lsel = reinterpret_cast<int32_t *>(b + x->L.lsel);
+    x->lpool = reinterpret_cast<int32_t *>(b + x->L.lpool);
+    x->latt = reinterpret_cast<int32_t *>(b + x->L.latt);
+    x->lout = b + x->L.lout;
+    x->mS = reinterpret_cast<float *>(b + x->L.mS);
+    x->mcpos = reinterpret_cast<int32_t *>(b + x->L.mcpos);
+    x->mcount = reinterpret_cast<int32_t *>(b + x->L.mcount);
+    x->mhist = reinterpret_cast<uint32_t *>(b + x->L.mhist);
+    x->mspill = reinterpret_cast<uint64_t *>(b + x->L.mspill);
+    return PRISM_OK;
+}
+
+CpPrepArgs cp_prep_args(const prism_config_t &c, const prism_cp_shard_t &sh, const CpWs &x,
+                        const int32_t *len) {
+    CpPrepArgs pa{};
+    pa.what = kCpPrepLen;
+    pa.len = len;
+    pa.B = c.batch; pa.Hkv = c.n_kv_heads; pa.Lmax = c.max_len;
+    pa.lo = sh.rank * sh.shard_len; pa.cap = sh.shard_len;
+    pa.llen = x.llen; pa.st = x.w.st;
+    return pa;
+}
+
+prism_status_t cp_pack(const prism_config_t &c, const prism_cp_shard_t &sh, const CpWs &x,
+                       const int32_t *sel, int n, const float *S, const int32_t *cpos,
+                       int32_t *pos_out, float *score_out, cudaStream_t s) {
+    CpPackArgs pk{};
+    pk.sel = sel; pk.rows = c.batch * c.n_kv_heads; pk.n = n; pk.lo = sh.rank * sh.shard_len;
+    pk.S = S; pk.sstride = sh.shard_len; pk.cpos = cpos;
+    pk.n_off = x.lsrc_off; pk.n_src = x.L.lsrc_k;
+    pk.pos_out = pos_out; pk.score_out = score_out; pk.st = x.w.st;
+    return cuda_status(launch_cp_pack(pk, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+prism_status_t prism_cp_workspace_size(const prism_config_t *cfg, const prism_cp_shard_t *shard,
+                                       size_t *bytes) {
+    PRISM_TRY(check_cp(cfg, shard));
+    if (!bytes) return PRISM_ERR_INVALID_ARG;
+    *bytes = make_cp_layout(*cfg, *shard).total;
+    return PRISM_OK;
+}
+
+prism_status_t prism_cp_index_local(const prism_config_t *cfg, const prism_cp_shard_t *shard,
+                                    const void *q, const void *k, const int32_t *len,
+                                    const int32_t *src, int32_t *cand_pos, float *cand_score,
+                                    int32_t *pool_pos, float *pool_score, void *ws,
+                                    size_t ws_bytes, void *stream) {
+    PRISM_TRY(check_cp(cfg, shard));
+    if (!q || !k || !len || !cand_pos || !cand_score) return PRISM_ERR_INVALID_ARG;
+    const bool pool = pool_mode(*cfg);
+    const bool want_pool = pool && !src;
+    if (want_pool != (pool_pos != nullptr) || want_pool != (pool_score != nullptr))
+        return PRISM_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(len, 4) || !aligned(cand_pos, 4) ||
+        !aligned(cand_score, 4) || (src && !aligned(src, 4)) ||
+        (pool_pos && !aligned(pool_pos, 4)) || (pool_score && !aligned(pool_score, 4)))
+        return PRISM_ERR_INVALID_ARG;
+    CpWs x;
+    PRISM_TRY(carve_cp(*cfg, *shard, ws, ws_bytes, &x));
+    const prism_config_t lc = local_config(*cfg, *shard);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CpPrepArgs pa = cp_prep_args(*cfg, *shard, x, len);
+    if (src) {
+        pa.what = kCpPrepProposal;
+        pa.src = src; pa.src_kappa = src_kappa_of(*cfg); pa.radius = cp_radius(*cfg);
+        pa.out = x.lsrc; pa.out_off = x.lsrc_off; pa.out_kappa = x.L.lsrc_k;
+    }
+    PRISM_CUDA(launch_cp_prepare(pa, s));
+    // A plain stream operation between the kernel above and the ones below:
+    // those may read the shard lengths before their grid-dependency wait.
+    PRISM_TRY(zero_control(x.w, s));
+    if (!src) {
+        PRISM_TRY(run_anchor_score(lc, x.w, 0, q, k, x.llen, nullptr, s));
+        if (pool)
+            PRISM_TRY(run_pool_select(lc, x.w, 0, x.llen, x.lpool, nullptr, x.lsel, s));
+        else
+            PRISM_TRY(run_anchor_select(lc, x.w, 0, x.llen, x.lsel, nullptr, s));
+        PRISM_TRY(cp_pack(*cfg, *shard, x, x.lsel, cfg->kappa, x.w.slot[0].S, nullptr, cand_pos,
+                          cand_score, s));
+        if (pool)
+            PRISM_TRY(cp_pack(*cfg, *shard, x, x.lpool, src_kappa_of(*cfg), x.w.slot[0].S,
+                              nullptr, pool_pos, pool_score, s));
+        return PRISM_OK;
+    }
+    const Slot &sl = x.w.slot[kRefineSlot];
+    ScoreArgs sa = score_args(lc, x.w, sl, q, k, x.llen);
+    sa.src = x.lsrc; sa.src_off = x.lsrc_off;
+    sa.kappa = x.L.lsrc_k; sa.radius = 0;
+    PRISM_CUDA(launch_refine_rescore(sa, num_sms(), s));
+    SelectArgs se = select_args(lc, x.w, sl, sl.S, sl.cpos, x.lsrc_off, x.llen, x.lsel, nullptr);
+    se.src_kappa = x.L.lsrc_k; se.radius = 0; se.n_bound = x.L.lsrc_k;
+    PRISM_CUDA(launch_select(se, s));
+    return cp_pack(*cfg, *shard, x, x.lsel, cfg->kappa, sl.S, sl.cpos, cand_pos, cand_score, s);
+}
+
+prism_status_t prism_cp_merge(const prism_config_t *cfg, const prism_cp_shard_t *shard,
+                              int32_t n_out, const int32_t *cand_pos, const float *cand_score,
+                              const int32_t *len, int32_t *idx_out, void *ws, size_t ws_bytes,
+                              void *stream) {
+    PRISM_TRY(check_cp(cfg, shard));
+    if (!cand_pos || !cand_score || !len || !idx_out) return PRISM_ERR_INVALID_ARG;
+    if (n_out != cfg->kappa && !(pool_mode(*cfg) && n_out == src_kappa_of(*cfg)))
+        return PRISM_ERR_INVALID_ARG;
+    if (!aligned(cand_pos, 4) || !aligned(cand_score, 4) || !aligned(len, 4) ||
+        !aligned(idx_out, 4))
+        return PRISM_ERR_INVALID_ARG;
+    CpWs x;
+    PRISM_TRY(carve_cp(*cfg, *shard, ws, ws_bytes, &x));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int R = shard->n_ranks;
+    CpMergeArgs ma{};
+    ma.pos = cand_pos; ma.score = cand_score;
+    ma.R = R; ma.rows = cfg->batch * cfg->n_kv_heads; ma.n = n_out;
+    ma.B = cfg->batch; ma.Hkv = cfg->n_kv_heads; ma.Lmax = cfg->max_len; ma.len = len;
+    ma.S = x.mS; ma.cpos = x.mcpos; ma.cstride = x.L.cs_m; ma.count_out = x.mcount;
+    ma.hist = x.mhist; ma.st = x.w.st;
+    PRISM_CUDA(launch_cp_merge_prepare(ma, s));
+    SelectArgs se = select_args(*cfg, x.w, x.w.slot[0], x.mS, x.mcpos, x.mcount, len, idx_out,
+                                nullptr);
+    se.kappa = n_out; se.radius = 0;
+    se.src_kappa = R * n_out; se.n_bound = R * n_out;
+    se.cstride = x.L.cs_m; se.hist = x.mhist; se.cspill = x.mspill;
+    return cuda_status(launch_select(se, s));
+}
+
+prism_status_t prism_cp_attn_local(const prism_config_t *cfg, const prism_cp_shard_t *shard,
+                                   const void *q, const void *k, const void *v,
+                                   const int32_t *len, const int32_t *idx, float *part_out,
+                                   void *ws, size_t ws_bytes, void *stream) {
+    PRISM_TRY(check_cp(cfg, shard));
+    if (!q || !k || !v || !len || !idx || !part_out) return PRISM_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(len, 4) ||
+        !aligned(idx, 4) || !aligned(part_out, 4))
+        return PRISM_ERR_INVALID_ARG;
+    CpWs x;
+    PRISM_TRY(carve_cp(*cfg, *shard, ws, ws_bytes, &x));
+    const prism_config_t lc = local_config(*cfg, *shard);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CpPrepArgs pa = cp_prep_args(*cfg, *shard, x, len);
+    pa.what = kCpPrepSelection;
+    pa.src = idx; pa.src_kappa = cfg->kappa;
+    pa.out = x.latt; pa.out_kappa = cfg->kappa;
+    PRISM_CUDA(launch_cp_prepare(pa, s));
+    // plain stream operation (see prism_cp_index_local), and the attention's row counters
+    PRISM_CUDA(cudaMemsetAsync(x.w.attn_ctl, 0,
+                               (size_t)cfg->batch * cfg->n_kv_heads * sizeof(RowCtl), s));
+    PRISM_TRY(run_attn(lc, x.w, q, k, v, x.llen, x.latt, cfg->kappa, cfg->kappa, x.lout, s));
+    CpReduceArgs ra{};
+    ra.part_acc = x.w.pacc; ra.part_ml = x.w.pml;
+    ra.rows = cfg->batch * cfg->n_kv_heads;
+    ra.nsplit = (cfg->kappa + kAttnChunk - 1) / kAttnChunk;
+    ra.G = cfg->n_q_heads / cfg->n_kv_heads; ra.d = cfg->head_dim;
+    ra.out = part_out;
+    return cuda_status(launch_cp_reduce(ra, s));
+}
+
+prism_status_t prism_cp_combine(const prism_config_t *cfg, int32_t n_ranks,
+                                const float *part_all, void *out, void *stream) {
+    PRISM_TRY(check_config(cfg));
+    if (n_ranks < 1 || !part_all || !out) return PRISM_ERR_INVALID_ARG;
+    if (!aligned(part_all, 4) || !aligned(out, 16)) return PRISM_ERR_INVALID_ARG;
+    CpCombineArgs ca{};
+    ca.part = part_all; ca.R = n_ranks;
+    ca.heads = cfg->batch * cfg->n_q_heads; ca.d = cfg->head_dim; ca.out = out;
+    return cuda_status(launch_cp_combine(ca, static_cast<cudaStream_t>(stream)));
+}
 
 }  // extern "C"

@@ -1,7 +1,8 @@
 """C-ABI boundary on the CPU: the library loads, exports every entry point
-that include/prism.h declares, and rejects invalid arguments on the host
+that include/*.h declare, and rejects invalid arguments on the host
 before anything is launched (no GPU needed, no device memory touched)."""
 import ctypes
+import glob
 import os
 import re
 
@@ -11,7 +12,7 @@ import long_context_decoding_anchor_b200 as prism
 from long_context_decoding_anchor_b200 import build as prism_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "prism.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 @pytest.fixture(scope="module")
@@ -21,14 +22,15 @@ def L():
 
 
 def declared_symbols():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"PRISM_API\s+[\w\s\*]+?\b(prism_\w+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():
     names = declared_symbols()
     for required in ("prism_index_anchor", "prism_index_refine", "prism_sparse_decode",
-                     "prism_decode_step", "prism_workspace_size"):
+                     "prism_decode_step", "prism_workspace_size", "prism_cp_index_local",
+                     "prism_cp_merge", "prism_cp_attn_local", "prism_cp_combine"):
         assert required in names
 
 
@@ -201,3 +203,60 @@ def test_int2_key_validation(L):
     assert q(ctypes.byref(c), A16, A4, -1, A16, ws, 256, None) == 1          # negative start
     assert q(ctypes.byref(c), A16, A4, 0, MIS, ws, 256, None) == 1           # kq misaligned
     assert q(ctypes.byref(c), A16, A4, 0, A16, None, 256, None) == 1         # no status word
+
+
+def _shard(n_ranks=2, rank=0, shard_len=2048):
+    return prism.CpShard(n_ranks, rank, shard_len)
+
+
+@pytest.mark.parametrize("sh,cfg_kw,status", [
+    (dict(n_ranks=0), {}, 1), (dict(rank=2), {}, 1), (dict(rank=-1), {}, 1),
+    (dict(shard_len=0), {}, 1), (dict(shard_len=1000), {}, 1),     # 2 x 1000 < Lmax 4096
+    (dict(), dict(mode=3, pool_factor=2, flags=2), 2),              # 2-bit keys
+    (dict(), dict(head_dim=96), 2),
+])
+def test_cp_invalid_shard_rejected(L, sh, cfg_kw, status):
+    c, s = _cfg(**cfg_kw), _shard(**sh)
+    n = ctypes.c_size_t(0)
+    assert L.prism_cp_workspace_size(ctypes.byref(c), ctypes.byref(s), ctypes.byref(n)) == status
+
+
+def test_cp_workspace_grows_with_ranks_and_shard(L):
+    c = _cfg()
+    a = prism.prism_cp_workspace_size(c, _shard(2, 0, 2048))
+    assert prism.prism_cp_workspace_size(c, _shard(4, 0, 2048)) > a       # merge buffers
+    assert prism.prism_cp_workspace_size(c, _shard(2, 0, 4096)) > a       # shard buffers
+    assert prism.prism_cp_workspace_size(c, _shard(2, 1, 2048)) == a
+
+
+def test_cp_argument_validation(L):
+    c, s = _cfg(), _shard()
+    ws_n = prism.prism_cp_workspace_size(c, s)
+    ws = ctypes.c_void_p(0x100000)
+    cp_, sp = ctypes.byref(c), ctypes.byref(s)
+    f = L.prism_cp_index_local
+    assert f(cp_, sp, None, A16, A4, None, A4, A4, None, None, ws, ws_n, None) == 1   # null q
+    assert f(cp_, sp, A16, A16, A4, None, None, A4, None, None, ws, ws_n, None) == 1  # null pos
+    assert f(cp_, sp, MIS, A16, A4, None, A4, A4, None, None, ws, ws_n, None) == 1    # q align
+    assert f(cp_, sp, A16, A16, A4, None, A4, A4, A4, A4, ws, ws_n, None) == 1        # pool bufs
+    assert f(cp_, sp, A16, A16, A4, None, A4, A4, None, None, ws, ws_n - 1, None) == 3
+    assert f(cp_, sp, A16, A16, A4, None, A4, A4, None, None, None, ws_n, None) == 1
+    assert f(cp_, None, A16, A16, A4, None, A4, A4, None, None, ws, ws_n, None) == 1  # no shard
+    pc = _cfg(mode=3, pool_factor=2)
+    pws = prism.prism_cp_workspace_size(pc, s)
+    pcp = ctypes.byref(pc)
+    assert f(pcp, sp, A16, A16, A4, None, A4, A4, None, None, ws, pws, None) == 1     # pool anchor
+    assert f(pcp, sp, A16, A16, A4, A4, A4, A4, A4, A4, ws, pws, None) == 1           # refined
+    m = L.prism_cp_merge
+    assert m(cp_, sp, c.kappa + 1, A4, A4, A4, A4, ws, ws_n, None) == 1                # n_out
+    assert m(pcp, sp, 3 * pc.kappa, A4, A4, A4, A4, ws, pws, None) == 1
+    assert m(cp_, sp, c.kappa, None, A4, A4, A4, ws, ws_n, None) == 1
+    assert m(cp_, sp, c.kappa, A4, A4, A4, A4, ws, ws_n - 1, None) == 3
+    a = L.prism_cp_attn_local
+    assert a(cp_, sp, A16, A16, None, A4, A4, A4, ws, ws_n, None) == 1                 # null v
+    assert a(cp_, sp, A16, A16, MIS, A4, A4, A4, ws, ws_n, None) == 1
+    assert a(cp_, sp, A16, A16, A16, A4, A4, A4, ws, ws_n - 1, None) == 3
+    cb = L.prism_cp_combine
+    assert cb(cp_, 0, A4, A16, None) == 1
+    assert cb(cp_, 2, None, A16, None) == 1
+    assert cb(cp_, 2, A4, MIS, None) == 1
