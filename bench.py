@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-q2", action="store_true", help="skip the 2-bit key measurement")
+    ap.add_argument("--skip-cp", action="store_true",
+                    help="skip the context-parallel measurement (512K workload)")
     ap.add_argument("--profile", action="store_true",
                     help="only run --steps eager decode steps (for ncu captures)")
     ap.add_argument("--layers", type=int, default=0,
@@ -239,6 +241,95 @@ def run_reference(args, rank, world):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def measure_context_parallel(args, rank, world, dev):
+    """The context-parallel step (cp.decode_step_cp) on the 512K workload,
+    its context split over the job's ranks (strong scaling: total work fixed).
+    Eager schedule timed with CUDA events (max over ranks); with one rank also
+    replayed from a CUDA graph, beside the single-GPU step's graph."""
+    import math
+
+    import torch
+    import long_context_decoding_anchor_b200 as prism
+    from long_context_decoding_anchor_b200 import cp, synth
+    from long_context_decoding_anchor_b200.runner import DecodeStepGraph
+
+    w = synth.WORKLOADS[5]
+    inp = synth.make_inputs(w, device=dev)
+    cfg = prism.Config.from_workload(w)
+    R, N = world, w.n_layers
+    shard_len = math.ceil(w.max_len / R)
+    sh = prism.CpShard(R, rank, shard_len)
+    if R == 1:
+        ks, vs = inp["k"], inp["v"]
+    else:
+        ks = [cp.shard_rows(k, sh) for k in inp["k"]]
+        vs = [cp.shard_rows(v, sh) for v in inp["v"]]
+        inp["k"] = inp["v"] = None
+        torch.cuda.empty_cache()
+    me = cp.CudaShard(cfg, sh, inp["q"], ks, vs, inp["lens"])
+    gather = cp.local_gather if R == 1 else cp.dist_gather()
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return cp.decode_step_cp(cfg, [me], gather)
+
+    n0 = prism.lib().prism_launch_count()
+    outs, sel = step()
+    launches = int(prism.lib().prism_launch_count() - n0)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    st, detail = prism.prism_check_device_status(me.ws)
+    if st != 0:
+        raise RuntimeError(f"context-parallel step: device status {st} {detail}")
+    barrier_if_distributed()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_eager = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
+    res = {
+        "workload": f"{w.name}: {w.describe()}", "ranks": R, "shard_len": shard_len,
+        "scaling": "strong", "launches_per_step": launches,
+        "eager_us_per_layer": ms_eager * 1e3 / N,
+        "exchange_bytes_per_layer_per_rank": {
+            "selection": w.rows * w.kappa * 8,
+            "attention_partials": w.batch * w.n_q_heads * (w.head_dim + 2) * 4},
+        "how": "per layer: shard-local selection (+ scores), all_gather, exact merge; "
+               "shard-local split-softmax partials, all_gather, combine",
+    }
+    if R == 1:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        res["graph_us_per_layer"] = a.elapsed_time(b) / args.steps * 1e3 / N
+        single = DecodeStepGraph(cfg, inp["q"], inp["k"], inp["v"], inp["lens"])
+        for _ in range(3):
+            single.replay()
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(args.steps):
+            single.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        res["single_gpu_graph_us_per_layer"] = a.elapsed_time(b) / args.steps * 1e3 / N
+        _, idx_s = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                           want_idx=True)
+        res["selections_equal_single_gpu"] = all(torch.equal(sel[l], idx_s[l]) for l in range(N))
+        del g, single
+    return res
 
 
 def run_prism(args, rank, world, dev):
@@ -636,6 +727,16 @@ def run_prism(args, rank, world, dev):
                          f"{w.n_kv_heads} KV heads of the 128K workload, mean of {reps} passes "
                          f"({t_cpu * reps:.1f} s)"}
 
+    # -- context parallel (512K workload split over the job's ranks)
+    cpar = None
+    if not args.skip_cp:
+        del runner
+        runner = None
+        try:
+            cpar = measure_context_parallel(args, rank, world, dev)
+        except Exception as e:          # reported in the line; the headline stands
+            cpar = {"error": f"{type(e).__name__}: {e}"}
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -668,6 +769,7 @@ def run_prism(args, rank, world, dev):
             "breakdown_us": br,
             "pool_mode": pool,
             "pool_mode_int2": pool_q2,
+            "context_parallel": cpar,
             "gpu_launches": launches_per_step * args.steps,
             "launches_per_step": launches_per_step,
             "clocks": clk,

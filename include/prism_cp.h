@@ -5,9 +5,10 @@
  * Source of the operations: "Prism Attention: Proposal-Refined Index Sharing
  * Mechanism for Efficient LLMs Inference", section 4.1 (Eq. (1)-(6)),
  * section 4.2 (Eq. (4), (9): the pool variant) and Algorithm 1.  The paper
- * itself runs one KV head per GPU (tensor parallel, section 5); splitting the
- * context is this library's own extension for contexts whose KV cache
- * outgrows one GPU.  It changes no result:
+ * itself times its kernels at the shapes of one tensor-parallel rank (TP8: one
+ * KV head per GPU; Appendix D, per-layer timing under the SGLang integration);
+ * splitting the context is this library's own extension for contexts whose
+ * KV cache outgrows one GPU.  It changes no result:
  *
  *  - Exact distributed top-k.  Order tokens by (score descending, position
  *    ascending).  A token among the k first of the whole sequence is among
