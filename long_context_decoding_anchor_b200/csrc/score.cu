@@ -341,6 +341,36 @@ k_refine_rescore(ScoreArgs a) {
     if (warp == C::kConsumerWarps) {
         // ---------------- producer warp: the position tables ---------------------
         const int32_t *src = a.src + (size_t)row * a.kappa;
+        if (a.radius == 0) {
+            // Radius 0 (a pool, or a proposal already cut into single
+            // positions): each entry of the canonical source owns exactly its
+            // own position, so slot s is entry s and a window's table is a
+            // copy of the source.  A malformed entry (outside [0, L), or not
+            // above its predecessor) is reported and reads row 0.
+            for (int it = 0; it < nwin; ++it) {
+                const int s = it % C::kPosDepth;
+                const uint32_t ph = (uint32_t)(it / C::kPosDepth) & 1u;
+                if (!mbar_wait(&pos_empty[s], ph ^ 1u, a.wait_ns)) {
+                    if (lane == 0) report(a.st, kDevErrTimeout, kWhereRescore, (uint32_t)it);
+                    break;
+                }
+                const int w0 = s_begin + it * C::kTileRows;
+                const int wend = min(w0 + C::kTileRows, s_end);
+                int *pos = pos_s + s * C::kTileRows;
+                for (int t = w0 + lane; t < wend; t += 32) {
+                    int p = __ldcg(src + t);
+                    const int prev = t > 0 ? __ldcg(src + t - 1) : -1;
+                    if (p < 0 || p >= L || p <= prev) {
+                        report(a.st, kDevErrBadIndex, kWhereRescore, (uint32_t)p);
+                        p = 0;
+                    }
+                    pos[t - w0] = p;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pos_full[s]);
+            }
+            return;
+        }
         // First entry to look at: the last one starting at or before s_begin,
         // by a 64-way search over the offsets (off[0] = 0 <= s_begin).
         int lo = 0, hi = a.kappa;
