@@ -7,7 +7,8 @@
 //    ("Prism Attention", Eq. (5): every position within r of a source token,
 //    clipped to [0, len)) restricted to the shard, as a radius-0 source; or a
 //    global selection in local positions for the attention.
-//  - k_cp_pack: a local selection as (global position, score) pairs.
+//  - k_cp_scatter / k_cp_pack: a local selection as (global position, score)
+//    pairs (a refined layer's candidate scores are first put by position).
 //  - k_cp_merge_compact / k_cp_merge_hist: the gathered pairs of all ranks as
 //    one candidate list per row, for the exact selection (the top-k of a
 //    union is the top-k of the union of the parts' top-k).
@@ -20,22 +21,26 @@
 namespace prism {
 
 constexpr int kCpThreads = 256;
+constexpr int kCpSplit = 8;          // CTAs per row of k_cp_prepare and k_cp_scatter
 
+// Grid (rows, kCpSplit).  For a proposal, every CTA of a row counts the
+// positions of all entries (one run of entries per thread, a block scan) and
+// writes the positions of its own share of the output slots.
 __global__ void __launch_bounds__(kCpThreads)
 k_cp_prepare(CpPrepArgs a) {
     __shared__ int scratch[40];
-    const int row = blockIdx.x;
+    const int row = blockIdx.x, part = blockIdx.y;
     const int b = row / a.Hkv, h = row % a.Hkv;
     const int tid = threadIdx.x;
     pdl_wait();
     const int L = load_len(a.len, b, a.Lmax, a.st, kWhereCanon);
     const int n_loc = max(0, min(L - a.lo, a.cap));
-    if (h == 0 && tid == 0) a.llen[b] = n_loc;
+    if (h == 0 && part == 0 && tid == 0) a.llen[b] = n_loc;
     if (a.what == kCpPrepLen) return;
     const int32_t *src = a.src + (size_t)row * a.src_kappa;
     int32_t *out = a.out + (size_t)row * a.out_kappa;
     if (a.what == kCpPrepSelection) {
-        for (int t = tid; t < a.src_kappa; t += kCpThreads) {
+        for (int t = part * kCpThreads + tid; t < a.src_kappa; t += kCpSplit * kCpThreads) {
             const int p = __ldg(src + t);
             out[t] = (p >= a.lo && p < a.lo + n_loc) ? p - a.lo : -1;
         }
@@ -43,42 +48,62 @@ k_cp_prepare(CpPrepArgs a) {
     }
     // The proposal inside the shard: entry j owns the positions of its window
     // that no earlier entry's window covers (owned_range), here cut to the
-    // shard [lo, lo + n_loc).  Thread t takes a contiguous run of entries.
+    // shard [lo, lo + n_loc).
     const int per = (a.src_kappa + kCpThreads - 1) / kCpThreads;
     const int j0 = min(a.src_kappa, tid * per), j1 = min(a.src_kappa, j0 + per);
     const long long shard_hi = (long long)a.lo + n_loc - 1;
     int cnt = 0;
     for (int j = j0; j < j1; ++j) {
         int lo_j = 0;
-        const int own = owned_range(src, j, a.radius, L, &lo_j, a.st, kWhereCanon);
+        const int own = owned_range(src, j, a.radius, L, &lo_j, part == 0 ? a.st : nullptr,
+                                    kWhereCanon);
         const long long s = max((long long)lo_j, (long long)a.lo);
         const long long e = min((long long)lo_j + own - 1, shard_hi);
         if (own > 0 && e >= s) cnt += (int)(e - s + 1);
     }
     int total;
     int at = block_exclusive_scan(cnt, scratch, &total);
-    for (int j = j0; j < j1; ++j) {
+    const int cap_total = min(total, a.out_kappa);
+    const int o_begin = (int)((long long)part * cap_total / kCpSplit);
+    const int o_end = (int)((long long)(part + 1) * cap_total / kCpSplit);
+    for (int j = j0; j < j1 && at < o_end; ++j) {
         int lo_j = 0;
         const int own = owned_range(src, j, a.radius, L, &lo_j, nullptr, kWhereCanon);
         const long long s = max((long long)lo_j, (long long)a.lo);
         const long long e = min((long long)lo_j + own - 1, shard_hi);
         if (own <= 0 || e < s) continue;
-        for (long long p = s; p <= e; ++p) {
-            if (at < a.out_kappa) out[at] = (int)(p - a.lo);
-            ++at;
-        }
+        const int len = (int)(e - s + 1);
+        // this entry's slots [at, at + len) within this CTA's [o_begin, o_end)
+        const int t0 = max(at, o_begin), t1 = min(at + len, o_end);
+        for (int t = t0; t < t1; ++t) out[t] = (int)(s - a.lo) + (t - at);
+        at += len;
     }
-    if (total > a.out_kappa) {
-        if (tid == 0) report(a.st, kDevErrInternal, kWhereCanon, (uint32_t)total);
-        total = a.out_kappa;
+    if (part == 0 && tid == 0) {
+        if (total > a.out_kappa) report(a.st, kDevErrInternal, kWhereCanon, (uint32_t)total);
+        a.out_off[(size_t)row * (a.out_kappa + 1) + a.out_kappa] = cap_total;
     }
-    for (int e = total + tid; e < a.out_kappa; e += kCpThreads) out[e] = -1;
-    int32_t *off = a.out_off + (size_t)row * (a.out_kappa + 1);
-    for (int e = tid; e <= a.out_kappa; e += kCpThreads) off[e] = min(e, total);
 }
 
 cudaError_t launch_cp_prepare(const CpPrepArgs &a, cudaStream_t s) {
-    return launch_kernel(k_cp_prepare, dim3(a.B * a.Hkv), dim3(kCpThreads), 0, s, a);
+    return launch_kernel(k_cp_prepare, dim3(a.B * a.Hkv, kCpSplit), dim3(kCpThreads), 0, s, a);
+}
+
+__global__ void __launch_bounds__(kCpThreads)
+k_cp_scatter(CpScatterArgs a) {
+    const int row = blockIdx.x, part = blockIdx.y;
+    pdl_wait();
+    const int n = __ldcg(a.n_off + (size_t)row * (a.n_src + 1) + a.n_src);
+    const float *S = a.S + (size_t)row * a.stride;
+    const int32_t *cpos = a.cpos + (size_t)row * a.stride;
+    float *dst = a.S_pos + (size_t)row * a.stride;
+    for (int t = part * kCpThreads + threadIdx.x; t < n; t += kCpSplit * kCpThreads) {
+        const int p = __ldcg(cpos + t);
+        if (p >= 0 && p < a.stride) dst[p] = __ldcg(S + t);
+    }
+}
+
+cudaError_t launch_cp_scatter(const CpScatterArgs &a, cudaStream_t s) {
+    return launch_kernel(k_cp_scatter, dim3(a.rows, kCpSplit), dim3(kCpThreads), 0, s, a);
 }
 
 __global__ void __launch_bounds__(kCpThreads)
@@ -87,39 +112,11 @@ k_cp_pack(CpPackArgs a) {
     pdl_wait();
     const int32_t *sel = a.sel + (size_t)row * a.n;
     const float *S = a.S + (size_t)row * a.sstride;
-    int count = 0;
-    const int32_t *cpos = nullptr;
-    if (a.cpos) {
-        cpos = a.cpos + (size_t)row * a.sstride;
-        count = __ldcg(a.n_off + (size_t)row * (a.n_src + 1) + a.n_src);
-    }
     for (int t = threadIdx.x; t < a.n; t += kCpThreads) {
         const int i = __ldcg(sel + t);
-        int pos = -1;
-        float sc = -INFINITY;
-        if (i >= 0) {
-            int slot = i;
-            if (cpos) {                       // the slot holding local position i
-                int lo = 0, hi = count;
-                while (lo < hi) {
-                    const int mid = (lo + hi) >> 1;
-                    if (__ldcg(cpos + mid) < i) lo = mid + 1;
-                    else hi = mid;
-                }
-                if (lo >= count || __ldcg(cpos + lo) != i) {
-                    report(a.st, kDevErrInternal, kWhereFinalize, (uint32_t)i);
-                    slot = -1;
-                } else {
-                    slot = lo;
-                }
-            }
-            if (slot >= 0) {
-                pos = a.lo + i;
-                sc = __ldcg(S + slot);
-            }
-        }
-        a.pos_out[(size_t)row * a.n + t] = pos;
-        a.score_out[(size_t)row * a.n + t] = sc;
+        const bool ok = i >= 0 && i < a.sstride;
+        a.pos_out[(size_t)row * a.n + t] = ok ? a.lo + i : -1;
+        a.score_out[(size_t)row * a.n + t] = ok ? __ldcg(S + i) : -INFINITY;
     }
 }
 

@@ -16,10 +16,12 @@ struct CpPrepArgs {
     int B, Hkv, Lmax;          // Lmax: global capacity
     int lo, cap;               // the shard
     int32_t *llen;             // [B] shard lengths, clamp(len - lo, 0, cap)
-    // kCpPrepProposal: the canonical global source selection and the radius;
-    // out/out_off receive the proposal inside the shard in local positions,
-    // as a radius-0 source of out_kappa entries (ascending, -1 padded; offsets
-    // e -> min(e, count)).
+    // kCpPrepProposal: src is the canonical global source selection and
+    // radius its proposal radius; out receives the proposal inside the shard
+    // in local positions, ascending (a radius-0 source of at most out_kappa
+    // entries), and out_off[row * (out_kappa + 1) + out_kappa] its count --
+    // the one offset that the rescoring and the selection read for a
+    // radius-0 source.
     // kCpPrepSelection: src is a global selection of src_kappa entries; out
     // receives it in local positions, -1 where outside the shard.
     const int32_t *src;
@@ -31,21 +33,27 @@ struct CpPrepArgs {
 };
 cudaError_t launch_cp_prepare(const CpPrepArgs &a, cudaStream_t s);
 
-// (global position, score) of each entry of a local selection.  Anchor form
-// (cpos == nullptr): S holds scores by local position.  Refined form: S holds
-// candidate scores by slot, cpos/n_off the slots' local positions (ascending)
-// and counts (cpos row stride cstride, count at n_off[row * (n_src + 1) + n_src]).
+// A refined layer's candidate scores (by slot, positions cpos, row stride
+// stride, count at n_off[row * (n_src + 1) + n_src]) written by position into
+// S_pos (row stride stride), so that they can be looked up like an anchor's.
+struct CpScatterArgs {
+    const float *S;
+    const int32_t *cpos;
+    const int32_t *n_off;
+    int n_src, rows, stride;
+    float *S_pos;
+};
+cudaError_t launch_cp_scatter(const CpScatterArgs &a, cudaStream_t s);
+
+// (global position, score) of each entry of a local selection; S holds the
+// scores by local position (row stride sstride).
 struct CpPackArgs {
     const int32_t *sel;        // [rows][n] local positions, ascending, -1 padded
     int rows, n, lo;
     const float *S;
     int sstride;
-    const int32_t *cpos;
-    const int32_t *n_off;
-    int n_src;
     int32_t *pos_out;          // [rows][n]
     float *score_out;          // [rows][n]
-    DevStatus *st;
 };
 cudaError_t launch_cp_pack(const CpPackArgs &a, cudaStream_t s);
 

@@ -1013,14 +1013,13 @@ CpPrepArgs cp_prep_args(const prism_config_t &c, const prism_cp_shard_t &sh, con
     return pa;
 }
 
-prism_status_t cp_pack(const prism_config_t &c, const prism_cp_shard_t &sh, const CpWs &x,
-                       const int32_t *sel, int n, const float *S, const int32_t *cpos,
-                       int32_t *pos_out, float *score_out, cudaStream_t s) {
+prism_status_t cp_pack(const prism_config_t &c, const prism_cp_shard_t &sh, const int32_t *sel,
+                       int n, const float *S, int32_t *pos_out, float *score_out,
+                       cudaStream_t s) {
     CpPackArgs pk{};
     pk.sel = sel; pk.rows = c.batch * c.n_kv_heads; pk.n = n; pk.lo = sh.rank * sh.shard_len;
-    pk.S = S; pk.sstride = sh.shard_len; pk.cpos = cpos;
-    pk.n_off = x.lsrc_off; pk.n_src = x.L.lsrc_k;
-    pk.pos_out = pos_out; pk.score_out = score_out; pk.st = x.w.st;
+    pk.S = S; pk.sstride = sh.shard_len;
+    pk.pos_out = pos_out; pk.score_out = score_out;
     return cuda_status(launch_cp_pack(pk, s));
 }
 
@@ -1071,11 +1070,11 @@ prism_status_t prism_cp_index_local(const prism_config_t *cfg, const prism_cp_sh
             PRISM_TRY(run_pool_select(lc, x.w, 0, x.llen, x.lpool, nullptr, x.lsel, s));
         else
             PRISM_TRY(run_anchor_select(lc, x.w, 0, x.llen, x.lsel, nullptr, s));
-        PRISM_TRY(cp_pack(*cfg, *shard, x, x.lsel, cfg->kappa, x.w.slot[0].S, nullptr, cand_pos,
+        PRISM_TRY(cp_pack(*cfg, *shard, x.lsel, cfg->kappa, x.w.slot[0].S, cand_pos,
                           cand_score, s));
         if (pool)
-            PRISM_TRY(cp_pack(*cfg, *shard, x, x.lpool, src_kappa_of(*cfg), x.w.slot[0].S,
-                              nullptr, pool_pos, pool_score, s));
+            PRISM_TRY(cp_pack(*cfg, *shard, x.lpool, src_kappa_of(*cfg), x.w.slot[0].S, pool_pos,
+                              pool_score, s));
         return PRISM_OK;
     }
     const Slot &sl = x.w.slot[kRefineSlot];
@@ -1086,7 +1085,13 @@ prism_status_t prism_cp_index_local(const prism_config_t *cfg, const prism_cp_sh
     SelectArgs se = select_args(lc, x.w, sl, sl.S, sl.cpos, x.lsrc_off, x.llen, x.lsel, nullptr);
     se.src_kappa = x.L.lsrc_k; se.radius = 0; se.n_bound = x.L.lsrc_k;
     PRISM_CUDA(launch_select(se, s));
-    return cp_pack(*cfg, *shard, x, x.lsel, cfg->kappa, sl.S, sl.cpos, cand_pos, cand_score, s);
+    // the candidates' scores by position (slot 0's score rows are free here)
+    CpScatterArgs sc{};
+    sc.S = sl.S; sc.cpos = sl.cpos; sc.n_off = x.lsrc_off; sc.n_src = x.L.lsrc_k;
+    sc.rows = cfg->batch * cfg->n_kv_heads; sc.stride = shard->shard_len;
+    sc.S_pos = x.w.slot[0].S;
+    PRISM_CUDA(launch_cp_scatter(sc, s));
+    return cp_pack(*cfg, *shard, x.lsel, cfg->kappa, x.w.slot[0].S, cand_pos, cand_score, s);
 }
 
 prism_status_t prism_cp_merge(const prism_config_t *cfg, const prism_cp_shard_t *shard,
