@@ -7,8 +7,8 @@ partials, a second all_gather and the combine -- with OracleShard ranks in
 place of the CUDA ones.  The result must equal the oracle's single-process
 decode step: the selections exactly (the top-k of a union is the top-k of the
 union of the parts' top-k), the outputs to fp64 rounding (split softmax).
-Shards past a sequence's end, uneven shards (3 ranks), every mode, both
-chains and the F/R/S layer kinds are covered."""
+Shards past a sequence's end, shards reaching past the capacity (4 x 80 >
+300), every mode, both chains and the F/R/S layer kinds are covered."""
 import datetime
 import os
 import socket
@@ -105,7 +105,7 @@ def _run(world, shard_len, names):
     return res
 
 
-@pytest.mark.parametrize("world,shard_len", [(2, 150), (3, 100)])
+@pytest.mark.parametrize("world,shard_len", [(2, 150), (3, 100), (4, 80)])
 def test_cp_schedule_matches_single_process(oracle, world, shard_len):
     names = list(CASES)
     res = _run(world, shard_len, names)
@@ -119,3 +119,26 @@ def test_cp_schedule_matches_single_process(oracle, world, shard_len):
             np.testing.assert_array_equal(idx, ref_idx, err_msg=f"{name}, rank {rank}")
             np.testing.assert_allclose(out, ref_out, rtol=1e-12, atol=1e-12,
                                        err_msg=f"{name}, rank {rank}")
+
+
+def test_layer_kinds_and_shard_rows():
+    """Host helpers of the schedule: the layer kinds it walks and the shard
+    copy of a cache (rows past the capacity are zero)."""
+    import long_context_decoding_anchor_b200 as prism
+    from long_context_decoding_anchor_b200 import cp
+    c = prism.Config.make(1, 4, 2, 64, 300, 8, 1, 4, [1, 0, 2, 1])
+    assert cp.layer_kinds(c) == [1, 0, 2, 1]
+    d = prism.Config.make(1, 4, 2, 64, 300, 8, 1, 3, None, mode=prism.MODE_DENSE_ANCHOR)
+    assert cp.layer_kinds(d) == [1, 1, 1]
+    for bad in ([0, 1, 1, 1], [1, 3, 0, 0]):
+        with pytest.raises(ValueError):
+            cp.layer_kinds(prism.Config.make(1, 4, 2, 64, 300, 8, 1, 4, bad))
+    with pytest.raises(ValueError):
+        cp.layer_kinds(prism.Config.make(1, 4, 2, 64, 300, 8, 1, 4, None))
+    t = torch.arange(2 * 3 * 10 * 2, dtype=torch.float32).reshape(2, 3, 10, 2)
+    sh = prism.CpShard(3, 2, 4)                    # rows 8..11 of a capacity of 10
+    part = cp.shard_rows(t, sh)
+    assert part.shape == (2, 3, 4, 2)
+    assert torch.equal(part[:, :, :2], t[:, :, 8:10])
+    assert bool((part[:, :, 2:] == 0).all())
+    assert torch.equal(cp.local_gather([t[0], t[1]]), t)
