@@ -11,7 +11,8 @@
  * Efficient LLMs Inference" (arXiv 2610.22985), section 4.1, equations (1)-(6),
  * and Algorithm 1 (PrismAttention decoding at step t).
  *
- * Variant implemented (the readings are listed in the design doc):
+ * Variant implemented (where the paper leaves a step open, the plainest
+ * reading that the rest of it supports):
  *   - relevance score phi(q, k_i) = scale * sum_{j in G(h)} <q_j, k_i> on the
  *     bf16 key cache, accumulated in fp64 (Eq. (1));
  *   - TopK returns the kappa largest scores, ties broken by the lower token
