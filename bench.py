@@ -164,6 +164,22 @@ def anchor_bytes(w, lens):
     return int(sum(int(L) for L in lens)) * w.n_kv_heads * w.head_dim * 2
 
 
+def selection_recall(sel, exact) -> list:
+    """Per (batch, KV head) row: the fraction of the exact top-kappa `exact`
+    (-1 padded) that the selection `sel` holds -- how much of each layer's
+    own best set the shared-and-refined index keeps (the paper's Fig. 3 view
+    of index sharing)."""
+    import torch
+    s_all = sel.reshape(-1, sel.shape[-1]).cpu()
+    e_all = exact.reshape(-1, exact.shape[-1]).cpu()
+    out = []
+    for s_row, e_row in zip(s_all, e_all):
+        e_row = e_row[e_row >= 0]
+        s_row = s_row[s_row >= 0]
+        out.append(float(torch.isin(e_row, s_row).sum()) / max(1, e_row.numel()))
+    return out
+
+
 def kernel_traffic(src_paths, profile_md):
     """DRAM bytes per launch of the anchor scoring kernel from a committed ncu
     summary, valid only while the kernel's sources are unchanged."""
@@ -381,6 +397,7 @@ def run_prism(args, rank, world, dev):
         raise RuntimeError(f"device status {st} {detail}")
     mask = w.anchor_mask()
     prop_sizes = []
+    refine_diag = []
     last_anchor = 0
     for l in range(N):
         if mask[l]:
@@ -389,6 +406,15 @@ def run_prism(args, rank, world, dev):
         _, _, _, cc = prism.prism_index_refine(cfg, inp["q"][l], inp["k"][l], inp["lens"],
                                                idx_e[l - 1].contiguous(), cand_cap=1, ws=ws)
         prop_sizes.append(int(cc.sum()))
+        # the layer's own exact top-kappa (an anchor selection of this layer), for recall
+        try:
+            exact = prism.prism_index_anchor(cfg, inp["q"][l], inp["k"][l], inp["lens"], ws=ws)
+            rec = selection_recall(idx_e[l], exact)
+            refine_diag.append({"layer": l, "proposal_mean_per_row": float(cc.float().mean()),
+                                "proposal_max_per_row": int(cc.max()),
+                                "recall_mean": statistics.mean(rec), "recall_min": min(rec)})
+        except Exception as e:          # a diagnostic: never costs the line
+            refine_diag.append({"layer": l, "error": f"{type(e).__name__}: {e}"})
     n_anchor = sum(mask)
     kappa_eff = sum(min(w.kappa, int(L)) for L in lens_h) * w.n_kv_heads
     gather = kappa_eff * w.head_dim * 2 * 2
@@ -753,6 +779,14 @@ def run_prism(args, rank, world, dev):
                          "frac": step_gbs / peak, "peak": peak, "peak_kind": peak_kind,
                          "proposal_sizes": {"mean_per_row": statistics.mean(prop_sizes)
                                             / w.rows if prop_sizes else 0}},
+            "refine_diagnostics": {
+                "how": "per refined layer of the timed step: proposal |P| per (batch, KV head) "
+                       "row, and the recall of the layer's selection against its own exact "
+                       "top-kappa (an anchor selection of the same layer)",
+                "recall_mean": (statistics.mean(d["recall_mean"] for d in refine_diag
+                                                if "recall_mean" in d)
+                                if any("recall_mean" in d for d in refine_diag) else None),
+                "layers": refine_diag},
             "roofline": {"kernel": "k_anchor_score", "bound": "hbm", "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "traffic": traffic,
                          "bytes_per_launch": a_bytes, "us_per_launch": t_score * 1e6,

@@ -71,3 +71,16 @@ def test_reference_arm_is_rank0_only(capsys):
         workload, ref_layers, steps, warmup = 3, 8, 1, 0
     assert bench.run_reference(A(), rank=1, world=2) is None
     assert capsys.readouterr().out == ""
+
+
+def test_selection_recall():
+    """The bench's recall diagnostic: the share of the exact top-kappa (padding
+    ignored) that a selection holds, per (batch, KV head) row."""
+    sys.path.insert(0, ROOT)
+    import bench
+    sel = torch.tensor([[[0, 3, 5, -1], [1, 2, 3, 4]], [[-1, -1, -1, -1], [9, 10, 11, 12]]],
+                       dtype=torch.int32)
+    exact = torch.tensor([[[0, 5, 7, -1], [1, 2, 3, 4]], [[2, -1, -1, -1], [1, 2, 3, 4]]],
+                         dtype=torch.int32)
+    assert bench.selection_recall(sel, exact) == pytest.approx([2 / 3, 1.0, 0.0, 0.0])
+    assert bench.selection_recall(exact, exact) == [1.0, 1.0, 1.0, 1.0]
