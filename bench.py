@@ -166,9 +166,10 @@ def anchor_bytes(w, lens):
 
 def selection_recall(sel, exact) -> list:
     """Per (batch, KV head) row: the fraction of the exact top-kappa `exact`
-    (-1 padded) that the selection `sel` holds -- how much of each layer's
-    own best set the shared-and-refined index keeps (the paper's Fig. 3 view
-    of index sharing)."""
+    (-1 padded) that the selection `sel` holds.  For a refined layer this is
+    the coverage of the layer's own top-kappa by its proposal (the quantity of
+    the paper's Fig. 3): an exact top-kappa token inside the proposal ranks
+    among the proposal's kappa best and is selected."""
     import torch
     s_all = sel.reshape(-1, sel.shape[-1]).cpu()
     e_all = exact.reshape(-1, exact.shape[-1]).cpu()
