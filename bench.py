@@ -211,14 +211,24 @@ def oracle_sample(w, inp, layers, heads):
     return q, ks, vs, lens, mask
 
 
-def time_oracle(w, sample, reps=1):
+def time_oracle(w, sample, reps=1, threads=None):
+    """Seconds per pass of the oracle's decode step over `sample`, and the
+    threads it used (all host cores unless `threads` is given)."""
     import oracle
     o = oracle.load()
     q, ks, vs, lens, mask = sample
-    t0 = time.perf_counter()
-    for _ in range(reps):
-        o.decode_step(q, ks, vs, lens, w.kappa, w.radius, mask)
-    return (time.perf_counter() - t0) / reps, o.num_threads()
+    full = o.num_threads()
+    if threads:
+        o.set_num_threads(threads)
+    try:
+        used = o.num_threads()
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            o.decode_step(q, ks, vs, lens, w.kappa, w.radius, mask)
+        return (time.perf_counter() - t0) / reps, used
+    finally:
+        if threads:
+            o.set_num_threads(full)
 
 
 # --------------------------------------------------------------------------- arms
@@ -753,6 +763,13 @@ def run_prism(args, rank, world, dev):
                "sample": f"layers 0-{layers[-1]} ({na} anchor + {len(layers) - na} refined) x all "
                          f"{w.n_kv_heads} KV heads of the 128K workload, mean of {reps} passes "
                          f"({t_cpu * reps:.1f} s)"}
+        # the same on one thread, on the first anchor group only (about 1-2 s)
+        g_layers = layers[:min(len(layers), w.anchor_every)]
+        g_sample = oracle_sample(w, inp, g_layers, (0, w.n_kv_heads))
+        t_1, _ = time_oracle(w, g_sample, threads=1)
+        cpu["single_thread"] = {"value": t_1 * 1e6 / len(g_layers), "unit": UNIT, "cores": 1,
+                                "sample": f"layers 0-{g_layers[-1]} x all {w.n_kv_heads} KV "
+                                          f"heads, one pass ({t_1:.1f} s)"}
 
     # -- context parallel (512K workload split over the job's ranks)
     cpar = None

@@ -78,6 +78,16 @@ int prism_ref_num_threads(void)
 #endif
 }
 
+/* Threads of the row-parallel loops from now on (n >= 1); for timing only. */
+void prism_ref_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 int prism_ref_plant(void) { return PRISM_REF_PLANT; }
 
 /*

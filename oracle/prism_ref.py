@@ -60,6 +60,8 @@ class Oracle:
             _vp, _vp, _vp, _vp, _vp, _vp, _vp]
         lib.prism_ref_decode_step.restype = _i32
         lib.prism_ref_num_threads.restype = _i32
+        lib.prism_ref_set_num_threads.argtypes = [_i32]
+        lib.prism_ref_set_num_threads.restype = None
         lib.prism_ref_plant.restype = _i32
         self.lib = lib
 
@@ -69,6 +71,10 @@ class Oracle:
 
     def num_threads(self) -> int:
         return self.lib.prism_ref_num_threads()
+
+    def set_num_threads(self, n: int) -> None:
+        """Threads of the row-parallel loops from now on (timing only)."""
+        self.lib.prism_ref_set_num_threads(int(n))
 
     # -- single (batch, KV head) row ----------------------------------------
     def score(self, q_group, k_rows, pos=None, scale=None, n=None, agg="sum"):
