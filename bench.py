@@ -717,6 +717,25 @@ def run_prism(args, rank, world, dev):
     br["anchor_layer"] = br["anchor_index"] + br["sparse_attn"]
     br["refine_layer"] = br["refine_index"] + br["sparse_attn"]
 
+    # -- the same step as eager launches (no graph), inputs resident
+    eager = None
+    if not args.no_graph:
+        for _ in range(3):
+            prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], out=out_e,
+                                    ws=ws, stream=stream)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"], out=out_e,
+                                    ws=ws, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_eager = max_over_ranks(a.elapsed_time(b) / args.steps, dev)
+        eager = {"value": whole_job_us_per_layer(ms_eager, N, world), "unit": UNIT,
+                 "ms_per_step": ms_eager,
+                 "how": "prism_decode_step launched eagerly each step (host launch cost included)"}
+
     # -- end to end through the public call, host buffers, copies in the timed region
     e2e = None
     if not args.skip_e2e:
@@ -825,6 +844,7 @@ def run_prism(args, rank, world, dev):
             "gpu_launches": launches_per_step * args.steps,
             "launches_per_step": launches_per_step,
             "clocks": clk,
+            "eager": eager,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
