@@ -211,6 +211,20 @@ def oracle_sample(w, inp, layers, heads):
     return q, ks, vs, lens, mask
 
 
+def host_cpu() -> dict:
+    """The host's CPU model and logical core count (for the CPU baseline)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "nproc": os.cpu_count()}
+
+
 def time_oracle(w, sample, reps=1, threads=None):
     """Seconds per pass of the oracle's decode step over `sample`, and the
     threads it used (all host cores unless `threads` is given)."""
@@ -262,6 +276,7 @@ def run_reference(args, rank, world):
         "config": {"workload": f"{w.name}: {w.describe()}", "sample_layers": layers,
                    "kv_heads": w.n_kv_heads},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "host": host_cpu(),
                          "sample": f"layers {layers[0]}-{layers[-1]} ({n_anchor} anchor + "
                                    f"{len(layers) - n_anchor} refined) x all {w.n_kv_heads} KV "
                                    f"heads of the 128K workload, per step"},
@@ -786,6 +801,7 @@ def run_prism(args, rank, world, dev):
         g_layers = layers[:min(len(layers), w.anchor_every)]
         g_sample = oracle_sample(w, inp, g_layers, (0, w.n_kv_heads))
         t_1, _ = time_oracle(w, g_sample, threads=1)
+        cpu["host"] = host_cpu()
         cpu["single_thread"] = {"value": t_1 * 1e6 / len(g_layers), "unit": UNIT, "cores": 1,
                                 "sample": f"layers 0-{g_layers[-1]} x all {w.n_kv_heads} KV "
                                           f"heads, one pass ({t_1:.1f} s)"}
