@@ -370,6 +370,25 @@ def measure_context_parallel(args, rank, world, dev):
         _, idx_s = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
                                            want_idx=True)
         res["selections_equal_single_gpu"] = all(torch.equal(sel[l], idx_s[l]) for l in range(N))
+        # algorithmic HBM bytes of the step (as for the headline step: anchor K, measured
+        # proposal K rows, gathered K/V rows) over the graph-replayed time
+        mask = w.anchor_mask()
+        lens_h = inp["lens"].cpu().tolist()
+        props = []
+        for l in range(N):
+            if not mask[l]:
+                _, _, _, cc = prism.prism_index_refine(cfg, inp["q"][l], inp["k"][l], inp["lens"],
+                                                       idx_s[l - 1].contiguous(), cand_cap=1)
+                props.append(int(cc.sum()))
+        kappa_eff = sum(min(w.kappa, int(L)) for L in lens_h) * w.n_kv_heads
+        step_bytes = (sum(mask) * anchor_bytes(w, lens_h) + sum(props) * w.head_dim * 2
+                      + N * kappa_eff * w.head_dim * 4)
+        peak, peak_kind = peaks()
+        for key in ("graph_us_per_layer", "single_gpu_graph_us_per_layer"):
+            gbs = step_bytes / (res[key] * N * 1e-6) / 1e9
+            res[key.replace("us_per_layer", "step_hbm")] = {"gbs": gbs, "frac": gbs / peak}
+        res["step_algorithmic_bytes"] = step_bytes
+        res["peak"] = {"gbs": peak, "kind": peak_kind}
         del g, single
     return res
 
