@@ -142,3 +142,23 @@ def test_layer_kinds_and_shard_rows():
     assert torch.equal(part[:, :, :2], t[:, :, 8:10])
     assert bool((part[:, :, 2:] == 0).all())
     assert torch.equal(cp.local_gather([t[0], t[1]]), t)
+
+
+@pytest.mark.parametrize("world,shard_len", [(1, 300), (2, 151), (5, 61)])
+def test_cp_schedule_emulated_ranks(oracle, world, shard_len):
+    """The same schedule with every rank in one process (local_gather), as the
+    one-GPU tests run it, against the oracle's single-process step."""
+    from cp_oracle_shard import OracleShard
+    from long_context_decoding_anchor_b200 import cp
+    w, q, ks, vs, lens = _inputs()
+    for name in ("refine-prev", "pool", "frs"):
+        mode, chain, kinds, rho = CASES[name]
+        cfg = _cfg(w, mode, chain, kinds, rho)
+        ranks = [OracleShard(oracle, cfg, world, r, shard_len, q, ks, vs, lens)
+                 for r in range(world)]
+        outs, sel = cp.decode_step_cp(cfg, ranks, cp.local_gather)
+        ref_out, ref_idx = oracle.decode_step(q, ks, vs, lens, w.kappa, w.radius, kinds,
+                                              mode=mode, chain=chain, rho=rho)
+        np.testing.assert_array_equal(np.stack([x.numpy() for x in sel]), ref_idx, err_msg=name)
+        np.testing.assert_allclose(np.stack([x.numpy() for x in outs]), ref_out, rtol=1e-12,
+                                   atol=1e-12, err_msg=name)
