@@ -260,3 +260,41 @@ def test_cp_argument_validation(L):
     assert cb(cp_, 0, A4, A16, None) == 1
     assert cb(cp_, 2, None, A16, None) == 1
     assert cb(cp_, 2, A4, MIS, None) == 1
+
+
+def test_headers_compile_as_c_and_match_the_library(L, tmp_path):
+    """include/prism.h and include/prism_cp.h are plain C: a C program built
+    with gcc against them links libprism.so, and the struct layouts it sees
+    give the same workspace sizes as the Python binding's."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "prism.h"
+#include "prism_cp.h"
+int main(void) {
+    uint8_t mask[4] = {1, 0, 2, 0};
+    prism_config_t c = {1, 8, 2, 64, 4096, 256, 4, 4, mask, PRISM_MODE_REFINE,
+                        PRISM_CHAIN_PREV, 0.0f, 0, 1};
+    prism_cp_shard_t sh = {2, 1, 2048};
+    size_t a = 0, b = 0;
+    if (prism_workspace_size(&c, &a) != PRISM_OK) return 2;
+    if (prism_cp_workspace_size(&c, &sh, &b) != PRISM_OK) return 3;
+    printf("%d %zu %zu\n", prism_version(), a, b);
+    return 0;
+}
+""")
+    lib_dir = os.path.dirname(prism.LIB_PATH)
+    exe = tmp_path / "abi"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), f"-L{lib_dir}", "-l:libprism.so",
+                    f"-Wl,-rpath,{lib_dir}"], check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    c = _cfg(anchor_mask=[1, 0, 2, 0])
+    assert int(out[0]) == L.prism_version()
+    assert int(out[1]) == prism.prism_workspace_size(c)
+    assert int(out[2]) == prism.prism_cp_workspace_size(c, prism.CpShard(2, 1, 2048))
