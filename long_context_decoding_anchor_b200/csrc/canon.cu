@@ -8,8 +8,8 @@
 // a caller's selection may come in any order, with duplicates.  One CTA per
 // (batch, KV head) marks the selected positions in a shared-memory bitmap
 // (duplicates vanish there) and a block-wide popcount scan writes them back in
-// ascending order, followed by the enumeration offsets of the proposal around
-// them.
+// ascending order, followed (when asked) by the enumeration offsets of the
+// proposal around them.
 #include "prism_internal.cuh"
 
 namespace prism {
@@ -58,9 +58,11 @@ k_canonicalize(CanonArgs a) {
         }
     }
     for (int e = total + tid; e < a.kappa; e += blockDim.x) out[e] = -1;
-    __syncthreads();
-    proposal_offsets(out, a.kappa, a.radius, L, a.out_off + (size_t)row * (a.kappa + 1), scratch,
-                     a.st);
+    if (a.out_off) {
+        __syncthreads();
+        proposal_offsets(out, a.kappa, a.radius, L, a.out_off + (size_t)row * (a.kappa + 1),
+                         scratch, a.st);
+    }
 }
 
 cudaError_t launch_canonicalize(const CanonArgs &a, cudaStream_t s) {

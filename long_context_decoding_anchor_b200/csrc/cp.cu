@@ -7,8 +7,8 @@
 //    ("Prism Attention", Eq. (5): every position within r of a source token,
 //    clipped to [0, len)) restricted to the shard, as a radius-0 source; or a
 //    global selection in local positions for the attention.
-//  - k_cp_scatter / k_cp_pack: a local selection as (global position, score)
-//    pairs (a refined layer's candidate scores are first put by position).
+//  - k_cp_pack: a local selection as (global position, score) pairs (the
+//    rescoring of a refined layer leaves its candidates' scores by position).
 //  - k_cp_merge_compact / k_cp_merge_hist: the gathered pairs of all ranks as
 //    one candidate list per row, for the exact selection (the top-k of a
 //    union is the top-k of the union of the parts' top-k).
@@ -21,7 +21,7 @@
 namespace prism {
 
 constexpr int kCpThreads = 256;
-constexpr int kCpSplit = 8;          // CTAs per row of k_cp_prepare and k_cp_scatter
+constexpr int kCpSplit = 8;          // CTAs per row of k_cp_prepare
 
 // Grid (rows, kCpSplit).  For a proposal, every CTA of a row counts the
 // positions of all entries (one run of entries per thread, a block scan) and
@@ -78,32 +78,15 @@ k_cp_prepare(CpPrepArgs a) {
         for (int t = t0; t < t1; ++t) out[t] = (int)(s - a.lo) + (t - at);
         at += len;
     }
-    if (part == 0 && tid == 0) {
-        if (total > a.out_kappa) report(a.st, kDevErrInternal, kWhereCanon, (uint32_t)total);
-        a.out_off[(size_t)row * (a.out_kappa + 1) + a.out_kappa] = cap_total;
-    }
+    // the rest of the source is padding
+    for (int t = cap_total + part * kCpThreads + tid; t < a.out_kappa; t += kCpSplit * kCpThreads)
+        out[t] = -1;
+    if (part == 0 && tid == 0 && total > a.out_kappa)
+        report(a.st, kDevErrInternal, kWhereCanon, (uint32_t)total);
 }
 
 cudaError_t launch_cp_prepare(const CpPrepArgs &a, cudaStream_t s) {
     return launch_kernel(k_cp_prepare, dim3(a.B * a.Hkv, kCpSplit), dim3(kCpThreads), 0, s, a);
-}
-
-__global__ void __launch_bounds__(kCpThreads)
-k_cp_scatter(CpScatterArgs a) {
-    const int row = blockIdx.x, part = blockIdx.y;
-    pdl_wait();
-    const int n = __ldcg(a.n_off + (size_t)row * (a.n_src + 1) + a.n_src);
-    const float *S = a.S + (size_t)row * a.stride;
-    const int32_t *cpos = a.cpos + (size_t)row * a.stride;
-    float *dst = a.S_pos + (size_t)row * a.stride;
-    for (int t = part * kCpThreads + threadIdx.x; t < n; t += kCpSplit * kCpThreads) {
-        const int p = __ldcg(cpos + t);
-        if (p >= 0 && p < a.stride) dst[p] = __ldcg(S + t);
-    }
-}
-
-cudaError_t launch_cp_scatter(const CpScatterArgs &a, cudaStream_t s) {
-    return launch_kernel(k_cp_scatter, dim3(a.rows, kCpSplit), dim3(kCpThreads), 0, s, a);
 }
 
 __global__ void __launch_bounds__(kCpThreads)

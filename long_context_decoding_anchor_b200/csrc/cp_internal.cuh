@@ -18,32 +18,17 @@ struct CpPrepArgs {
     int32_t *llen;             // [B] shard lengths, clamp(len - lo, 0, cap)
     // kCpPrepProposal: src is the canonical global source selection and
     // radius its proposal radius; out receives the proposal inside the shard
-    // in local positions, ascending (a radius-0 source of at most out_kappa
-    // entries), and out_off[row * (out_kappa + 1) + out_kappa] its count --
-    // the one offset that the rescoring and the selection read for a
-    // radius-0 source.
+    // in local positions, ascending, -1 padded (a radius-0 source of
+    // out_kappa entries).
     // kCpPrepSelection: src is a global selection of src_kappa entries; out
     // receives it in local positions, -1 where outside the shard.
     const int32_t *src;
     int src_kappa, radius;
     int32_t *out;
-    int32_t *out_off;
     int out_kappa;
     DevStatus *st;
 };
 cudaError_t launch_cp_prepare(const CpPrepArgs &a, cudaStream_t s);
-
-// A refined layer's candidate scores (by slot, positions cpos, row stride
-// stride, count at n_off[row * (n_src + 1) + n_src]) written by position into
-// S_pos (row stride stride), so that they can be looked up like an anchor's.
-struct CpScatterArgs {
-    const float *S;
-    const int32_t *cpos;
-    const int32_t *n_off;
-    int n_src, rows, stride;
-    float *S_pos;
-};
-cudaError_t launch_cp_scatter(const CpScatterArgs &a, cudaStream_t s);
 
 // (global position, score) of each entry of a local selection; S holds the
 // scores by local position (row stride sstride).

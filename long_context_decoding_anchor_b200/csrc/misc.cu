@@ -5,29 +5,46 @@
 namespace prism {
 
 // Diagnostic copy of a refined layer's candidates (ascending positions and
-// their scores) into caller buffers of capacity cand_cap per row.
+// their scores) into caller buffers of capacity cand_cap per row: the
+// proposal of the canonical source enumerated by its owned ranges (one
+// contiguous run of entries a thread, a block scan), the scores read by
+// position.  One block per row.
 __global__ void __launch_bounds__(256)
-k_export_candidates(const float *cscore, const int32_t *cpos, const int32_t *src_off, int Lmax,
-                    int kappa, int32_t *cand_pos, float *cand_score, int32_t *cand_count,
-                    int cand_cap) {
+k_export_candidates(const int32_t *src, int E, int radius, const int32_t *len, int Hkv, int Lmax,
+                    const float *Spos, int32_t *cand_pos, float *cand_score, int32_t *cand_count,
+                    int cand_cap, DevStatus *st) {
+    __shared__ int scratch[40];
     pdl_wait();
-    const int row = blockIdx.y;
-    const int n = min(src_off[(size_t)row * (kappa + 1) + kappa], Lmax);
-    if (blockIdx.x == 0 && threadIdx.x == 0) cand_count[row] = n;
-    const int lim = min(n, cand_cap);
-    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < lim; e += gridDim.x * blockDim.x) {
-        cand_pos[(size_t)row * cand_cap + e] = cpos[(size_t)row * Lmax + e];
-        cand_score[(size_t)row * cand_cap + e] = cscore[(size_t)row * Lmax + e];
+    const int row = blockIdx.x, tid = threadIdx.x;
+    const int L = load_len(len, row / Hkv, Lmax, st, kWhereCanon);
+    const int32_t *sr = src + (size_t)row * E;
+    const float *sp = Spos + (size_t)row * Lmax;
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int j0 = min(E, tid * per), j1 = min(E, j0 + per);
+    int cnt = 0;
+    for (int j = j0; j < j1; ++j) {
+        int lo;
+        cnt += owned_range(sr, j, radius, L, &lo, nullptr, 0);
+    }
+    int total;
+    int o = block_exclusive_scan(cnt, scratch, &total);
+    if (tid == 0) cand_count[row] = total;
+    for (int j = j0; j < j1 && o < cand_cap; ++j) {
+        int lo = 0;
+        const int c = owned_range(sr, j, radius, L, &lo, nullptr, 0);
+        for (int t = 0; t < c && o < cand_cap; ++t, ++o) {
+            cand_pos[(size_t)row * cand_cap + o] = lo + t;
+            cand_score[(size_t)row * cand_cap + o] = sp[lo + t];
+        }
     }
 }
 
-cudaError_t launch_export_candidates(const float *cscore, const int32_t *cpos,
-                                     const int32_t *src_off, int rows, int Lmax, int kappa,
+cudaError_t launch_export_candidates(const int32_t *src, int E, int radius, const int32_t *len,
+                                     int B, int Hkv, int Lmax, const float *Spos,
                                      int32_t *cand_pos, float *cand_score, int32_t *cand_count,
-                                     int cand_cap, cudaStream_t s) {
-    const int blocks = max(1, min(64, (cand_cap + 255) / 256));
-    return launch_kernel(k_export_candidates, dim3(blocks, rows), dim3(256), 0, s, cscore, cpos,
-                         src_off, Lmax, kappa, cand_pos, cand_score, cand_count, cand_cap);
+                                     int cand_cap, DevStatus *st, cudaStream_t s) {
+    return launch_kernel(k_export_candidates, dim3(B * Hkv), dim3(256), 0, s, src, E, radius, len,
+                         Hkv, Lmax, Spos, cand_pos, cand_score, cand_count, cand_cap, st);
 }
 
 // Waits on an mbarrier that nothing will ever complete, for at most limit_ns,

@@ -24,6 +24,7 @@
 // helpers of cp.cu around them.
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -57,23 +58,29 @@ namespace {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 constexpr int kAnchorAhead = 2;     // anchors indexed ahead of the chain (ring of anchor slots)
-constexpr int kSlots = kAnchorAhead + 1;   // selection slots: the anchor ring, then refined layers
-constexpr int kRefineSlot = kAnchorAhead;
 
-// Buffers of one selection slot.
+// Buffers of one anchor selection slot.
 struct SlotLayout {
-    size_t hist, S, cpos, cspill;
+    size_t hist, S, cspill;
+};
+
+// The rescoring of a refined layer with source entries E and radius r, in
+// launches of up to nzmax batched layers: runs per row (the largest P * K of
+// refine_parts over the batch sizes) and the ties' overflow capacity.
+struct RunLayout {
+    int E, radius, nzmax, nruns, tie_cap;
+    int parts1;                     // parts of a single-layer launch (the fused selection)
 };
 
 struct Layout {
     size_t status;
     size_t ctl_begin, ctl_end;      // [ctl_begin, ctl_end): histograms and counters; zeroed per call
-    SlotLayout slot[kSlots];
+    SlotLayout slot[kAnchorAhead];
     size_t attn_ctl;
-    // pool mode: kMaxZ candidate slots of refined layers scored together
-    size_t phist, pS, pcpos, pspill;
-    int cstride;                    // their row stride: rho*kappa (at most Lmax), 4-aligned
-    size_t canon, canon_off, idx_all, off_all, pool_all, pool_off_all, pacc, pml, total;
+    RunLayout rl;
+    size_t rhist, runs, run_cnt, ties;   // [nzmax][rows][...] candidate runs of refined layers
+    size_t rbar, part_cnt;               // fused selection: arrivals [rows], counts [rows][parts1][2]
+    size_t canon, idx_all, pool_all, pacc, pml, total;
 };
 
 int n_layers_of(const prism_config_t &c) { return c.n_layers > 0 ? c.n_layers : 1; }
@@ -86,44 +93,54 @@ int src_kappa_of(const prism_config_t &c) {
     return pool_mode(c) ? c.pool_factor * c.kappa : c.kappa;
 }
 
-Layout make_layout(const prism_config_t &c) {
+// Radius of a refined layer's proposal: the pool is rescored as it is.
+int refine_radius_of(const prism_config_t &c) { return pool_mode(c) ? 0 : c.radius; }
+
+RunLayout run_layout(const prism_config_t &c, int E, int radius, int nzmax) {
+    const int rows = c.batch * c.n_kv_heads;
+    RunLayout r{E, radius, nzmax, 1, 1, refine_parts(E, radius, c.max_len, rows, 1).parts};
+    for (int nz = 1; nz <= nzmax; ++nz) {
+        const RefineParts rp = refine_parts(E, radius, c.max_len, rows, nz);
+        r.nruns = std::max(r.nruns, rp.parts * rp.run_k);
+    }
+    r.tie_cap = (int)std::min<long long>(c.max_len, (long long)r.nruns * kRunCap);
+    return r;
+}
+
+// The layout of a workspace.  A context-parallel rank passes its shard's
+// refined-layer source (E entries, radius 0) instead of the config's.
+Layout make_layout(const prism_config_t &c, int src_E = -1, int src_r = -1) {
     const size_t rows = (size_t)c.batch * c.n_kv_heads;
     const size_t G = (size_t)(c.n_q_heads / c.n_kv_heads);
     const size_t nsplit = ((size_t)c.kappa + kAttnChunk - 1) / kAttnChunk;
     const size_t sel_elems = rows * (size_t)c.kappa;
-    const size_t off_elems = rows * ((size_t)c.kappa + 1);
     const size_t src_elems = rows * (size_t)src_kappa_of(c);
-    const size_t src_off_elems = rows * ((size_t)src_kappa_of(c) + 1);
     const size_t n_pools = pool_mode(c) ? (size_t)n_layers_of(c) : 0;
     Layout l{};
+    l.rl = run_layout(c, src_E >= 0 ? src_E : src_kappa_of(c), src_r >= 0 ? src_r : refine_radius_of(c),
+                      pool_mode(c) ? kMaxZ : 1);
+    const size_t nzs = (size_t)l.rl.nzmax;
     size_t off = 0;
     l.status = off; off = align256(off + sizeof(DevStatus));
     l.ctl_begin = off;
-    for (int s = 0; s < kSlots; ++s) {
+    for (int s = 0; s < kAnchorAhead; ++s) {
         l.slot[s].hist = off;   off = align256(off + rows * kHistBins * sizeof(uint32_t));
     }
     l.attn_ctl = off; off = align256(off + rows * sizeof(RowCtl));
-    const size_t nzs = pool_mode(c) ? (size_t)kMaxZ : 0;
-    l.phist = off;    off = align256(off + nzs * rows * kHistBins * sizeof(uint32_t));
+    l.rhist = off;    off = align256(off + nzs * rows * kHistBins * sizeof(uint32_t));
+    l.rbar = off;     off = align256(off + rows * sizeof(uint32_t));
     l.ctl_end = off;
-    {
-        const long long n = (long long)src_kappa_of(c) < c.max_len ? src_kappa_of(c) : c.max_len;
-        l.cstride = (int)((n + 3) & ~3LL);
-    }
-    l.pS = off;       off = align256(off + nzs * rows * (size_t)l.cstride * sizeof(float));
-    l.pcpos = off;    off = align256(off + nzs * rows * (size_t)l.cstride * sizeof(int32_t));
-    l.pspill = off;   off = align256(off + nzs * rows * 2 * (size_t)l.cstride * sizeof(uint64_t));
-    for (int s = 0; s < kSlots; ++s) {
-        l.slot[s].S = off;    off = align256(off + rows * (size_t)c.max_len * sizeof(float));
-        l.slot[s].cpos = off; off = align256(off + (s == kRefineSlot ? rows * (size_t)c.max_len : 1) * sizeof(int32_t));
+    l.part_cnt = off; off = align256(off + rows * (size_t)l.rl.parts1 * 2 * sizeof(int32_t));
+    l.runs = off;     off = align256(off + nzs * rows * (size_t)l.rl.nruns * kRunCap * sizeof(uint64_t));
+    l.run_cnt = off;  off = align256(off + nzs * rows * (size_t)l.rl.nruns * sizeof(int32_t));
+    l.ties = off;     off = align256(off + nzs * rows * (size_t)l.rl.tie_cap * sizeof(uint64_t));
+    for (int s = 0; s < kAnchorAhead; ++s) {
+        l.slot[s].S = off;      off = align256(off + rows * (size_t)c.max_len * sizeof(float));
         l.slot[s].cspill = off; off = align256(off + rows * 2 * (size_t)c.max_len * sizeof(uint64_t));
     }
     l.canon = off;     off = align256(off + src_elems * sizeof(int32_t));
-    l.canon_off = off; off = align256(off + src_off_elems * sizeof(int32_t));
     l.idx_all = off;   off = align256(off + (size_t)n_layers_of(c) * sel_elems * sizeof(int32_t));
-    l.off_all = off;   off = align256(off + (size_t)n_layers_of(c) * off_elems * sizeof(int32_t));
     l.pool_all = off;  off = align256(off + n_pools * src_elems * sizeof(int32_t));
-    l.pool_off_all = off; off = align256(off + n_pools * src_off_elems * sizeof(int32_t));
     l.pacc = off;      off = align256(off + rows * nsplit * G * (size_t)c.head_dim * sizeof(float));
     l.pml = off;       off = align256(off + rows * nsplit * G * 2 * sizeof(float));
     l.total = off;
@@ -225,50 +242,52 @@ prism_status_t helpers_for_current_device(size_t n_events, DeviceHelpers **out) 
 struct Slot {
     uint32_t *hist;
     float *S;
-    int32_t *cpos;
     uint64_t *cspill;
 };
 
 struct Ws {
     DevStatus *st;
-    Slot slot[kSlots];
+    Slot slot[kAnchorAhead];
     RowCtl *attn_ctl;
-    int32_t *canon, *canon_off;
-    int32_t *idx_all, *off_all;
-    int32_t *pool_all, *pool_off_all;     // pool mode: [N][rows][rho*kappa], [N][rows][rho*kappa + 1]
-    uint32_t *phist;                      // pool mode: [kMaxZ][rows][kHistBins]
-    float *pS;                            // pool mode: [kMaxZ][rows][cstride]
-    int32_t *pcpos;                       // pool mode: [kMaxZ][rows][cstride]
-    uint64_t *pspill;                     // pool mode: [kMaxZ][rows][2][cstride]
+    uint32_t *rhist;                      // [nzmax][rows][kHistBins]
+    uint64_t *runs;                       // [nzmax][rows][nruns][kRunCap]
+    int32_t *run_cnt;                     // [nzmax][rows][nruns]
+    uint64_t *ties;                       // [nzmax][rows][tie_cap]
+    uint32_t *rbar;                       // fused selection: arrival counters [rows]
+    int32_t *part_cnt;                    // fused selection: [rows][parts][2]
+    mutable uint32_t bar_arrivals = 0;    // arrivals enqueued so far in this call (host side)
+    int32_t *canon;
+    int32_t *idx_all;
+    int32_t *pool_all;                    // pool mode: [N][rows][rho*kappa]
     float *pacc, *pml;
     uint8_t *base;
     Layout l;
 };
 
-prism_status_t carve(const prism_config_t &c, void *ws, size_t ws_bytes, Ws *w) {
+prism_status_t carve(const prism_config_t &c, void *ws, size_t ws_bytes, Ws *w, int src_E = -1,
+                     int src_r = -1) {
     if (!ws || !aligned(ws, 256)) return PRISM_ERR_INVALID_ARG;
-    w->l = make_layout(c);
+    w->l = make_layout(c, src_E, src_r);
     if (ws_bytes < w->l.total) return PRISM_ERR_WORKSPACE;
     uint8_t *b = static_cast<uint8_t *>(ws);
     w->base = b;
     w->st = reinterpret_cast<DevStatus *>(b + w->l.status);
-    for (int s = 0; s < kSlots; ++s) {
+    for (int s = 0; s < kAnchorAhead; ++s) {
         w->slot[s].hist = reinterpret_cast<uint32_t *>(b + w->l.slot[s].hist);
         w->slot[s].S = reinterpret_cast<float *>(b + w->l.slot[s].S);
-        w->slot[s].cpos = reinterpret_cast<int32_t *>(b + w->l.slot[s].cpos);
         w->slot[s].cspill = reinterpret_cast<uint64_t *>(b + w->l.slot[s].cspill);
     }
     w->attn_ctl = reinterpret_cast<RowCtl *>(b + w->l.attn_ctl);
+    w->rhist = reinterpret_cast<uint32_t *>(b + w->l.rhist);
+    w->runs = reinterpret_cast<uint64_t *>(b + w->l.runs);
+    w->run_cnt = reinterpret_cast<int32_t *>(b + w->l.run_cnt);
+    w->ties = reinterpret_cast<uint64_t *>(b + w->l.ties);
+    w->rbar = reinterpret_cast<uint32_t *>(b + w->l.rbar);
+    w->part_cnt = reinterpret_cast<int32_t *>(b + w->l.part_cnt);
+    w->bar_arrivals = 0;
     w->canon = reinterpret_cast<int32_t *>(b + w->l.canon);
-    w->canon_off = reinterpret_cast<int32_t *>(b + w->l.canon_off);
     w->idx_all = reinterpret_cast<int32_t *>(b + w->l.idx_all);
-    w->off_all = reinterpret_cast<int32_t *>(b + w->l.off_all);
     w->pool_all = reinterpret_cast<int32_t *>(b + w->l.pool_all);
-    w->pool_off_all = reinterpret_cast<int32_t *>(b + w->l.pool_off_all);
-    w->phist = reinterpret_cast<uint32_t *>(b + w->l.phist);
-    w->pS = reinterpret_cast<float *>(b + w->l.pS);
-    w->pcpos = reinterpret_cast<int32_t *>(b + w->l.pcpos);
-    w->pspill = reinterpret_cast<uint64_t *>(b + w->l.pspill);
     w->pacc = reinterpret_cast<float *>(b + w->l.pacc);
     w->pml = reinterpret_cast<float *>(b + w->l.pml);
     return PRISM_OK;
@@ -287,28 +306,26 @@ prism_status_t zero_control(const Ws &w, cudaStream_t s) {
     return cuda_status(cudaMemsetAsync(w.base + w.l.ctl_begin, 0, w.l.ctl_end - w.l.ctl_begin, s));
 }
 
-ScoreArgs score_args(const prism_config_t &c, const Ws &w, const Slot &sl, const void *q,
-                     const void *k, const int32_t *len) {
+ScoreArgs score_args(const prism_config_t &c, const Ws &w, const void *q, const void *k,
+                     const int32_t *len) {
     ScoreArgs sa{};
     sa.q = q; sa.k = k; sa.len = len;
     sa.B = c.batch; sa.Hkv = c.n_kv_heads; sa.G = c.n_q_heads / c.n_kv_heads;
     sa.d = c.head_dim; sa.Lmax = c.max_len; sa.scale = eff_scale(c);
-    sa.S = sl.S; sa.cpos = sl.cpos; sa.hist = sl.hist; sa.src = nullptr; sa.src_off = nullptr;
     sa.kappa = c.kappa; sa.radius = c.radius; sa.st = w.st; sa.wait_ns = wait_limit_ns();
     sa.agg = pool_mode(c) ? kAggMax : kAggSum;
     sa.q2 = (c.flags & PRISM_FLAG_INT2_KEYS) ? 1 : 0;
     return sa;
 }
 
-SelectArgs select_args(const prism_config_t &c, const Ws &w, const Slot &sl, const float *S,
-                       const int32_t *cpos, const int32_t *src_off, const int32_t *len,
-                       int32_t *idx_out, int32_t *prop_off) {
+SelectArgs select_args(const prism_config_t &c, const Ws &w, const Slot &sl, const int32_t *len,
+                       int32_t *idx_out) {
     SelectArgs se{};
-    se.S = S; se.cpos = cpos; se.src_off = src_off; se.len = len;
+    se.S = sl.S; se.len = len;
     se.B = c.batch; se.Hkv = c.n_kv_heads; se.Lmax = c.max_len; se.kappa = c.kappa;
     se.radius = c.radius;
     se.hist = sl.hist; se.cspill = sl.cspill;
-    se.idx_out = idx_out; se.prop_off = prop_off; se.st = w.st; se.wait_ns = wait_limit_ns();
+    se.idx_out = idx_out; se.st = w.st; se.wait_ns = wait_limit_ns();
     return se;
 }
 
@@ -316,84 +333,104 @@ SelectArgs select_args(const prism_config_t &c, const Ws &w, const Slot &sl, con
 prism_status_t run_anchor_score(const prism_config_t &c, const Ws &w, int slot, const void *q,
                                 const void *k, const int32_t *len, float *scores,
                                 cudaStream_t s) {
-    ScoreArgs sa = score_args(c, w, w.slot[slot], q, k, len);
-    if (scores) sa.S = scores;
+    ScoreArgs sa = score_args(c, w, q, k, len);
+    sa.S = scores ? scores : w.slot[slot].S;
+    sa.hist = w.slot[slot].hist;
     return cuda_status(launch_anchor_score(sa, num_sms(), s));
 }
 
-// Anchor top-kappa (Eq. (2)) from slot `slot`; prop_off (nullable) receives
-// the offsets of the proposal around the selection.
+// Anchor top-kappa (Eq. (2)) from slot `slot`.
 prism_status_t run_anchor_select(const prism_config_t &c, const Ws &w, int slot,
-                                 const int32_t *len, int32_t *idx_out, int32_t *prop_off,
-                                 cudaStream_t s) {
-    const Slot &sl = w.slot[slot];
-    return cuda_status(launch_select(select_args(c, w, sl, sl.S, nullptr, nullptr, len, idx_out,
-                                                 prop_off), s));
+                                 const int32_t *len, int32_t *idx_out, cudaStream_t s) {
+    return cuda_status(launch_select(select_args(c, w, w.slot[slot], len, idx_out), s));
 }
 
 // Pool mode, proposal layer: from the scores and histogram in slot `slot`,
-// the pool of Eq. (4) (rho * kappa tokens, with its enumeration offsets at
-// radius 0 when pool_off is given) and the layer's own top-kappa.  The first
-// selection leaves the histogram for the second, which clears it.
+// the pool of Eq. (4) (rho * kappa tokens) and the layer's own top-kappa.
+// The first selection leaves the histogram for the second, which clears it.
 prism_status_t run_pool_select(const prism_config_t &c, const Ws &w, int slot, const int32_t *len,
-                               int32_t *pool_out, int32_t *pool_off, int32_t *idx_out,
-                               cudaStream_t s) {
-    const Slot &sl = w.slot[slot];
-    SelectArgs p = select_args(c, w, sl, sl.S, nullptr, nullptr, len, pool_out, pool_off);
+                               int32_t *pool_out, int32_t *idx_out, cudaStream_t s) {
+    SelectArgs p = select_args(c, w, w.slot[slot], len, pool_out);
     p.kappa = src_kappa_of(c);
     p.radius = 0;
     p.keep_hist = 1;
     PRISM_CUDA(launch_select(p, s));
-    return cuda_status(launch_select(select_args(c, w, sl, sl.S, nullptr, nullptr, len, idx_out,
-                                                 nullptr), s));
+    return cuda_status(launch_select(select_args(c, w, w.slot[slot], len, idx_out), s));
 }
 
-// Refined layer: +-r proposal around the canonical source selection `src`
-// (with its offsets `src_off`), Eq. (5) on it, Eq. (6).
-prism_status_t run_refine(const prism_config_t &c, const Ws &w, const void *q, const void *k,
-                          const int32_t *len, const int32_t *src, const int32_t *src_off,
-                          int32_t *idx_out, int32_t *prop_off, cudaStream_t s) {
-    const Slot &sl = w.slot[kRefineSlot];
-    ScoreArgs sa = score_args(c, w, sl, q, k, len);
-    sa.src = src;
-    sa.src_off = src_off;
-    PRISM_CUDA(launch_refine_rescore(sa, num_sms(), s));
-    return cuda_status(launch_select(select_args(c, w, sl, sl.S, sl.cpos, src_off, len, idx_out,
-                                                 prop_off), s));
-}
-
-// Pool mode: nz (<= kMaxZ) refined layers that share one anchor's pool
-// (`pool`, with its radius-0 enumeration offsets `pool_off`): Eq. (5) on the
-// pool with each layer's own q and K, then Eq. (6), one launch of each kernel
-// for all of them (layer z in grid z).  Layer z's selection goes to outs[z];
-// its candidates stay in candidate slot z.
-prism_status_t run_refine_pool(const prism_config_t &c, const Ws &w, const void *const *qs,
-                               const void *const *ks, int32_t *const *outs, int nz,
-                               const int32_t *len, const int32_t *pool, const int32_t *pool_off,
-                               cudaStream_t s) {
-    if (nz < 1 || nz > kMaxZ) return PRISM_ERR_INVALID_ARG;
+// Refined layers: Eq. (5) over the proposal of the canonical source `src` (E
+// entries, radius r) with each of nz layers' own q and K, then Eq. (6): one
+// launch of each kernel for all of them (layer z in grid z).  Layer z's
+// selection goes to outs[z].  Spos (nullable, nz == 1) receives every
+// candidate's score by position (row stride spos_stride).  `alone` says that
+// no other kernel of the call can run beside this one (no anchor scan in
+// flight): only then may a co-resident launch select in place.
+prism_status_t run_refine_batch(const prism_config_t &c, const Ws &w, const void *const *qs,
+                                const void *const *ks, int32_t *const *outs, int nz,
+                                const int32_t *len, const int32_t *src, int E, int radius,
+                                float *Spos, int spos_stride, cudaStream_t s, bool alone = true) {
+    if (nz < 1 || nz > w.l.rl.nzmax || E != w.l.rl.E || radius != w.l.rl.radius)
+        return PRISM_ERR_INVALID_ARG;
     const size_t rows = (size_t)c.batch * c.n_kv_heads;
-    const int cs = w.l.cstride;
-    ScoreArgs sa = score_args(c, w, w.slot[kRefineSlot], qs[0], ks[0], len);
-    sa.S = w.pS; sa.cpos = w.pcpos; sa.hist = w.phist;
-    sa.src = pool; sa.src_off = pool_off;
-    sa.kappa = src_kappa_of(c); sa.radius = 0;
-    sa.nz = nz; sa.cstride = cs;
-    sa.zS = rows * (size_t)cs; sa.zhist = rows * kHistBins;
+    const RefineParts rp = refine_parts(E, radius, c.max_len, (int)rows, nz);
+    const int nruns = rp.parts * rp.run_k;
+    if (nruns > w.l.rl.nruns) return PRISM_ERR_INVALID_ARG;
+    ScoreArgs sa = score_args(c, w, qs[0], ks[0], len);
+    sa.src = src; sa.kappa = E; sa.radius = radius;
+    sa.hist = w.rhist; sa.runs = w.runs; sa.run_cnt = w.run_cnt;
+    sa.parts = rp.parts; sa.run_k = rp.run_k;
+    sa.Spos = nz == 1 ? Spos : nullptr; sa.spos_stride = spos_stride;
+    sa.nz = nz;
+    sa.zruns = rows * (size_t)nruns * kRunCap; sa.zcnt = rows * (size_t)nruns;
+    sa.zhist = rows * kHistBins;
     for (int z = 0; z < nz; ++z) {
         sa.qz[z] = qs[z];
         sa.kz[z] = ks[z];
     }
-    PRISM_CUDA(launch_refine_rescore(sa, num_sms(), s));
-    SelectArgs se = select_args(c, w, w.slot[kRefineSlot], w.pS, w.pcpos, pool_off, len, outs[0],
-                                nullptr);
-    se.hist = w.phist; se.cspill = w.pspill;
-    se.src_kappa = src_kappa_of(c); se.radius = 0;
-    se.n_bound = cs;
-    se.nz = nz; se.cstride = cs;
-    se.zS = rows * (size_t)cs; se.zhist = rows * kHistBins; se.zspill = rows * 2 * (size_t)cs;
+    // One layer whose parts all fit the GPU at once (one block per SM), one
+    // run each: the rescoring blocks of a row select together (no second
+    // kernel); otherwise the selection kernel reads the runs.  The blocks of a
+    // row wait for one another, so the launch must have the GPU to itself: a
+    // concurrent anchor scan (a block on every SM) leaves no room for some of
+    // them until it ends, and the whole row waits (measured: ~50 against ~22
+    // us a layer).
+    if (alone && nz == 1 && rp.run_k == 1 && rp.parts <= 256 && rp.parts == w.l.rl.parts1 &&
+        (long long)rp.parts * (long long)rows <= num_sms()) {
+        sa.fused = 1;
+        sa.row_bar = w.rbar;
+        sa.bar_base = w.bar_arrivals;
+        w.bar_arrivals += 2u * (uint32_t)rp.parts;
+        sa.part_cnt = w.part_cnt;
+        sa.sel_out = outs[0];
+        sa.kap_out = c.kappa;
+        sa.tie_spill = w.ties;
+        sa.tie_cap = w.l.rl.tie_cap;
+        return cuda_status(launch_refine_rescore(sa, s));
+    }
+    PRISM_CUDA(launch_refine_rescore(sa, s));
+    RunSelectArgs se{};
+    se.runs = w.runs; se.run_cnt = w.run_cnt; se.nruns = nruns;
+    se.hist = w.rhist; se.len = len;
+    se.B = c.batch; se.Hkv = c.n_kv_heads; se.Lmax = c.max_len; se.kappa = c.kappa;
+    se.tie_spill = w.ties; se.tie_cap = w.l.rl.tie_cap;
+    se.nz = nz; se.zruns = sa.zruns; se.zcnt = sa.zcnt; se.zhist = sa.zhist;
+    se.ztie = rows * (size_t)w.l.rl.tie_cap;
     for (int z = 0; z < nz; ++z) se.outz[z] = outs[z];
-    return cuda_status(launch_select(se, s));
+    se.idx_out = outs[0];
+    se.st = w.st;
+    return cuda_status(launch_select_runs(se, s));
+}
+
+// One refined layer: Eq. (5) over the +-r proposal (pool mode: the pool) of
+// the canonical source selection `src`, then Eq. (6).
+prism_status_t run_refine(const prism_config_t &c, const Ws &w, const void *q, const void *k,
+                          const int32_t *len, const int32_t *src, int32_t *idx_out,
+                          cudaStream_t s, float *Spos = nullptr, bool alone = true) {
+    const void *qs[1] = {q};
+    const void *ks[1] = {k};
+    int32_t *outs[1] = {idx_out};
+    return run_refine_batch(c, w, qs, ks, outs, 1, len, src, src_kappa_of(c), refine_radius_of(c),
+                            Spos, c.max_len, s, alone);
 }
 
 prism_status_t run_attn(const prism_config_t &c, const Ws &w, const void *q, const void *k,
@@ -422,13 +459,9 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     const uint16_t *qb = static_cast<const uint16_t *>(q);
     uint16_t *ob = static_cast<uint16_t *>(out);
     int32_t *idx_base = idx_out ? idx_out : w.idx_all;
-    const size_t off_elems = rows * ((size_t)c.kappa + 1);
-    // A layer's proposal offsets are needed when a later layer refines from it.
-    const bool refining = c.mode == PRISM_MODE_REFINE;
-    // Pool mode: each anchor's pool and its offsets, by layer.
+    // Pool mode: each anchor's pool, by layer.
     const bool pool = pool_mode(c);
     const size_t pool_elems = rows * (size_t)src_kappa_of(c);
-    const size_t pool_off_elems = rows * ((size_t)src_kappa_of(c) + 1);
     // Layer kinds: 1 anchor (F), 0 the mode's other layer (R), 2 shared (S,
     // Table 9: keeps the previous layer's selection).
     auto kind_of = [&](int l) { return c.mode == PRISM_MODE_DENSE_ANCHOR ? 1 : (int)c.anchor_mask[l]; };
@@ -488,16 +521,13 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         PRISM_CUDA(cudaEventRecord(ev_scored[g], sA));
         PRISM_CUDA(cudaStreamWaitEvent(sX, ev_scored[g], 0));
         const Slot &sl = w.slot[slot];
-        SelectArgs p = select_args(c, w, sl, sl.S, nullptr, nullptr, len,
-                                   w.pool_all + (size_t)l * pool_elems,
-                                   w.pool_off_all + (size_t)l * pool_off_elems);
+        SelectArgs p = select_args(c, w, sl, len, w.pool_all + (size_t)l * pool_elems);
         p.kappa = src_kappa_of(c);
         p.radius = 0;
         p.keep_hist = 1;
         PRISM_CUDA(launch_select(p, sX));
         PRISM_CUDA(cudaEventRecord(ev_pool[g], sX));
-        SelectArgs t = select_args(c, w, sl, sl.S, nullptr, nullptr, len,
-                                   idx_base + (size_t)l * sel_elems, nullptr);
+        SelectArgs t = select_args(c, w, sl, len, idx_base + (size_t)l * sel_elems);
         t.keep_hist = 1;
         PRISM_CUDA(launch_select(t, sX));
         PRISM_CUDA(cudaEventRecord(ev_kdone[g], sX));
@@ -509,18 +539,15 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     auto index_anchor = [&](int g) -> prism_status_t {
         if (pool && hp) return index_anchor_pool(g);
         const int l = anchors[g];
-        const bool next_refines = refining && l + 1 < N && !is_anchor(l + 1);
         if (hp && g >= kAnchorAhead) PRISM_CUDA(cudaStreamWaitEvent(sA, ev_reached[g - kAnchorAhead], 0));
         PRISM_TRY(run_anchor_score(c, w, g % kAnchorAhead, qb + (size_t)l * q_elems,
                                    kq ? kq[l] : k[l], len,
                                    nullptr, sA));
         if (pool) {
             PRISM_TRY(run_pool_select(c, w, g % kAnchorAhead, len, w.pool_all + (size_t)l * pool_elems,
-                                      w.pool_off_all + (size_t)l * pool_off_elems,
                                       idx_base + (size_t)l * sel_elems, sA));
         } else {
             PRISM_TRY(run_anchor_select(c, w, g % kAnchorAhead, len, idx_base + (size_t)l * sel_elems,
-                                        next_refines ? w.off_all + (size_t)l * off_elems : nullptr,
                                         sA));
         }
         if (hp) PRISM_CUDA(cudaEventRecord(ev_indexed[g], sA));
@@ -530,8 +557,7 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         for (int g = 0; g < NA && g < kAnchorAhead; ++g) PRISM_TRY(index_anchor(g));
     }
 
-    const int32_t *anchor_sel = nullptr, *anchor_off = nullptr;
-    const int32_t *prev_sel = nullptr, *prev_off = nullptr;
+    const int32_t *anchor_sel = nullptr, *prev_sel = nullptr;
     int anchor_layer = 0;
     std::vector<char> batched(pool ? (size_t)N : 0, 0);   // pool mode: refined layers enqueued
     bool prev_is_anchor_sel = false;     // the previous layer's selection is an anchor's own
@@ -539,11 +565,8 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
     for (int l = 0; l < N; ++l) {
         const void *ql = qb + (size_t)l * q_elems;
         const int32_t *src = c.chain == PRISM_CHAIN_ANCHOR ? anchor_sel : prev_sel;
-        const int32_t *src_off = c.chain == PRISM_CHAIN_ANCHOR ? anchor_off : prev_off;
         int32_t *dst = idx_base + (size_t)l * sel_elems;
-        int32_t *dst_off = w.off_all + (size_t)l * off_elems;
-        const bool next_refines = refining && l + 1 < N && !is_anchor(l + 1);
-        const int32_t *cur = dst, *cur_off = dst_off;
+        const int32_t *cur = dst;
         if (is_anchor(l)) {
             if (hp) {
                 PRISM_CUDA(cudaStreamWaitEvent(sM, pool ? ev_pool[g] : ev_indexed[g], 0));
@@ -552,13 +575,11 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
             } else {
                 PRISM_TRY(index_anchor(g));
             }
-            anchor_off = dst_off;
             anchor_sel = dst;
             anchor_layer = l;
             ++g;
         } else if (is_shared(l)) {
-            // Table 9's shared layer: the previous layer's selection, unchanged
-            // (and still described by the previous layer's proposal offsets).
+            // Table 9's shared layer: the previous layer's selection, unchanged.
             // In pool mode an anchor's own selection comes from the aux
             // stream, so a copy of it waits for that selection.
             if (pool && hp && prev_is_anchor_sel) PRISM_CUDA(cudaStreamWaitEvent(sM, ev_kdone[g - 1], 0));
@@ -568,7 +589,6 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
             } else {
                 cur = prev_sel;
             }
-            cur_off = prev_off;
         } else if (pool) {
             // Eq. (5)-(6) over the nearest preceding anchor's pool.  The
             // refined layers of a group depend on that pool alone, so up to
@@ -587,10 +607,9 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
                     batched[e] = 1;
                     ++nz;
                 }
-                PRISM_TRY(run_refine_pool(c, w, qs, ks, outs, nz, len,
-                                          w.pool_all + (size_t)anchor_layer * pool_elems,
-                                          w.pool_off_all + (size_t)anchor_layer * pool_off_elems,
-                                          sM));
+                PRISM_TRY(run_refine_batch(c, w, qs, ks, outs, nz, len,
+                                           w.pool_all + (size_t)anchor_layer * pool_elems,
+                                           src_kappa_of(c), 0, nullptr, 0, sM, !hp || g >= NA));
             }
         } else if (c.mode == PRISM_MODE_STATIC_REUSE) {
             if (idx_out) {
@@ -599,11 +618,9 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
             } else {
                 cur = src;
             }
-            cur_off = nullptr;
         } else {
-            const bool need_off = c.chain == PRISM_CHAIN_PREV && next_refines;
-            PRISM_TRY(run_refine(c, w, ql, k[l], len, src, src_off, dst, need_off ? dst_off : nullptr,
-                                 sM));
+            // alone: on one stream, or once no anchor scan remains ahead of the chain
+            PRISM_TRY(run_refine(c, w, ql, k[l], len, src, dst, sM, nullptr, !hp || g >= NA));
         }
         if (hp) {
             PRISM_CUDA(cudaEventRecord(ev_sel[l], sM));
@@ -614,7 +631,6 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
         PRISM_TRY(run_attn(c, w, ql, k[l], v[l], len, cur, c.kappa, c.kappa,
                            ob + (size_t)l * q_elems, sC));
         prev_sel = cur;
-        prev_off = cur_off;
         if (!is_shared(l)) prev_is_anchor_sel = is_anchor(l);
     }
     if (hp) {
@@ -653,7 +669,7 @@ prism_status_t prism_index_anchor(const prism_config_t *cfg, const void *q, cons
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     PRISM_TRY(zero_control(w, s));
     PRISM_TRY(run_anchor_score(*cfg, w, 0, q, k, len, nullptr, s));
-    PRISM_TRY(run_anchor_select(*cfg, w, 0, len, idx_out, nullptr, s));
+    PRISM_TRY(run_anchor_select(*cfg, w, 0, len, idx_out, s));
     if (scores_out) {
         // The selection reads the workspace copy (its staged copies may round
         // a row's end up to 16 bytes); the caller gets the scores afterwards.
@@ -677,7 +693,7 @@ prism_status_t prism_index_pool(const prism_config_t *cfg, const void *q, const 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     PRISM_TRY(zero_control(w, s));
     PRISM_TRY(run_anchor_score(*cfg, w, 0, q, k, len, nullptr, s));
-    PRISM_TRY(run_pool_select(*cfg, w, 0, len, pool_out, nullptr, idx_out, s));
+    PRISM_TRY(run_pool_select(*cfg, w, 0, len, pool_out, idx_out, s));
     if (scores_out) {
         const size_t bytes = (size_t)cfg->batch * cfg->n_kv_heads * cfg->max_len * sizeof(float);
         PRISM_CUDA(cudaMemcpyAsync(scores_out, w.slot[0].S, bytes, cudaMemcpyDeviceToDevice, s));
@@ -719,27 +735,17 @@ prism_status_t prism_index_refine(const prism_config_t *cfg, const void *q, cons
     CanonArgs ca{};
     ca.idx = idx_prev; ca.len = len; ca.B = cfg->batch; ca.Hkv = cfg->n_kv_heads;
     ca.Lmax = cfg->max_len; ca.kappa = src_kappa_of(*cfg);
-    ca.radius = pool_mode(*cfg) ? 0 : cfg->radius;
-    ca.out = w.canon; ca.out_off = w.canon_off; ca.st = w.st;
+    ca.radius = refine_radius_of(*cfg);
+    ca.out = w.canon; ca.out_off = nullptr; ca.st = w.st;
     PRISM_CUDA(launch_canonicalize(ca, s));
-    if (pool_mode(*cfg)) {
-        const void *qs[1] = {q};
-        const void *ks[1] = {k};
-        int32_t *outs[1] = {idx_out};
-        PRISM_TRY(run_refine_pool(*cfg, w, qs, ks, outs, 1, len, w.canon, w.canon_off, s));
-        if (all)
-            PRISM_CUDA(launch_export_candidates(w.pS, w.pcpos, w.canon_off,
-                                                cfg->batch * cfg->n_kv_heads, w.l.cstride,
-                                                src_kappa_of(*cfg), cand_pos, cand_score,
-                                                cand_count, cand_cap, s));
-        return PRISM_OK;
-    }
-    PRISM_TRY(run_refine(*cfg, w, q, k, len, w.canon, w.canon_off, idx_out, nullptr, s));
+    // With an export, the rescoring also leaves every candidate's score by
+    // position in anchor slot 0 (unused by this call).
+    float *Spos = all ? w.slot[0].S : nullptr;
+    PRISM_TRY(run_refine(*cfg, w, q, k, len, w.canon, idx_out, s, Spos));
     if (all)
-        PRISM_CUDA(launch_export_candidates(w.slot[kRefineSlot].S, w.slot[kRefineSlot].cpos,
-                                            w.canon_off, cfg->batch * cfg->n_kv_heads,
-                                            cfg->max_len, cfg->kappa, cand_pos, cand_score,
-                                            cand_count, cand_cap, s));
+        PRISM_CUDA(launch_export_candidates(w.canon, src_kappa_of(*cfg), refine_radius_of(*cfg), len,
+                                            cfg->batch, cfg->n_kv_heads, cfg->max_len, Spos,
+                                            cand_pos, cand_score, cand_count, cand_cap, w.st, s));
     return PRISM_OK;
 }
 
@@ -915,35 +921,32 @@ prism_config_t local_config(const prism_config_t &c, const prism_cp_shard_t &sh)
     return lc;
 }
 
-// Radius of a refined layer's proposal: the pool is rescored as it is.
-int cp_radius(const prism_config_t &c) { return pool_mode(c) ? 0 : c.radius; }
-
 // Entries of the radius-0 source that a refined layer's proposal becomes
 // inside one shard: at most |source| * (2r + 1) positions, at most shard_len.
 int cp_local_src(const prism_config_t &c, const prism_cp_shard_t &sh) {
-    const long long n = (long long)src_kappa_of(c) * (2LL * cp_radius(c) + 1);
+    const long long n = (long long)src_kappa_of(c) * (2LL * refine_radius_of(c) + 1);
     return (int)(n < sh.shard_len ? n : sh.shard_len);
 }
 
 struct CpLayout {
     Layout l;
     int lsrc_k, kmax, R, cs_m;
-    size_t llen, lsrc, lsrc_off, lsel, lpool, latt, lout;
+    size_t llen, lsrc, lsel, lpool, latt, lout;
     size_t mS, mcpos, mcount, mhist, mspill, total;
 };
 
 CpLayout make_cp_layout(const prism_config_t &c, const prism_cp_shard_t &sh) {
     CpLayout L{};
-    L.l = make_layout(local_config(c, sh));
     const size_t rows = (size_t)c.batch * c.n_kv_heads;
     L.lsrc_k = cp_local_src(c, sh);
+    // a refined layer rescores the shard's cut of its proposal, a radius-0 source
+    L.l = make_layout(local_config(c, sh), L.lsrc_k, 0);
     L.kmax = src_kappa_of(c);
     L.R = sh.n_ranks;
     L.cs_m = (int)(((long long)L.R * L.kmax + 3) & ~3LL);
     size_t off = L.l.total;
     L.llen = off;     off = align256(off + (size_t)c.batch * sizeof(int32_t));
     L.lsrc = off;     off = align256(off + rows * (size_t)L.lsrc_k * sizeof(int32_t));
-    L.lsrc_off = off; off = align256(off + rows * ((size_t)L.lsrc_k + 1) * sizeof(int32_t));
     L.lsel = off;     off = align256(off + rows * (size_t)c.kappa * sizeof(int32_t));
     L.lpool = off;    off = align256(off + rows * (size_t)L.kmax * sizeof(int32_t));
     L.latt = off;     off = align256(off + rows * (size_t)c.kappa * sizeof(int32_t));
@@ -962,7 +965,10 @@ prism_status_t check_cp(const prism_config_t *c, const prism_cp_shard_t *sh) {
     if (!sh) return PRISM_ERR_INVALID_ARG;
     if (sh->n_ranks < 1 || sh->rank < 0 || sh->rank >= sh->n_ranks || sh->shard_len < 1)
         return PRISM_ERR_INVALID_ARG;
+    // the shards cover the capacity; a shard's positions (up to
+    // n_ranks * shard_len) must fit the 32-bit positions of the kernels
     if ((long long)sh->n_ranks * sh->shard_len < c->max_len) return PRISM_ERR_INVALID_ARG;
+    if ((long long)sh->n_ranks * sh->shard_len > INT32_MAX) return PRISM_ERR_INVALID_ARG;
     if (c->flags & PRISM_FLAG_INT2_KEYS) return PRISM_ERR_UNSUPPORTED;
     if (sh->shard_len > PRISM_MAX_LEN) return PRISM_ERR_UNSUPPORTED;
     if ((long long)sh->n_ranks * src_kappa_of(*c) > PRISM_MAX_LEN) return PRISM_ERR_UNSUPPORTED;
@@ -972,7 +978,7 @@ prism_status_t check_cp(const prism_config_t *c, const prism_cp_shard_t *sh) {
 struct CpWs {
     Ws w;
     CpLayout L;
-    int32_t *llen, *lsrc, *lsrc_off, *lsel, *lpool, *latt;
+    int32_t *llen, *lsrc, *lsel, *lpool, *latt;
     void *lout;
     float *mS;
     int32_t *mcpos, *mcount;
@@ -985,11 +991,10 @@ prism_status_t carve_cp(const prism_config_t &c, const prism_cp_shard_t &sh, voi
     if (!ws || !aligned(ws, 256)) return PRISM_ERR_INVALID_ARG;
     x->L = make_cp_layout(c, sh);
     if (ws_bytes < x->L.total) return PRISM_ERR_WORKSPACE;
-    PRISM_TRY(carve(local_config(c, sh), ws, ws_bytes, &x->w));
+    PRISM_TRY(carve(local_config(c, sh), ws, ws_bytes, &x->w, x->L.lsrc_k, 0));
     uint8_t *b = static_cast<uint8_t *>(ws);
     x->llen = reinterpret_cast<int32_t *>(b + x->L.llen);
     x->lsrc = reinterpret_cast<int32_t *>(b + x->L.lsrc);
-    x->lsrc_off = reinterpret_cast<int32_t *>(b + x->L.lsrc_off);
     x->lsel = reinterpret_cast<int32_t *>(b + x->L.lsel);
     x->lpool = reinterpret_cast<int32_t *>(b + x->L.lpool);
     x->latt = reinterpret_cast<int32_t *>(b + x->L.latt);
@@ -1057,8 +1062,8 @@ prism_status_t prism_cp_index_local(const prism_config_t *cfg, const prism_cp_sh
     CpPrepArgs pa = cp_prep_args(*cfg, *shard, x, len);
     if (src) {
         pa.what = kCpPrepProposal;
-        pa.src = src; pa.src_kappa = src_kappa_of(*cfg); pa.radius = cp_radius(*cfg);
-        pa.out = x.lsrc; pa.out_off = x.lsrc_off; pa.out_kappa = x.L.lsrc_k;
+        pa.src = src; pa.src_kappa = src_kappa_of(*cfg); pa.radius = refine_radius_of(*cfg);
+        pa.out = x.lsrc; pa.out_kappa = x.L.lsrc_k;
     }
     PRISM_CUDA(launch_cp_prepare(pa, s));
     // A plain stream operation between the kernel above and the ones below:
@@ -1067,9 +1072,9 @@ prism_status_t prism_cp_index_local(const prism_config_t *cfg, const prism_cp_sh
     if (!src) {
         PRISM_TRY(run_anchor_score(lc, x.w, 0, q, k, x.llen, nullptr, s));
         if (pool)
-            PRISM_TRY(run_pool_select(lc, x.w, 0, x.llen, x.lpool, nullptr, x.lsel, s));
+            PRISM_TRY(run_pool_select(lc, x.w, 0, x.llen, x.lpool, x.lsel, s));
         else
-            PRISM_TRY(run_anchor_select(lc, x.w, 0, x.llen, x.lsel, nullptr, s));
+            PRISM_TRY(run_anchor_select(lc, x.w, 0, x.llen, x.lsel, s));
         PRISM_TRY(cp_pack(*cfg, *shard, x.lsel, cfg->kappa, x.w.slot[0].S, cand_pos,
                           cand_score, s));
         if (pool)
@@ -1077,20 +1082,13 @@ prism_status_t prism_cp_index_local(const prism_config_t *cfg, const prism_cp_sh
                               pool_score, s));
         return PRISM_OK;
     }
-    const Slot &sl = x.w.slot[kRefineSlot];
-    ScoreArgs sa = score_args(lc, x.w, sl, q, k, x.llen);
-    sa.src = x.lsrc; sa.src_off = x.lsrc_off;
-    sa.kappa = x.L.lsrc_k; sa.radius = 0;
-    PRISM_CUDA(launch_refine_rescore(sa, num_sms(), s));
-    SelectArgs se = select_args(lc, x.w, sl, sl.S, sl.cpos, x.lsrc_off, x.llen, x.lsel, nullptr);
-    se.src_kappa = x.L.lsrc_k; se.radius = 0; se.n_bound = x.L.lsrc_k;
-    PRISM_CUDA(launch_select(se, s));
-    // the candidates' scores by position (slot 0's score rows are free here)
-    CpScatterArgs sc{};
-    sc.S = sl.S; sc.cpos = sl.cpos; sc.n_off = x.lsrc_off; sc.n_src = x.L.lsrc_k;
-    sc.rows = cfg->batch * cfg->n_kv_heads; sc.stride = shard->shard_len;
-    sc.S_pos = x.w.slot[0].S;
-    PRISM_CUDA(launch_cp_scatter(sc, s));
+    // Eq. (5)-(6) over the shard's cut of the proposal (a radius-0 source);
+    // the candidates' scores are left by local position in slot 0 for the pack.
+    const void *qs[1] = {q};
+    const void *ks[1] = {k};
+    int32_t *outs[1] = {x.lsel};
+    PRISM_TRY(run_refine_batch(lc, x.w, qs, ks, outs, 1, x.llen, x.lsrc, x.L.lsrc_k, 0,
+                               x.w.slot[0].S, shard->shard_len, s));
     return cp_pack(*cfg, *shard, x.lsel, cfg->kappa, x.w.slot[0].S, cand_pos, cand_score, s);
 }
 
@@ -1116,8 +1114,8 @@ prism_status_t prism_cp_merge(const prism_config_t *cfg, const prism_cp_shard_t 
     ma.S = x.mS; ma.cpos = x.mcpos; ma.cstride = x.L.cs_m; ma.count_out = x.mcount;
     ma.hist = x.mhist; ma.st = x.w.st;
     PRISM_CUDA(launch_cp_merge_prepare(ma, s));
-    SelectArgs se = select_args(*cfg, x.w, x.w.slot[0], x.mS, x.mcpos, x.mcount, len, idx_out,
-                                nullptr);
+    SelectArgs se = select_args(*cfg, x.w, x.w.slot[0], len, idx_out);
+    se.S = x.mS; se.cpos = x.mcpos; se.src_off = x.mcount;
     se.kappa = n_out; se.radius = 0;
     se.src_kappa = R * n_out; se.n_bound = R * n_out;
     se.cstride = x.L.cs_m; se.hist = x.mhist; se.cspill = x.mspill;

@@ -74,16 +74,29 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// <k, q> over 8 bf16 key elements and 8 fp32 query elements: two fp32
+// accumulators (even and odd elements), each a chain of round-to-nearest FMAs
+// issued in pairs (fma.rn.f32x2), added at the end.  Every kernel that scores
+// with it forms bit-identical scores for the same key and query.
+__device__ __forceinline__ unsigned long long f32x2_pack(float lo, float hi) {
+    return ((unsigned long long)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ unsigned long long fma_f32x2(unsigned long long a, unsigned long long b,
+                                                        unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
 __device__ __forceinline__ float dot8(const uint4 &kv, const float *q) {
-    float a = bf16_lo(kv.x) * q[0];
-    a = fmaf(bf16_hi(kv.x), q[1], a);
-    a = fmaf(bf16_lo(kv.y), q[2], a);
-    a = fmaf(bf16_hi(kv.y), q[3], a);
-    a = fmaf(bf16_lo(kv.z), q[4], a);
-    a = fmaf(bf16_hi(kv.z), q[5], a);
-    a = fmaf(bf16_lo(kv.w), q[6], a);
-    a = fmaf(bf16_hi(kv.w), q[7], a);
-    return a;
+    // word w holds elements 2w (low half) and 2w + 1 (high half); the
+    // accumulators start at -0.0, so the first step is exactly a product
+    // (signed zeros survive: a key of -0.0 scores -0.0)
+    unsigned long long acc = 0x8000000080000000ull;
+    acc = fma_f32x2(((unsigned long long)(kv.x & 0xffff0000u) << 32) | (kv.x << 16), f32x2_pack(q[0], q[1]), acc);
+    acc = fma_f32x2(((unsigned long long)(kv.y & 0xffff0000u) << 32) | (kv.y << 16), f32x2_pack(q[2], q[3]), acc);
+    acc = fma_f32x2(((unsigned long long)(kv.z & 0xffff0000u) << 32) | (kv.z << 16), f32x2_pack(q[4], q[5]), acc);
+    acc = fma_f32x2(((unsigned long long)(kv.w & 0xffff0000u) << 32) | (kv.w << 16), f32x2_pack(q[6], q[7]), acc);
+    return __uint_as_float((uint32_t)acc) + __uint_as_float((uint32_t)(acc >> 32));
 }
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
@@ -256,6 +269,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
     }
     return false;
 }
+// Acquire load at GPU scope (pairs with a fence + atomic arrival elsewhere).
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Barrier of blocks that are resident together (the caller guarantees it):
+// thread 0 makes the block's earlier global writes visible, adds one arrival
+// to *ctr and waits until *ctr reaches `target`, bounded by limit_ns (then it
+// records a timeout and lets the block continue; the results are void).  The
+// whole block calls it; *ok (shared) says whether the wait completed.
+__device__ __forceinline__ void block_group_barrier(uint32_t *ctr, uint32_t target, uint64_t limit_ns,
+                                                    DevStatus *st, uint32_t where, int *ok) {
+    __threadfence();                   // every thread's writes, before the arrival
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        atomicAdd(ctr, 1u);
+        const uint64_t t0 = global_timer_ns();
+        int good = 1;
+        for (uint32_t it = 0; ld_acquire_gpu(ctr) < target; ++it) {
+            if ((it & 15u) == 15u && global_timer_ns() - t0 > limit_ns) {
+                report(st, kDevErrTimeout, where, target);
+                good = 0;
+                break;
+            }
+        }
+        *ok = good;
+    }
+    __syncthreads();
+}
+
 // Evict-first L2 policy for data read exactly once (the streamed key cache).
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     uint64_t pol;
@@ -448,28 +492,73 @@ struct ScoreArgs {
     const int32_t *len;     // [B]
     int B, Hkv, G, d, Lmax;
     float scale;
-    float *S;               // fp32 [rows][Lmax]: anchor scores by position; refine
-                            // candidate scores in enumeration (= ascending position) order
-    int32_t *cpos;          // refine: [rows][Lmax] candidate positions
-    uint32_t *hist;         // [rows][kHistBins]
+    float *S;               // anchor: fp32 [rows][Lmax] scores by position
+    uint32_t *hist;         // [rows][kHistBins] first-digit histogram (accumulated)
     const int32_t *src;     // refine: canonical source selection [rows][kappa]
-    const int32_t *src_off; // refine: its proposal enumeration offsets [rows][kappa + 1]
     int kappa, radius;      // refine: entries of the source selection, proposal radius
     int agg;                // kAggSum: Eq. (1) group sum; kAggMax: Eq. (9) group maximum
     int q2;                 // nonzero: k (and kz) are 2-bit key caches (Eq. (7)-(8),
                             // rows of d/2 bytes, q2_impl.cuh), scored by Eq. (9)
+    // refine: the candidates leave as runs (see RefineParts): run t of a row
+    // holds run_cnt[row * nruns + t] items (key << 32 | position), ordered by
+    // first radix digit, highest first, at runs + (row * nruns + t) * kRunCap
+    uint64_t *runs;
+    int32_t *run_cnt;
+    int parts, run_k;       // parts per row, runs per part (nruns = parts * run_k)
+    float *Spos;            // refine, nullable: every candidate's score by position
+    int spos_stride;        //   (row stride)
+    // refine, fused selection (Eq. (6) in the same launch; nz == 1, one run a
+    // part, every block of the grid resident at once): the blocks of a row
+    // meet at two barriers on row_bar[row] (arrivals counted from bar_base),
+    // exchange their first-digit ties through their runs and their counts
+    // through part_cnt [rows][parts][2], and each writes its selected
+    // positions to sel_out [rows][kap_out] at its offset; ties beyond the
+    // shared-memory cache go to tie_spill [rows][tie_cap]
+    int fused;
+    uint32_t *row_bar;
+    uint32_t bar_base;
+    int32_t *part_cnt;
+    int32_t *sel_out;
+    int kap_out;
+    uint64_t *tie_spill;
+    int tie_cap;
     // refine: several layers rescoring the same source in one launch (grid z);
-    // layer z reads qz[z] / kz[z] (z = 0: q / k) and writes S, cpos, hist
-    // shifted by z * zS, z * zS, z * zhist.  cstride is the row stride of S
-    // and cpos (0: Lmax).
+    // layer z reads qz[z] / kz[z] (z = 0: q / k) and writes runs, run_cnt and
+    // hist shifted by z * zruns, z * zcnt, z * zhist
     int nz;
     const void *qz[8];
     const void *kz[8];
-    int cstride;
-    size_t zS, zhist;
+    size_t zruns, zcnt, zhist;
     DevStatus *st;
     uint64_t wait_ns;
 };
+// Work split of a refined layer's rescoring.  Part p of a row takes the
+// source entries [p*E/P, (p+1)*E/P) -- at most kMaxPartEntries -- and the
+// proposal positions they own, at most run_k * kRunCap of them; each run of
+// kRunCap candidates is sorted by first digit for the selection.
+constexpr int kRunCap = 2048;
+constexpr int kMaxPartEntries = 512;
+constexpr int kTargetCtas = 148;   // rescoring blocks aimed at per launch (B200 SMs)
+struct RefineParts {
+    int parts, run_k;
+};
+inline RefineParts refine_parts(int E, int radius, int Lmax, int rows, int nz) {
+    const long long own = (long long)2 * radius + 1 < Lmax ? 2LL * radius + 1 : (long long)Lmax;
+    const long long per_run = own <= kRunCap ? kRunCap / own : 1;        // entries a run holds
+    long long per = per_run < kMaxPartEntries ? per_run : kMaxPartEntries;
+    long long P = (E + per - 1) / per;
+    const long long want = kTargetCtas / ((long long)rows * (nz > 0 ? nz : 1));
+    if (P < want) P = want < E ? want : E;
+    if (P < 1) P = 1;
+    const long long ent = (E + P - 1) / P;                                // entries of a part
+    long long slots = ent * own;
+    if (slots > Lmax) slots = Lmax;
+    RefineParts r;
+    r.parts = (int)P;
+    r.run_k = (int)((slots + kRunCap - 1) / kRunCap);
+    if (r.run_k < 1) r.run_k = 1;
+    return r;
+}
 enum : int { kAggSum = 0, kAggMax = 1 };
 constexpr int kMaxZ = 8;           // refined layers batched into one launch
 
@@ -481,14 +570,14 @@ cudaError_t launch_anchor_score_q2(const ScoreArgs &a, int num_sms, cudaStream_t
 cudaError_t launch_quantize_keys(const void *k, const int32_t *len, int B, int Hkv, int d, int Lmax,
                                  int start, void *kq, DevStatus *st, cudaStream_t s);
 
-cudaError_t launch_refine_rescore(const ScoreArgs &a, int num_sms, cudaStream_t s);
+cudaError_t launch_refine_rescore(const ScoreArgs &a, cudaStream_t s);
 
 struct CanonArgs {
     const int32_t *idx;        // [rows][kappa], any order, duplicates, -1 padding
     const int32_t *len;
     int B, Hkv, Lmax, kappa, radius;
     int32_t *out;              // [rows][kappa] canonical: ascending, distinct, -1 padded
-    int32_t *out_off;          // [rows][kappa + 1] its proposal enumeration offsets
+    int32_t *out_off;          // nullable: [rows][kappa + 1] its proposal enumeration offsets
     DevStatus *st;
 };
 cudaError_t launch_canonicalize(const CanonArgs &a, cudaStream_t s);
@@ -516,8 +605,35 @@ struct SelectArgs {
     int32_t *prop_off;         // nullable: [rows][kappa + 1] offsets of the next proposal
     DevStatus *st;
     uint64_t wait_ns;          // bound on the wait for the slice copies
+    int row_cap;               // one-block-per-row kernel: bound on a row's items (set by the launcher)
 };
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
+
+// Selection of a refined layer from the rescoring's runs (select_row.cu): one
+// block per row (and per batched layer z); the selection leaves as ascending
+// positions, -1 padded.
+struct RunSelectArgs {
+    const uint64_t *runs;      // [rows][nruns][kRunCap]
+    const int32_t *run_cnt;    // [rows][nruns]
+    int nruns;
+    uint32_t *hist;            // [rows][kHistBins], left zeroed
+    const int32_t *len;
+    int B, Hkv, Lmax, kappa;
+    uint64_t *tie_spill;       // [rows][tie_cap] overflow of the first-digit ties
+    int tie_cap;
+    int nz;                    // z > 0: shifted by z * zruns, z * zcnt, z * zhist, z * ztie
+    size_t zruns, zcnt, zhist, ztie;
+    int32_t *outz[8];          // nz > 1: layer z's selection; else idx_out
+    int32_t *idx_out;          // [rows][kappa]
+    DevStatus *st;
+};
+cudaError_t launch_select_runs(const RunSelectArgs &a, cudaStream_t s);
+// One block per row (select_row.cu), for rows of at most kRowMaxItems items
+// and budgets of at most kRowMaxKappa.
+constexpr int kRowMaxItems = 1 << 18;
+constexpr int kRowMaxKappa = 8192;
+bool select_row_fits(int items, int kappa);
+cudaError_t launch_select_row(const SelectArgs &a, int items, cudaStream_t s);
 
 struct AttnArgs {
     const void *q;             // bf16 [B][Hq][d]
@@ -546,10 +662,13 @@ struct StaticAttnScratch {
 };
 cudaError_t static_attn_scratch(StaticAttnScratch *out);
 
-cudaError_t launch_export_candidates(const float *cscore, const int32_t *cpos,
-                                     const int32_t *src_off, int rows, int Lmax, int kappa,
+// Diagnostic export of a refined layer's candidates (misc.cu): the proposal
+// of the canonical source `src` ([rows][E], radius r) in ascending order, with
+// the scores the rescoring left by position in Spos (row stride Lmax).
+cudaError_t launch_export_candidates(const int32_t *src, int E, int radius, const int32_t *len,
+                                     int B, int Hkv, int Lmax, const float *Spos,
                                      int32_t *cand_pos, float *cand_score, int32_t *cand_count,
-                                     int cand_cap, cudaStream_t s);
+                                     int cand_cap, DevStatus *st, cudaStream_t s);
 
 cudaError_t launch_debug_wait(DevStatus *st, uint64_t limit_ns, cudaStream_t s);
 

@@ -21,6 +21,7 @@
 // are stored contiguously at their enumeration index.
 #include "prism_internal.cuh"
 #include "q2_impl.cuh"
+#include "select_impl.cuh"
 #include "tiles.cuh"
 
 namespace prism {
@@ -215,20 +216,26 @@ k_anchor_score(ScoreArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Refined layer: score only the proposal positions (Eq. (5)).  The proposal
-// of a row is enumerated slot by slot from the owned ranges of the canonical
-// source selection (the offsets src_off give each entry's first slot), so a
-// row's n slots split evenly into P contiguous parts, one CTA each.  A CTA
-// walks its part in windows of 128 slots.  The producer warp finds the
-// entries overlapping each window (one coalesced load of 32 entries at a
-// time, the next batch in flight) and writes every slot's key row into a ring
-// of position tables, up to kPosDepth windows ahead.  Each consumer warp owns
-// 16 slots of every window: it gathers exactly the 16-byte pieces of those
-// key rows that its lanes will read (cp.async, a 3-stage pipeline per warp,
-// no hand-off between warps), forms the dot products and stores the
-// (score, position) candidates at their slot index.  (A run of the proposal
-// is only ~11-17 rows, 3-4 KB: issuing one bulk copy per run from a single
-// warp, not DRAM, limited an earlier version to ~25 GB/s per SM.)
+// Refined layer: score only the proposal positions (Eq. (5)), and hand the
+// selection (Eq. (6)) its candidates already ordered by first radix digit.
+//
+// The source selection is canonical (ascending, distinct, -1 padded), so the
+// proposal -- every position within r of a source entry, clipped to [0, L) --
+// splits into the owned ranges of consecutive entries (owned_range): entry j
+// owns the positions of its window that no earlier window covers.  Part p of
+// a row (blockIdx.x) takes the entries [p*E/P, (p+1)*E/P), counts their
+// ranges with one block scan, and lists the positions they own ("slots",
+// ascending) in a shared-memory table, one run of kRunCap slots at a time.
+// Each warp owns 16 slots of every window of 128 and gathers exactly the
+// 16-byte pieces of those key rows that its lanes will read (cp.async, a
+// kStages pipeline per warp, no hand-off between warps).  (One 1-D bulk copy
+// per 256-byte row was measured slower: the copy engine's rate for small
+// copies, not DRAM, then sets the pace.)
+// The scores' order-preserving keys go into the table beside the positions;
+// at the end of the run the block sorts the (key, position) items by first
+// radix digit (a counting sort on its own histogram, which it also adds to
+// the row's) and writes them out as one run, highest digit first.  The
+// selection then reads only the head of each run.
 // Key formats of the rescoring kernel: bf16 keys with the group sum
 // (Eq. (1)), bf16 keys with the group maximum (Eq. (9)), 2-bit keys with the
 // group maximum (Eq. (7)-(9), row format of q2_impl.cuh).
@@ -236,27 +243,34 @@ enum : int { kFmtSum = 0, kFmtMax = 1, kFmtQ2 = 2 };
 
 template <int D, int FMT = kFmtSum>
 struct RescoreCfg {
-    static constexpr int kTileRows = 128;
-    static constexpr int kStages = 3;                  // data stages per consumer warp
-    static constexpr int kPosDepth = 8;                // position tables in the ring
-    static constexpr int kConsumerWarps = 8;
-    static constexpr int kThreads = 32 * (kConsumerWarps + 1);
+    static constexpr int kTileRows = 128;              // slots of a window
+    static constexpr int kStages = 3;                  // windows in a warp's pipeline
+    static constexpr int kWarps = 8;
+    static constexpr int kThreads = 32 * kWarps;
     static constexpr int kRowBytes = FMT == kFmtQ2 ? q2_row_bytes(D) : D * 2;
+    // rows read by ldmatrix are padded by 16 bytes: eight consecutive rows
+    // then start in eight different bank quads (conflict-free, no swizzle)
+    static constexpr int kRowStride = FMT == kFmtMax ? kRowBytes + 16 : kRowBytes;
     static constexpr int kNL = kRowBytes / 16;         // lanes (16-byte pieces) per key row
     static constexpr int kRPI = 32 / kNL;
-    static constexpr int kRowsPerWarp = kTileRows / kConsumerWarps;   // 16
+    static constexpr int kRowsPerWarp = kTileRows / kWarps;   // 16
     static constexpr int kSteps = kRowsPerWarp / kRPI;
-    static constexpr int kTileBytes = kTileRows * kRowBytes;
-    static constexpr int kPosOff = kStages * kTileBytes;
-    static constexpr int kBarOff = kPosOff + kPosDepth * kTileRows * 4;
-    static constexpr int kHistOff = kBarOff + 2 * kPosDepth * 8;
-    static constexpr int kSmemBytes = kHistOff + kHistBins * 4;
+    static constexpr int kWarpStage = kRowsPerWarp * kRowStride;
+    static constexpr int kStageBytes = kStages * kWarps * kWarpStage;
+    static constexpr int kItemOff = kStageBytes;                   // u64 [kRunCap]: key << 32 | position
+    static constexpr int kHistOff = kItemOff + kRunCap * 8;
+    static constexpr int kScratchOff = kHistOff + kHistBins * 4;
+    static constexpr int kSmemBytes = kScratchOff + 48 * 4;
+    // each run is sorted in the (then idle) stages
+    static constexpr bool kStageSort = kStageBytes >= kRunCap * 8;
+    static_assert(kMaxPartEntries % kThreads == 0, "entries split evenly over the threads");
 };
 
 // Group maximum (Eq. (9) form) of a warp's 16 gathered rows: the [16 x d] x
 // [d x 8] products of mma.sync m16n8k16 (bf16 in, fp32 accumulate; one or two
-// n-tiles of 8 heads), A fragments by ldmatrix from rows whose 16-byte chunk c
-// sits at chunk c ^ (row % 8) (conflict-free), B fragments (the group's
+// n-tiles of 8 heads), A fragments by ldmatrix from rows RS bytes apart
+// (conflict-free: rows padded to D*2 + 16 bytes, or rows of D*2 bytes whose
+// 16-byte chunk c sits at chunk c ^ (row % 8)), B fragments (the group's
 // queries, head n % G in column n) held in registers.  Returns the maxima of
 // rows lane/4 (.x) and lane/4 + 8 (.y) of the warp's block, in every lane of
 // the quad.
@@ -275,17 +289,19 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-template <int D>
+template <int D, int RS>
 __device__ __forceinline__ float2 group_max_16rows(const uint8_t *rows16, const uint32_t (&qf)[2][D / 16][2],
                                                    bool two_tiles, int lane) {
     float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
     const int r = (lane & 7) + ((lane >> 3) & 1) * 8;       // row this lane addresses
-    const uint32_t base = smem_addr(rows16 + r * (D * 2));
+    const uint32_t base = smem_addr(rows16 + r * RS);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
         const int chunk = 2 * kk + (lane >> 4);
+        // rows of D*2 bytes are swizzled (chunk c at c ^ (row % 8)); padded rows are not
+        const int at = RS == D * 2 ? (chunk ^ (lane & 7)) : chunk;
         uint32_t a0, a1, a2, a3;
-        ldmatrix_x4(base + (uint32_t)((chunk ^ (lane & 7)) << 4), a0, a1, a2, a3);
+        ldmatrix_x4(base + (uint32_t)(at << 4), a0, a1, a2, a3);
         mma_bf16_16816(c0, a0, a1, a2, a3, qf[0][kk][0], qf[0][kk][1]);
         if (two_tiles) mma_bf16_16816(c1, a0, a1, a2, a3, qf[1][kk][0], qf[1][kk][1]);
     }
@@ -301,130 +317,357 @@ __device__ __forceinline__ float2 group_max_16rows(const uint8_t *rows16, const 
     return make_float2(lo, hi);
 }
 
+// ---------------------------------------------------------------------------
+// Fused selection of a refined layer (Eq. (6)): the blocks of a row, resident
+// together, each holding its part's candidates (key << 32 | position, in
+// ascending position order) in shared memory.
+//   1. every block adds its histogram to the row's; barrier;
+//   2. every block reads the row's histogram (the first digit b1 of the
+//      kappa-th key), counts its candidates above b1 and publishes its ties
+//      (first digit b1) and both counts; barrier;
+//   3. every block gathers all ties of the row and resolves the exact kappa-th
+//      key T and the cutoff position among the items equal to T (the next 11
+//      bits; a handful of items in that bin ranked directly, a crowded bin by
+//      histograms); then every part's selected count, hence its offset;
+//   4. every block writes its selected positions, in order, at its offset:
+//      parts hold ascending disjoint position ranges, so the selection comes
+//      out in ascending order.
+// The block scans here are warp scans joined by one barrier.
+struct EpiView {              // the shared-memory view the threshold helpers take
+    uint32_t *hist;
+    int *scratch;
+    int *thr;
+};
+
+// Exclusive prefix of x over the block (NW warps); wsum holds NW ints and is
+// free again after the next barrier.  One barrier.
+template <int NW>
+__device__ __forceinline__ int block_excl_scan_fast(int x, int *wsum, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        const int v = wsum[w];
+        before += w < warp ? v : 0;
+        tot += v;
+    }
+    *total = tot;
+    return before + incl - x;
+}
+
+template <int NW>
+__device__ void fused_select(const ScoreArgs &a, int row, int part, int P, int n, const uint64_t *items,
+                             uint32_t *hist_s, int *scratch, uint8_t *area, int area_bytes,
+                             uint64_t *ties_out_g, const uint64_t *runs_row, int run_stride) {
+    constexpr int NTH = NW * 32;
+    constexpr int kPmax = 256;             // parts of a row in one fused launch (<= SMs)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int *cnt_sure = reinterpret_cast<int *>(area);        // [kPmax]
+    int *cnt_tie = cnt_sure + kPmax;                     // [kPmax]
+    int *tie_off = cnt_tie + kPmax;                      // [kPmax]
+    int *chosen = tie_off + kPmax;                       // [kPmax]
+    int *misc = chosen + kPmax;                          // [64]: ok, thr[2], counters, wsum
+    int *ok = misc, *thr = misc + 2, *acc = misc + 4, *wsum = misc + 16;
+    uint64_t *small = reinterpret_cast<uint64_t *>(misc + 64);   // [kSmallCap]
+    uint64_t *tcache = small + kSmallCap;                // the row's ties
+    const int tcap = (area_bytes - (int)((uint8_t *)tcache - area)) / 8;
+    uint32_t *hist_g = a.hist + (size_t)row * kHistBins;
+    uint32_t *bar = a.row_bar + row;
+    uint64_t *spill = a.tie_spill + (size_t)row * a.tie_cap;
+    const int kap = a.kap_out;
+    EpiView sv{hist_s, scratch, thr};
+
+    // 1. this part's histogram into the row's
+    for (int i = tid; i < kHistBins; i += NTH) {
+        const uint32_t v = hist_s[i];
+        if (v) atomicAdd(hist_g + i, v);
+    }
+    if (tid < 8) acc[tid] = 0;
+    block_group_barrier(bar, a.bar_base + (uint32_t)P, a.wait_ns, a.st, kWhereRescore, ok);
+
+    // 2. the row's histogram: candidates of the row, first digit of the kappa-th
+    {
+        const uint4 *g4 = reinterpret_cast<const uint4 *>(hist_g);
+        uint4 *s4 = reinterpret_cast<uint4 *>(hist_s);
+        int mine = 0;
+        for (int i = tid; i < kHistBins / 4; i += NTH) {
+            const uint4 v = __ldcg(g4 + i);
+            s4[i] = v;
+            mine += (int)(v.x + v.y + v.z + v.w);
+        }
+        mine = __reduce_add_sync(0xffffffffu, mine);
+        if (lane == 0) atomicAdd(&acc[0], mine);
+    }
+    __syncthreads();
+    const int n_row = acc[0];
+    const bool all = n_row <= kap;
+    int b1i = 0, above1 = 0;
+    if (!all) find_bin_2048<NW>(hist_s, kap, wsum, thr, &b1i, &above1);
+    const uint32_t b1 = (uint32_t)b1i;
+    const int need1 = kap - above1;
+    // this part's candidates above b1, and its ties (published through its run)
+    {
+        const unsigned lt = (1u << lane) - 1u;
+        int sure = 0, nt = 0;
+        unsigned tm_all[kRunCap / NTH];
+#pragma unroll
+        for (int i = 0; i < kRunCap / NTH; ++i) {
+            const int e = i * NTH + tid;
+            bool tie = false;
+            if (e < n) {
+                const uint32_t d = (uint32_t)(items[e] >> 32) >> (32 - kHistBits);
+                sure += (all || d > b1) ? 1 : 0;
+                tie = !all && d == b1;
+            }
+            tm_all[i] = __ballot_sync(0xffffffffu, tie);
+            nt += __popc(tm_all[i]);
+        }
+        sure = __reduce_add_sync(0xffffffffu, sure);
+        int base = 0;
+        if (lane == 0) {
+            atomicAdd(&acc[1], sure);
+            if (nt) base = atomicAdd(&acc[2], nt);
+        }
+        base = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+        for (int i = 0; i < kRunCap / NTH; ++i) {
+            if ((tm_all[i] >> lane) & 1u) ties_out_g[base + __popc(tm_all[i] & lt)] = items[i * NTH + tid];
+            base += __popc(tm_all[i]);
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        a.part_cnt[((size_t)row * P + part) * 2 + 0] = acc[1];
+        a.part_cnt[((size_t)row * P + part) * 2 + 1] = acc[2];
+    }
+    block_group_barrier(bar, a.bar_base + 2u * (uint32_t)P, a.wait_ns, a.st, kWhereRescore, ok);
+    // Every block of the grid has passed its arrivals: the next kernel may set up.
+    pdl_launch_dependents();
+    // every block of the row has read the row's histogram: left zeroed for the next use
+    if (part == 0)
+        for (int i = tid; i < kHistBins / 4; i += NTH)
+            reinterpret_cast<uint4 *>(hist_g)[i] = make_uint4(0u, 0u, 0u, 0u);
+
+    // 3. every part's counts and the head of its ties, fetched together (the
+    //    run areas and the counts are in L2); the ties are used in place,
+    //    part p's i-th at stage[p * kSpec + i]
+    constexpr int kSpec = 64;
+    uint64_t *stage_t = tcache;                          // [P][kSpec]
+    const bool spec_fits = (long long)P * kSpec <= tcap;
+    if (spec_fits) {
+        for (int q = tid; q < P * (kSpec / 2); q += NTH) {
+            const int p = q / (kSpec / 2), e2 = 2 * (q - p * (kSpec / 2));
+            cp_async16(stage_t + p * kSpec + e2, runs_row + (size_t)p * run_stride + e2, 16u);
+        }
+        cp_async_commit();
+    }
+    int cs = 0, ct = 0;
+    if (tid < P) {
+        cs = __ldcg(a.part_cnt + ((size_t)row * P + tid) * 2 + 0);
+        ct = __ldcg(a.part_cnt + ((size_t)row * P + tid) * 2 + 1);
+        cnt_sure[tid] = cs;
+        cnt_tie[tid] = ct;
+    }
+    for (int i = tid; i < kHistBins; i += NTH) hist_s[i] = 0;   // next 11 bits of the ties
+    if (tid == 0) acc[3] = 0;
+    if (spec_fits) cp_async_wait<0>();
+    int m;
+    const int toff = block_excl_scan_fast<NW>(ct, wsum, &m);     // barrier: counts, ties in place
+    if (tid < P) tie_off[tid] = toff;
+    const int big = __syncthreads_or(tid < P && ct > kSpec);
+    // The ties in one list: in place (every part's ties fit the fetched head)
+    // or compacted in order into tcache / the spill (a part with more).
+    const bool in_place = spec_fits && !big;
+    const int nslot = in_place ? P * kSpec : m;
+    auto tie_slot = [&](int f, uint64_t *it) -> bool {  // f-th slot of the list: a tie?
+        if (in_place) {
+            const int p = f / kSpec;
+            if (f - p * kSpec >= cnt_tie[p]) return false;
+            *it = stage_t[f];
+            return true;
+        }
+        *it = f < tcap ? tcache[f] : __ldcg(spill + f);
+        return true;
+    };
+    uint32_t T = 0u;
+    int cutoff = 0x7fffffff;
+    if (!all && m > 0) {
+        if (!in_place) {
+            // compaction (into tcache, which overwrites the fetched heads)
+            __syncthreads();
+            for (int p = warp; p < P; p += NW) {
+                const int c = cnt_tie[p], o = tie_off[p];
+                for (int i = lane; i < c; i += 32) {
+                    const uint64_t it = __ldcg(runs_row + (size_t)p * run_stride + i);
+                    const int e = o + i;
+                    if (e < tcap) tcache[e] = it;
+                    else if (e < a.tie_cap) spill[e] = it;
+                }
+            }
+            __syncthreads();
+        }
+        for (int f = tid; f < nslot; f += NTH) {
+            uint64_t it;
+            if (tie_slot(f, &it)) atomicAdd(&hist_s[((uint32_t)(it >> 32) >> 10) & 0x7ffu], 1u);
+        }
+        __syncthreads();
+        if (need1 < m) {
+            int b2, above2;
+            find_bin_2048<NW>(hist_s, need1, wsum, thr, &b2, &above2);
+            const int need2 = need1 - above2;
+            const uint32_t hi21 = (b1 << 21) | ((uint32_t)b2 << 10);
+            if ((int)hist_s[b2] <= kSmallCap) {
+                for (int f = tid; f < nslot; f += NTH) {
+                    uint64_t it;
+                    if (tie_slot(f, &it) && ((uint32_t)(it >> 32) & 0xfffffc00u) == hi21)
+                        small[atomicAdd(&acc[3], 1)] = it;
+                }
+                __syncthreads();
+                // the need2-th item of the bin in (key descending, position ascending) order
+                const int ns = acc[3];
+                for (int i = tid; i < ns; i += NTH) {
+                    const uint64_t u = small[i];
+                    const uint32_t ku = (uint32_t)(u >> 32), pu = (uint32_t)u;
+                    int rk = 0;
+                    for (int j = 0; j < ns; ++j) {
+                        const uint64_t w = small[j];
+                        const uint32_t kw = (uint32_t)(w >> 32);
+                        rk += kw > ku || (kw == ku && (uint32_t)w < pu);
+                    }
+                    if (rk == need2 - 1) {
+                        thr[0] = (int)ku;
+                        thr[1] = (int)pu;
+                    }
+                }
+                __syncthreads();
+                T = (uint32_t)thr[0];
+                cutoff = thr[1];
+            } else {
+                if (in_place) {
+                    // the histogram fallback takes the ties as one list
+                    __syncthreads();
+                    for (int p = warp; p < P; p += NW) {
+                        const int c = cnt_tie[p], o = tie_off[p];
+                        for (int i = lane; i < c; i += 32) spill[o + i] = stage_t[p * kSpec + i];
+                    }
+                    __threadfence_block();
+                    __syncthreads();
+                }
+                auto tie_at = [&](int e) -> uint64_t {
+                    return in_place ? __ldcg(spill + e) : (e < tcap ? tcache[e] : __ldcg(spill + e));
+                };
+                resolve_threshold(sv, tie_at, m, b1, need1, &T, &cutoff);
+            }
+        }
+    }
+    // every part's chosen ties (all of them when need1 >= m)
+    for (int p = tid; p < P; p += NTH) chosen[p] = 0;
+    __syncthreads();
+    if (!all && m > 0) {
+        if (in_place) {
+            for (int f = tid; f < nslot; f += NTH) {
+                uint64_t it;
+                if (!tie_slot(f, &it)) continue;
+                const uint32_t ku = (uint32_t)(it >> 32);
+                if (ku > T || (ku == T && (int)(uint32_t)it <= cutoff)) atomicAdd(&chosen[f / kSpec], 1);
+            }
+        } else {
+            for (int p = warp; p < P; p += NW) {
+                const int c = cnt_tie[p], o = tie_off[p];
+                int k = 0;
+                for (int i = lane; i < c; i += 32) {
+                    const int e = o + i;
+                    const uint64_t it = e < tcap ? tcache[e] : __ldcg(spill + e);
+                    const uint32_t ku = (uint32_t)(it >> 32);
+                    k += (ku > T || (ku == T && (int)(uint32_t)it <= cutoff)) ? 1 : 0;
+                }
+                k = __reduce_add_sync(0xffffffffu, k);
+                if (lane == 0) chosen[p] = k;
+            }
+        }
+    }
+    __syncthreads();
+    // this part's offset in the selection, and the selection's size
+    int total_sel;
+    const int poff = block_excl_scan_fast<NW>(tid < P ? cnt_sure[tid] + chosen[tid] : 0, wsum, &total_sel);
+    if (tid == part) acc[5] = poff;
+    __syncthreads();
+    const int my_off = acc[5];
+
+    // 4. this part's selected positions, in order, at its offset: item
+    //    i * NTH + t is thread t's i-th (conflict-free reads); its output
+    //    index comes from the per-(round, warp) counts after one barrier
+    int32_t *out = a.sel_out + (size_t)row * kap;
+    auto picked = [&](uint64_t it) {
+        const uint32_t ku = (uint32_t)(it >> 32);
+        const uint32_t d = ku >> (32 - kHistBits);
+        return all || d > b1 || (d == b1 && (ku > T || (ku == T && (int)(uint32_t)it <= cutoff)));
+    };
+    constexpr int R = kRunCap / NTH;
+    int *rw = cnt_tie;                                   // [R][NW] counts (cnt_tie is done)
+    unsigned pm[R];
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        const int e = i * NTH + tid;
+        pm[i] = __ballot_sync(0xffffffffu, e < n && picked(items[e]));
+        if (lane == 0) rw[i * NW + warp] = __popc(pm[i]);
+    }
+    __syncthreads();
+    int o = my_off;
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+        int before = 0, rt = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const int v = rw[i * NW + w];
+            before += w < warp ? v : 0;
+            rt += v;
+        }
+        if ((pm[i] >> lane) & 1u) {
+            const int j = o + before + __popc(pm[i] & lt);
+            if (j < kap) out[j] = (int)(uint32_t)items[i * NTH + tid];
+        }
+        o += rt;
+    }
+    if (part == P - 1)
+        for (int j = total_sel + tid; j < kap; j += NTH) out[j] = -1;
+    if (part == 0 && tid == 0 && total_sel != min(kap, n_row))
+        report(a.st, kDevErrInternal, kWhereRescore, (uint32_t)total_sel);
+}
+
 template <int D, int FMT, int NT = 1>
 __global__ void __launch_bounds__(RescoreCfg<D, FMT>::kThreads, 1)
 k_refine_rescore(ScoreArgs a) {
     using C = RescoreCfg<D, FMT>;
     constexpr bool MAXAGG = FMT != kFmtSum;
+    constexpr int EPT = kMaxPartEntries / C::kThreads;     // source entries a thread
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *stages = smem;
-    int *pos_s = reinterpret_cast<int *>(smem + C::kPosOff);
-    uint64_t *pos_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
-    uint64_t *pos_empty = pos_full + C::kPosDepth;
+    uint64_t *items = reinterpret_cast<uint64_t *>(smem + C::kItemOff);
     uint32_t *hist_s = reinterpret_cast<uint32_t *>(smem + C::kHistOff);
+    int *scratch = reinterpret_cast<int *>(smem + C::kScratchOff);
     const int row = blockIdx.y, part = blockIdx.x, P = gridDim.x, z = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = row / a.Hkv, h = row % a.Hkv;
-    const int cstride = a.cstride > 0 ? a.cstride : a.Lmax;
     const int L = load_len(a.len, b, a.Lmax, a.st, kWhereRescore);
     for (int i = tid; i < kHistBins; i += C::kThreads) hist_s[i] = 0;
-    if (tid == 0) {
-        for (int s = 0; s < C::kPosDepth; ++s) {
-            mbar_init(&pos_full[s], 1);
-            mbar_init(&pos_empty[s], C::kConsumerWarps);
-        }
-        fence_mbar_init();
-    }
-    __syncthreads();
-    // The source selection and its offsets come from the preceding kernels.
-    pdl_wait();
-    const int32_t *off = a.src_off + (size_t)row * (a.kappa + 1);
-    const int n = min(min(__ldcg(off + a.kappa), L), a.Lmax);
-    const int s_begin = (int)((long long)part * n / P);
-    const int s_end = (int)((long long)(part + 1) * n / P);
-    const int nwin = (s_end - s_begin + C::kTileRows - 1) / C::kTileRows;
-    if (nwin <= 0) {
-        pdl_launch_dependents();
-        return;
-    }
 
-    if (warp == C::kConsumerWarps) {
-        // ---------------- producer warp: the position tables ---------------------
-        const int32_t *src = a.src + (size_t)row * a.kappa;
-        if (a.radius == 0) {
-            // Radius 0 (a pool, or a proposal already cut into single
-            // positions): each entry of the canonical source owns exactly its
-            // own position, so slot s is entry s and a window's table is a
-            // copy of the source.  A malformed entry (outside [0, L), or not
-            // above its predecessor) is reported and reads row 0.
-            for (int it = 0; it < nwin; ++it) {
-                const int s = it % C::kPosDepth;
-                const uint32_t ph = (uint32_t)(it / C::kPosDepth) & 1u;
-                if (!mbar_wait(&pos_empty[s], ph ^ 1u, a.wait_ns)) {
-                    if (lane == 0) report(a.st, kDevErrTimeout, kWhereRescore, (uint32_t)it);
-                    break;
-                }
-                const int w0 = s_begin + it * C::kTileRows;
-                const int wend = min(w0 + C::kTileRows, s_end);
-                int *pos = pos_s + s * C::kTileRows;
-                for (int t = w0 + lane; t < wend; t += 32) {
-                    int p = __ldcg(src + t);
-                    const int prev = t > 0 ? __ldcg(src + t - 1) : -1;
-                    if (p < 0 || p >= L || p <= prev) {
-                        report(a.st, kDevErrBadIndex, kWhereRescore, (uint32_t)p);
-                        p = 0;
-                    }
-                    pos[t - w0] = p;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&pos_full[s]);
-            }
-            return;
-        }
-        // First entry to look at: the last one starting at or before s_begin,
-        // by a 64-way search over the offsets (off[0] = 0 <= s_begin).
-        int lo = 0, hi = a.kappa;
-        while (hi - lo > 32) {
-            const int st = (hi - lo + 63) / 64;
-            const int x0 = lo + 2 * lane * st, x1 = x0 + st;
-            const bool p0 = x0 < hi && __ldcg(off + x0) <= s_begin;
-            const bool p1 = x1 < hi && __ldcg(off + x1) <= s_begin;
-            const unsigned m0 = __ballot_sync(0xffffffffu, p0), m1 = __ballot_sync(0xffffffffu, p1);
-            const int k0 = m0 ? 2 * (31 - __clz(m0)) : 0;
-            const int k1 = m1 ? 2 * (31 - __clz(m1)) + 1 : 0;
-            lo += max(k0, k1) * st;
-            hi = min(hi, lo + st);
-        }
-        int jb = lo;
-        EntryRun e = make_entry(load_entry_raw(src, off, a.kappa, jb + lane), jb + lane, a.kappa, n,
-                                a.radius, L, a.st);
-        EntryRaw next = load_entry_raw(src, off, a.kappa, jb + 32 + lane);
-        for (int it = 0; it < nwin; ++it) {
-            const int s = it % C::kPosDepth;
-            const uint32_t ph = (uint32_t)(it / C::kPosDepth) & 1u;
-            if (!mbar_wait(&pos_empty[s], ph ^ 1u, a.wait_ns)) {
-                if (lane == 0) report(a.st, kDevErrTimeout, kWhereRescore, (uint32_t)it);
-                break;
-            }
-            const int w0 = s_begin + it * C::kTileRows;
-            const int wend = min(w0 + C::kTileRows, s_end);
-            int *pos = pos_s + s * C::kTileRows;
-            for (;;) {
-                const int g0 = max(e.o0, w0), g1 = min(e.o1, wend);
-                if (g0 < g1) {
-                    // keep the rows inside this row of the key cache whatever the offsets say
-                    const int r0 = min(e.lo + (g0 - e.o0), a.Lmax - (g1 - g0));
-                    for (int t = g0; t < g1; ++t) pos[t - w0] = r0 + (t - g0);
-                }
-                const int reach = __shfl_sync(0xffffffffu, e.o1, 31);
-                if (reach >= wend || jb + 32 >= a.kappa) break;
-                jb += 32;
-                e = make_entry(next, jb + lane, a.kappa, n, a.radius, L, a.st);
-                next = load_entry_raw(src, off, a.kappa, jb + 32 + lane);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&pos_full[s]);
-        }
-        return;
-    }
-
-    // ---------------- consumers ------------------------------------------------
-    const int slice = lane % C::kNL, sub = lane / C::kNL;
-    const uint16_t *qb = static_cast<const uint16_t *>(z == 0 ? a.q : a.qz[z]);
-    const int Hq = a.Hkv * a.G;
+    // This lane's query data (an input: read while the predecessor finishes).
     // Group sum: qbar, this lane's 8 elements.  Group maximum: the B fragments
     // of the group's queries (column n of n-tile t is head (8t + n) % G; k
     // pairs 2*(lane%4) and +8 of each 16-wide k step).
+    const int slice = lane % C::kNL, sub = lane / C::kNL;
+    const uint16_t *qb = static_cast<const uint16_t *>(z == 0 ? a.q : a.qz[z]);
+    const int Hq = a.Hkv * a.G;
     float qreg[8];
     uint32_t qf[2][D / 16][2];
     Q2Query<D, NT> Q;
@@ -454,91 +697,196 @@ k_refine_rescore(ScoreArgs a) {
         }
     }
     const bool two_tiles = a.G > 8;
+    __syncthreads();                                    // histogram zeroed
+
+    // The source selection comes from the preceding kernels.
+    pdl_wait();
+    const int E = a.kappa;
+    const int j0 = (int)((long long)part * E / P), j1 = (int)((long long)(part + 1) * E / P);
+    const int ne = min(j1 - j0, kMaxPartEntries);
+    const int32_t *src = a.src + (size_t)row * E + j0;
+    // The ranges owned by this thread's entries [t0, t0 + EPT) of the part:
+    // first slot, length, first position (kept in registers).
+    const int t0 = tid * EPT;
+    int cnt[EPT], lo_[EPT], off_[EPT];
+    {
+        int prev = (t0 < ne && j0 + t0 > 0) ? __ldcg(src + t0 - 1) : -1;
+        int cur[EPT];
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) cur[e] = t0 + e < ne ? __ldcg(src + t0 + e) : -1;
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+            const int i = cur[e];
+            cnt[e] = 0;
+            lo_[e] = 0;
+            if (i >= 0) {
+                if (i >= L || (prev >= 0 && i <= prev)) {
+                    report(a.st, kDevErrBadIndex, kWhereRescore, (uint32_t)i);
+                } else {
+                    long long lo = (long long)i - a.radius;
+                    if (prev >= 0 && (long long)prev + a.radius + 1 > lo) lo = (long long)prev + a.radius + 1;
+                    if (lo < 0) lo = 0;
+                    long long hi = (long long)i + a.radius;
+                    if (hi > L - 1) hi = L - 1;
+                    if (hi >= lo) {
+                        lo_[e] = (int)lo;
+                        cnt[e] = (int)(hi - lo + 1);
+                    }
+                }
+            }
+            prev = i;
+        }
+    }
+    int n;
+    {
+        int mine = 0;
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) mine += cnt[e];
+        int run = block_exclusive_scan(mine, scratch, &n);
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+            off_[e] = run;
+            run += cnt[e];
+        }
+    }
+    const int K = a.run_k;
+    if (n > K * kRunCap) {
+        if (tid == 0) report(a.st, kDevErrInternal, kWhereRescore, (uint32_t)n);
+        n = K * kRunCap;
+    }
+
     const uint8_t *kb = static_cast<const uint8_t *>(z == 0 ? a.k : a.kz[z]) +
                         (size_t)row * a.Lmax * C::kRowBytes;
-    float *S = a.S + (size_t)z * a.zS + (size_t)row * cstride;
-    int32_t *cpos = a.cpos + (size_t)z * a.zS + (size_t)row * cstride;
+    const size_t nruns = (size_t)P * K;
+    uint64_t *runs_row = a.runs + (size_t)z * a.zruns + (size_t)row * nruns * kRunCap;
+    int32_t *cnt_row = a.run_cnt + (size_t)z * a.zcnt + (size_t)row * nruns;
+    uint32_t *hist_g = a.hist + (size_t)z * a.zhist + (size_t)row * kHistBins;
+    float *Spos = a.Spos ? a.Spos + (size_t)row * a.spos_stride : nullptr;
     const int r_base = warp * C::kRowsPerWarp;
-    // The row whose score this lane stores, if it is a writer.
-    const int r_item = MAXAGG ? r_base + (lane >> 2) + ((lane & 3) == 1 ? 8 : 0)
-                              : r_base + transpose_item<C::kSteps, C::kNL>(lane) * C::kRPI + sub;
+    // The row (of the warp's 16) whose score this lane stores, if it is a writer.
+    const int rr_item = MAXAGG ? (lane >> 2) + ((lane & 3) == 1 ? 8 : 0)
+                               : transpose_item<C::kSteps, C::kNL>(lane) * C::kRPI + sub;
     const bool writer = MAXAGG ? (lane & 3) < 2 : transpose_writer<C::kSteps, C::kNL>(lane);
-    bool failed = false;
-    // Issue this lane's pieces of window `it` (rows r_base + st*kRPI + sub,
-    // bytes [16*slice, 16*slice + 16)); rows past the window are zero-filled.
-    auto gather = [&](int it) {
-        const int s = it % C::kPosDepth;
-        const uint32_t ph = (uint32_t)(it / C::kPosDepth) & 1u;
-        if (!failed && !mbar_wait(&pos_full[s], ph, a.wait_ns)) {
-            if (lane == 0) report(a.st, kDevErrTimeout, kWhereRescore, 0x40000000u | (uint32_t)it);
-            failed = true;
+    uint32_t *item_w = reinterpret_cast<uint32_t *>(items);   // [2e]: position, [2e + 1]: key
+    const int last = n > 0 ? (n - 1) / kRunCap : -1;
+
+    for (int k = 0; k <= last; ++k) {
+        const int s0 = k * kRunCap;
+        const int nk = min(kRunCap, n - s0);
+        // The run's position table.
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+            const int a0 = max(off_[e], s0), a1 = min(off_[e] + cnt[e], s0 + nk);
+            for (int t = a0; t < a1; ++t) item_w[2 * (t - s0)] = (uint32_t)(lo_[e] + (t - off_[e]));
         }
-        const int nrows = min(C::kTileRows, s_end - (s_begin + it * C::kTileRows));
-        const int *pos = pos_s + s * C::kTileRows;
-        uint8_t *tile = stages + (it % C::kStages) * C::kTileBytes;
+        __syncthreads();
+        const int nwin = (nk + C::kTileRows - 1) / C::kTileRows;
+        // This lane's pieces of window w (rows st*kRPI + sub of the warp's 16,
+        // bytes [16*slice, 16*slice + 16)); rows past the run are zero-filled.
+        auto gather = [&](int w) {
+            const int first = w * C::kTileRows + r_base;
+            uint8_t *dst = stages + ((w % C::kStages) * C::kWarps + warp) * C::kWarpStage + slice * 16;
 #pragma unroll
-        for (int st = 0; st < C::kSteps; ++st) {
-            const int r = r_base + st * C::kRPI + sub;
-            const bool ok = !failed && r < nrows;
-            const int krow = ok ? pos[r] : 0;
-            // the bf16 group-maximum path reads the rows by ldmatrix: swizzled chunks
-            const int chunk = FMT == kFmtMax ? (slice ^ (r & 7)) : slice;
-            cp_async16(tile + r * C::kRowBytes + chunk * 16,
-                       kb + (size_t)krow * C::kRowBytes + slice * 16, ok ? 16u : 0u);
+            for (int sp = 0; sp < C::kSteps; ++sp) {
+                const int rr = sp * C::kRPI + sub;
+                const bool ok = first + rr < nk;
+                const int p = ok ? (int)item_w[2 * (first + rr)] : 0;
+                cp_async16(dst + rr * C::kRowStride, kb + (size_t)p * C::kRowBytes + slice * 16, ok ? 16u : 0u);
+            }
+            cp_async_commit();
+        };
+#pragma unroll
+        for (int w = 0; w < C::kStages - 1; ++w) {
+            if (w < nwin) gather(w);
+            else cp_async_commit();
         }
-        cp_async_commit();
-    };
+        for (int w = 0; w < nwin; ++w) {
+            if (w + C::kStages - 1 < nwin) gather(w + C::kStages - 1);
+            else cp_async_commit();
+            cp_async_wait<C::kStages - 1>();             // this lane's pieces of window w
+            const uint8_t *tw = stages + ((w % C::kStages) * C::kWarps + warp) * C::kWarpStage;
+            float part_[C::kSteps];
+            if constexpr (FMT == kFmtQ2) {
+                __syncwarp();                            // the warp reads rows of all its lanes
+                const float2 m = q2_group_max_16rows<D, NT>(tw, Q, lane);
+                part_[0] = (lane & 3) == 1 ? m.y : m.x;
+            } else if constexpr (MAXAGG) {
+                __syncwarp();
+                const float2 m = group_max_16rows<D, C::kRowStride>(tw, qf, two_tiles, lane);
+                part_[0] = (lane & 3) == 1 ? m.y : m.x;
+            } else {
 #pragma unroll
-    for (int it = 0; it < C::kStages - 1; ++it) {
-        if (it < nwin) gather(it);
-        else cp_async_commit();
-    }
-    for (int it = 0; it < nwin; ++it) {
-        if (it + C::kStages - 1 < nwin) gather(it + C::kStages - 1);
-        else cp_async_commit();
-        cp_async_wait<C::kStages - 1>();                // this lane's pieces of window `it`
-        const uint8_t *tile = stages + (it % C::kStages) * C::kTileBytes;
-        float part_[C::kSteps];
-        if constexpr (FMT == kFmtQ2) {
-            // The warp reads rows gathered by all of its lanes.
-            __syncwarp();
-            const float2 m = q2_group_max_16rows<D, NT>(tile + r_base * C::kRowBytes, Q, lane);
-            part_[0] = (lane & 3) == 1 ? m.y : m.x;
-        } else if constexpr (MAXAGG) {
-            // The warp reads rows gathered by all of its lanes.
-            __syncwarp();
-            const float2 m = group_max_16rows<D>(tile + r_base * C::kRowBytes, qf, two_tiles, lane);
-            part_[0] = (lane & 3) == 1 ? m.y : m.x;
-        } else {
-#pragma unroll
-            for (int st = 0; st < C::kSteps; ++st) {
-                const int r = r_base + st * C::kRPI + sub;
-                const uint4 kv = *reinterpret_cast<const uint4 *>(tile + r * C::kRowBytes + slice * 16);
-                part_[st] = dot8(kv, qreg);
+                for (int sp = 0; sp < C::kSteps; ++sp) {
+                    const uint4 kv = *reinterpret_cast<const uint4 *>(
+                        tw + (sp * C::kRPI + sub) * C::kRowStride + slice * 16);
+                    part_[sp] = dot8(kv, qreg);
+                }
+                transpose_reduce<C::kSteps, C::kNL>(part_, lane);
+            }
+            __syncwarp();                                // the stage is free for the next gather
+            const int t = w * C::kTileRows + r_base + rr_item;     // run-local slot
+            if (writer && t < nk) {
+                const float sc = part_[0] * a.scale;
+                const uint32_t key = score_key(sc);
+                item_w[2 * t + 1] = key;
+                atomicAdd(&hist_s[key >> (32 - kHistBits)], 1u);
+                if (Spos) Spos[item_w[2 * t]] = sc;
             }
         }
-        const int s = it % C::kPosDepth;
-        const int p_item = pos_s[s * C::kTileRows + r_item];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pos_empty[s]);
-        if constexpr (!MAXAGG) transpose_reduce<C::kSteps, C::kNL>(part_, lane);
-        const int w0 = s_begin + it * C::kTileRows;
-        const int nrows = min(C::kTileRows, s_end - w0);
-        if (!failed && writer && r_item < nrows) {
-            const float sc = part_[0] * a.scale;
-            S[w0 + r_item] = sc;
-            cpos[w0 + r_item] = p_item;
-            atomicAdd(&hist_s[score_key(sc) >> (32 - kHistBits)], 1u);
+        cp_async_wait<0>();
+        __syncthreads();                         // every copy landed, every key in place
+        if (a.fused) break;                      // one run: the fused selection below
+        // The selection may set up now; it waits for this grid before reading.
+        if (k == last) pdl_launch_dependents();
+
+        // Counting sort of the run by first digit, highest first: this run's
+        // histogram goes to the row's and becomes the bins' start offsets.
+        constexpr int BPT = kHistBins / C::kThreads;
+        const int hb = kHistBins - (tid + 1) * BPT;   // thread 0 owns the top bins
+        uint32_t hv[BPT];
+        int mine = 0;
+#pragma unroll
+        for (int i = 0; i < BPT; ++i) {
+            hv[i] = hist_s[hb + i];
+            mine += (int)hv[i];
+            if (hv[i]) atomicAdd(hist_g + hb + i, hv[i]);
         }
+        int tot;
+        int cur = block_exclusive_scan(mine, scratch, &tot);   // items in higher bins
+#pragma unroll
+        for (int i = BPT - 1; i >= 0; --i) {
+            hist_s[hb + i] = (uint32_t)cur;
+            cur += (int)hv[i];
+        }
+        __syncthreads();
+        uint64_t *dst_g = runs_row + (size_t)(part * K + k) * kRunCap;
+        uint64_t *dst = C::kStageSort ? reinterpret_cast<uint64_t *>(stages) : dst_g;
+        for (int e = tid; e < nk; e += C::kThreads) {
+            const uint64_t it = items[e];
+            const uint32_t o = atomicAdd(&hist_s[(uint32_t)(it >> 32) >> (32 - kHistBits)], 1u);
+            if (o < (uint32_t)nk) dst[o] = it;
+        }
+        __syncthreads();
+        if constexpr (C::kStageSort) {
+            const uint4 *s4 = reinterpret_cast<const uint4 *>(stages);
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst_g);
+            for (int e = tid; 2 * e < nk; e += C::kThreads) {
+                if (2 * e + 1 < nk) d4[e] = s4[e];
+                else dst_g[2 * e] = reinterpret_cast<const uint64_t *>(stages)[2 * e];
+            }
+        }
+        if (tid == 0) cnt_row[part * K + k] = nk;
+        for (int i = tid; i < kHistBins; i += C::kThreads) hist_s[i] = 0;
+        __syncthreads();                         // stages, table and histogram free again
     }
-    cp_async_wait<0>();
-    consumer_sync();
-    pdl_launch_dependents();
-    uint32_t *hist_g = a.hist + (size_t)z * a.zhist + (size_t)row * kHistBins;
-    for (int i = tid; i < kHistBins; i += 32 * C::kConsumerWarps) {
-        const uint32_t v = hist_s[i];
-        if (v) atomicAdd(hist_g + i, v);
+    if (a.fused) {
+        fused_select<C::kWarps>(a, row, part, P, n, items, hist_s, scratch, stages, C::kStageBytes,
+                                runs_row + (size_t)part * K * kRunCap, runs_row, K * kRunCap);
+        return;
     }
+    if (last < 0) pdl_launch_dependents();
+    if (tid == 0)
+        for (int k = last + 1; k < K; ++k) cnt_row[part * K + k] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -563,33 +911,32 @@ cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s)
 
 
 template <int D, int FMT, int NT = 1>
-static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, int num_sms, cudaStream_t s) {
+static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, cudaStream_t s) {
     using C = RescoreCfg<D, FMT>;
     cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D, FMT, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    // About one CTA per SM over all rows (of all batched layers); each row's
-    // proposal is split evenly.
     const int nz = a.nz > 1 ? a.nz : 1;
     const int rows = a.B * a.Hkv;
-    const int parts = rows * nz >= num_sms ? 1 : num_sms / (rows * nz);
-    return launch_kernel(k_refine_rescore<D, FMT, NT>, dim3((unsigned)parts, (unsigned)rows, (unsigned)nz),
+    return launch_kernel(k_refine_rescore<D, FMT, NT>, dim3((unsigned)a.parts, (unsigned)rows, (unsigned)nz),
                          dim3(C::kThreads), C::kSmemBytes, s, a);
 }
 
-cudaError_t launch_refine_rescore(const ScoreArgs &a, int num_sms, cudaStream_t s) {
+cudaError_t launch_refine_rescore(const ScoreArgs &a, cudaStream_t s) {
+    if (a.parts < 1 || a.run_k < 1 || (long long)(a.kappa + a.parts - 1) / a.parts > kMaxPartEntries)
+        return cudaErrorInvalidValue;
     if (a.agg == kAggMax && a.q2) {
         if (a.G > 8)
-            return a.d == 128 ? launch_refine_rescore_d<128, kFmtQ2, 2>(a, num_sms, s)
-                              : launch_refine_rescore_d<64, kFmtQ2, 2>(a, num_sms, s);
-        return a.d == 128 ? launch_refine_rescore_d<128, kFmtQ2, 1>(a, num_sms, s)
-                          : launch_refine_rescore_d<64, kFmtQ2, 1>(a, num_sms, s);
+            return a.d == 128 ? launch_refine_rescore_d<128, kFmtQ2, 2>(a, s)
+                              : launch_refine_rescore_d<64, kFmtQ2, 2>(a, s);
+        return a.d == 128 ? launch_refine_rescore_d<128, kFmtQ2, 1>(a, s)
+                          : launch_refine_rescore_d<64, kFmtQ2, 1>(a, s);
     }
     if (a.agg == kAggMax)
-        return a.d == 128 ? launch_refine_rescore_d<128, kFmtMax>(a, num_sms, s)
-                          : launch_refine_rescore_d<64, kFmtMax>(a, num_sms, s);
-    return a.d == 128 ? launch_refine_rescore_d<128, kFmtSum>(a, num_sms, s)
-                      : launch_refine_rescore_d<64, kFmtSum>(a, num_sms, s);
+        return a.d == 128 ? launch_refine_rescore_d<128, kFmtMax>(a, s)
+                          : launch_refine_rescore_d<64, kFmtMax>(a, s);
+    return a.d == 128 ? launch_refine_rescore_d<128, kFmtSum>(a, s)
+                      : launch_refine_rescore_d<64, kFmtSum>(a, s);
 }
 
 }  // namespace prism

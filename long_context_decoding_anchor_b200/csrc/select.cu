@@ -11,6 +11,8 @@
 // candidates (first digit >= b1) in position order, and select_finish
 // (select_impl.cuh) resolves the exact threshold across the cluster and
 // writes the selection.
+#include <atomic>
+
 #include "select_impl.cuh"
 
 namespace prism {
@@ -199,22 +201,27 @@ int select_cluster_size(int items, bool refine) {
 }
 
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s) {
-    static bool attr_done[64] = {false};
+    // per device: the kernel's attributes are set (setting them twice is harmless)
+    static std::atomic<bool> attr_done[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+    if (dev < 0 || dev >= 64 || !attr_done[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kSelDynSmem);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(k_select, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_done[dev] = true;
+        if (dev >= 0 && dev < 64) attr_done[dev].store(true, std::memory_order_release);
     }
     const int rows = a.B * a.Hkv;
     const bool refine = a.cpos != nullptr;
     const long long bound = a.n_bound > 0 ? (long long)a.n_bound
                             : refine ? (long long)a.kappa * (2LL * a.radius + 1) : (long long)a.Lmax;
     const int items = (int)(bound < a.Lmax ? bound : a.Lmax);
+    // A refined row (a proposal or a pool, tens of thousands of candidates)
+    // is selected by one block: its latency is a few block barriers, where a
+    // cluster pays cluster barriers and distributed gathers.
+    if (refine && select_row_fits(items, a.kappa)) return launch_select_row(a, items, s);
     const int C = select_cluster_size(items, refine);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(C, rows, a.nz > 1 ? a.nz : 1);

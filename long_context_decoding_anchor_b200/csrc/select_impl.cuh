@@ -1,7 +1,7 @@
-// select_impl.cuh -- the cluster-wide part of the exact top-kappa selection
-// (Eq. (2) and Eq. (6) of "Prism Attention", section 4.1), shared by the
-// anchor selection kernel (select.cu) and the fused rescoring + selection
-// kernel of refined layers (refine.cu).
+// select_impl.cuh -- the exact top-kappa selection (Eq. (2) and Eq. (6) of
+// "Prism Attention", section 4.1): the radix-threshold helpers shared by the
+// cluster selection kernel (select.cu) and the one-CTA-per-row selection
+// kernel (select_row.cu), and the cluster-wide part of the former.
 //
 // A row's items are split among the C CTAs of a thread-block cluster in
 // contiguous slices, slice r = [r*n/C, (r+1)*n/C).  Before select_finish runs,
@@ -94,8 +94,8 @@ __device__ __forceinline__ int warp_offsets(SelShared &sm, int wcount, int *tota
 // by value, the top bin last) and the number of items above it.  nbins is a
 // multiple of 256; the first 256 threads own nbins / 256 bins each.  All
 // threads; contains __syncthreads().
-__device__ __forceinline__ void threshold_bin(SelShared &sm, int nbins, int need, int *bin,
-                                              int *above) {
+template <class SM>
+__device__ __forceinline__ void threshold_bin(SM &sm, int nbins, int need, int *bin, int *above) {
     const int t = threadIdx.x;
     const int per = nbins / 256;
     const int hi = nbins - t * per;                // thread t owns [hi - per, hi): thread 0 the top
@@ -123,16 +123,74 @@ __device__ __forceinline__ void threshold_bin(SelShared &sm, int nbins, int need
     __syncthreads();                               // thr may be reset by the next call
 }
 
-__device__ __forceinline__ void zero_hist(SelShared &sm, int nbins) {
+template <class SM>
+__device__ __forceinline__ void zero_hist(SM &sm, int nbins) {
     for (int i = threadIdx.x; i < nbins; i += blockDim.x) sm.hist[i] = 0;
     __syncthreads();
+}
+
+// The bin of h[0, 2048) holding the need-th largest item (bins ordered by
+// value, the top bin last) and the number of items above it, by the NW warps
+// of the block: lane l of warp w holds the 2048 / (32 NW) bins of descending
+// ranks starting at (32w + l) * 2048 / (32 NW); hardware warp sums, then one
+// scan in the warp that holds the answer.  wsum holds NW ints, thr two.  A
+// block-wide scan costs a few hundred cycles of dependent shuffles and
+// barriers; this costs two barriers.  Whole block.
+template <int NW>
+__device__ __forceinline__ void find_bin_2048(const uint32_t *h, int need, int *wsum, int *thr,
+                                              int *bin, int *above) {
+    constexpr int BPL = kHistBins / (32 * NW);            // bins a lane, a multiple of 4
+    static_assert(BPL >= 4 && BPL % 4 == 0, "whole 16-byte groups of bins a lane");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int b0 = kHistBins - BPL * (32 * warp + lane + 1);
+    uint32_t c[BPL];                                      // descending: c[0] is bin b0 + BPL - 1
+    int ls = 0;
+#pragma unroll
+    for (int g = 0; g < BPL / 4; ++g) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(h + b0 + 4 * g);
+        c[BPL - 1 - 4 * g] = v.x;
+        c[BPL - 2 - 4 * g] = v.y;
+        c[BPL - 3 - 4 * g] = v.z;
+        c[BPL - 4 - 4 * g] = v.w;
+        ls += (int)(v.x + v.y + v.z + v.w);
+    }
+    const int ws = __reduce_add_sync(0xffffffffu, ls);
+    if (lane == 0) wsum[warp] = ws;
+    if (threadIdx.x == 0) thr[0] = thr[1] = 0;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    if (before < need && before + ws >= need) {
+        int incl = ls;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const int ab = before + incl - ls;
+        if (ab < need && ab + ls >= need) {
+            int acc = ab;
+#pragma unroll
+            for (int i = 0; i < BPL; ++i) {
+                if (acc + (int)c[i] >= need) {
+                    thr[0] = b0 + BPL - 1 - i;
+                    thr[1] = acc;
+                    break;
+                }
+                acc += (int)c[i];
+            }
+        }
+    }
+    __syncthreads();
+    *bin = thr[0];
+    *above = thr[1];
 }
 
 // Items equal to key T: the position of the rank-th (0-based) lowest, by two
 // radix digits of the position (10 + 10 bits; positions < 2^20).  Bins are
 // reversed so that the lowest position sits in the top bin.
-template <class Get>
-__device__ int tie_cutoff(SelShared &sm, Get tie, int m, uint32_t T, int rank) {
+template <class SM, class Get>
+__device__ int tie_cutoff(SM &sm, Get tie, int m, uint32_t T, int rank) {
     zero_hist(sm, 1024);
     for (int e = threadIdx.x; e < m; e += blockDim.x) {
         const uint64_t it = tie(e);
@@ -157,8 +215,8 @@ __device__ int tie_cutoff(SelShared &sm, Get tie, int m, uint32_t T, int rank) {
 // The exact kappa-th key T from the items of first digit b1 among the m given
 // (need1 = places left after the items above that bin), and the cutoff
 // position among the items equal to T.  All threads.
-template <class Get>
-__device__ void resolve_threshold(SelShared &sm, Get tie, int m, uint32_t b1, int need1,
+template <class SM, class Get>
+__device__ void resolve_threshold(SM &sm, Get tie, int m, uint32_t b1, int need1,
                                   uint32_t *T_out, int *cutoff_out) {
     zero_hist(sm, kHistBins);                        // bits 20..10
     for (int e = threadIdx.x; e < m; e += blockDim.x) {

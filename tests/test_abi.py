@@ -212,6 +212,7 @@ def _shard(n_ranks=2, rank=0, shard_len=2048):
 @pytest.mark.parametrize("sh,cfg_kw,status", [
     (dict(n_ranks=0), {}, 1), (dict(rank=2), {}, 1), (dict(rank=-1), {}, 1),
     (dict(shard_len=0), {}, 1), (dict(shard_len=1000), {}, 1),     # 2 x 1000 < Lmax 4096
+    (dict(n_ranks=2049, shard_len=1 << 20), {}, 1),               # positions past 2^31 - 1
     (dict(), dict(mode=3, pool_factor=2, flags=2), 2),              # 2-bit keys
     (dict(), dict(head_dim=96), 2),
 ])

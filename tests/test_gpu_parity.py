@@ -45,6 +45,14 @@ SHAPES = {
                                                radius=2, ragged=(1, 777), n_clusters=3),
     "d64-g8": synth.WORKLOADS[1].replace(max_len=1500, n_layers=2, n_q_heads=16,
                                          n_kv_heads=2, kappa=300, radius=4),
+    # a budget of 9000 over 30011 tokens (the anchor's cluster selection
+    # with large tie lists)
+    "d64-kappa-9000": synth.WORKLOADS[1].replace(max_len=30011, n_layers=2, kappa=9000,
+                                                 radius=1, n_clusters=40),
+    # more rows than SMs: the rescoring's blocks cannot all be resident at
+    # once, so refined rows go through the run selection kernel
+    "d128-160-rows": synth.WORKLOADS[4].replace(batch=20, max_len=2000, n_layers=2, kappa=128,
+                                                ragged=(500, 2000), n_clusters=4),
 }
 
 
