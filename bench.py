@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-q2", action="store_true", help="skip the 2-bit key measurement")
+    ap.add_argument("--configs", default="2,4,5",
+                    help="other workloads measured into per_config ('' to skip)")
     ap.add_argument("--skip-cp", action="store_true",
                     help="skip the context-parallel measurement (512K workload)")
     ap.add_argument("--profile", action="store_true",
@@ -61,8 +63,10 @@ def parse_args():
                     help="override the workload's layer count (profiling a smaller case)")
     ap.add_argument("--pool", type=int, default=4,
                     help="rho of the pool-mode measurement (0: skip it)")
-    ap.add_argument("--mode", choices=["refine", "pool", "pool-int2"], default="refine",
-                    help="decode-step mode of a --profile run (pool uses --pool as rho; "
+    ap.add_argument("--mode", choices=["refine", "refine-chain", "pool", "pool-int2"],
+                    default="refine",
+                    help="decode-step mode of a --profile run (refine-chain: one anchor at "
+                         "layer 0, every other layer refined; pool uses --pool as rho; "
                          "pool-int2 scores on 2-bit keys)")
     return ap.parse_args()
 
@@ -179,6 +183,161 @@ def selection_recall(sel, exact) -> list:
         s_row = s_row[s_row >= 0]
         out.append(float(torch.isin(e_row, s_row).sum()) / max(1, e_row.numel()))
     return out
+
+
+def proposal_counts(prism, cfg, inp, idx, mask, ws) -> list:
+    """Per refined layer: the proposal size |P| of every (batch, KV head) row
+    (int tensor on the host), from the public refine call's candidate count."""
+    out = []
+    for l in range(cfg.n_layers):
+        if mask[l]:
+            continue
+        _, _, _, cc = prism.prism_index_refine(cfg, inp["q"][l], inp["k"][l], inp["lens"],
+                                               idx[l - 1].contiguous(), cand_cap=1, ws=ws)
+        out.append(cc.flatten().cpu())
+    return out
+
+
+def graph_step_ms(prism, cfg, inp, reps, dev, ws=None):
+    """Mean device time (CUDA events) of one CUDA-graph replay of the step."""
+    import torch
+    from long_context_decoding_anchor_b200.runner import DecodeStepGraph
+    n = cfg.n_layers
+    r = DecodeStepGraph(cfg, inp["q"][:n], inp["k"][:n], inp["v"][:n], inp["lens"], ws=ws)
+    for _ in range(3):
+        r.replay()
+    stream = torch.cuda.current_stream(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for _ in range(reps):
+        r.replay()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = r.launches
+    del r
+    return a.elapsed_time(b) / reps, launches
+
+
+def anchor_kernel_s(prism, cfg, inp, anchors, ws, reps, dev):
+    """Mean seconds of one prism_score_anchor launch (a single scoring kernel),
+    CUDA events around each launch on the launching stream."""
+    import ctypes
+
+    import torch
+    L = prism.lib()
+    stream = torch.cuda.current_stream(dev)
+    S = torch.empty((cfg.batch, cfg.n_kv_heads, cfg.max_len), dtype=torch.float32, device=dev)
+    cfgp = ctypes.byref(cfg)
+
+    def launch(l):
+        rc = L.prism_score_anchor(cfgp, ctypes.c_void_p(inp["q"][l].data_ptr()),
+                                  ctypes.c_void_p(inp["k"][l].data_ptr()),
+                                  ctypes.c_void_p(inp["lens"].data_ptr()),
+                                  ctypes.c_void_p(S.data_ptr()), ctypes.c_void_p(ws.data_ptr()),
+                                  ws.numel(), ctypes.c_void_p(stream.cuda_stream))
+        if rc != 0:
+            raise RuntimeError(f"prism_score_anchor: {rc}")
+    for i in range(3):
+        launch(anchors[i % len(anchors)])
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for i in range(reps):
+        evs[i][0].record(stream)
+        launch(anchors[i % len(anchors)])
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    del S
+    return statistics.mean(a.elapsed_time(b) for a, b in evs) * 1e-3
+
+
+def kernel_table(replay, dev) -> dict:
+    """Per kernel of one replay: launches, total and mean device microseconds
+    (CUPTI activity records through torch.profiler; no host launch cost,
+    overlapping kernels each counted in full), plus the replay's span."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    torch.cuda.synchronize(dev)
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        replay()
+        torch.cuda.synchronize(dev)
+    fd, fn = tempfile.mkstemp(prefix="prism_trace_", suffix=".json")
+    os.close(fd)
+    try:
+        prof.export_chrome_trace(fn)
+        with open(fn) as f:
+            ev = [e for e in json.load(f)["traceEvents"] if e.get("cat") == "kernel"]
+    finally:
+        os.unlink(fn)
+    rows = {}
+    for e in ev:
+        name = e["name"].replace("void ", "").replace("prism::", "").split("(")[0][:60]
+        r = rows.setdefault(name, [0, 0.0])
+        r[0] += 1
+        r[1] += float(e["dur"])
+    span = (max(e["ts"] + e["dur"] for e in ev) - min(e["ts"] for e in ev)) if ev else 0.0
+    return {"span_us": round(span, 2),
+            "kernels": {n: {"launches": c, "total_us": round(t, 2), "mean_us": round(t / c, 3)}
+                        for n, (c, t) in sorted(rows.items(), key=lambda x: -x[1][1])}}
+
+
+def measure_workload(args, prism, synth, wid, dev, peak, reps, world) -> dict:
+    """One of the pages' workloads at one GPU: graph-replayed step (us/layer),
+    its algorithmic HBM fraction, the anchor scoring kernel's roofline, the
+    refined layers alone, and the proposal sizes |P|."""
+    import torch
+    w = synth.WORKLOADS[wid]
+    inp = synth.make_inputs(w, device=dev)
+    cfg = prism.Config.from_workload(w)
+    ws = prism.workspace(cfg, dev)
+    N = w.n_layers
+    mask = w.anchor_mask()
+    lens_h = inp["lens"].cpu().tolist()
+    _, idx = prism.prism_decode_step(cfg, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                     want_idx=True, ws=ws)
+    st, detail = prism.prism_check_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"{w.name}: device status {st} {detail}")
+    props = proposal_counts(prism, cfg, inp, idx, mask, ws)
+    n_anchor = sum(mask)
+    kappa_eff = sum(min(w.kappa, int(L)) for L in lens_h) * w.n_kv_heads
+    gather = kappa_eff * w.head_dim * 2 * 2
+    a_bytes = anchor_bytes(w, lens_h)
+    prop_total = sum(int(p.sum()) for p in props)
+    step_bytes = n_anchor * a_bytes + prop_total * w.head_dim * 2 + N * gather
+    ms, launches = graph_step_ms(prism, cfg, inp, reps, dev, ws=ws)
+    ms = max_over_ranks(ms, dev)
+    anchors = [l for l in range(N) if mask[l]]
+    t_a = anchor_kernel_s(prism, cfg, inp, anchors, ws, max(8, reps), dev)
+    # refined layers alone: one anchor then every other layer refined, minus the anchor layer
+    cfg_r = prism.Config.from_workload(w, anchor_mask=[1] + [0] * (N - 1))
+    cfg_0 = prism.Config.from_workload(w.replace(n_layers=1))
+    t_r, _ = graph_step_ms(prism, cfg_r, inp, reps, dev)
+    t_0, _ = graph_step_ms(prism, cfg_0, inp, reps, dev)
+    _, idx_r = prism.prism_decode_step(cfg_r, inp["q"], inp["k"], inp["v"], inp["lens"],
+                                       want_idx=True, ws=ws)
+    props_r = proposal_counts(prism, cfg_r, inp, idx_r, [1] + [0] * (N - 1), ws)
+    r_us = (t_r - t_0) * 1e3 / (N - 1)
+    r_bytes = statistics.mean(int(p.sum()) for p in props_r) * w.head_dim * 2 + gather
+    allp = torch.cat(props).float() if props else torch.zeros(1)
+    step_gbs = step_bytes / (ms * 1e-3) / 1e9
+    res = {
+        "workload": f"{w.name}: {w.describe()}",
+        "value": whole_job_us_per_layer(ms, N, world), "unit": UNIT, "ms_per_step": ms,
+        "launches_per_step": launches,
+        "anchor_kernel": {"bound": "hbm", "achieved": a_bytes / t_a / 1e9, "peak": peak,
+                          "unit": "GB/s", "frac": a_bytes / t_a / 1e9 / peak,
+                          "us_per_launch": t_a * 1e6, "bytes_per_launch": a_bytes},
+        "proposal": {"mean_per_row": float(allp.mean()), "max_per_row": int(allp.max()),
+                     "min_per_row": int(allp.min()),
+                     "kappa_2r1": w.kappa * (2 * w.radius + 1)},
+        "refine_attn": {"bytes_per_layer": r_bytes, "us_per_layer": r_us,
+                        "frac": r_bytes / (r_us * 1e-6) / 1e9 / peak},
+        "step_hbm": {"algorithmic_bytes": step_bytes, "gbs": step_gbs, "frac": step_gbs / peak},
+    }
+    del inp, ws, idx, idx_r
+    torch.cuda.empty_cache()
+    return res
 
 
 def kernel_traffic(src_paths, profile_md):
@@ -409,9 +568,11 @@ def run_prism(args, rank, world, dev):
     if args.profile:
         pool_run = args.mode in ("pool", "pool-int2")
         q2_run = args.mode == "pool-int2"
+        chain = [1] + [0] * (w.n_layers - 1) if args.mode == "refine-chain" else None
         cfg = (prism.Config.from_workload(w, mode=prism.MODE_POOL, pool_factor=args.pool,
                                           flags=prism.FLAG_INT2_KEYS if q2_run else 0)
-               if pool_run else prism.Config.from_workload(w))
+               if pool_run else prism.Config.from_workload(
+                   w, **({"anchor_mask": chain} if chain else {})))
         ws = prism.workspace(cfg, dev)
         kq = [prism.prism_quantize_keys(cfg, kk, inp["lens"], ws=ws) for kk in inp["k"]] \
             if q2_run else None
@@ -721,35 +882,34 @@ def run_prism(args, rank, world, dev):
         }
         del kq
 
-    # -- per-stage breakdown (events around each public stage call)
-    def timed(fn, reps=8):
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(reps)]
-        fn(0)
-        for i in range(reps):
-            ev[i][0].record(stream)
-            fn(i)
-            ev[i][1].record(stream)
-        torch.cuda.synchronize(dev)
-        return statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+    # -- per-kernel breakdown: device durations (CUPTI) of every kernel of one
+    #    replay of the timed step, and of one serial call of each public stage
     refines = [l for l in range(N) if not mask[l]]
     idx_tmp = torch.empty((w.batch, w.n_kv_heads, w.kappa), dtype=torch.int32, device=dev)
     out_tmp = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
-    br = {
-        "anchor_index": timed(lambda i: prism.prism_index_anchor(
-            cfg, inp["q"][anchors[i % len(anchors)]], inp["k"][anchors[i % len(anchors)]],
-            inp["lens"], idx_out=idx_tmp, ws=ws, stream=stream)),
-        "refine_index": timed(lambda i: prism.prism_index_refine(
-            cfg, inp["q"][refines[i % len(refines)]], inp["k"][refines[i % len(refines)]],
-            inp["lens"], idx_e[refines[i % len(refines)] - 1].contiguous(), idx_out=idx_tmp,
-            ws=ws, stream=stream)),
-        "sparse_attn": timed(lambda i: prism.prism_sparse_decode(
-            cfg, inp["q"][i % N], inp["k"][i % N], inp["v"][i % N], inp["lens"],
-            idx_e[i % N].contiguous(), out=out_tmp, ws=ws, stream=stream)),
-        "anchor_score_kernel": t_score * 1e6,
-    }
-    br["anchor_layer"] = br["anchor_index"] + br["sparse_attn"]
-    br["refine_layer"] = br["refine_index"] + br["sparse_attn"]
+
+    def stages_once():
+        la, lr = anchors[0], refines[0]
+        prism.prism_index_anchor(cfg, inp["q"][la], inp["k"][la], inp["lens"], idx_out=idx_tmp,
+                                 ws=ws, stream=stream)
+        prism.prism_index_refine(cfg, inp["q"][lr], inp["k"][lr], inp["lens"],
+                                 idx_e[lr - 1].contiguous(), idx_out=idx_tmp, ws=ws,
+                                 stream=stream)
+        prism.prism_sparse_decode(cfg, inp["q"][lr], inp["k"][lr], inp["v"][lr], inp["lens"],
+                                  idx_e[lr].contiguous(), out=out_tmp, ws=ws, stream=stream)
+    br = {"how": "device time of each kernel (CUPTI activity records): 'step' over one replay "
+                 "of the timed graph (kernels overlap across streams, each counted in full), "
+                 "'stages' over one serial call each of prism_index_anchor, prism_index_refine "
+                 "and prism_sparse_decode; anchor_score_kernel_us from CUDA events around "
+                 "single launches",
+          "anchor_score_kernel_us": t_score * 1e6}
+    try:
+        stages_once()
+        br["stages"] = kernel_table(stages_once, dev)["kernels"]
+        if runner is not None:
+            br["step"] = kernel_table(runner.replay, dev)
+    except Exception as e:              # a diagnostic: never costs the line
+        br["error"] = f"{type(e).__name__}: {e}"
 
     # -- the same step as eager launches (no graph), inputs resident
     eager = None
@@ -825,6 +985,18 @@ def run_prism(args, rank, world, dev):
                                 "sample": f"layers 0-{g_layers[-1]} x all {w.n_kv_heads} KV "
                                           f"heads, one pass ({t_1:.1f} s)"}
 
+    # -- the pages' other workloads at one GPU (replicas per rank, like the headline)
+    per_config = None
+    if args.configs.strip():
+        per_config = {}
+        for wid in [int(x) for x in args.configs.split(",") if x.strip()]:
+            try:
+                per_config[f"c{wid}"] = measure_workload(args, prism, synth, wid, dev, peak,
+                                                         max(5, args.steps // 2), world)
+            except Exception as e:      # reported in the line; the headline stands
+                per_config[f"c{wid}"] = {"error": f"{type(e).__name__}: {e}"}
+        per_config["c3"] = {"headline": True, "value": value, "unit": UNIT}
+
     # -- context parallel (512K workload split over the job's ranks)
     cpar = None
     if not args.skip_cp:
@@ -847,18 +1019,6 @@ def run_prism(args, rank, world, dev):
                        "l2": "no flush: each step reads ~%.1f GB of distinct K/V, > 126 MB L2"
                              % (step_bytes / 1e9)},
             "layers_per_s": 1e6 / value,
-            "step_hbm": {"algorithmic_bytes": step_bytes, "gbs": step_gbs,
-                         "frac": step_gbs / peak, "peak": peak, "peak_kind": peak_kind,
-                         "proposal_sizes": {"mean_per_row": statistics.mean(prop_sizes)
-                                            / w.rows if prop_sizes else 0}},
-            "refine_diagnostics": {
-                "how": "per refined layer of the timed step: proposal |P| per (batch, KV head) "
-                       "row, and the recall of the layer's selection against its own exact "
-                       "top-kappa (an anchor selection of the same layer)",
-                "recall_mean": (statistics.mean(d["recall_mean"] for d in refine_diag
-                                                if "recall_mean" in d)
-                                if any("recall_mean" in d for d in refine_diag) else None),
-                "layers": refine_diag},
             "roofline": {"kernel": "k_anchor_score", "bound": "hbm", "achieved": ach,
                          "peak": peak, "unit": "GB/s", "frac": ach / peak, "traffic": traffic,
                          "bytes_per_launch": a_bytes, "us_per_launch": t_score * 1e6,
@@ -866,22 +1026,37 @@ def run_prism(args, rank, world, dev):
                          "share_of_step": n_anchor * t_score * 1e3 / ms,
                          "why": "largest HBM consumer of the step (anchor K: "
                                 f"{n_anchor * a_bytes / step_bytes:.0%} of its bytes)"},
-            "refine_attn": {"bytes_per_layer": refine_bytes, "us_per_layer": refine_us,
-                            "gbs": refine_bytes / (refine_us * 1e-6) / 1e9,
-                            "frac": refine_bytes / (refine_us * 1e-6) / 1e9 / peak,
-                            "how": "one anchor then 31 refined layers, graph-timed, minus the "
-                                   "anchor layer alone, per refined layer; bytes = measured "
-                                   "proposal K rows + gathered K/V rows"},
-            "breakdown_us": br,
-            "pool_mode": pool,
-            "pool_mode_int2": pool_q2,
-            "context_parallel": cpar,
             "gpu_launches": launches_per_step * args.steps,
             "launches_per_step": launches_per_step,
             "clocks": clk,
             "eager": eager,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "breakdown_us": br,
+            "pool_mode": pool,
+            "pool_mode_int2": pool_q2,
+            "context_parallel": cpar,
+            "refine_diagnostics": {
+                "how": "per refined layer of the timed step: recall of the layer's selection "
+                       "against its own exact top-kappa (an anchor selection of the same "
+                       "layer), and the proposal |P| per (batch, KV head) row",
+                "recall_mean": (statistics.mean(d["recall_mean"] for d in refine_diag
+                                                if "recall_mean" in d)
+                                if any("recall_mean" in d for d in refine_diag) else None),
+                "recall_min": (min(d["recall_min"] for d in refine_diag if "recall_min" in d)
+                               if any("recall_min" in d for d in refine_diag) else None),
+                "errors": [d for d in refine_diag if "error" in d]},
+            "per_config": per_config,
+            "refine_attn": {"bytes_per_layer": refine_bytes, "us_per_layer": refine_us,
+                            "gbs": refine_bytes / (refine_us * 1e-6) / 1e9,
+                            "frac": refine_bytes / (refine_us * 1e-6) / 1e9 / peak,
+                            "how": "one anchor then 31 refined layers, graph-timed, minus the "
+                                   "anchor layer alone, per refined layer; bytes = measured "
+                                   "proposal K rows + gathered K/V rows"},
+            "step_hbm": {"algorithmic_bytes": step_bytes, "gbs": step_gbs,
+                         "frac": step_gbs / peak, "peak": peak, "peak_kind": peak_kind,
+                         "proposal_mean_per_row": (statistics.mean(prop_sizes) / w.rows
+                                                   if prop_sizes else 0)},
         }
         print(json.dumps(line), flush=True)
     if runner is not None:

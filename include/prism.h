@@ -18,7 +18,16 @@
  *    the current CUDA device; the caller owns every buffer.  The library
  *    allocates no device memory.  Between calls it keeps only per-device
  *    caches: the SM count, and (for prism_decode_step) four helper streams
- *    and a pool of events, created on first use and kept until exit.
+ *    and a pool of events, created on first use and kept until exit.  These
+ *    per-device caches are the library's only global state; the helper
+ *    streams carry the step's multi-stream schedule.
+ *  - A refined layer's selection may run inside its rescoring kernel, whose
+ *    blocks of one row then wait for one another at bounded barriers; this
+ *    is chosen only when the launch's blocks fit the device's SMs at once.
+ *    Kernels of the caller running concurrently on other streams delay such
+ *    a launch but do not change its result, unless they hold SMs for longer
+ *    than the wait limit (PRISM_WAIT_LIMIT_MS, default 4000), which is then
+ *    reported as PRISM_ERR_TIMEOUT in the status word.
  *  - Layouts (row-major, no padding between rows):
  *      q    bf16 [B][Hq][d]            one decode query per sequence
  *      k, v bf16 [B][Hkv][Lmax][d]     KV cache of one layer; position i of
