@@ -471,10 +471,13 @@ def measure_context_parallel(args, rank, world, dev):
         torch.cuda.empty_cache()
     me = cp.CudaShard(cfg, sh, inp["q"], ks, vs, inp["lens"])
     gather = cp.local_gather if R == 1 else cp.dist_gather()
+    # the attention half trails on its own stream, with its own exchange group
+    attn_gather = cp.local_gather if R == 1 else cp.dist_gather(torch.distributed.new_group())
+    side = torch.cuda.Stream(device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        return cp.decode_step_cp(cfg, [me], gather)
+        return cp.decode_step_cp(cfg, [me], gather, attn_stream=side, attn_gather=attn_gather)
 
     n0 = prism.lib().prism_launch_count()
     outs, sel = step()
@@ -501,7 +504,8 @@ def measure_context_parallel(args, rank, world, dev):
             "selection": w.rows * w.kappa * 8,
             "attention_partials": w.batch * w.n_q_heads * (w.head_dim + 2) * 4},
         "how": "per layer: shard-local selection (+ scores), all_gather, exact merge; "
-               "shard-local split-softmax partials, all_gather, combine",
+               "shard-local split-softmax partials, all_gather, combine (the attention half "
+               "on a second stream behind the merge)",
     }
     if R == 1:
         g = torch.cuda.CUDAGraph()

@@ -72,6 +72,7 @@ class CudaShard:
         self.cfg, self.shard = cfg, shard
         self.q, self.k, self.v, self.lens = q, list(k_layers), list(v_layers), lens
         self.ws = cp_workspace(cfg, shard, q.device) if ws is None else ws
+        self.ws_side = None      # the attention half's workspace when it trails on its own stream
 
     def index_local(self, layer: int, src=None):
         return prism_cp_index_local(self.cfg, self.shard, self.q[layer], self.k[layer],
@@ -80,9 +81,12 @@ class CudaShard:
     def merge(self, pos_all, score_all):
         return prism_cp_merge(self.cfg, self.shard, pos_all, score_all, self.lens, ws=self.ws)
 
-    def attn_local(self, layer: int, idx):
+    def attn_local(self, layer: int, idx, side: bool = False):
+        if side and self.ws_side is None:
+            self.ws_side = cp_workspace(self.cfg, self.shard, self.q.device)
         return prism_cp_attn_local(self.cfg, self.shard, self.q[layer], self.k[layer],
-                                   self.v[layer], self.lens, idx, ws=self.ws)
+                                   self.v[layer], self.lens, idx,
+                                   ws=self.ws_side if side else self.ws)
 
     def combine(self, part_all):
         return prism_cp_combine(self.cfg, part_all)
@@ -113,12 +117,18 @@ def dist_gather(group=None) -> Gather:
     return gather
 
 
-def decode_step_cp(cfg: Config, ranks: Sequence, gather: Gather):
+def decode_step_cp(cfg: Config, ranks: Sequence, gather: Gather, attn_stream=None,
+                   attn_gather: Gather = None):
     """Algorithm 1 over all layers, context parallel.
 
     ranks: the rank handles this process runs (one per process under
     torch.distributed; all of them when emulating), each with index_local,
-    merge, attn_local and combine.  Returns (out [N] of [B][Hq][d], idx [N]
+    merge, attn_local and combine.  attn_stream (optional, a CUDA stream):
+    every layer's attention half runs there, each rank on a second workspace,
+    behind the layer's merge, so the next layer's selection does not wait
+    for it; attn_gather is then its exchange, which under torch.distributed
+    must be a second process group (the two streams' collectives must not
+    interleave on one communicator).  Returns (out [N] of [B][Hq][d], idx [N]
     of [B][Hkv][kappa]) as every rank sees them."""
     kinds = layer_kinds(cfg)
     pool_mode = cfg.mode == MODE_POOL
@@ -142,8 +152,22 @@ def decode_step_cp(cfg: Config, ranks: Sequence, gather: Gather):
             src = pool if pool_mode else sel[src_layer]
             parts = [r.index_local(l, src) for r in ranks]
             sel[l] = lead.merge(gather([p[0] for p in parts]), gather([p[1] for p in parts]))
-        partials = [r.attn_local(l, sel[l]) for r in ranks]
-        outs[l] = lead.combine(gather(partials))
+        if attn_stream is None:
+            partials = [r.attn_local(l, sel[l]) for r in ranks]
+            outs[l] = lead.combine(gather(partials))
+        else:
+            # the attention half trails on its own stream (own workspace, own
+            # exchange group), so the next layer's selection need not wait for it
+            main = torch.cuda.current_stream()
+            attn_stream.wait_stream(main)
+            sel[l].record_stream(attn_stream)
+            with torch.cuda.stream(attn_stream):
+                partials = [r.attn_local(l, sel[l], side=True) for r in ranks]
+                outs[l] = lead.combine((attn_gather or gather)(partials))
         if kind == 1:
             last_anchor = l
+    if attn_stream is not None:
+        torch.cuda.current_stream().wait_stream(attn_stream)
+        for o in outs:
+            o.record_stream(torch.cuda.current_stream())
     return outs, sel

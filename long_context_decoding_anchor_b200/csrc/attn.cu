@@ -33,39 +33,52 @@ struct AttnCfg {
 
 // Merge the split-K partials of one (batch, KV head) row:
 //   O_j = sum_s exp(m_s - M) acc_s / sum_s exp(m_s - M) l_s,  M = max_s m_s.
-// `wbuf` holds at least G * kAttnChunk floats (the split weights are cached
-// there when the row has at most kAttnChunk splits).
+// Every split's (m, l) is read once, by all threads together, into `mlbuf`
+// (at least kAttnChunk * G float2: the row's K tile, free by now) when the
+// row has at most kAttnChunk splits; `wbuf` (at least G * kAttnChunk floats)
+// then caches the split weights.  Longer rows read (m, l) from L2 as they go.
 template <int D, int G>
-__device__ void combine_row(const AttnArgs &a, int row, int b, int h, int nsplit, float *wbuf) {
-    __shared__ float Mh[G], inv_den[G];
+__device__ void combine_row(const AttnArgs &a, int row, int b, int h, int nsplit, float *wbuf,
+                            float2 *mlbuf) {
+    __shared__ float Mh[G], inv_den[G], den_h[G];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const float *pm = a.part_ml + (size_t)row * nsplit * G * 2;
     const bool cache = nsplit <= kAttnChunk;
+    constexpr int kC4 = G * D / 4;
+    constexpr int kBatch = 16;
+    const float4 *pa4 = reinterpret_cast<const float4 *>(a.part_acc + (size_t)row * nsplit * G * D);
+    if (cache) {
+        const float2 *pm2 = reinterpret_cast<const float2 *>(pm);
+        for (int i = tid; i < nsplit * G; i += blockDim.x) mlbuf[i] = __ldcg(pm2 + i);
+        __syncthreads();
+    }
+    auto ml_at = [&](int s, int g) -> float2 {
+        return cache ? mlbuf[s * G + g]
+                     : make_float2(__ldcg(pm + ((size_t)s * G + g) * 2), __ldcg(pm + ((size_t)s * G + g) * 2 + 1));
+    };
     for (int g = warp; g < G; g += 4) {
         float M = -INFINITY;
-        for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, __ldcg(pm + ((size_t)s * G + g) * 2));
+        for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, ml_at(s, g).x);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float den = 0.f;
         for (int s = lane; s < nsplit; s += 32) {
-            const float m = __ldcg(pm + ((size_t)s * G + g) * 2);
-            const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : __expf(m - M);
+            const float2 ml = ml_at(s, g);
+            const float w = (M == -INFINITY || ml.x == -INFINITY) ? 0.f : __expf(ml.x - M);
             if (cache) wbuf[g * kAttnChunk + s] = w;
-            den = fmaf(w, __ldcg(pm + ((size_t)s * G + g) * 2 + 1), den);
+            den = fmaf(w, ml.y, den);
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
         if (lane == 0) {
             Mh[g] = M;
+            den_h[g] = den;
             inv_den[g] = den > 0.f ? 1.f / den : 0.f;
         }
     }
     __syncthreads();
     // Each thread owns float4 columns of the [G][D] accumulator; the partials
     // of 16 splits are loaded at a time so their L2 round trips overlap.
-    constexpr int kC4 = G * D / 4;
-    constexpr int kBatch = 16;
-    const float4 *pa4 = reinterpret_cast<const float4 *>(a.part_acc + (size_t)row * nsplit * G * D);
     uint16_t *out = static_cast<uint16_t *>(a.out) + ((size_t)b * a.Hkv * G + (size_t)h * G) * D;
     for (int c4 = threadIdx.x; c4 < kC4; c4 += blockDim.x) {
         const int g = (c4 * 4) / D;
@@ -95,6 +108,20 @@ __device__ void combine_row(const AttnArgs &a, int row, int b, int h, int nsplit
                     acc.w = fmaf(w, v[u].w, acc.w);
                 }
             }
+        }
+        if (a.cp_part) {
+            // this rank's partial of the row: the accumulator unnormalised, M, l
+            float *cp = a.cp_part + ((size_t)row * G + g) * (D + 2);
+            const int c = (c4 * 4) % D;
+            cp[c] = acc.x;
+            cp[c + 1] = acc.y;
+            cp[c + 2] = acc.z;
+            cp[c + 3] = acc.w;
+            if (c == 0) {
+                cp[D] = Mg;
+                cp[D + 1] = den_h[g];
+            }
+            continue;
         }
         const float sc = inv_den[g];
         const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * sc, acc.y * sc);
@@ -269,7 +296,7 @@ k_sparse_attn(AttnArgs a) {
     __syncthreads();
     if (!is_last) return;
     __threadfence();
-    combine_row<D, G>(a, row, b, h, gridDim.x, &z[0][0]);
+    combine_row<D, G>(a, row, b, h, gridDim.x, &z[0][0], reinterpret_cast<float2 *>(Ks));
     if (tid == 0) a.ctl[row].done_attn = 0;
 }
 

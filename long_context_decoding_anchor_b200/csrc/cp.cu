@@ -3,16 +3,16 @@
 // One rank holds the positions [lo, lo + cap) of every sequence.  It runs the
 // single-GPU kernels (scoring, rescoring, selection, attention) on its shard
 // in local positions; these kernels adapt their inputs and outputs:
-//  - k_cp_prepare: the shard lengths, and the refined layer's proposal
-//    ("Prism Attention", Eq. (5): every position within r of a source token,
-//    clipped to [0, len)) restricted to the shard, as a radius-0 source; or a
-//    global selection in local positions for the attention.
+//  - k_cp_prepare: the shard lengths, and a global selection in local
+//    positions for the attention.  (A refined layer's rescoring cuts the
+//    proposal of the global source to the shard itself.)
 //  - k_cp_pack: a local selection as (global position, score) pairs (the
 //    rescoring of a refined layer leaves its candidates' scores by position).
 //  - k_cp_merge_compact / k_cp_merge_hist: the gathered pairs of all ranks as
 //    one candidate list per row, for the exact selection (the top-k of a
 //    union is the top-k of the union of the parts' top-k).
-//  - k_cp_reduce / k_cp_combine: split softmax across ranks,
+//  - k_cp_combine: split softmax across ranks (each rank's attention kernel
+//    leaves its merged partial (acc, m, l)),
 //    o = sum_r e^(m_r - M) acc_r / sum_r e^(m_r - M) l_r.
 #include <cuda_bf16.h>
 
@@ -23,12 +23,10 @@ namespace prism {
 constexpr int kCpThreads = 256;
 constexpr int kCpSplit = 8;          // CTAs per row of k_cp_prepare
 
-// Grid (rows, kCpSplit).  For a proposal, every CTA of a row counts the
-// positions of all entries (one run of entries per thread, a block scan) and
-// writes the positions of its own share of the output slots.
+// Grid (rows, kCpSplit): the shard lengths, and the selection's entries
+// strided over the row's CTAs.
 __global__ void __launch_bounds__(kCpThreads)
 k_cp_prepare(CpPrepArgs a) {
-    __shared__ int scratch[40];
     const int row = blockIdx.x, part = blockIdx.y;
     const int b = row / a.Hkv, h = row % a.Hkv;
     const int tid = threadIdx.x;
@@ -39,72 +37,32 @@ k_cp_prepare(CpPrepArgs a) {
     if (a.what == kCpPrepLen) return;
     const int32_t *src = a.src + (size_t)row * a.src_kappa;
     int32_t *out = a.out + (size_t)row * a.out_kappa;
-    if (a.what == kCpPrepSelection) {
-        for (int t = part * kCpThreads + tid; t < a.src_kappa; t += kCpSplit * kCpThreads) {
-            const int p = __ldg(src + t);
-            out[t] = (p >= a.lo && p < a.lo + n_loc) ? p - a.lo : -1;
-        }
-        return;
+    for (int t = part * kCpThreads + tid; t < a.src_kappa; t += kCpSplit * kCpThreads) {
+        const int p = __ldg(src + t);
+        out[t] = (p >= a.lo && p < a.lo + n_loc) ? p - a.lo : -1;
     }
-    // The proposal inside the shard: entry j owns the positions of its window
-    // that no earlier entry's window covers (owned_range), here cut to the
-    // shard [lo, lo + n_loc).
-    const int per = (a.src_kappa + kCpThreads - 1) / kCpThreads;
-    const int j0 = min(a.src_kappa, tid * per), j1 = min(a.src_kappa, j0 + per);
-    const long long shard_hi = (long long)a.lo + n_loc - 1;
-    int cnt = 0;
-    for (int j = j0; j < j1; ++j) {
-        int lo_j = 0;
-        const int own = owned_range(src, j, a.radius, L, &lo_j, part == 0 ? a.st : nullptr,
-                                    kWhereCanon);
-        const long long s = max((long long)lo_j, (long long)a.lo);
-        const long long e = min((long long)lo_j + own - 1, shard_hi);
-        if (own > 0 && e >= s) cnt += (int)(e - s + 1);
-    }
-    int total;
-    int at = block_exclusive_scan(cnt, scratch, &total);
-    const int cap_total = min(total, a.out_kappa);
-    const int o_begin = (int)((long long)part * cap_total / kCpSplit);
-    const int o_end = (int)((long long)(part + 1) * cap_total / kCpSplit);
-    for (int j = j0; j < j1 && at < o_end; ++j) {
-        int lo_j = 0;
-        const int own = owned_range(src, j, a.radius, L, &lo_j, nullptr, kWhereCanon);
-        const long long s = max((long long)lo_j, (long long)a.lo);
-        const long long e = min((long long)lo_j + own - 1, shard_hi);
-        if (own <= 0 || e < s) continue;
-        const int len = (int)(e - s + 1);
-        // this entry's slots [at, at + len) within this CTA's [o_begin, o_end)
-        const int t0 = max(at, o_begin), t1 = min(at + len, o_end);
-        for (int t = t0; t < t1; ++t) out[t] = (int)(s - a.lo) + (t - at);
-        at += len;
-    }
-    // the rest of the source is padding
-    for (int t = cap_total + part * kCpThreads + tid; t < a.out_kappa; t += kCpSplit * kCpThreads)
-        out[t] = -1;
-    if (part == 0 && tid == 0 && total > a.out_kappa)
-        report(a.st, kDevErrInternal, kWhereCanon, (uint32_t)total);
 }
 
 cudaError_t launch_cp_prepare(const CpPrepArgs &a, cudaStream_t s) {
     return launch_kernel(k_cp_prepare, dim3(a.B * a.Hkv, kCpSplit), dim3(kCpThreads), 0, s, a);
 }
 
+// Grid (ceil(n / kCpThreads), rows): one entry a thread.
 __global__ void __launch_bounds__(kCpThreads)
 k_cp_pack(CpPackArgs a) {
-    const int row = blockIdx.x;
+    const int row = blockIdx.y;
+    const int t = blockIdx.x * kCpThreads + threadIdx.x;
     pdl_wait();
-    const int32_t *sel = a.sel + (size_t)row * a.n;
-    const float *S = a.S + (size_t)row * a.sstride;
-    for (int t = threadIdx.x; t < a.n; t += kCpThreads) {
-        const int i = __ldcg(sel + t);
-        const bool ok = i >= 0 && i < a.sstride;
-        a.pos_out[(size_t)row * a.n + t] = ok ? a.lo + i : -1;
-        a.score_out[(size_t)row * a.n + t] = ok ? __ldcg(S + i) : -INFINITY;
-    }
+    if (t >= a.n) return;
+    const int i = __ldcg(a.sel + (size_t)row * a.n + t);
+    const bool ok = i >= 0 && i < a.sstride;
+    a.pos_out[(size_t)row * a.n + t] = ok ? a.lo + i : -1;
+    a.score_out[(size_t)row * a.n + t] = ok ? __ldcg(a.S + (size_t)row * a.sstride + i) : -INFINITY;
 }
 
 cudaError_t launch_cp_pack(const CpPackArgs &a, cudaStream_t s) {
-    return launch_kernel(k_cp_pack, dim3(a.rows), dim3(kCpThreads), 0, s, a);
+    return launch_kernel(k_cp_pack, dim3((a.n + kCpThreads - 1) / kCpThreads, a.rows), dim3(kCpThreads),
+                         0, s, a);
 }
 
 // The rows of the R lists are consecutive shards, so keeping the valid
@@ -169,64 +127,6 @@ cudaError_t launch_cp_merge_prepare(const CpMergeArgs &a, cudaStream_t s) {
     cudaError_t e = launch_kernel(k_cp_merge_compact, dim3(a.rows), dim3(kMergeThreads), 0, s, a);
     if (e != cudaSuccess) return e;
     return launch_kernel(k_cp_merge_hist, dim3(a.rows), dim3(512), 0, s, a);
-}
-
-// One CTA per (row, query head); thread c owns column c of the accumulator.
-__global__ void __launch_bounds__(128)
-k_cp_reduce(CpReduceArgs a) {
-    __shared__ float wts[kAttnChunk * 4];
-    __shared__ float stat[2];
-    const int row = blockIdx.x, g = blockIdx.y;
-    const int tid = threadIdx.x;
-    pdl_wait();
-    const float *pm = a.part_ml + (size_t)row * a.nsplit * a.G * 2;
-    if (tid < 32) {
-        float M = -INFINITY;
-        for (int s = tid; s < a.nsplit; s += 32) M = fmaxf(M, __ldcg(pm + ((size_t)s * a.G + g) * 2));
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float den = 0.f;
-        for (int s = tid; s < a.nsplit; s += 32) {
-            const float m = __ldcg(pm + ((size_t)s * a.G + g) * 2);
-            const float w = (M == -INFINITY || m == -INFINITY) ? 0.f : __expf(m - M);
-            den = fmaf(w, __ldcg(pm + ((size_t)s * a.G + g) * 2 + 1), den);
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-        if (tid == 0) {
-            stat[0] = M;
-            stat[1] = den;
-        }
-    }
-    __syncthreads();
-    const float M = stat[0];
-    float *out = a.out + ((size_t)row * a.G + g) * (a.d + 2);
-    for (int s0 = 0; s0 < a.nsplit; s0 += kAttnChunk * 4) {
-        const int cnt = min(kAttnChunk * 4, a.nsplit - s0);
-        __syncthreads();
-        for (int s = tid; s < cnt; s += 128) {
-            const float m = __ldcg(pm + ((size_t)(s0 + s) * a.G + g) * 2);
-            wts[s] = (M == -INFINITY || m == -INFINITY) ? 0.f : __expf(m - M);
-        }
-        __syncthreads();
-        if (tid < a.d) {
-            float acc = s0 == 0 ? 0.f : out[tid];
-            for (int s = 0; s < cnt; ++s) {
-                const float w = wts[s];
-                if (w != 0.f)
-                    acc = fmaf(w, __ldcg(a.part_acc + (((size_t)row * a.nsplit + s0 + s) * a.G + g) * a.d + tid), acc);
-            }
-            out[tid] = acc;
-        }
-    }
-    if (tid == 0) {
-        out[a.d] = M;
-        out[a.d + 1] = stat[1];
-    }
-}
-
-cudaError_t launch_cp_reduce(const CpReduceArgs &a, cudaStream_t s) {
-    return launch_kernel(k_cp_reduce, dim3(a.rows, a.G), dim3(128), 0, s, a);
 }
 
 // One CTA per query head; thread c owns column c.

@@ -8,7 +8,7 @@
 
 namespace prism {
 
-enum : int { kCpPrepLen = 0, kCpPrepProposal = 1, kCpPrepSelection = 2 };
+enum : int { kCpPrepLen = 0, kCpPrepSelection = 1 };
 
 struct CpPrepArgs {
     int what;                  // kCpPrep*
@@ -16,14 +16,10 @@ struct CpPrepArgs {
     int B, Hkv, Lmax;          // Lmax: global capacity
     int lo, cap;               // the shard
     int32_t *llen;             // [B] shard lengths, clamp(len - lo, 0, cap)
-    // kCpPrepProposal: src is the canonical global source selection and
-    // radius its proposal radius; out receives the proposal inside the shard
-    // in local positions, ascending, -1 padded (a radius-0 source of
-    // out_kappa entries).
     // kCpPrepSelection: src is a global selection of src_kappa entries; out
     // receives it in local positions, -1 where outside the shard.
     const int32_t *src;
-    int src_kappa, radius;
+    int src_kappa;
     int32_t *out;
     int out_kappa;
     DevStatus *st;
@@ -60,14 +56,6 @@ struct CpMergeArgs {
 cudaError_t launch_cp_merge_prepare(const CpMergeArgs &a, cudaStream_t s);
 
 // Split-K partials of the attention kernel -> one (acc[d], m, l) per query head.
-struct CpReduceArgs {
-    const float *part_acc;     // [rows][nsplit][G][d]
-    const float *part_ml;      // [rows][nsplit][G][2]
-    int rows, nsplit, G, d;
-    float *out;                // [rows * G][d + 2]
-};
-cudaError_t launch_cp_reduce(const CpReduceArgs &a, cudaStream_t s);
-
 struct CpCombineArgs {
     const float *part;         // [R][heads][d + 2]
     int R, heads, d;

@@ -365,10 +365,18 @@ prism_status_t run_pool_select(const prism_config_t &c, const Ws &w, int slot, c
 // candidate's score by position (row stride spos_stride).  `alone` says that
 // no other kernel of the call can run beside this one (no anchor scan in
 // flight): only then may a co-resident launch select in place.
+// A context-parallel rank's refined layer: the source is global, len is the
+// shard's, and the proposal is cut to [lo, lo + len) (see ScoreArgs::glen).
+struct CutToShard {
+    const int32_t *glen;
+    int glmax, lo;
+};
+
 prism_status_t run_refine_batch(const prism_config_t &c, const Ws &w, const void *const *qs,
                                 const void *const *ks, int32_t *const *outs, int nz,
                                 const int32_t *len, const int32_t *src, int E, int radius,
-                                float *Spos, int spos_stride, cudaStream_t s, bool alone = true) {
+                                float *Spos, int spos_stride, cudaStream_t s, bool alone = true,
+                                const CutToShard *cut = nullptr) {
     if (nz < 1 || nz > w.l.rl.nzmax || E != w.l.rl.E || radius != w.l.rl.radius)
         return PRISM_ERR_INVALID_ARG;
     const size_t rows = (size_t)c.batch * c.n_kv_heads;
@@ -380,6 +388,9 @@ prism_status_t run_refine_batch(const prism_config_t &c, const Ws &w, const void
     sa.hist = w.rhist; sa.runs = w.runs; sa.run_cnt = w.run_cnt;
     sa.parts = rp.parts; sa.run_k = rp.run_k;
     sa.Spos = nz == 1 ? Spos : nullptr; sa.spos_stride = spos_stride;
+    if (cut) {
+        sa.glen = cut->glen; sa.glmax = cut->glmax; sa.shard_lo = cut->lo;
+    }
     sa.nz = nz;
     sa.zruns = rows * (size_t)nruns * kRunCap; sa.zcnt = rows * (size_t)nruns;
     sa.zhist = rows * kHistBins;
@@ -435,13 +446,14 @@ prism_status_t run_refine(const prism_config_t &c, const Ws &w, const void *q, c
 
 prism_status_t run_attn(const prism_config_t &c, const Ws &w, const void *q, const void *k,
                         const void *v, const int32_t *len, const int32_t *idx, int idx_stride,
-                        int n_idx, void *out, cudaStream_t s) {
+                        int n_idx, void *out, cudaStream_t s, float *cp_part = nullptr) {
     AttnArgs aa{};
     aa.q = q; aa.k = k; aa.v = v; aa.len = len; aa.idx = idx;
     aa.idx_stride = idx_stride; aa.n_idx = n_idx;
     aa.B = c.batch; aa.Hkv = c.n_kv_heads; aa.G = c.n_q_heads / c.n_kv_heads;
     aa.d = c.head_dim; aa.Lmax = c.max_len; aa.scale = eff_scale(c);
     aa.part_acc = w.pacc; aa.part_ml = w.pml; aa.ctl = w.attn_ctl; aa.out = out; aa.st = w.st;
+    aa.cp_part = cp_part;
     return cuda_status(launch_sparse_attn(aa, s));
 }
 
@@ -926,36 +938,26 @@ prism_config_t local_config(const prism_config_t &c, const prism_cp_shard_t &sh)
     return lc;
 }
 
-// Entries of the radius-0 source that a refined layer's proposal becomes
-// inside one shard: at most |source| * (2r + 1) positions, at most shard_len.
-int cp_local_src(const prism_config_t &c, const prism_cp_shard_t &sh) {
-    const long long n = (long long)src_kappa_of(c) * (2LL * refine_radius_of(c) + 1);
-    return (int)(n < sh.shard_len ? n : sh.shard_len);
-}
-
 struct CpLayout {
     Layout l;
-    int lsrc_k, kmax, R, cs_m;
-    size_t llen, lsrc, lsel, lpool, latt, lout;
+    int kmax, R, cs_m;
+    size_t llen, lsel, lpool, latt;
     size_t mS, mcpos, mcount, mhist, mspill, total;
 };
 
 CpLayout make_cp_layout(const prism_config_t &c, const prism_cp_shard_t &sh) {
     CpLayout L{};
     const size_t rows = (size_t)c.batch * c.n_kv_heads;
-    L.lsrc_k = cp_local_src(c, sh);
-    // a refined layer rescores the shard's cut of its proposal, a radius-0 source
-    L.l = make_layout(local_config(c, sh), L.lsrc_k, 0);
+    // a refined layer rescores its proposal cut to the shard, from the global source
+    L.l = make_layout(local_config(c, sh));
     L.kmax = src_kappa_of(c);
     L.R = sh.n_ranks;
     L.cs_m = (int)(((long long)L.R * L.kmax + 3) & ~3LL);
     size_t off = L.l.total;
     L.llen = off;     off = align256(off + (size_t)c.batch * sizeof(int32_t));
-    L.lsrc = off;     off = align256(off + rows * (size_t)L.lsrc_k * sizeof(int32_t));
     L.lsel = off;     off = align256(off + rows * (size_t)c.kappa * sizeof(int32_t));
     L.lpool = off;    off = align256(off + rows * (size_t)L.kmax * sizeof(int32_t));
     L.latt = off;     off = align256(off + rows * (size_t)c.kappa * sizeof(int32_t));
-    L.lout = off;     off = align256(off + (size_t)c.batch * c.n_q_heads * c.head_dim * 2);
     L.mS = off;       off = align256(off + rows * (size_t)L.cs_m * sizeof(float));
     L.mcpos = off;    off = align256(off + rows * (size_t)L.cs_m * sizeof(int32_t));
     L.mcount = off;   off = align256(off + rows * ((size_t)L.R * L.kmax + 1) * sizeof(int32_t));
@@ -983,8 +985,7 @@ prism_status_t check_cp(const prism_config_t *c, const prism_cp_shard_t *sh) {
 struct CpWs {
     Ws w;
     CpLayout L;
-    int32_t *llen, *lsrc, *lsel, *lpool, *latt;
-    void *lout;
+    int32_t *llen, *lsel, *lpool, *latt;
     float *mS;
     int32_t *mcpos, *mcount;
     uint32_t *mhist;
@@ -996,14 +997,12 @@ prism_status_t carve_cp(const prism_config_t &c, const prism_cp_shard_t &sh, voi
     if (!ws || !aligned(ws, 256)) return PRISM_ERR_INVALID_ARG;
     x->L = make_cp_layout(c, sh);
     if (ws_bytes < x->L.total) return PRISM_ERR_WORKSPACE;
-    PRISM_TRY(carve(local_config(c, sh), ws, ws_bytes, &x->w, x->L.lsrc_k, 0));
+    PRISM_TRY(carve(local_config(c, sh), ws, ws_bytes, &x->w));
     uint8_t *b = static_cast<uint8_t *>(ws);
     x->llen = reinterpret_cast<int32_t *>(b + x->L.llen);
-    x->lsrc = reinterpret_cast<int32_t *>(b + x->L.lsrc);
     x->lsel = reinterpret_cast<int32_t *>(b + x->L.lsel);
     x->lpool = reinterpret_cast<int32_t *>(b + x->L.lpool);
     x->latt = reinterpret_cast<int32_t *>(b + x->L.latt);
-    x->lout = b + x->L.lout;
     x->mS = reinterpret_cast<float *>(b + x->L.mS);
     x->mcpos = reinterpret_cast<int32_t *>(b + x->L.mcpos);
     x->mcount = reinterpret_cast<int32_t *>(b + x->L.mcount);
@@ -1065,11 +1064,6 @@ prism_status_t prism_cp_index_local(const prism_config_t *cfg, const prism_cp_sh
     const prism_config_t lc = local_config(*cfg, *shard);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     CpPrepArgs pa = cp_prep_args(*cfg, *shard, x, len);
-    if (src) {
-        pa.what = kCpPrepProposal;
-        pa.src = src; pa.src_kappa = src_kappa_of(*cfg); pa.radius = refine_radius_of(*cfg);
-        pa.out = x.lsrc; pa.out_kappa = x.L.lsrc_k;
-    }
     PRISM_CUDA(launch_cp_prepare(pa, s));
     // A plain stream operation between the kernel above and the ones below:
     // those may read the shard lengths before their grid-dependency wait.
@@ -1087,13 +1081,15 @@ prism_status_t prism_cp_index_local(const prism_config_t *cfg, const prism_cp_sh
                               pool_score, s));
         return PRISM_OK;
     }
-    // Eq. (5)-(6) over the shard's cut of the proposal (a radius-0 source);
+    // Eq. (5)-(6) over the proposal of the global source cut to the shard;
     // the candidates' scores are left by local position in slot 0 for the pack.
     const void *qs[1] = {q};
     const void *ks[1] = {k};
     int32_t *outs[1] = {x.lsel};
-    PRISM_TRY(run_refine_batch(lc, x.w, qs, ks, outs, 1, x.llen, x.lsrc, x.L.lsrc_k, 0,
-                               x.w.slot[0].S, shard->shard_len, s));
+    const CutToShard cut{len, cfg->max_len, shard->rank * shard->shard_len};
+    PRISM_TRY(run_refine_batch(lc, x.w, qs, ks, outs, 1, x.llen, src, src_kappa_of(*cfg),
+                               refine_radius_of(*cfg), x.w.slot[0].S, shard->shard_len, s, true,
+                               &cut));
     return cp_pack(*cfg, *shard, x.lsel, cfg->kappa, x.w.slot[0].S, cand_pos, cand_score, s);
 }
 
@@ -1112,6 +1108,13 @@ prism_status_t prism_cp_merge(const prism_config_t *cfg, const prism_cp_shard_t 
     PRISM_TRY(carve_cp(*cfg, *shard, ws, ws_bytes, &x));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int R = shard->n_ranks;
+    if (R == 1) {
+        // One shard: its list (ascending, -1 padded, n_out entries a row) is
+        // the selection.
+        return cuda_status(cudaMemcpyAsync(idx_out, cand_pos,
+                                           (size_t)cfg->batch * cfg->n_kv_heads * n_out * sizeof(int32_t),
+                                           cudaMemcpyDeviceToDevice, s));
+    }
     CpMergeArgs ma{};
     ma.pos = cand_pos; ma.score = cand_score;
     ma.R = R; ma.rows = cfg->batch * cfg->n_kv_heads; ma.n = n_out;
@@ -1148,14 +1151,8 @@ prism_status_t prism_cp_attn_local(const prism_config_t *cfg, const prism_cp_sha
     // plain stream operation (see prism_cp_index_local), and the attention's row counters
     PRISM_CUDA(cudaMemsetAsync(x.w.attn_ctl, 0,
                                (size_t)cfg->batch * cfg->n_kv_heads * sizeof(RowCtl), s));
-    PRISM_TRY(run_attn(lc, x.w, q, k, v, x.llen, x.latt, cfg->kappa, cfg->kappa, x.lout, s));
-    CpReduceArgs ra{};
-    ra.part_acc = x.w.pacc; ra.part_ml = x.w.pml;
-    ra.rows = cfg->batch * cfg->n_kv_heads;
-    ra.nsplit = (cfg->kappa + kAttnChunk - 1) / kAttnChunk;
-    ra.G = cfg->n_q_heads / cfg->n_kv_heads; ra.d = cfg->head_dim;
-    ra.out = part_out;
-    return cuda_status(launch_cp_reduce(ra, s));
+    // the attention's row merge leaves this rank's partial (acc, m, l)
+    return run_attn(lc, x.w, q, k, v, x.llen, x.latt, cfg->kappa, cfg->kappa, nullptr, s, part_out);
 }
 
 prism_status_t prism_cp_combine(const prism_config_t *cfg, int32_t n_ranks,

@@ -507,6 +507,12 @@ struct ScoreArgs {
     int parts, run_k;       // parts per row, runs per part (nruns = parts * run_k)
     float *Spos;            // refine, nullable: every candidate's score by position
     int spos_stride;        //   (row stride)
+    // refine on one shard of a context-parallel rank (glen nullable): the
+    // source holds global positions, len is the shard's, and the proposal is
+    // cut to the shard [shard_lo, shard_lo + len) in local positions; glen
+    // (capacity glmax) are the global lengths the windows are clipped to
+    const int32_t *glen;
+    int glmax, shard_lo;
     // refine, fused selection (Eq. (6) in the same launch; nz == 1, one run a
     // part, every block of the grid resident at once): the blocks of a row
     // meet at two barriers on row_bar[row] (arrivals counted from bar_base),
@@ -647,6 +653,10 @@ struct AttnArgs {
     float *part_ml;            // [rows][nsplit][G][2]
     RowCtl *ctl;
     void *out;                 // bf16 [B][Hq][d]
+    // nullable: instead of out, the row's merged split softmax unnormalised,
+    // [B*Hq][d + 2] fp32 = (sum_s e^(m_s - M) acc_s, M, sum_s e^(m_s - M) l_s),
+    // the partial of one context-parallel rank
+    float *cp_part;
     DevStatus *st;
 };
 constexpr int kAttnChunk = 64;

@@ -458,14 +458,18 @@ __device__ void fused_select(const ScoreArgs &a, int row, int part, int P, int n
 
     // 3. every part's counts and the head of its ties, fetched together (the
     //    run areas and the counts are in L2); the ties are used in place,
-    //    part p's i-th at stage[p * kSpec + i]
-    constexpr int kSpec = 64;
-    uint64_t *stage_t = tcache;                          // [P][kSpec]
-    const bool spec_fits = (long long)P * kSpec <= tcap;
+    //    part p's i-th at stage[p * spec + i].  A head of 128 (64 when that
+    //    does not fit) holds a part's ties nearly always: a part of ~1000
+    //    candidates has ~50 of the threshold's first digit, and a part over
+    //    the head costs a second round trip for the whole row.
+    const int spec_sh = (long long)P * 128 <= tcap ? 7 : 6;
+    const int spec = 1 << spec_sh;
+    uint64_t *stage_t = tcache;                          // [P][spec]
+    const bool spec_fits = (long long)P * spec <= tcap;
     if (spec_fits) {
-        for (int q = tid; q < P * (kSpec / 2); q += NTH) {
-            const int p = q / (kSpec / 2), e2 = 2 * (q - p * (kSpec / 2));
-            cp_async16(stage_t + p * kSpec + e2, runs_row + (size_t)p * run_stride + e2, 16u);
+        for (int q = tid; q < P * (spec / 2); q += NTH) {
+            const int p = q >> (spec_sh - 1), e2 = 2 * (q - p * (spec / 2));
+            cp_async16(stage_t + p * spec + e2, runs_row + (size_t)p * run_stride + e2, 16u);
         }
         cp_async_commit();
     }
@@ -482,15 +486,15 @@ __device__ void fused_select(const ScoreArgs &a, int row, int part, int P, int n
     int m;
     const int toff = block_excl_scan_fast<NW>(ct, wsum, &m);     // barrier: counts, ties in place
     if (tid < P) tie_off[tid] = toff;
-    const int big = __syncthreads_or(tid < P && ct > kSpec);
+    const int big = __syncthreads_or(tid < P && ct > spec);
     // The ties in one list: in place (every part's ties fit the fetched head)
     // or compacted in order into tcache / the spill (a part with more).
     const bool in_place = spec_fits && !big;
-    const int nslot = in_place ? P * kSpec : m;
+    const int nslot = in_place ? P * spec : m;
     auto tie_slot = [&](int f, uint64_t *it) -> bool {  // f-th slot of the list: a tie?
         if (in_place) {
-            const int p = f / kSpec;
-            if (f - p * kSpec >= cnt_tie[p]) return false;
+            const int p = f >> spec_sh;
+            if (f - (p << spec_sh) >= cnt_tie[p]) return false;
             *it = stage_t[f];
             return true;
         }
@@ -556,7 +560,7 @@ __device__ void fused_select(const ScoreArgs &a, int row, int part, int P, int n
                     __syncthreads();
                     for (int p = warp; p < P; p += NW) {
                         const int c = cnt_tie[p], o = tie_off[p];
-                        for (int i = lane; i < c; i += 32) spill[o + i] = stage_t[p * kSpec + i];
+                        for (int i = lane; i < c; i += 32) spill[o + i] = stage_t[p * spec + i];
                     }
                     __threadfence_block();
                     __syncthreads();
@@ -577,7 +581,7 @@ __device__ void fused_select(const ScoreArgs &a, int row, int part, int P, int n
                 uint64_t it;
                 if (!tie_slot(f, &it)) continue;
                 const uint32_t ku = (uint32_t)(it >> 32);
-                if (ku > T || (ku == T && (int)(uint32_t)it <= cutoff)) atomicAdd(&chosen[f / kSpec], 1);
+                if (ku > T || (ku == T && (int)(uint32_t)it <= cutoff)) atomicAdd(&chosen[f >> spec_sh], 1);
             }
         } else {
             for (int p = warp; p < P; p += NW) {
@@ -702,6 +706,10 @@ k_refine_rescore(ScoreArgs a) {
     // The source selection comes from the preceding kernels.
     pdl_wait();
     const int E = a.kappa;
+    // the windows' global bounds and the shard they are cut to (the whole row
+    // on one GPU)
+    const int Lg = a.glen ? load_len(a.glen, b, a.glmax, a.st, kWhereRescore) : L;
+    const long long slo = a.glen ? a.shard_lo : 0, shi = slo + L - 1;
     const int j0 = (int)((long long)part * E / P), j1 = (int)((long long)(part + 1) * E / P);
     const int ne = min(j1 - j0, kMaxPartEntries);
     const int32_t *src = a.src + (size_t)row * E + j0;
@@ -720,16 +728,18 @@ k_refine_rescore(ScoreArgs a) {
             cnt[e] = 0;
             lo_[e] = 0;
             if (i >= 0) {
-                if (i >= L || (prev >= 0 && i <= prev)) {
+                if (i >= Lg || (prev >= 0 && i <= prev)) {
                     report(a.st, kDevErrBadIndex, kWhereRescore, (uint32_t)i);
                 } else {
                     long long lo = (long long)i - a.radius;
                     if (prev >= 0 && (long long)prev + a.radius + 1 > lo) lo = (long long)prev + a.radius + 1;
                     if (lo < 0) lo = 0;
                     long long hi = (long long)i + a.radius;
-                    if (hi > L - 1) hi = L - 1;
+                    if (hi > Lg - 1) hi = Lg - 1;
+                    if (lo < slo) lo = slo;
+                    if (hi > shi) hi = shi;
                     if (hi >= lo) {
-                        lo_[e] = (int)lo;
+                        lo_[e] = (int)(lo - slo);
                         cnt[e] = (int)(hi - lo + 1);
                     }
                 }

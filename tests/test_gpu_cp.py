@@ -113,6 +113,32 @@ def test_cp_rank_counts(oracle, R):
     layerwise_step_check(oracle, cfg, inp, torch.stack(outs), torch.stack(sel))
 
 
+@pytest.mark.parametrize("mode", ["refine", "pool-frs"])
+@pytest.mark.parametrize("R", [1, 3])
+def test_cp_attention_on_its_own_stream_matches(mode, R):
+    """The attention half trailing on its own stream (second workspace per
+    rank) gives the same selections and outputs as the one-stream schedule,
+    eagerly and replayed from a CUDA graph."""
+    w, cfg, inp = _setup("d128-g4", mode)
+    ranks = _ranks(cfg, inp, R)
+    outs0, sel0 = cp.decode_step_cp(cfg, ranks, cp.local_gather)
+    side = torch.cuda.Stream()
+    outs1, sel1 = cp.decode_step_cp(cfg, ranks, cp.local_gather, attn_stream=side)
+    torch.cuda.synchronize()
+    _check_status(ranks)
+    for l in range(cfg.n_layers):
+        assert torch.equal(sel1[l], sel0[l]), f"layer {l}: selection differs"
+        assert torch.equal(outs1[l], outs0[l]), f"layer {l}: output differs"
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        outs2, sel2 = cp.decode_step_cp(cfg, ranks, cp.local_gather, attn_stream=side)
+    g.replay()
+    torch.cuda.synchronize()
+    for l in range(cfg.n_layers):
+        assert torch.equal(sel2[l], sel0[l]) and torch.equal(outs2[l], outs0[l]), f"graph, layer {l}"
+    del g
+
+
 def test_cp_local_scores_are_the_single_gpu_scores():
     """A shard's (position, score) pairs are the single-GPU anchor scores at
     those positions, bit for bit; the merge of all shards is the single-GPU
