@@ -364,7 +364,7 @@ prism_status_t run_pool_select(const prism_config_t &c, const Ws &w, int slot, c
 // selection goes to outs[z].  Spos (nullable, nz == 1) receives every
 // candidate's score by position (row stride spos_stride).  `alone` says that
 // no other kernel of the call can run beside this one (no anchor scan in
-// flight): only then may a co-resident launch select in place.
+// flight); it decides how a layer selects in place (below).
 // A context-parallel rank's refined layer: the source is global, len is the
 // shard's, and the proposal is cut to [lo, lo + len) (see ScoreArgs::glen).
 struct CutToShard {
@@ -401,13 +401,19 @@ prism_status_t run_refine_batch(const prism_config_t &c, const Ws &w, const void
     // One layer whose parts all fit the GPU at once (one block per SM), one
     // run each: the rescoring blocks of a row select together (no second
     // kernel); otherwise the selection kernel reads the runs.  The blocks of a
-    // row wait for one another, so the launch must have the GPU to itself: a
-    // concurrent anchor scan (a block on every SM) leaves no room for some of
-    // them until it ends, and the whole row waits (measured: ~50 against ~22
-    // us a layer).
-    if (alone && nz == 1 && rp.run_k == 1 && rp.parts <= 256 && rp.parts == w.l.rl.parts1 &&
+    // row wait for one another, so each of them must find room on an SM.
+    // Beside an anchor scan (a block on every SM) the full-size rescoring
+    // block leaves no room for an attention block, and a row whose block
+    // waits behind attention blocks stalls (measured: ~50 against ~22 us a
+    // layer); the two-stage block (group sum) leaves room for one.  So the
+    // group sum uses it while an anchor scan may be in flight (`alone`
+    // false), the full-size block otherwise; the group maximum selects in
+    // place only when alone.
+    const bool sum_fmt = sa.agg == kAggSum && !sa.q2;
+    if ((alone || sum_fmt) && nz == 1 && rp.run_k == 1 && rp.parts <= 256 && rp.parts == w.l.rl.parts1 &&
         (long long)rp.parts * (long long)rows <= num_sms()) {
         sa.fused = 1;
+        sa.two_stages = alone ? 0 : 1;
         sa.row_bar = w.rbar;
         sa.bar_base = w.bar_arrivals;
         w.bar_arrivals += 2u * (uint32_t)rp.parts;
@@ -632,7 +638,8 @@ prism_status_t enqueue_step(const prism_config_t &c, const Ws &w, const void *q,
             }
         } else {
             // alone: on one stream, or once no anchor scan remains ahead of the
-            // chain.  (A schedule that ran every group's refined layers alone,
+            // chain (it picks the rescoring block size; see run_refine_batch).
+            // (A schedule that ran every group's refined layers alone,
             // the next anchor's scan overlapping only the current anchor's
             // selection, was measured slower: 38.7 against 30.6 us a layer at
             // 128K; the scans' streaming then no longer hides under the

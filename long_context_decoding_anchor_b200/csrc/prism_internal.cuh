@@ -521,6 +521,7 @@ struct ScoreArgs {
     // positions to sel_out [rows][kap_out] at its offset; ties beyond the
     // shared-memory cache go to tie_spill [rows][tie_cap]
     int fused;
+    int two_stages;         // group sum: the smaller rescoring CTA (two gather stages)
     uint32_t *row_bar;
     uint32_t bar_base;
     int32_t *part_cnt;

@@ -241,10 +241,14 @@ k_anchor_score(ScoreArgs a) {
 // group maximum (Eq. (7)-(9), row format of q2_impl.cuh).
 enum : int { kFmtSum = 0, kFmtMax = 1, kFmtQ2 = 2 };
 
-template <int D, int FMT = kFmtSum>
+// ST: windows in a warp's gather pipeline.  Three keep more bytes in
+// flight; two (an 89 KB CTA at d = 128) let a rescoring CTA share an SM with
+// an anchor-scan CTA and an attention CTA, which a layer whose rows' blocks
+// wait for one another needs while anchor scans are in flight.
+template <int D, int FMT = kFmtSum, int ST = 3>
 struct RescoreCfg {
     static constexpr int kTileRows = 128;              // slots of a window
-    static constexpr int kStages = 3;                  // windows in a warp's pipeline
+    static constexpr int kStages = ST;                 // windows in a warp's pipeline
     static constexpr int kWarps = 8;
     static constexpr int kThreads = 32 * kWarps;
     static constexpr int kRowBytes = FMT == kFmtQ2 ? q2_row_bytes(D) : D * 2;
@@ -648,10 +652,10 @@ __device__ void fused_select(const ScoreArgs &a, int row, int part, int P, int n
         report(a.st, kDevErrInternal, kWhereRescore, (uint32_t)total_sel);
 }
 
-template <int D, int FMT, int NT = 1>
-__global__ void __launch_bounds__(RescoreCfg<D, FMT>::kThreads, 1)
+template <int D, int FMT, int NT = 1, int ST = 3>
+__global__ void __launch_bounds__(RescoreCfg<D, FMT, ST>::kThreads, 1)
 k_refine_rescore(ScoreArgs a) {
-    using C = RescoreCfg<D, FMT>;
+    using C = RescoreCfg<D, FMT, ST>;
     constexpr bool MAXAGG = FMT != kFmtSum;
     constexpr int EPT = kMaxPartEntries / C::kThreads;     // source entries a thread
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -920,15 +924,15 @@ cudaError_t launch_anchor_score(const ScoreArgs &a, int num_sms, cudaStream_t s)
 }
 
 
-template <int D, int FMT, int NT = 1>
+template <int D, int FMT, int NT = 1, int ST = 3>
 static cudaError_t launch_refine_rescore_d(const ScoreArgs &a, cudaStream_t s) {
-    using C = RescoreCfg<D, FMT>;
-    cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D, FMT, NT>,
+    using C = RescoreCfg<D, FMT, ST>;
+    cudaError_t e = cudaFuncSetAttribute(k_refine_rescore<D, FMT, NT, ST>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int nz = a.nz > 1 ? a.nz : 1;
     const int rows = a.B * a.Hkv;
-    return launch_kernel(k_refine_rescore<D, FMT, NT>, dim3((unsigned)a.parts, (unsigned)rows, (unsigned)nz),
+    return launch_kernel(k_refine_rescore<D, FMT, NT, ST>, dim3((unsigned)a.parts, (unsigned)rows, (unsigned)nz),
                          dim3(C::kThreads), C::kSmemBytes, s, a);
 }
 
@@ -945,6 +949,9 @@ cudaError_t launch_refine_rescore(const ScoreArgs &a, cudaStream_t s) {
     if (a.agg == kAggMax)
         return a.d == 128 ? launch_refine_rescore_d<128, kFmtMax>(a, s)
                           : launch_refine_rescore_d<64, kFmtMax>(a, s);
+    if (a.two_stages)
+        return a.d == 128 ? launch_refine_rescore_d<128, kFmtSum, 1, 2>(a, s)
+                          : launch_refine_rescore_d<64, kFmtSum, 1, 2>(a, s);
     return a.d == 128 ? launch_refine_rescore_d<128, kFmtSum>(a, s)
                       : launch_refine_rescore_d<64, kFmtSum>(a, s);
 }
