@@ -424,6 +424,9 @@ prism_status_t run_refine_batch(const prism_config_t &c, const Ws &w, const void
         sa.tie_cap = w.l.rl.tie_cap;
         return cuda_status(launch_refine_rescore(sa, s));
     }
+    // A grid of more blocks than SMs runs in waves of one full-size block per
+    // SM; two two-stage blocks fit an SM, which halves the waves.
+    if (sum_fmt && (long long)rp.parts * (long long)rows * nz > num_sms()) sa.two_stages = 1;
     PRISM_CUDA(launch_refine_rescore(sa, s));
     RunSelectArgs se{};
     se.runs = w.runs; se.run_cnt = w.run_cnt; se.nruns = nruns;
