@@ -480,7 +480,7 @@ def measure_context_parallel(args, rank, world, dev):
         return cp.decode_step_cp(cfg, [me], gather, attn_stream=side, attn_gather=attn_gather)
 
     n0 = prism.lib().prism_launch_count()
-    outs, sel = step()
+    _, sel = step()
     launches = int(prism.lib().prism_launch_count() - n0)
     for _ in range(max(3, args.warmup)):
         step()
@@ -608,10 +608,8 @@ def run_prism(args, rank, world, dev):
     mask = w.anchor_mask()
     prop_sizes = []
     refine_diag = []
-    last_anchor = 0
     for l in range(N):
         if mask[l]:
-            last_anchor = l
             continue
         _, _, _, cc = prism.prism_index_refine(cfg, inp["q"][l], inp["k"][l], inp["lens"],
                                                idx_e[l - 1].contiguous(), cand_cap=1, ws=ws)
