@@ -290,12 +290,16 @@ k_sparse_attn(AttnArgs a) {
     // The last CTA of the row to finish merges the partials (no waiting: an
     // atomic counter decides which CTA that is).
     __shared__ int is_last;
-    __threadfence();
     __syncthreads();
-    if (tid == 0) is_last = atomicAdd(&a.ctl[row].done_attn, 1u) == gridDim.x - 1;
+    if (tid == 0) {
+        // the block's partials (ordered before this thread by the barrier)
+        // become visible before the count: the fence is cumulative
+        __threadfence();
+        is_last = atomicAdd(&a.ctl[row].done_attn, 1u) == gridDim.x - 1;
+        if (is_last) __threadfence();
+    }
     __syncthreads();
     if (!is_last) return;
-    __threadfence();
     combine_row<D, G>(a, row, b, h, gridDim.x, &z[0][0], reinterpret_cast<float2 *>(Ks));
     if (tid == 0) a.ctl[row].done_attn = 0;
 }

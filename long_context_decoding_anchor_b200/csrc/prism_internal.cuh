@@ -282,9 +282,11 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
 // whole block calls it; *ok (shared) says whether the wait completed.
 __device__ __forceinline__ void block_group_barrier(uint32_t *ctr, uint32_t target, uint64_t limit_ns,
                                                     DevStatus *st, uint32_t where, int *ok) {
-    __threadfence();                   // every thread's writes, before the arrival
     __syncthreads();
     if (threadIdx.x == 0) {
+        // the block's writes (ordered before this thread by the barrier)
+        // become visible before the arrival: the fence is cumulative
+        __threadfence();
         atomicAdd(ctr, 1u);
         const uint64_t t0 = global_timer_ns();
         int good = 1;
